@@ -1,0 +1,391 @@
+"""Benchmark of the BRA forward pass (bra_forward = bra_route + bra_attend) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload stage1] [--impl ours|reference]
+
+A step is one pass of the whole hot path (region means, affinity + top-k, gather-attention)
+over one batch of the workload. Inputs are seeded synthetic data of the workload's shape,
+resident in HBM before timing starts; the step rotates through enough input/output buffer
+sets (copies of the batch, rolled along the image axis) that the set it reads was evicted
+from L2 by the others. Each set's route and attend calls are captured once as CUDA graphs
+(eager launches if capture is refused) and replayed; CUDA events on the launching stream
+time every step and every attention kernel. With N > 1 (torchrun), each rank runs its own
+batch (weak scaling, no data-path collective) and the time is the max over ranks.
+
+Prints one JSON line on rank 0. `--impl reference` times the CPU oracle on the host cores
+instead (a bounded sample of the same workload per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "BRA forward tokens/s on 1 B200 (device-timed) and % of roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = {"attend_gather_mma": "bi_level_routing_b200/csrc/bra_attend_mma.cu",
+                  "attend_dense_mma": "bi_level_routing_b200/csrc/bra_attend_mma.cu",
+                  "attend_simt": "bi_level_routing_b200/csrc/bra_attend_simt.cu"}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="stage1")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="do not capture CUDA graphs")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha(rel: str) -> str:
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        table = json.load(f)
+    rec = table.get(kernel, {}).get(workload)
+    if not rec or rec.get("source_sha256") != source_sha(KERNEL_SOURCES[kernel]):
+        return None
+    return rec.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        else:
+            self.lines = []
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline(w, inp, seconds: float):
+    """The oracle's forward pass, as it stands, on the first images of the batch."""
+    import oracle
+    orc = oracle.default()
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    t0 = time.perf_counter()
+    orc.forward(q[:1], k[:1], v[:1], w.n_win, w.topk, w.heads)
+    t1 = time.perf_counter() - t0
+    n = int(max(1, min(w.B, math.floor(seconds / max(t1, 1e-6)))))
+    if n > 1:
+        t0 = time.perf_counter()
+        orc.forward(q[:n], k[:n], v[:n], w.n_win, w.topk, w.heads)
+        t1 = time.perf_counter() - t0
+    return {"value": n * w.N / t1, "unit": UNIT, "cores": orc.max_threads(), "kind": "oracle",
+            "sample": f"oracle forward (route + attend, float64) on the first {n} of {w.B} images "
+                      f"({n * w.N} query tokens), {t1:.2f} s"}
+
+
+def run_reference(args, w, rank):
+    """Reference arm: the CPU oracle timed on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    from bi_level_routing_b200.workloads import make_inputs
+    import oracle
+    sample = w.with_(B=1)
+    inp = make_inputs(sample)
+    orc = oracle.default()
+    for _ in range(args.warmup):
+        orc.forward(inp["q"], inp["k"], inp["v"], w.n_win, w.topk, w.heads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.forward(inp["q"], inp["k"], inp["v"], w.n_win, w.topk, w.heads)
+    dt = time.perf_counter() - t0
+    value = args.steps * sample.N / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(1, args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {**w.describe(), "sample_per_step": f"1 of {w.B} images ({sample.N} query tokens)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": orc.max_threads(), "kind": "oracle",
+                             "sample": f"1 image of {w.name} per step, {args.steps} steps"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from bi_level_routing_b200.workloads import WORKLOADS, make_inputs
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import bi_level_routing_b200 as bra
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    # ---- inputs: one seeded batch per rank, resident in HBM; rotation sets are rolled copies
+    inp = make_inputs(w, seed=w.seed + 1000 * rank)
+    if w.dtype == "bf16":
+        host = [torch.from_numpy(inp[n + "_bits"].view(np.int16)).view(torch.bfloat16) for n in "qkv"]
+    else:
+        host = [torch.from_numpy(inp[n]) for n in "qkv"]
+    base = [t.to(dev) for t in host]
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2**20))
+    set_bytes = w.unique_bytes() + w.B * w.R * w.topk * 4
+    nsets = max(2, math.ceil(2 * l2 / set_bytes) + 1)
+    sets = []
+    for i in range(nsets):
+        q, k, v = (torch.roll(t, shifts=i, dims=0).contiguous() for t in base)
+        out = torch.empty_like(q)
+        idx = torch.empty((w.B, w.R, w.topk), dtype=torch.int32, device=dev)
+        sets.append((q, k, v, out, idx))
+    torch.cuda.synchronize()
+
+    def route(s):
+        q, k, v, out, idx = s
+        bra.route(q, k, w.n_win, w.topk, idx=idx)
+
+    def attend(s):
+        q, k, v, out, idx = s
+        bra.attend(q, k, v, idx, w.heads, w.n_win, out=out)
+
+    # eager warm-up (also initialises the library's per-device state before any capture)
+    for i in range(max(3, args.warmup)):
+        route(sets[i % nsets])
+        attend(sets[i % nsets])
+    torch.cuda.synchronize()
+
+    launch = "eager"
+    graphs = None
+    if not args.eager:
+        try:
+            graphs = []
+            for s in sets:
+                ga, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+                with torch.cuda.graph(ga):
+                    route(s)
+                with torch.cuda.graph(gb):
+                    attend(s)
+                graphs.append((ga, gb))
+            launch = "cuda_graph"
+        except Exception as e:  # capture refused: time eager launches
+            graphs = None
+            launch = f"eager (graph capture failed: {type(e).__name__})"
+            torch.cuda.synchronize()
+
+    def step(i):
+        if graphs:
+            ga, gb = graphs[i % nsets]
+            return ga.replay, gb.replay
+        s = sets[i % nsets]
+        return (lambda: route(s)), (lambda: attend(s))
+
+    for i in range(args.warmup):
+        a, b = step(i)
+        a()
+        b()
+    torch.cuda.synchronize()
+
+    # ---- clock samples over a soak of identical steps around the timed region
+    sampler = ClockSampler(local_rank)
+    K = args.steps
+    ev_route = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_attend = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_end = torch.cuda.Event(enable_timing=True)
+    with sampler:
+        t_soak = time.perf_counter()
+        i = 0
+        while time.perf_counter() - t_soak < 1.0:
+            a, b = step(i)
+            a()
+            b()
+            i += 1
+            if i % 64 == 0:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(K):
+            a, b = step(i)
+            ev_route[i].record()
+            a()
+            ev_attend[i].record()
+            b()
+        ev_end.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        # keep the GPU busy while the sampler catches the tail
+        t_tail = time.perf_counter()
+        i = 0
+        while time.perf_counter() - t_tail < 0.5:
+            a, b = step(i)
+            a()
+            b()
+            i += 1
+            if i % 64 == 0:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+
+    total_ms = ev_route[0].elapsed_time(ev_end)
+    attend_ms = [ev_attend[i].elapsed_time(ev_route[i + 1] if i + 1 < K else ev_end) for i in range(K)]
+    route_ms = [ev_route[i].elapsed_time(ev_attend[i]) for i in range(K)]
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    tokens = w.tokens * world
+    value = tokens * K / (total_ms / 1e3)
+    ms_per_step = total_ms / K
+
+    # ---- roofline of the dominant kernel
+    pk, pk_kind = peaks()
+    hbm = float(pk["hbm_gbs"])
+    kernel = bra.selected_attend_kernel(w.B, w.H, w.W, w.C, w.heads, w.n_win, w.topk,
+                                        torch.bfloat16 if w.dtype == "bf16" else torch.float32)
+    kname = "attend_" + kernel
+    mean_attend = statistics.mean(attend_ms)
+    mean_route = statistics.mean(route_ms)
+    attend_bytes = w.unique_bytes()  # q, k, v read once, out written once
+    achieved = attend_bytes / (mean_attend / 1e3) / 1e9
+    traffic = recorded_traffic(kname, w.name)
+    roof_step_ms = max(w.unique_bytes() / (hbm * 1e9),
+                       w.attention_flops() / (float(pk["bf16_tflops"]) * 1e12)) * 1e3
+    roofline = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": traffic,
+                "peak_source": f"{pk_kind} hbm_gbs (MEASURED_PEAKS.json)" if pk_kind == "measured" else "fallback",
+                "algorithmic_bytes_per_launch": attend_bytes, "mean_launch_us": mean_attend * 1e3,
+                "route_kernels_mean_us": mean_route * 1e3,
+                "step_roofline_us": roof_step_ms * 1e3, "step_frac": roof_step_ms / ms_per_step,
+                "step_frac_vs_8tbs": (w.unique_bytes() / 8e12 * 1e3) / ms_per_step}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic",
+            "config": {**w.describe(), "l2": f"rotating {nsets} buffer sets of {set_bytes / 1e6:.1f} MB "
+                                             f"(> 2x the {l2 / 2**20:.0f} MiB L2)",
+                       "launch": launch, "parallelism": f"dp{world} (images split, no collective)"},
+            "roofline": roofline,
+            "gpu_launches": K * bra.kernels_per_call("bra_forward", w.B),
+            "clocks": sampler.summary()}
+
+    # ---- end to end through the host entry point (pinned buffers, copies inside the timed region)
+    if not args.no_e2e:
+        hq, hk, hv = (t.pin_memory() for t in host)
+        hout = torch.empty_like(hq).pin_memory()
+        hidx = torch.empty((w.B, w.R, w.topk), dtype=torch.int32).pin_memory()
+        for _ in range(2):
+            bra.forward_host(hq, hk, hv, w.n_win, w.topk, w.heads, out=hout, idx=hidx)
+        ke = max(3, min(20, K))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(ke):
+            bra.forward_host(hq, hk, hv, w.n_win, w.topk, w.heads, out=hout, idx=hidx)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        line["e2e"] = {"value": tokens * ke / (e2e_ms / 1e3), "unit": UNIT,
+                       "h2d_bytes_per_step": 3 * w.B * w.N * w.C * w.elem_bytes,
+                       "d2h_bytes_per_step": w.B * w.N * w.C * w.elem_bytes + w.B * w.R * w.topk * 4,
+                       "steps": ke, "entry_point": "bra_forward_host"}
+
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_seconds)
+
+    del graphs
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

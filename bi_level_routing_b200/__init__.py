@@ -1,7 +1,9 @@
 """Bi-Level Routing Attention (BRA) forward pass for NVIDIA B200 (sm_100a).
 
 The compute lives in ``libbra.so`` (hand-written CUDA behind a C ABI, declared in
-``include/bra.h``); this package only marshals torch tensors into it. The binding is
-loaded on first use and raises if the library is missing: there is no CPU fallback.
+``include/bra.h``); this package only marshals torch tensors into it. The library is loaded
+on first use and a missing library raises: there is no CPU fallback.
 """
+from .api import (BraError, attend, check_device_error, forward, forward_host, kernels_per_call,  # noqa: F401
+                  route, route_scratch_bytes, selected_attend_kernel, set_attend_kernel)
 from .workloads import HEADLINE, WORKLOADS, Workload, make_inputs  # noqa: F401

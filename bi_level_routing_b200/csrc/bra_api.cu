@@ -1,0 +1,353 @@
+// bra_api.cu -- the C ABI of libbra.so (declared in include/bra.h): argument validation,
+// kernel selection, TMA descriptors, the per-device scratch pool and the device error word.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "bra.h"
+#include "bra_launch.h"
+
+namespace {
+
+// Sticky device error word (kErrIndex | kErrTimeout), one per device.
+__device__ unsigned g_device_error;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool ready = false;
+    unsigned *error_word = nullptr;
+    cudaMemPool_t pool = nullptr;
+    int num_sms = 0;
+};
+
+std::mutex g_mutex;
+DeviceState g_devices[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::atomic<int> g_forced_kernel{BRA_ATTEND_AUTO};
+thread_local std::string g_last_error;
+
+bra_status cuda_fail(cudaError_t e, const char *what)
+{
+    g_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+    return BRA_ERR_CUDA;
+}
+
+// Per-device set-up on first use: error word address, SM count, scratch pool, TMA encoder.
+bra_status device_state(DeviceState **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) {
+        g_last_error = "device ordinal out of range";
+        return BRA_ERR_UNSUPPORTED;
+    }
+    DeviceState &st = g_devices[dev];
+    if (!st.ready) {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!st.ready) {
+            void *p = nullptr;
+            if ((e = cudaGetSymbolAddress(&p, g_device_error)) != cudaSuccess)
+                return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+            st.error_word = static_cast<unsigned *>(p);
+            if ((e = cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+                return cuda_fail(e, "cudaDeviceGetAttribute");
+            cudaMemPoolProps props;
+            std::memset(&props, 0, sizeof(props));
+            props.allocType = cudaMemAllocationTypePinned;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            if ((e = cudaMemPoolCreate(&st.pool, &props)) != cudaSuccess) return cuda_fail(e, "cudaMemPoolCreate");
+            uint64_t keep = ~0ull;  // keep freed scratch in the pool
+            if ((e = cudaMemPoolSetAttribute(st.pool, cudaMemPoolAttrReleaseThreshold, &keep)) != cudaSuccess)
+                return cuda_fail(e, "cudaMemPoolSetAttribute");
+            if (!g_encode) {
+                void *fn = nullptr;
+                cudaDriverEntryPointQueryResult q;
+                e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
+                if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) {
+                    g_last_error = "cuTensorMapEncodeTiled not available from the driver";
+                    return BRA_ERR_CUDA;
+                }
+                g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+            }
+            st.ready = true;
+        }
+    }
+    *out = &st;
+    return BRA_OK;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shape checks shared by every entry point (pointers are checked by the callers).
+bra_status check_shape(int B, int H, int W, int C, int heads, int n_win, int topk, bra_dtype dtype,
+                       bra::Geometry *g)
+{
+    if (dtype != BRA_F32 && dtype != BRA_BF16) return BRA_ERR_INVALID_ARG;
+    if (B < 0 || H <= 0 || W <= 0 || C <= 0 || heads <= 0 || n_win <= 0 || topk <= 0) return BRA_ERR_INVALID_ARG;
+    if (H % n_win != 0 || W % n_win != 0 || C % heads != 0) return BRA_ERR_INVALID_ARG;
+    const long long R = (long long)n_win * n_win;
+    if (topk > R) return BRA_ERR_INVALID_ARG;
+    const int elem = dtype == BRA_BF16 ? 2 : 4;
+    if (((long long)C * elem) % 16 != 0) return BRA_ERR_INVALID_ARG;
+    if (R > bra::kMaxRegions) return BRA_ERR_UNSUPPORTED;
+    if ((long long)H * W > 0x7fffffffLL / 2) return BRA_ERR_UNSUPPORTED;
+    g->B = B;
+    g->H = H;
+    g->W = W;
+    g->C = C;
+    g->heads = heads;
+    g->n_win = n_win;
+    g->topk = topk;
+    g->R = (int)R;
+    g->hr = H / n_win;
+    g->wr = W / n_win;
+    g->rs = g->hr * g->wr;
+    g->hd = C / heads;
+    g->N = H * W;
+    // The means kernel keeps one region column's partial sums (wr x C fp32) in 48 KB.
+    if ((long long)g->wr * C * 4 > 48 * 1024) return BRA_ERR_UNSUPPORTED;
+    return BRA_OK;
+}
+
+int choose_attend_kernel(const bra::Geometry &g, bra_dtype dtype)
+{
+    const bool bf16 = dtype == BRA_BF16;
+    const bool simt_ok = g.hd <= bra::kSimtMaxHeadDim;
+    const bool gather_ok = bf16 && bra::gather_mma_supports(g);
+    const bool dense_ok = bf16 && bra::dense_mma_supports(g);
+    switch (g_forced_kernel.load()) {
+    case BRA_ATTEND_SIMT: return simt_ok ? BRA_ATTEND_SIMT : -1;
+    case BRA_ATTEND_GATHER_MMA: return gather_ok ? BRA_ATTEND_GATHER_MMA : -1;
+    case BRA_ATTEND_DENSE_MMA: return dense_ok ? BRA_ATTEND_DENSE_MMA : -1;
+    default: break;
+    }
+    // Dense attention over the whole image wastes at most 4x the routed work here.
+    if (dense_ok && 4LL * g.topk * g.rs >= g.N) return BRA_ATTEND_DENSE_MMA;
+    if (gather_ok) return BRA_ATTEND_GATHER_MMA;
+    if (dense_ok) return BRA_ATTEND_DENSE_MMA;
+    return simt_ok ? BRA_ATTEND_SIMT : -1;
+}
+
+// 4-D bf16 tensor map of a [B, H, W, C] array, 128-byte swizzle, box (64, bw, bh, 1).
+bra_status encode_map(CUtensorMap *map, const void *base, const bra::Geometry &g, int bw, int bh)
+{
+    cuuint64_t dims[4] = {(cuuint64_t)g.C, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.B};
+    cuuint64_t strides[3] = {(cuuint64_t)g.C * 2, (cuuint64_t)g.W * g.C * 2, (cuuint64_t)g.H * g.W * g.C * 2};
+    cuuint32_t box[4] = {64u, (cuuint32_t)bw, (cuuint32_t)bh, 1u};
+    cuuint32_t elem_strides[4] = {1u, 1u, 1u, 1u};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
+                          elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_error = "cuTensorMapEncodeTiled failed with CUresult " + std::to_string((int)r);
+        return BRA_ERR_CUDA;
+    }
+    return BRA_OK;
+}
+
+bra_status route_impl(const void *q, const void *k, int32_t *idx, const bra::Geometry &g, bra_dtype dtype,
+                      cudaStream_t stream)
+{
+    DeviceState *st = nullptr;
+    bra_status s = device_state(&st);
+    if (s != BRA_OK) return s;
+    const size_t bytes = (size_t)2 * g.B * g.R * g.C * sizeof(float);
+    void *scratch = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(&scratch, bytes, st->pool, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync(route scratch)");
+    float *qm = static_cast<float *>(scratch);
+    float *km = qm + (size_t)g.B * g.R * g.C;
+    e = bra::launch_region_means(q, k, qm, km, g, dtype == BRA_BF16, st->num_sms, stream);
+    if (e == cudaSuccess) e = bra::launch_route_topk(qm, km, idx, g, stream);
+    cudaError_t f = cudaFreeAsync(scratch, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "routing kernels");
+    if (f != cudaSuccess) return cuda_fail(f, "cudaFreeAsync(route scratch)");
+    return BRA_OK;
+}
+
+bra_status attend_impl(const void *q, const void *k, const void *v, const int32_t *idx, void *out,
+                       const bra::Geometry &g, bra_dtype dtype, cudaStream_t stream)
+{
+    const int kernel = choose_attend_kernel(g, dtype);
+    if (kernel < 0) return BRA_ERR_UNSUPPORTED;
+    DeviceState *st = nullptr;
+    bra_status s = device_state(&st);
+    if (s != BRA_OK) return s;
+    cudaError_t e = cudaSuccess;
+    if (kernel == BRA_ATTEND_SIMT) {
+        e = bra::launch_attend_simt(q, k, v, idx, out, g, dtype == BRA_BF16, st->error_word, stream);
+    } else if (kernel == BRA_ATTEND_GATHER_MMA) {
+        CUtensorMap tq, tk, tv, to;
+        int box[4];
+        bra::gather_mma_box(g, box);
+        if ((s = encode_map(&tq, q, g, box[1], box[2])) != BRA_OK) return s;
+        if ((s = encode_map(&tk, k, g, box[1], box[2])) != BRA_OK) return s;
+        if ((s = encode_map(&tv, v, g, box[1], box[2])) != BRA_OK) return s;
+        if ((s = encode_map(&to, out, g, box[1], box[2])) != BRA_OK) return s;
+        e = bra::launch_attend_gather_mma(tq, tk, tv, to, idx, g, st->error_word, stream);
+    } else {
+        const int rows = bra::dense_mma_rows_per_split(g, st->num_sms);
+        CUtensorMap tq, tk, tv, to;
+        if ((s = encode_map(&tq, q, g, g.W, rows)) != BRA_OK) return s;
+        if ((s = encode_map(&tk, k, g, g.W, g.H)) != BRA_OK) return s;
+        if ((s = encode_map(&tv, v, g, g.W, g.H)) != BRA_OK) return s;
+        if ((s = encode_map(&to, out, g, g.W, rows)) != BRA_OK) return s;
+        e = bra::launch_attend_dense_mma(tq, tk, tv, to, idx, g, rows, st->error_word, stream);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "attention kernel");
+    return BRA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+bra_status bra_route(const void *q, const void *k, int32_t *idx, int B, int H, int W, int C, int n_win, int topk,
+                     bra_dtype dtype, void *stream)
+{
+    bra::Geometry g;
+    bra_status s = check_shape(B, H, W, C, 1, n_win, topk, dtype, &g);
+    if (s != BRA_OK) return s;
+    if (B == 0) return BRA_OK;
+    if (!q || !k || !idx) return BRA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(idx, 4)) return BRA_ERR_INVALID_ARG;
+    return route_impl(q, k, idx, g, dtype, static_cast<cudaStream_t>(stream));
+}
+
+bra_status bra_attend(const void *q, const void *k, const void *v, const int32_t *idx, void *out, int B, int H,
+                      int W, int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream)
+{
+    bra::Geometry g;
+    bra_status s = check_shape(B, H, W, C, heads, n_win, topk, dtype, &g);
+    if (s != BRA_OK) return s;
+    if (B == 0) return BRA_OK;
+    if (!q || !k || !v || !idx || !out) return BRA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(idx, 4))
+        return BRA_ERR_INVALID_ARG;
+    return attend_impl(q, k, v, idx, out, g, dtype, static_cast<cudaStream_t>(stream));
+}
+
+bra_status bra_forward(const void *q, const void *k, const void *v, int32_t *idx, void *out, int B, int H, int W,
+                       int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream)
+{
+    bra::Geometry g;
+    bra_status s = check_shape(B, H, W, C, heads, n_win, topk, dtype, &g);
+    if (s != BRA_OK) return s;
+    if (B == 0) return BRA_OK;
+    if (!q || !k || !v || !idx || !out) return BRA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(idx, 4))
+        return BRA_ERR_INVALID_ARG;
+    if (choose_attend_kernel(g, dtype) < 0) return BRA_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((s = route_impl(q, k, idx, g, dtype, st)) != BRA_OK) return s;
+    return attend_impl(q, k, v, idx, out, g, dtype, st);
+}
+
+bra_status bra_forward_host(const void *q, const void *k, const void *v, int32_t *idx, void *out, int B, int H,
+                            int W, int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream)
+{
+    bra::Geometry g;
+    bra_status s = check_shape(B, H, W, C, heads, n_win, topk, dtype, &g);
+    if (s != BRA_OK) return s;
+    if (B == 0) return BRA_OK;
+    if (!q || !k || !v || !idx || !out) return BRA_ERR_INVALID_ARG;
+    if (choose_attend_kernel(g, dtype) < 0) return BRA_ERR_UNSUPPORTED;
+    DeviceState *dst = nullptr;
+    if ((s = device_state(&dst)) != BRA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t elem = dtype == BRA_BF16 ? 2 : 4;
+    const size_t tensor = (size_t)B * H * W * C * elem;
+    const size_t tensor_padded = (tensor + 255) & ~(size_t)255;
+    const size_t idx_bytes = (size_t)B * g.R * topk * sizeof(int32_t);
+    uint8_t *buf = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&buf), 4 * tensor_padded + idx_bytes, dst->pool, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync(host staging)");
+    uint8_t *dq = buf, *dk = buf + tensor_padded, *dv = buf + 2 * tensor_padded, *dout = buf + 3 * tensor_padded;
+    int32_t *didx = reinterpret_cast<int32_t *>(buf + 4 * tensor_padded);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dq, q, tensor, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dk, k, tensor, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dv, v, tensor, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) {
+        s = route_impl(dq, dk, didx, g, dtype, st);
+        if (s == BRA_OK) s = attend_impl(dq, dk, dv, didx, dout, g, dtype, st);
+        if (s == BRA_OK) e = cudaMemcpyAsync(idx, didx, idx_bytes, cudaMemcpyDeviceToHost, st);
+        if (s == BRA_OK && e == cudaSuccess) e = cudaMemcpyAsync(out, dout, tensor, cudaMemcpyDeviceToHost, st);
+    }
+    cudaError_t f = cudaFreeAsync(buf, st);
+    cudaError_t y = cudaStreamSynchronize(st);
+    if (s != BRA_OK) return s;
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync");
+    if (f != cudaSuccess) return cuda_fail(f, "cudaFreeAsync(host staging)");
+    if (y != cudaSuccess) return cuda_fail(y, "cudaStreamSynchronize");
+    return BRA_OK;
+}
+
+bra_status bra_set_attend_kernel(bra_attend_kernel kernel)
+{
+    if (kernel < BRA_ATTEND_AUTO || kernel > BRA_ATTEND_DENSE_MMA) return BRA_ERR_INVALID_ARG;
+    g_forced_kernel.store(kernel);
+    return BRA_OK;
+}
+
+int bra_selected_attend_kernel(int B, int H, int W, int C, int heads, int n_win, int topk, bra_dtype dtype)
+{
+    bra::Geometry g;
+    if (check_shape(B, H, W, C, heads, n_win, topk, dtype, &g) != BRA_OK) return -1;
+    return choose_attend_kernel(g, dtype);
+}
+
+bra_status bra_check_device_error(void *stream)
+{
+    DeviceState *st = nullptr;
+    bra_status s = device_state(&st);
+    if (s != BRA_OK) return s;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned word = 0;
+    if ((e = cudaMemcpy(&word, st->error_word, sizeof(word), cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(e, "read error word");
+    if ((e = cudaMemset(st->error_word, 0, sizeof(word))) != cudaSuccess) return cuda_fail(e, "clear error word");
+    if (word & bra::kErrTimeout) return BRA_ERR_TIMEOUT;
+    if (word & bra::kErrIndex) return BRA_ERR_INDEX;
+    return BRA_OK;
+}
+
+size_t bra_route_scratch_bytes(int B, int H, int W, int C, int n_win)
+{
+    if (B <= 0 || H <= 0 || W <= 0 || C <= 0 || n_win <= 0) return 0;
+    return (size_t)2 * B * n_win * n_win * C * sizeof(float);
+}
+
+int bra_kernels_per_call(const char *entry_point, int B)
+{
+    if (!entry_point || B <= 0) return 0;
+    if (!std::strcmp(entry_point, "bra_route")) return 2;
+    if (!std::strcmp(entry_point, "bra_attend")) return 1;
+    if (!std::strcmp(entry_point, "bra_forward") || !std::strcmp(entry_point, "bra_forward_host")) return 3;
+    return 0;
+}
+
+const char *bra_status_string(bra_status status)
+{
+    switch (status) {
+    case BRA_OK: return "BRA_OK";
+    case BRA_ERR_INVALID_ARG: return "BRA_ERR_INVALID_ARG";
+    case BRA_ERR_UNSUPPORTED: return "BRA_ERR_UNSUPPORTED";
+    case BRA_ERR_CUDA: return "BRA_ERR_CUDA";
+    case BRA_ERR_INDEX: return "BRA_ERR_INDEX";
+    case BRA_ERR_TIMEOUT: return "BRA_ERR_TIMEOUT";
+    default: return "BRA_ERR_UNKNOWN";
+    }
+}
+
+const char *bra_last_error_message(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,535 @@
+// bra_attend_mma.cu -- token-to-token attention over the routed regions on tensor cores (bf16).
+//
+// What it computes ("从零构建BiFormer", §2.2 TokenAttention; "医学图像分割模块：BiFormer /
+// 双层路由注意力", §五 steps ⑤-⑦): for every query token of region r and every head, softmax
+// (scale head_dim^-1/2) over the tokens of the regions idx[b, r, 0..topk-1], then the weighted
+// sum of their values. Accumulation, softmax and normalisation are fp32; P is rounded to bf16
+// for the PV product; out is rounded to bf16.
+//
+// Two kernels, both with K/V staged in shared memory by TMA (cp.async.bulk.tensor, 128-byte
+// swizzle, no multicast) and the gathered K/V never written to HBM:
+//
+// * gather: one CTA per (image, query region, group of 64-channel blocks). The query tile and,
+//   per routed region, its K and V tiles (rs tokens x 64 channels each) arrive by TMA on
+//   mbarriers, up to four regions in flight. Each warp owns 16 query rows of one head and runs
+//   S = Q K^T and O += P V with mma.sync m16n8k16, folding the softmax online (exp2 with a
+//   log2(e) pre-scale, running max and sum in registers). The output tile is staged in the
+//   query tile's shared memory and written back by one TMA store. Needs rs % 16 == 0, rs <= 64.
+//
+// * dense: for tiny regions (rs of 1 or 4 tokens, where a 16-row MMA tile spans several query
+//   regions). One CTA per (image, 64-channel block, band of query rows) stages the whole
+//   image's K and V once; every query row attends to every key of the image with weight
+//   cnt[region(query), region(key)] = number of times the key's region occurs in the query
+//   region's idx row (0 masks it). That is exactly the gather semantics, duplicates included:
+//   softmax over a concatenated key list weights each distinct key by its multiplicity. The
+//   weight enters as +log2(cnt) on the logit. Needs R <= 64 and H * W <= 256.
+#include "bra_device.cuh"
+#include "bra_launch.h"
+
+namespace bra {
+
+constexpr int kRowBytes = 128;  // one token's 64 bf16 channels
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current device, once per
+// (kernel, device, size high-water mark): later calls, including those made during CUDA
+// graph capture, issue no attribute call.
+template <typename Kernel>
+static cudaError_t ensure_smem_limit(Kernel kernel, size_t bytes, int (&granted)[64])
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if ((int)bytes <= granted[dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) granted[dev] = (int)bytes;
+    return e;
+}
+
+struct GatherArgs {
+    const int32_t *idx;
+    unsigned *err;
+    int n_win, topk, R, hr, wr;
+    int ncb;          // 64-channel blocks in C
+    int ncb_per_cta;  // channel blocks one CTA covers
+    int groups;       // CTAs per (image, region)
+    int nstage;       // routed regions in flight
+    float scale_log2;
+};
+
+__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v)
+{
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Rescales the running output and sum of one row pair by corr0 (row g) and corr1 (row g+8).
+__device__ __forceinline__ void rescale(float (&o)[4][4], float (&l)[2], float corr0, float corr1)
+{
+    l[0] *= corr0;
+    l[1] *= corr1;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+        o[nt][0] *= corr0;
+        o[nt][1] *= corr0;
+        o[nt][2] *= corr1;
+        o[nt][3] *= corr1;
+    }
+}
+
+__device__ __forceinline__ float quad_max(float x)
+{
+    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
+    return fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
+}
+
+__device__ __forceinline__ float quad_sum(float x)
+{
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    return x + __shfl_xor_sync(0xffffffffu, x, 2);
+}
+
+// O += P V for KSTEPS 16-key steps; P in the S accumulators sc (fp32, rounded to bf16 here),
+// V tile at vtile (keys x 64 channels, swizzled), key offset key0, head hb of the block.
+template <int KSTEPS>
+__device__ __forceinline__ void pv_product(float (&o)[4][4], const float (*sc)[4], uint32_t vtile, int key0, int hb,
+                                           int lane)
+{
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+        uint32_t pa[4];
+        pa[0] = pack_bf16x2(sc[2 * kk][0], sc[2 * kk][1]);
+        pa[1] = pack_bf16x2(sc[2 * kk][2], sc[2 * kk][3]);
+        pa[2] = pack_bf16x2(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
+        pa[3] = pack_bf16x2(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {
+            uint32_t b0, b1, b2, b3;
+            const int row = key0 + kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+            ldmatrix_x4_trans(vtile + sw128(row, hb * 4 + np * 2 + (lane >> 4)), b0, b1, b2, b3);
+            mma_bf16_16816(o[2 * np], pa, b0, b1);
+            mma_bf16_16816(o[2 * np + 1], pa, b2, b3);
+        }
+    }
+}
+
+// Writes this warp's normalised 16 x 32 output (rows row0.., head hb) into a swizzled tile.
+__device__ __forceinline__ void stage_output(uint32_t tile, const float (&o)[4][4], const float (&l)[2], int row0,
+                                             int hb, int lane)
+{
+    const float l0 = quad_sum(l[0]), l1 = quad_sum(l[1]);
+    const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+        st_shared_u32(tile + sw128(row0 + g, hb * 4 + nt) + 4 * t, pack_bf16x2(o[nt][0] * inv0, o[nt][1] * inv0));
+        st_shared_u32(tile + sw128(row0 + g + 8, hb * 4 + nt) + 4 * t, pack_bf16x2(o[nt][2] * inv1, o[nt][3] * inv1));
+    }
+}
+
+template <int RS>
+__global__ void __launch_bounds__(256) attend_gather_mma_kernel(const __grid_constant__ CUtensorMap tq,
+                                                                const __grid_constant__ CUtensorMap tk,
+                                                                const __grid_constant__ CUtensorMap tv,
+                                                                const __grid_constant__ CUtensorMap tout,
+                                                                const GatherArgs a)
+{
+    constexpr int RT = RS / 16;             // 16-row tiles per region
+    constexpr int NT = RS / 8;              // 8-key n-tiles per region
+    constexpr int TILE = RS * kRowBytes;    // one (region, 64-channel block) tile
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int NCB = a.ncb_per_cta;
+    uint8_t *sQ = smem;
+    uint8_t *sKV = smem + NCB * TILE;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sKV + (size_t)a.nstage * 2 * NCB * TILE);
+    int *stage_ok = reinterpret_cast<int *>(bars + 1 + a.nstage);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int64_t item = blockIdx.x;
+    const int grp = (int)(item % a.groups);
+    item /= a.groups;
+    const int r = (int)(item % a.R);
+    const int b = (int)(item / a.R);
+    const int qx = (r % a.n_win) * a.wr, qy = (r / a.n_win) * a.hr;
+    const int cb0 = grp * NCB;
+    const int ncb_here = min(NCB, a.ncb - cb0);
+    const int32_t *routed = a.idx + ((int64_t)b * a.R + r) * a.topk;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[0], 1);
+        for (int i = 0; i < a.nstage; ++i) mbar_init(&bars[1 + i], 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+
+    // Thread 0 only: load routed region j's K and V tiles into stage slot j % nstage.
+    auto issue_stage = [&](int j) {
+        const int slot = j % a.nstage;
+        const int s = routed[j];
+        const bool ok = (s >= 0 && s < a.R);
+        stage_ok[slot] = ok;
+        uint64_t *bar = &bars[1 + slot];
+        if (!ok) {
+            flag_error(a.err, kErrIndex);
+            mbar_arrive_expect_tx(bar, 0);
+            return;
+        }
+        mbar_arrive_expect_tx(bar, (uint32_t)(2 * ncb_here * TILE));
+        const int sx = (s % a.n_win) * a.wr, sy = (s / a.n_win) * a.hr;
+        uint8_t *kt = sKV + (size_t)slot * 2 * NCB * TILE;
+        uint8_t *vt = kt + NCB * TILE;
+        for (int cb = 0; cb < ncb_here; ++cb) {
+            tma_load_4d(kt + cb * TILE, &tk, (cb0 + cb) * 64, sx, sy, b, bar);
+            tma_load_4d(vt + cb * TILE, &tv, (cb0 + cb) * 64, sx, sy, b, bar);
+        }
+    };
+
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(&bars[0], (uint32_t)(ncb_here * TILE));
+        for (int cb = 0; cb < ncb_here; ++cb) tma_load_4d(sQ + cb * TILE, &tq, (cb0 + cb) * 64, qx, qy, b, &bars[0]);
+        const int first = min(a.nstage, a.topk);
+        for (int j = 0; j < first; ++j) issue_stage(j);
+    }
+
+    const int rt = warp % RT, hb = (warp / RT) & 1, cbl = warp / (2 * RT);
+    const bool active = cbl < ncb_here;
+    const uint32_t qtile = smem_u32(sQ + cbl * TILE);
+
+    uint32_t qf[2][4];
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    float o[4][4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+
+    bool alive = mbar_wait(&bars[0], 0, a.err);
+    if (alive && active) {
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+            ldmatrix_x4(qtile + sw128(rt * 16 + (lane & 15), hb * 4 + ks * 2 + (lane >> 4)), qf[ks][0], qf[ks][1],
+                        qf[ks][2], qf[ks][3]);
+    }
+
+    for (int j = 0; j < a.topk; ++j) {
+        const int slot = j % a.nstage;
+        if (alive) alive = mbar_wait(&bars[1 + slot], (uint32_t)((j / a.nstage) & 1), a.err);
+        if (alive && active && stage_ok[slot]) {
+            const uint32_t ktile = smem_u32(sKV + (size_t)slot * 2 * NCB * TILE + cbl * TILE);
+            const uint32_t vtile = ktile + NCB * TILE;
+            float sc[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4(ktile + sw128(nt * 8 + (lane & 7), hb * 4 + (lane >> 3)), b0, b1, b2, b3);
+                mma_bf16_16816(sc[nt], qf[0], b0, b1);
+                mma_bf16_16816(sc[nt], qf[1], b2, b3);
+            }
+            float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
+                mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
+            }
+            const float mn0 = fmaxf(m[0], quad_max(mx0) * a.scale_log2);
+            const float mn1 = fmaxf(m[1], quad_max(mx1) * a.scale_log2);
+            rescale(o, l, exp2f(m[0] - mn0), exp2f(m[1] - mn1));
+            m[0] = mn0;
+            m[1] = mn1;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                sc[nt][0] = exp2f(fmaf(sc[nt][0], a.scale_log2, -mn0));
+                sc[nt][1] = exp2f(fmaf(sc[nt][1], a.scale_log2, -mn0));
+                sc[nt][2] = exp2f(fmaf(sc[nt][2], a.scale_log2, -mn1));
+                sc[nt][3] = exp2f(fmaf(sc[nt][3], a.scale_log2, -mn1));
+                l[0] += sc[nt][0] + sc[nt][1];
+                l[1] += sc[nt][2] + sc[nt][3];
+            }
+            pv_product<RT>(o, sc, vtile, 0, hb, lane);
+        }
+        if (j + a.nstage < a.topk) {
+            __syncthreads();  // every warp is done with this slot
+            if (threadIdx.x == 0 && alive) issue_stage(j + a.nstage);
+        }
+    }
+
+    __syncthreads();  // the query tiles are free: stage the output there
+    if (alive && active) stage_output(qtile, o, l, rt * 16, hb, lane);
+    fence_async_shared();
+    __syncthreads();
+    if (threadIdx.x == 0 && alive) {
+        for (int cb = 0; cb < ncb_here; ++cb) tma_store_4d(&tout, sQ + cb * TILE, (cb0 + cb) * 64, qx, qy, b);
+        tma_store_commit();
+        tma_store_wait_read();
+    }
+}
+
+bool gather_mma_supports(const Geometry &g)
+{
+    return g.hd == 32 && g.C % 64 == 0 && g.rs % 16 == 0 && g.rs <= 64 && g.wr <= 256 && g.hr <= 256;
+}
+
+void gather_mma_box(const Geometry &g, int box[4])
+{
+    box[0] = 64;
+    box[1] = g.wr;
+    box[2] = g.hr;
+    box[3] = 1;
+}
+
+template <int RS>
+static cudaError_t launch_gather_rs(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                    const CUtensorMap &tout, const GatherArgs &a, int threads, size_t smem,
+                                    long long blocks, cudaStream_t stream)
+{
+    static_assert(RS % 16 == 0 && RS <= 64, "tokens per region");
+    static int granted[64] = {0};
+    cudaError_t e = ensure_smem_limit(attend_gather_mma_kernel<RS>, smem, granted);
+    if (e != cudaSuccess) return e;
+    attend_gather_mma_kernel<RS><<<(unsigned)blocks, threads, smem, stream>>>(tq, tk, tv, tout, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                     const CUtensorMap &tout, const int32_t *idx, const Geometry &g, unsigned *err,
+                                     cudaStream_t stream)
+{
+    GatherArgs a;
+    a.idx = idx;
+    a.err = err;
+    a.n_win = g.n_win;
+    a.topk = g.topk;
+    a.R = g.R;
+    a.hr = g.hr;
+    a.wr = g.wr;
+    a.ncb = g.C / 64;
+    const int rt = g.rs / 16;
+    int ncb_per_cta = 8 / (2 * rt);
+    if (ncb_per_cta < 1) ncb_per_cta = 1;
+    if (ncb_per_cta > a.ncb) ncb_per_cta = a.ncb;
+    a.ncb_per_cta = ncb_per_cta;
+    a.groups = (a.ncb + ncb_per_cta - 1) / ncb_per_cta;
+    a.nstage = g.topk < 4 ? g.topk : 4;
+    a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)g.hd));
+    const int threads = ncb_per_cta * 2 * rt * 32;
+    const size_t tile = (size_t)g.rs * kRowBytes;
+    const size_t smem = 1024 + tile * ncb_per_cta * (1 + 2 * (size_t)a.nstage) + 8 * (1 + a.nstage) + 4 * a.nstage;
+    const long long blocks = (long long)g.B * g.R * a.groups;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    switch (g.rs) {
+    case 16: return launch_gather_rs<16>(tq, tk, tv, tout, a, threads, smem, blocks, stream);
+    case 32: return launch_gather_rs<32>(tq, tk, tv, tout, a, threads, smem, blocks, stream);
+    case 48: return launch_gather_rs<48>(tq, tk, tv, tout, a, threads, smem, blocks, stream);
+    case 64: return launch_gather_rs<64>(tq, tk, tv, tout, a, threads, smem, blocks, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+// ------------------------------------------------------------------------- dense kernel
+
+struct DenseArgs {
+    const int32_t *idx;
+    unsigned *err;
+    int H, W, n_win, topk, R, hr, wr, N, npad;
+    int ncb;             // 64-channel blocks in C
+    int rows_per_split;  // image rows of queries per CTA
+    int nsplit;
+    float scale_log2;
+};
+
+__global__ void __launch_bounds__(256) attend_dense_mma_kernel(const __grid_constant__ CUtensorMap tq,
+                                                               const __grid_constant__ CUtensorMap tk,
+                                                               const __grid_constant__ CUtensorMap tv,
+                                                               const __grid_constant__ CUtensorMap tout,
+                                                               const DenseArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int nq = a.rows_per_split * a.W;  // query rows of this CTA (the last split may run past H)
+    const int nqpad = (nq + 15) & ~15;
+    uint8_t *sQ = smem;
+    uint8_t *sK = sQ + (size_t)nqpad * kRowBytes;
+    uint8_t *sV = sK + (size_t)a.npad * kRowBytes;
+    float *lw = reinterpret_cast<float *>(sV + (size_t)a.npad * kRowBytes);  // [R][R] log2(multiplicity)
+    uint8_t *cnt = reinterpret_cast<uint8_t *>(lw + a.R * a.R);                // [R][R]
+    uint8_t *reg = cnt + a.R * a.R;                                            // [npad] region of each key
+    uint64_t *bar = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(reg + a.npad) + 7) & ~uintptr_t(7));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+    int64_t item = blockIdx.x;
+    const int split = (int)(item % a.nsplit);
+    item /= a.nsplit;
+    const int cb = (int)(item % a.ncb);
+    const int b = (int)(item / a.ncb);
+    const int y0 = split * a.rows_per_split;
+    const int32_t *routed = a.idx + (int64_t)b * a.R * a.topk;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(bar, (uint32_t)((nq + 2 * a.N) * kRowBytes));
+        tma_load_4d(sQ, &tq, cb * 64, 0, y0, b, bar);
+        tma_load_4d(sK, &tk, cb * 64, 0, 0, b, bar);
+        tma_load_4d(sV, &tv, cb * 64, 0, 0, b, bar);
+    }
+    // zero the padding rows (TMA writes rows [0, nq) and [0, N) only)
+    for (int i = threadIdx.x; i < (nqpad - nq) * 8; i += blockDim.x)
+        reinterpret_cast<uint4 *>(sQ + (size_t)nq * kRowBytes)[i] = make_uint4(0, 0, 0, 0);
+    for (int i = threadIdx.x; i < (a.npad - a.N) * 8; i += blockDim.x) {
+        reinterpret_cast<uint4 *>(sK + (size_t)a.N * kRowBytes)[i] = make_uint4(0, 0, 0, 0);
+        reinterpret_cast<uint4 *>(sV + (size_t)a.N * kRowBytes)[i] = make_uint4(0, 0, 0, 0);
+    }
+    for (int t = threadIdx.x; t < a.npad; t += blockDim.x)
+        reg[t] = t < a.N ? (uint8_t)(((t / a.W) / a.hr) * a.n_win + (t % a.W) / a.wr) : 0;
+    for (int e = threadIdx.x; e < a.R * a.R; e += blockDim.x) cnt[e] = 0;
+    __syncthreads();
+    for (int r = threadIdx.x; r < a.R; r += blockDim.x)
+        for (int j = 0; j < a.topk; ++j) {
+            const int s = routed[r * a.topk + j];
+            if (s >= 0 && s < a.R)
+                ++cnt[r * a.R + s];
+            else if (cb == 0 && split == 0)
+                flag_error(a.err, kErrIndex);
+        }
+    __syncthreads();
+    for (int e = threadIdx.x; e < a.R * a.R; e += blockDim.x) lw[e] = cnt[e] ? log2f((float)cnt[e]) : -INFINITY;
+    __syncthreads();
+
+    const bool alive = mbar_wait(bar, 0, a.err);
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t qbase = smem_u32(sQ), kbase = smem_u32(sK), vbase = smem_u32(sV);
+    const int tasks = (nqpad / 16) * 2;
+
+    for (int task = warp; alive && task < tasks; task += nwarps) {
+        const int rt = task >> 1, hb = task & 1;
+        uint32_t qf[2][4];
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+            ldmatrix_x4(qbase + sw128(rt * 16 + (lane & 15), hb * 4 + ks * 2 + (lane >> 4)), qf[ks][0], qf[ks][1],
+                        qf[ks][2], qf[ks][3]);
+        const int tq0 = y0 * a.W + rt * 16 + g, tq1 = tq0 + 8;  // query tokens of rows g, g+8
+        const float *lw0 = lw + (tq0 < a.N ? reg[tq0] : 0) * a.R;
+        const float *lw1 = lw + (tq1 < a.N ? reg[tq1] : 0) * a.R;
+        float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+        float o[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+
+        for (int kb = 0; kb < a.npad; kb += 64) {
+            const int nk = min(64, a.npad - kb);  // multiple of 16
+            float sc[8][4];
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = -INFINITY;
+                if (nt * 8 < nk) {
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    uint32_t b0, b1, b2, b3;
+                    ldmatrix_x4(kbase + sw128(kb + nt * 8 + (lane & 7), hb * 4 + (lane >> 3)), b0, b1, b2, b3);
+                    mma_bf16_16816(acc, qf[0], b0, b1);
+                    mma_bf16_16816(acc, qf[1], b2, b3);
+                    const int key = kb + nt * 8 + 2 * t;
+                    const int rk0 = reg[key], rk1 = reg[key + 1];
+                    const bool in0 = key < a.N, in1 = key + 1 < a.N;
+                    sc[nt][0] = in0 ? fmaf(acc[0], a.scale_log2, lw0[rk0]) : -INFINITY;
+                    sc[nt][1] = in1 ? fmaf(acc[1], a.scale_log2, lw0[rk1]) : -INFINITY;
+                    sc[nt][2] = in0 ? fmaf(acc[2], a.scale_log2, lw1[rk0]) : -INFINITY;
+                    sc[nt][3] = in1 ? fmaf(acc[3], a.scale_log2, lw1[rk1]) : -INFINITY;
+                }
+            }
+            float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
+                mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
+            }
+            const float mn0 = fmaxf(m[0], quad_max(mx0)), mn1 = fmaxf(m[1], quad_max(mx1));
+            // a row with no unmasked key so far keeps m = -inf: nothing to rescale, p = 0
+            const float base0 = mn0 == -INFINITY ? 0.f : mn0, base1 = mn1 == -INFINITY ? 0.f : mn1;
+            rescale(o, l, mn0 == -INFINITY ? 1.f : exp2f(m[0] - mn0), mn1 == -INFINITY ? 1.f : exp2f(m[1] - mn1));
+            m[0] = mn0;
+            m[1] = mn1;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                sc[nt][0] = exp2f(sc[nt][0] - base0);
+                sc[nt][1] = exp2f(sc[nt][1] - base0);
+                sc[nt][2] = exp2f(sc[nt][2] - base1);
+                sc[nt][3] = exp2f(sc[nt][3] - base1);
+                l[0] += sc[nt][0] + sc[nt][1];
+                l[1] += sc[nt][2] + sc[nt][3];
+            }
+            if (nk == 64)
+                pv_product<4>(o, sc, vbase, kb, hb, lane);
+            else if (nk == 48)
+                pv_product<3>(o, sc, vbase, kb, hb, lane);
+            else if (nk == 32)
+                pv_product<2>(o, sc, vbase, kb, hb, lane);
+            else
+                pv_product<1>(o, sc, vbase, kb, hb, lane);
+        }
+        __syncwarp();
+        stage_output(qbase, o, l, rt * 16, hb, lane);  // overwrites only this warp's rows/head of the query tile
+    }
+    fence_async_shared();
+    __syncthreads();
+    if (threadIdx.x == 0 && alive) {
+        tma_store_4d(&tout, sQ, cb * 64, 0, y0, b);
+        tma_store_commit();
+        tma_store_wait_read();
+    }
+}
+
+bool dense_mma_supports(const Geometry &g)
+{
+    return g.hd == 32 && g.C % 64 == 0 && g.R <= 64 && g.N <= 256 && g.W <= 256 && g.H <= 256;
+}
+
+int dense_mma_rows_per_split(const Geometry &g, int num_sms)
+{
+    const long long base = (long long)g.B * (g.C / 64);
+    int nsplit = (int)((2LL * num_sms + base - 1) / base);
+    if (nsplit < 1) nsplit = 1;
+    if (nsplit > g.H) nsplit = g.H;
+    return (g.H + nsplit - 1) / nsplit;
+}
+
+static size_t dense_smem_bytes(const Geometry &g, int rows_per_split)
+{
+    const int nq = rows_per_split * g.W, nqpad = (nq + 15) & ~15;
+    const int npad = (g.N + 15) & ~15;
+    return 1024 + (size_t)(nqpad + 2 * npad) * kRowBytes + (size_t)g.R * g.R * 5 + npad + 16;
+}
+
+cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                    const CUtensorMap &tout, const int32_t *idx, const Geometry &g, int rows_per_split,
+                                    unsigned *err, cudaStream_t stream)
+{
+    DenseArgs a;
+    a.idx = idx;
+    a.err = err;
+    a.H = g.H;
+    a.W = g.W;
+    a.n_win = g.n_win;
+    a.topk = g.topk;
+    a.R = g.R;
+    a.hr = g.hr;
+    a.wr = g.wr;
+    a.N = g.N;
+    a.npad = (g.N + 15) & ~15;
+    a.ncb = g.C / 64;
+    a.rows_per_split = rows_per_split;
+    a.nsplit = (g.H + rows_per_split - 1) / rows_per_split;
+    a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)g.hd));
+    const size_t smem = dense_smem_bytes(g, rows_per_split);
+    const long long blocks = (long long)g.B * a.ncb * a.nsplit;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    static int granted[64] = {0};
+    cudaError_t e = ensure_smem_limit(attend_dense_mma_kernel, smem, granted);
+    if (e != cudaSuccess) return e;
+    attend_dense_mma_kernel<<<(unsigned)blocks, 256, smem, stream>>>(tq, tk, tv, tout, a);
+    return cudaGetLastError();
+}
+
+}  // namespace bra

@@ -1,0 +1,54 @@
+// bra_launch.h -- host-side launchers of the BRA kernels (internal to libbra.so).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace bra {
+
+// Bits of the sticky device error word.
+constexpr unsigned kErrIndex = 1u;    // an idx entry outside [0, R) was skipped
+constexpr unsigned kErrTimeout = 2u;  // a bounded wait gave up
+
+// Derived sizes of one call: R = n_win^2 regions of rs = hr * wr tokens, hd = C / heads.
+struct Geometry {
+    int B, H, W, C, heads, n_win, topk;
+    int R, hr, wr, rs, hd, N;
+};
+
+// Region means of q and k (fp32, [B, R, C] each) into qm and km.
+cudaError_t launch_region_means(const void *q, const void *k, float *qm, float *km, const Geometry &g,
+                                bool bf16, int num_sms, cudaStream_t stream);
+
+// Affinity rows and top-k: idx[b, r, :] from qm, km.
+cudaError_t launch_route_topk(const float *qm, const float *km, int32_t *idx, const Geometry &g,
+                              cudaStream_t stream);
+
+// Largest R the routing kernel handles.
+constexpr int kMaxRegions = 1024;
+
+// Generic attention on CUDA cores (fp32 or bf16, hd <= kSimtMaxHeadDim).
+constexpr int kSimtMaxHeadDim = 128;
+cudaError_t launch_attend_simt(const void *q, const void *k, const void *v, const int32_t *idx, void *out,
+                               const Geometry &g, bool bf16, unsigned *err, cudaStream_t stream);
+
+// Tensor-core attention kernels (bf16, hd == 32, C % 64 == 0). The tensor maps describe
+// q, k, v, out as 4-D (C, W, H, B) bf16 tensors, 128-byte swizzle; box sizes as each
+// launcher's `*_boxes` function states.
+bool gather_mma_supports(const Geometry &g);
+bool dense_mma_supports(const Geometry &g);
+
+// Boxes (channels, x, y, images) of the gather kernel: one region, 64 channels, for all four maps.
+void gather_mma_box(const Geometry &g, int box[4]);
+cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                     const CUtensorMap &tout, const int32_t *idx, const Geometry &g,
+                                     unsigned *err, cudaStream_t stream);
+
+// Boxes of the dense kernel: q and out (64, W, rows_per_split, 1); k and v (64, W, H, 1).
+int dense_mma_rows_per_split(const Geometry &g, int num_sms);
+cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                    const CUtensorMap &tout, const int32_t *idx, const Geometry &g,
+                                    int rows_per_split, unsigned *err, cudaStream_t stream);
+
+}  // namespace bra

@@ -1,0 +1,136 @@
+/*
+ * bra.h -- C ABI of libbra.so: the forward pass of Bi-Level Routing Attention (BRA) on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * BRA, as defined by the BiFormer pages this library restates:
+ *   1. cut the H x W feature map into n_win x n_win non-overlapping regions of
+ *      rs = (H / n_win) * (W / n_win) tokens ("从零构建BiFormer", §1 region_partition;
+ *      "手把手带你读懂BiFormer源码", §1.1 RegionPartition);
+ *   2. region-mean descriptors qm, km of q and k ("手把手带你读懂BiFormer源码", §1.2 step 1);
+ *   3. region affinity A = C^-1/2 qm km^T, R x R per image ("手把手带你读懂BiFormer源码",
+ *      §1.2 step 2; "从静态到动态", §2.1 TopkRouting);
+ *   4. routing index idx = the topk largest affinities of each row ("手把手带你读懂BiFormer源码",
+ *      §1.2 step 3);
+ *   5. for every query token of region r and every head: softmax attention, scale
+ *      head_dim^-1/2, over the tokens of the regions idx[r][0..topk-1] only
+ *      ("从零构建BiFormer", §2.2 TokenAttention; "医学图像分割模块：BiFormer / 双层路由注意力",
+ *      §五 steps ⑤-⑦).
+ * bra_route does steps 1-4, bra_attend step 5 and bra_forward all of them.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout. q, k, v and out are dense, contiguous [B, H, W, C] arrays (channels innermost,
+ *   then x, then y, then image) in DEVICE memory, of element type `dtype`. Head j owns
+ *   channels [j*hd, (j+1)*hd), hd = C / heads. Regions are numbered row-major over the
+ *   n_win x n_win grid: region r = (y / (H/n_win)) * n_win + x / (W/n_win). idx is a dense
+ *   int32 [B, R, topk] device array, R = n_win^2.
+ * Routing order. Each idx row lists regions by affinity descending; equal affinities put
+ *   the lower region index first; NaN affinities rank below every number. Routing is
+ *   shared by all heads and uses the full-C region means, accumulated in fp32.
+ * Precision. bf16 inputs are accumulated in fp32 (means, affinities, logits, softmax and
+ *   the weighted sum); out is rounded to bf16 (nearest even). fp32 inputs: fp32 throughout.
+ * Ownership. Every buffer belongs to the caller. Calls are asynchronous and ordered on
+ *   `stream` (a cudaStream_t; NULL = the legacy default stream) on the current device;
+ *   the library never synchronises, except bra_check_device_error and bra_forward_host.
+ *   bra_route and bra_forward take fp32 scratch for the region means, 2*B*R*C*4 bytes,
+ *   from a stream-ordered pool the library keeps per device (cudaMallocAsync /
+ *   cudaFreeAsync on `stream`).
+ * Validation. Every argument is checked on the host before anything is launched; a
+ *   rejected call launches nothing and returns BRA_ERR_INVALID_ARG: a NULL pointer (when
+ *   B > 0), B < 0, H, W, C, heads, n_win or topk <= 0, H or W not a multiple of n_win,
+ *   C not a multiple of heads, topk > R, a data pointer not 16-byte aligned, idx not
+ *   4-byte aligned, C * sizeof(element) not a multiple of 16 bytes, an unknown dtype.
+ *   B == 0 is an empty batch: nothing is launched and BRA_OK is returned.
+ *   BRA_ERR_UNSUPPORTED: valid but outside this build's limits (R > 1024, hd > 128).
+ *   BRA_ERR_CUDA: a CUDA call failed (the message is in bra_last_error_message()).
+ * Device-side checks. bra_attend checks every idx entry on the device; an entry outside
+ *   [0, R) is skipped (its region contributes no key; a query left with no key gets 0)
+ *   and a sticky device error word is set, which bra_check_device_error reports as
+ *   BRA_ERR_INDEX. A bounded wait that gave up sets BRA_ERR_TIMEOUT the same way.
+ */
+#ifndef BRA_H
+#define BRA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BRA_OK = 0,
+    BRA_ERR_INVALID_ARG = 1,
+    BRA_ERR_UNSUPPORTED = 2,
+    BRA_ERR_CUDA = 3,
+    BRA_ERR_INDEX = 4,
+    BRA_ERR_TIMEOUT = 5
+} bra_status;
+
+typedef enum { BRA_F32 = 0, BRA_BF16 = 1 } bra_dtype;
+
+/* Which attention kernel bra_attend / bra_forward use. AUTO picks per shape; the others
+   force one kernel (for tests and tuning) and make calls it cannot serve return
+   BRA_ERR_UNSUPPORTED. */
+typedef enum {
+    BRA_ATTEND_AUTO = 0,
+    BRA_ATTEND_SIMT = 1,      /* any dtype, hd <= 128: one thread per (query, head), CUDA cores */
+    BRA_ATTEND_GATHER_MMA = 2,/* bf16, hd == 32, C % 64 == 0, rs % 16 == 0, rs <= 64: per-region
+                                 tiles staged by TMA, tensor-core QK^T and PV */
+    BRA_ATTEND_DENSE_MMA = 3  /* bf16, hd == 32, C % 64 == 0, R <= 64, H*W <= 256: the image's
+                                 K/V staged once, masked by the routing multiplicities */
+} bra_attend_kernel;
+
+/* Steps 1-4: idx[b, r, :] = routing index of region r of image b.
+   q, k: device [B, H, W, C] of dtype. idx: device int32 [B, n_win^2, topk], written. */
+bra_status bra_route(const void *q, const void *k, int32_t *idx, int B, int H, int W, int C, int n_win,
+                     int topk, bra_dtype dtype, void *stream);
+
+/* Step 5: out = token-to-token attention of every query over the routed regions' keys.
+   q, k, v: device [B, H, W, C] of dtype. idx: device int32 [B, n_win^2, topk], read (any
+   values: duplicates are gathered as often as they occur; out-of-range entries are
+   skipped and flagged). out: device [B, H, W, C] of dtype, written; must not overlap the
+   inputs. */
+bra_status bra_attend(const void *q, const void *k, const void *v, const int32_t *idx, void *out, int B,
+                      int H, int W, int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream);
+
+/* Steps 1-5: bra_route then bra_attend on the same stream. idx is written (and then read). */
+bra_status bra_forward(const void *q, const void *k, const void *v, int32_t *idx, void *out, int B, int H,
+                       int W, int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream);
+
+/* bra_forward on HOST buffers: copies q, k, v (host, [B, H, W, C]) to device scratch from
+   the library's pool, runs the forward pass on `stream`, copies idx and out back to the
+   host buffers and synchronises `stream` before returning. Page-locked host memory gives
+   asynchronous, full-speed copies; pageable memory works too. */
+bra_status bra_forward_host(const void *q, const void *k, const void *v, int32_t *idx, void *out, int B,
+                            int H, int W, int C, int heads, int n_win, int topk, bra_dtype dtype,
+                            void *stream);
+
+/* Force (or, with AUTO, release) one attention kernel for later calls in this process.
+   Returns BRA_ERR_INVALID_ARG for an unknown value. */
+bra_status bra_set_attend_kernel(bra_attend_kernel kernel);
+
+/* The attention kernel a call with these arguments would use (after any forcing), or -1 if
+   the call would be rejected or unsupported. */
+int bra_selected_attend_kernel(int B, int H, int W, int C, int heads, int n_win, int topk, bra_dtype dtype);
+
+/* Synchronises `stream`, then reads and clears the current device's sticky error word:
+   BRA_OK, BRA_ERR_INDEX (an idx entry outside [0, R) was skipped) or BRA_ERR_TIMEOUT. */
+bra_status bra_check_device_error(void *stream);
+
+/* Bytes of scratch bra_route / bra_forward take from the pool for these sizes. */
+size_t bra_route_scratch_bytes(int B, int H, int W, int C, int n_win);
+
+/* Number of kernels one bra_route, bra_attend or bra_forward call launches (for launch
+   accounting); 0 for a call that would launch nothing. */
+int bra_kernels_per_call(const char *entry_point, int B);
+
+/* Static strings: the name of a status, and the last CUDA error message of this thread. */
+const char *bra_status_string(bra_status status);
+const char *bra_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BRA_H */

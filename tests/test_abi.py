@@ -1,0 +1,117 @@
+"""The C ABI on the host: the library loads, exports what include/bra.h declares, and
+rejects bad arguments before touching a GPU. No kernel is launched here."""
+import ctypes
+
+import pytest
+
+from bi_level_routing_b200 import api
+from bi_level_routing_b200.workloads import WORKLOADS
+
+OK, INVALID, UNSUPPORTED = 0, 1, 2
+
+
+@pytest.fixture(scope="module")
+def L():
+    from bi_level_routing_b200 import build
+    build.build()
+    return api.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = api.declared_symbols()
+    assert len(names) >= 11, names
+    for name in names:
+        assert hasattr(L, name), f"libbra.so does not export {name}"
+
+
+def test_status_strings(L):
+    for code, name in api.STATUS.items():
+        assert L.bra_status_string(code).decode() == name
+
+
+FAKE = 0x10000  # a 16-byte aligned non-NULL value; these calls must fail before using it
+
+
+def _route(L, q=FAKE, k=FAKE, idx=FAKE, B=1, H=28, W=28, C=64, n_win=7, topk=4, dtype=1):
+    return L.bra_route(q, k, idx, B, H, W, C, n_win, topk, dtype, None)
+
+
+def _attend(L, q=FAKE, k=FAKE, v=FAKE, idx=FAKE, out=FAKE, B=1, H=28, W=28, C=64, heads=2, n_win=7, topk=4,
+            dtype=1):
+    return L.bra_attend(q, k, v, idx, out, B, H, W, C, heads, n_win, topk, dtype, None)
+
+
+def _forward(L, q=FAKE, k=FAKE, v=FAKE, idx=FAKE, out=FAKE, B=1, H=28, W=28, C=64, heads=2, n_win=7, topk=4,
+             dtype=1):
+    return L.bra_forward(q, k, v, idx, out, B, H, W, C, heads, n_win, topk, dtype, None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(H=30),            # H % n_win != 0
+    dict(W=27),            # W % n_win != 0
+    dict(topk=50),         # topk > R
+    dict(topk=0), dict(n_win=0), dict(C=0), dict(H=-7), dict(B=-1),
+    dict(dtype=7),         # unknown dtype
+    dict(C=60),            # C * 2 bytes not a multiple of 16
+    dict(q=0), dict(k=0), dict(idx=0),
+    dict(q=FAKE + 8),      # not 16-byte aligned
+    dict(idx=FAKE + 2),    # not 4-byte aligned
+])
+def test_route_rejects(L, kw):
+    assert _route(L, **kw) == INVALID
+
+
+@pytest.mark.parametrize("kw", [
+    dict(heads=3),         # C % heads != 0
+    dict(heads=0), dict(v=0), dict(out=0), dict(v=FAKE + 4), dict(out=FAKE + 8),
+    dict(dtype=0, C=62, heads=2),  # fp32: C * 4 bytes not a multiple of 16
+    dict(topk=50),
+])
+def test_attend_and_forward_reject(L, kw):
+    assert _attend(L, **kw) == INVALID
+    assert _forward(L, **kw) == INVALID
+
+
+def test_empty_batch_is_a_no_op(L):
+    assert _route(L, B=0, q=0, k=0, idx=0) == OK
+    assert _attend(L, B=0, q=0, k=0, v=0, idx=0, out=0) == OK
+    assert _forward(L, B=0, q=0, k=0, v=0, idx=0, out=0) == OK
+    assert L.bra_kernels_per_call(b"bra_forward", 0) == 0
+
+
+def test_unsupported_sizes(L):
+    assert _route(L, H=33, W=33, n_win=33, topk=1) == UNSUPPORTED  # R = 1089 > 1024
+    assert L.bra_selected_attend_kernel(1, 8, 8, 1024, 4, 2, 1, 1) == -1  # head_dim 256 > 128
+
+
+def test_kernel_selection_per_workload(L):
+    assert L.bra_set_attend_kernel(0) == OK
+    want = {"tiny_f32": "simt", "stage1": "gather_mma", "stage2": "gather_mma", "stage3": "dense_mma",
+            "stage4": "dense_mma", "highres": "gather_mma"}
+    import torch
+    for name, kernel in want.items():
+        w = WORKLOADS[name]
+        dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+        assert api.selected_attend_kernel(w.B, w.H, w.W, w.C, w.heads, w.n_win, w.topk, dt) == kernel, name
+
+
+def test_forcing_a_kernel(L):
+    try:
+        assert L.bra_set_attend_kernel(9) == INVALID
+        assert L.bra_set_attend_kernel(1) == OK
+        assert L.bra_selected_attend_kernel(64, 56, 56, 64, 2, 7, 1, 1) == 1
+        assert L.bra_set_attend_kernel(3) == OK
+        assert L.bra_selected_attend_kernel(64, 56, 56, 64, 2, 7, 1, 1) == -1  # 3136 tokens > 256
+        assert L.bra_selected_attend_kernel(64, 14, 14, 256, 8, 7, 16, 1) == 3
+        assert L.bra_set_attend_kernel(2) == OK
+        assert L.bra_selected_attend_kernel(1, 28, 28, 64, 2, 7, 4, 0) == -1  # fp32 has no tensor-core kernel
+    finally:
+        L.bra_set_attend_kernel(0)
+
+
+def test_scratch_and_launch_accounting(L):
+    assert L.bra_route_scratch_bytes(64, 56, 56, 64, 7) == 2 * 64 * 49 * 64 * 4
+    assert L.bra_kernels_per_call(b"bra_route", 2) == 2
+    assert L.bra_kernels_per_call(b"bra_attend", 2) == 1
+    assert L.bra_kernels_per_call(b"bra_forward", 2) == 3
+    assert L.bra_kernels_per_call(b"nonsense", 2) == 0

@@ -1,0 +1,211 @@
+"""CUDA path against the CPU oracle, through the C ABI (via the ctypes binding)."""
+import numpy as np
+import pytest
+import torch
+
+import bi_level_routing_b200 as bra
+import oracle
+from bi_level_routing_b200.workloads import WORKLOADS, Workload, make_inputs, sample_tokens
+from parity import check_output, check_routing, device_tensors, host_values, make
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _auto_kernel():
+    bra.set_attend_kernel("auto")
+    yield
+    bra.set_attend_kernel("auto")
+
+
+# ------------------------------------------------------------------ the named workloads, full size
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_forward_full_size(name):
+    """bra_forward at full size, in the configuration the benchmark times: every routing row
+    checked (bit-exact outside near-ties), outputs checked on sampled tokens."""
+    w = WORKLOADS[name]
+    inp, (q, k, v) = make(w)
+    out, idx = bra.forward(q, k, v, w.n_win, w.topk, w.heads)
+    torch.cuda.synchronize()
+    assert bra.check_device_error() == 0
+    gidx = idx.cpu().numpy()
+    _, near = check_routing(gidx, inp["q"], inp["k"], w.n_win, w.topk)
+    assert near <= max(2, gidx.shape[0] * gidx.shape[1] // 1000), f"{near} near-tie rows"
+    toks = sample_tokens(w, 3000 if w.N * w.B > 3000 else w.N * w.B)
+    ref = oracle.attend_tokens(inp["q"], inp["k"], inp["v"], gidx, w.heads, w.n_win, toks)
+    got = host_values(out).reshape(-1, w.C)[toks]
+    check_output(got, ref, w.dtype, f"{name} sampled tokens")
+    # properties that hold at any size: finite, and each output channel inside the convex hull
+    # of the values (a softmax average)
+    o = host_values(out)
+    assert np.all(np.isfinite(o))
+    vmin, vmax = inp["v"].min(), inp["v"].max()
+    slack = 0.02 * max(abs(vmin), abs(vmax))
+    assert o.min() >= vmin - slack and o.max() <= vmax + slack
+
+
+# ------------------------------------------------------------------ small shapes, every element
+
+SMALL = [
+    # name, B, H, W, C, heads, n_win, topk, dtype
+    ("rect_rs15_bf16", 3, 12, 20, 64, 2, 4, 3, "bf16"),
+    ("rs64_ring_bf16", 2, 32, 32, 128, 4, 4, 5, "bf16"),
+    ("rs48_c192_bf16", 2, 16, 48, 192, 6, 4, 2, "bf16"),
+    ("rs16_c320_bf16", 1, 8, 8, 320, 10, 2, 4, "bf16"),
+    ("rs16_stage2_bf16", 2, 28, 28, 128, 4, 7, 4, "bf16"),
+    ("rs4_stage3_bf16", 3, 14, 14, 256, 8, 7, 16, "bf16"),
+    ("rs1_bf16", 2, 8, 8, 64, 2, 8, 5, "bf16"),
+    ("one_region_bf16", 2, 8, 8, 64, 2, 1, 1, "bf16"),
+    ("hd4_f32", 2, 9, 15, 12, 3, 3, 2, "f32"),
+    ("hd64_f32", 1, 16, 16, 128, 2, 4, 3, "f32"),
+    ("hd64_bf16", 1, 16, 16, 128, 2, 4, 3, "bf16"),
+    ("hd128_bf16", 1, 8, 8, 256, 2, 2, 2, "bf16"),
+    ("tiny_f32", 1, 28, 28, 64, 2, 7, 4, "f32"),
+    ("max_regions_bf16", 1, 32, 32, 8, 1, 32, 7, "bf16"),
+    ("topk_all_256_bf16", 1, 16, 16, 32, 1, 16, 256, "bf16"),
+]
+
+
+def _small(spec, values="region_offset", seed=1234):
+    name, B, H, W, C, heads, n, topk, dt = spec
+    return Workload(name, B, H, W, C, heads, n, topk, dt, values, seed)
+
+
+def _kernels_for(w):
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    out = []
+    for kname in ("simt", "gather_mma", "dense_mma"):
+        bra.set_attend_kernel(kname)
+        if bra.selected_attend_kernel(w.B, w.H, w.W, w.C, w.heads, w.n_win, w.topk, dt) == kname:
+            out.append(kname)
+    bra.set_attend_kernel("auto")
+    return out
+
+
+@pytest.mark.parametrize("spec", SMALL, ids=[s[0] for s in SMALL])
+def test_small_shapes_every_kernel(spec):
+    w = _small(spec)
+    inp, (q, k, v) = make(w)
+    idx = bra.route(q, k, w.n_win, w.topk)
+    torch.cuda.synchronize()
+    gidx = idx.cpu().numpy()
+    check_routing(gidx, inp["q"], inp["k"], w.n_win, w.topk)
+    ref = oracle.attend(inp["q"], inp["k"], inp["v"], gidx, w.heads, w.n_win)
+    kernels = _kernels_for(w)
+    assert kernels, "no kernel serves this shape"
+    for kname in kernels:
+        bra.set_attend_kernel(kname)
+        out = bra.attend(q, k, v, idx, w.heads, w.n_win)
+        torch.cuda.synchronize()
+        assert bra.check_device_error() == 0
+        check_output(host_values(out), ref, w.dtype, f"{w.name} / {kname}")
+    bra.set_attend_kernel("auto")
+    out, idx2 = bra.forward(q, k, v, w.n_win, w.topk, w.heads)
+    assert torch.equal(idx2, idx), "forward's routing differs from route's"
+    check_output(host_values(out), ref, w.dtype, f"{w.name} / forward")
+
+
+# ------------------------------------------------------------------ given indices: duplicates, order, bad entries
+
+GIVEN = [("rs64_bf16", 2, 16, 16, 64, 2, 2, 3, "bf16"),
+         ("rs16_bf16", 2, 16, 16, 128, 4, 4, 4, "bf16"),
+         ("rs4_bf16", 2, 14, 14, 128, 4, 7, 6, "bf16"),
+         ("rs9_f32", 2, 12, 12, 16, 2, 4, 3, "f32")]
+
+
+@pytest.mark.parametrize("spec", GIVEN, ids=[s[0] for s in GIVEN])
+def test_duplicates_and_row_order(spec):
+    w = _small(spec, values="iid", seed=99)
+    inp, (q, k, v) = make(w)
+    rng = np.random.Generator(np.random.PCG64(5))
+    R = w.R
+    dup = rng.integers(0, R, size=(w.B, R, w.topk)).astype(np.int32)
+    dup[:, :, -1] = dup[:, :, 0]  # at least one duplicate per row
+    ref = oracle.attend(inp["q"], inp["k"], inp["v"], dup, w.heads, w.n_win)
+    perm = np.ascontiguousarray(dup[:, :, rng.permutation(w.topk)])
+    for kname in _kernels_for(w):
+        bra.set_attend_kernel(kname)
+        out = bra.attend(q, k, v, torch.from_numpy(dup).cuda(), w.heads, w.n_win)
+        out_p = bra.attend(q, k, v, torch.from_numpy(perm).cuda(), w.heads, w.n_win)
+        torch.cuda.synchronize()
+        check_output(host_values(out), ref, w.dtype, f"duplicates / {kname}")
+        check_output(host_values(out_p), ref, w.dtype, f"permuted / {kname}")
+    assert bra.check_device_error() == 0
+
+
+@pytest.mark.parametrize("spec", GIVEN, ids=[s[0] for s in GIVEN])
+def test_out_of_range_entries_are_skipped_and_flagged(spec):
+    w = _small(spec, values="iid", seed=77)
+    inp, (q, k, v) = make(w)
+    rng = np.random.Generator(np.random.PCG64(6))
+    good = np.stack([np.stack([rng.choice(w.R, w.topk - 1, replace=False) for _ in range(w.R)])
+                     for _ in range(w.B)]).astype(np.int32)
+    bad = np.concatenate([good, np.full((w.B, w.R, 1), w.R + 3, np.int32)], axis=-1)
+    bad[:, ::2, -1] = -1
+    ref = oracle.attend(inp["q"], inp["k"], inp["v"], good, w.heads, w.n_win)
+    for kname in _kernels_for(w):
+        bra.set_attend_kernel(kname)
+        assert bra.check_device_error() == 0
+        out = bra.attend(q, k, v, torch.from_numpy(bad).cuda(), w.heads, w.n_win)
+        assert bra.check_device_error() == 4, f"{kname} did not flag BRA_ERR_INDEX"
+        assert bra.check_device_error() == 0, "the error word must clear after reading"
+        check_output(host_values(out), ref, w.dtype, f"bad entries skipped / {kname}")
+
+
+# ------------------------------------------------------------------ routing edge cases
+
+def test_route_exact_ties_go_to_the_lower_region():
+    w = Workload("ties", 2, 16, 16, 64, 2, 4, 16, "bf16", "region_offset", 4321)
+    inp = make_inputs(w)
+    for t in ("k_bits", "k"):  # region (1,2)=6 and region (3,0)=12 copy region (0,1)=1
+        inp[t][:, 4:8, 8:12, :] = inp[t][:, 0:4, 4:8, :]
+        inp[t][:, 12:16, 0:4, :] = inp[t][:, 0:4, 4:8, :]
+    q, k, _ = device_tensors(inp, w)
+    gidx = bra.route(q, k, w.n_win, w.topk).cpu().numpy()
+    orc = oracle.route(inp["q"], inp["k"], w.n_win, w.topk)
+    assert np.array_equal(gidx, orc)
+    for b in range(w.B):
+        for r in range(w.R):
+            row = list(gidx[b, r])
+            assert row.index(1) < row.index(6) < row.index(12)
+
+
+def test_route_nan_ranks_last():
+    w = Workload("nan", 1, 16, 16, 64, 2, 4, 16, "f32", "region_offset", 4322)
+    inp = make_inputs(w)
+    inp["k"][0, 4, 4, 3] = np.nan  # region (1,1) = 5 gets a NaN mean: column 5 is NaN in every row
+    q, k, _ = device_tensors(inp, w)
+    gidx = bra.route(q, k, w.n_win, w.topk).cpu().numpy()
+    orc = oracle.route(inp["q"], inp["k"], w.n_win, w.topk)
+    assert np.array_equal(gidx, orc)
+    assert np.all(gidx[0, :, -1] == 5)
+
+
+def test_empty_batch():
+    q = torch.empty((0, 8, 8, 64), dtype=torch.bfloat16, device="cuda")
+    out, idx = bra.forward(q, q, q, 2, 2, 2)
+    assert out.shape == (0, 8, 8, 64) and idx.shape == (0, 4, 2)
+
+
+def test_side_stream_and_host_entry_point():
+    w = WORKLOADS["stage2"].with_(B=4)
+    inp, (q, k, v) = make(w)
+    ref_out, ref_idx = bra.forward(q, k, v, w.n_win, w.topk, w.heads)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        out, idx = bra.forward(q, k, v, w.n_win, w.topk, w.heads)
+    s.synchronize()
+    assert torch.equal(out, ref_out) and torch.equal(idx, ref_idx)
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hout, hidx = bra.forward_host(hq, hk, hv, w.n_win, w.topk, w.heads)
+    assert torch.equal(hout, ref_out.cpu()) and torch.equal(hidx, ref_idx.cpu())
+
+
+def test_repeatable():
+    """Same inputs, same bits: the kernels use no atomics in their arithmetic."""
+    w = WORKLOADS["highres"].with_(B=2)
+    _, (q, k, v) = make(w)
+    a = bra.forward(q, k, v, w.n_win, w.topk, w.heads)
+    b = bra.forward(q, k, v, w.n_win, w.topk, w.heads)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
