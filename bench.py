@@ -6,9 +6,9 @@ A step is one pass of the whole hot path (region means, affinity + top-k, gather
 over one batch of the workload. Inputs are seeded synthetic data of the workload's shape,
 resident in HBM before timing starts; the step rotates through enough input/output buffer
 sets (copies of the batch, rolled along the image axis) that the set it reads was evicted
-from L2 by the others. Each set's route and attend calls are captured once as CUDA graphs
-(eager launches if capture is refused) and replayed; CUDA events on the launching stream
-time every step and every attention kernel. With N > 1 (torchrun), each rank runs its own
+from L2 by the others. The K timed steps are captured as one CUDA graph (eager launches if
+capture is refused), with timing events recorded as graph nodes on the launching stream
+around every route and every attention call. With N > 1 (torchrun), each rank runs its own
 batch (weak scaling, no data-path collective) and the time is the max over ranks.
 
 Prints one JSON line on rank 0. `--impl reference` times the CPU oracle on the host cores
@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true", help="do not capture CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--soak-seconds", type=float, default=1.0,
+                    help="identical untimed steps before the timed region, while clocks are sampled")
     return ap.parse_args()
 
 
@@ -232,83 +234,65 @@ def main():
         attend(sets[i % nsets])
     torch.cuda.synchronize()
 
-    launch = "eager"
-    graphs = None
+
+    # ---- the timed region: K steps, each [event, route, event, attend], captured as ONE CUDA
+    # graph (timing events as external event-record nodes) so that host launch overhead does
+    # not pace the GPU; eager launches if capture is refused.
+    K = args.steps
+    ev_route = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(K)]
+    ev_attend = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(K)]
+    ev_end = torch.cuda.Event(enable_timing=True, external=True)
+
+    def record_steps():
+        for i in range(K):
+            s = sets[i % nsets]
+            ev_route[i].record()
+            route(s)
+            ev_attend[i].record()
+            attend(s)
+        ev_end.record()
+
+    launch = "cuda_graph (all K steps in one graph)"
+    graph = None
     if not args.eager:
         try:
-            graphs = []
-            for s in sets:
-                ga, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-                with torch.cuda.graph(ga):
-                    route(s)
-                with torch.cuda.graph(gb):
-                    attend(s)
-                graphs.append((ga, gb))
-            launch = "cuda_graph"
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                record_steps()
         except Exception as e:  # capture refused: time eager launches
-            graphs = None
-            launch = f"eager (graph capture failed: {type(e).__name__})"
+            graph = None
+            launch = f"eager (graph capture failed: {type(e).__name__}: {e})"
             torch.cuda.synchronize()
+    if graph is None and launch.startswith("cuda_graph"):
+        launch = "eager"
+    run_steps = graph.replay if graph is not None else record_steps
 
-    def step(i):
-        if graphs:
-            ga, gb = graphs[i % nsets]
-            return ga.replay, gb.replay
-        s = sets[i % nsets]
-        return (lambda: route(s)), (lambda: attend(s))
-
-    for i in range(args.warmup):
-        a, b = step(i)
-        a()
-        b()
+    run_steps()  # untimed: the first replay also uploads the graph
     torch.cuda.synchronize()
 
     # ---- clock samples over a soak of identical steps around the timed region
     sampler = ClockSampler(local_rank)
-    K = args.steps
-    ev_route = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_attend = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_end = torch.cuda.Event(enable_timing=True)
     with sampler:
         t_soak = time.perf_counter()
-        i = 0
-        while time.perf_counter() - t_soak < 1.0:
-            a, b = step(i)
-            a()
-            b()
-            i += 1
-            if i % 64 == 0:
-                torch.cuda.synchronize()
+        while time.perf_counter() - t_soak < args.soak_seconds:
+            run_steps()
+            torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        run_steps()  # the timed K steps
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        for i in range(K):
-            a, b = step(i)
-            ev_route[i].record()
-            a()
-            ev_attend[i].record()
-            b()
-        ev_end.record()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        # keep the GPU busy while the sampler catches the tail
+        total_ms = ev_route[0].elapsed_time(ev_end)
+        attend_ms = [ev_attend[i].elapsed_time(ev_route[i + 1] if i + 1 < K else ev_end) for i in range(K)]
+        route_ms = [ev_route[i].elapsed_time(ev_attend[i]) for i in range(K)]
         t_tail = time.perf_counter()
-        i = 0
-        while time.perf_counter() - t_tail < 0.5:
-            a, b = step(i)
-            a()
-            b()
-            i += 1
-            if i % 64 == 0:
-                torch.cuda.synchronize()
-        torch.cuda.synchronize()
+        while time.perf_counter() - t_tail < min(0.5, args.soak_seconds):
+            run_steps()
+            torch.cuda.synchronize()
 
-    total_ms = ev_route[0].elapsed_time(ev_end)
-    attend_ms = [ev_attend[i].elapsed_time(ev_route[i + 1] if i + 1 < K else ev_end) for i in range(K)]
-    route_ms = [ev_route[i].elapsed_time(ev_attend[i]) for i in range(K)]
     if world > 1:
         t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -379,7 +363,7 @@ def main():
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_seconds)
 
-    del graphs
+    del graph
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

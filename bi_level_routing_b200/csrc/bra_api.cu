@@ -192,7 +192,7 @@ bra_status attend_impl(const void *q, const void *k, const void *v, const int32_
         if ((s = encode_map(&tk, k, g, box[1], box[2])) != BRA_OK) return s;
         if ((s = encode_map(&tv, v, g, box[1], box[2])) != BRA_OK) return s;
         if ((s = encode_map(&to, out, g, box[1], box[2])) != BRA_OK) return s;
-        e = bra::launch_attend_gather_mma(tq, tk, tv, to, idx, g, st->error_word, stream);
+        e = bra::launch_attend_gather_mma(tq, tk, tv, to, idx, g, st->num_sms, st->error_word, stream);
     } else {
         const int rows = bra::dense_mma_rows_per_split(g, st->num_sms);
         CUtensorMap tq, tk, tv, to;

@@ -46,17 +46,6 @@ static cudaError_t ensure_smem_limit(Kernel kernel, size_t bytes, int (&granted)
     return e;
 }
 
-struct GatherArgs {
-    const int32_t *idx;
-    unsigned *err;
-    int n_win, topk, R, hr, wr;
-    int ncb;          // 64-channel blocks in C
-    int ncb_per_cta;  // channel blocks one CTA covers
-    int groups;       // CTAs per (image, region)
-    int nstage;       // routed regions in flight
-    float scale_log2;
-};
-
 __device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v)
 {
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
@@ -126,141 +115,246 @@ __device__ __forceinline__ void stage_output(uint32_t tile, const float (&o)[4][
     }
 }
 
-template <int RS>
-__global__ void __launch_bounds__(256) attend_gather_mma_kernel(const __grid_constant__ CUtensorMap tq,
-                                                                const __grid_constant__ CUtensorMap tk,
-                                                                const __grid_constant__ CUtensorMap tv,
-                                                                const __grid_constant__ CUtensorMap tout,
-                                                                const GatherArgs a)
+struct GatherArgs {
+    const int32_t *idx;
+    unsigned *err;
+    int n_win, topk, R, hr, wr;
+    int ncb;          // 64-channel blocks in C
+    int ncb_per_cta;  // channel blocks one work item covers (NCB)
+    int groups;       // work items per (image, region)
+    int nitems;       // B * R * groups
+    int per_cta;      // contiguous work items per CTA
+    int ncw;          // consumer warps = NCB * 2 heads * rs / 16 row tiles
+    int qslots, kvslots, idx_chunk;
+    float scale_log2;
+};
+
+// S = Q K^T for one 16-row tile of one head against one routed region (NT 8-key n-tiles),
+// online-softmax update of (m, l, o), then O += P V. P is rounded down to bf16 (the low
+// half of the fp32 bits dropped) and the row sums accumulate exactly those values, so the
+// normalisation matches the weights used.
+template <int NT>
+__device__ __forceinline__ void attend_region(float (&o)[4][4], float (&m)[2], float (&l)[2], const uint32_t (&qf)[2][4],
+                                              uint32_t ktile, uint32_t vtile, int hb, int lane, float scale_log2)
 {
-    constexpr int RT = RS / 16;             // 16-row tiles per region
-    constexpr int NT = RS / 8;              // 8-key n-tiles per region
-    constexpr int TILE = RS * kRowBytes;    // one (region, 64-channel block) tile
+    float sc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4(ktile + sw128(nt * 8 + (lane & 7), hb * 4 + (lane >> 3)), b0, b1, b2, b3);
+        mma_bf16_16816(sc[nt], qf[0], b0, b1);
+        mma_bf16_16816(sc[nt], qf[1], b2, b3);
+    }
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
+        mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
+    }
+    const float mn0 = fmaxf(m[0], quad_max(mx0) * scale_log2);
+    const float mn1 = fmaxf(m[1], quad_max(mx1) * scale_log2);
+    rescale(o, l, fast_exp2(m[0] - mn0), fast_exp2(m[1] - mn1));
+    m[0] = mn0;
+    m[1] = mn1;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        sc[nt][0] = bf16_trunc(fast_exp2(fmaf(sc[nt][0], scale_log2, -mn0)));
+        sc[nt][1] = bf16_trunc(fast_exp2(fmaf(sc[nt][1], scale_log2, -mn0)));
+        sc[nt][2] = bf16_trunc(fast_exp2(fmaf(sc[nt][2], scale_log2, -mn1)));
+        sc[nt][3] = bf16_trunc(fast_exp2(fmaf(sc[nt][3], scale_log2, -mn1)));
+        l[0] += sc[nt][0] + sc[nt][1];
+        l[1] += sc[nt][2] + sc[nt][3];
+    }
+#pragma unroll
+    for (int kk = 0; kk < NT / 2; ++kk) {
+        uint32_t pa[4];
+        pa[0] = pack_bf16x2_trunc(sc[2 * kk][0], sc[2 * kk][1]);
+        pa[1] = pack_bf16x2_trunc(sc[2 * kk][2], sc[2 * kk][3]);
+        pa[2] = pack_bf16x2_trunc(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
+        pa[3] = pack_bf16x2_trunc(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {
+            uint32_t b0, b1, b2, b3;
+            const int row = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+            ldmatrix_x4_trans(vtile + sw128(row, hb * 4 + np * 2 + (lane >> 4)), b0, b1, b2, b3);
+            mma_bf16_16816(o[2 * np], pa, b0, b1);
+            mma_bf16_16816(o[2 * np + 1], pa, b2, b3);
+        }
+    }
+}
+
+// Persistent, warp-specialised gather attention. Each CTA owns a contiguous run of work
+// items (image, query region, group of NCB 64-channel blocks), in image order.
+//  * Warp `ncw` (producer): stages the idx rows of the next items in shared memory, then
+//    one lane issues the TMA loads: the query tile into a ring of `qslots` slots and, per
+//    routed region, its K and V tiles into a ring of `kvslots` slots; each slot has a
+//    "full" mbarrier (TMA transaction bytes) and an "empty" one (one arrival per consumer
+//    warp). An idx entry outside [0, R) fills its slot with nothing and is flagged.
+//  * Warps 0..ncw-1 (consumers): warp w owns 16 query rows (w % RT) of head (w / RT) % 2 of
+//    channel block w / (2 RT); it runs attend_region per routed region, then writes its
+//    normalised output into one of two output tiles; one thread stores the tile by TMA
+//    while the next item is computed.
+// Every wait is bounded; a wait that gives up flags kErrTimeout and the thread stops
+// computing but keeps arriving on barriers, so the CTA still finishes.
+template <int RS>
+__global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_constant__ CUtensorMap tq,
+                                                                   const __grid_constant__ CUtensorMap tk,
+                                                                   const __grid_constant__ CUtensorMap tv,
+                                                                   const __grid_constant__ CUtensorMap tout,
+                                                                   const GatherArgs a)
+{
+    constexpr int RT = RS / 16;           // 16-row tiles per region
+    constexpr int NT = RS / 8;            // 8-key n-tiles per region
+    constexpr int TILE = RS * kRowBytes;  // one (region, 64-channel block) tile
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int NCB = a.ncb_per_cta;
     uint8_t *sQ = smem;
-    uint8_t *sKV = smem + NCB * TILE;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sKV + (size_t)a.nstage * 2 * NCB * TILE);
-    int *stage_ok = reinterpret_cast<int *>(bars + 1 + a.nstage);
+    uint8_t *sKV = sQ + (size_t)a.qslots * NCB * TILE;
+    uint8_t *sO = sKV + (size_t)a.kvslots * 2 * NCB * TILE;
+    uint64_t *full_q = reinterpret_cast<uint64_t *>(sO + (size_t)2 * NCB * TILE);
+    uint64_t *empty_q = full_q + a.qslots;
+    uint64_t *full_kv = empty_q + a.qslots;
+    uint64_t *empty_kv = full_kv + a.kvslots;
+    int *kv_ok = reinterpret_cast<int *>(empty_kv + a.kvslots);
+    int *sidx = kv_ok + a.kvslots;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int64_t item = blockIdx.x;
-    const int grp = (int)(item % a.groups);
-    item /= a.groups;
-    const int r = (int)(item % a.R);
-    const int b = (int)(item / a.R);
-    const int qx = (r % a.n_win) * a.wr, qy = (r / a.n_win) * a.hr;
-    const int cb0 = grp * NCB;
-    const int ncb_here = min(NCB, a.ncb - cb0);
-    const int32_t *routed = a.idx + ((int64_t)b * a.R + r) * a.topk;
+    const int begin = blockIdx.x * a.per_cta;
+    const int end = min(a.nitems, begin + a.per_cta);
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars[0], 1);
-        for (int i = 0; i < a.nstage; ++i) mbar_init(&bars[1 + i], 1);
+        for (int i = 0; i < a.qslots; ++i) {
+            mbar_init(&full_q[i], 1);
+            mbar_init(&empty_q[i], a.ncw);
+        }
+        for (int i = 0; i < a.kvslots; ++i) {
+            mbar_init(&full_kv[i], 1);
+            mbar_init(&empty_kv[i], a.ncw);
+        }
         mbar_fence_init();
     }
     __syncthreads();
 
-    // Thread 0 only: load routed region j's K and V tiles into stage slot j % nstage.
-    auto issue_stage = [&](int j) {
-        const int slot = j % a.nstage;
-        const int s = routed[j];
-        const bool ok = (s >= 0 && s < a.R);
-        stage_ok[slot] = ok;
-        uint64_t *bar = &bars[1 + slot];
-        if (!ok) {
-            flag_error(a.err, kErrIndex);
-            mbar_arrive_expect_tx(bar, 0);
-            return;
+    if (warp == a.ncw) {
+        // ------------------------------------------------------------- producer warp
+        int qs = 0, kvs = 0;
+        uint32_t qph = 0, kvph = 0;
+        bool alive = true;
+        for (int c0 = begin; c0 < end; c0 += a.idx_chunk) {
+            const int n = min(a.idx_chunk, end - c0);
+            __syncwarp();
+            for (int e = lane; e < n * a.topk; e += 32) {
+                const int it = c0 + e / a.topk, j = e % a.topk;
+                sidx[e] = a.idx[(int64_t)(it / a.groups) * a.topk + j];
+            }
+            __syncwarp();
+            if (lane != 0 || !alive) continue;
+            for (int i = 0; i < n && alive; ++i) {
+                const int item = c0 + i;
+                const int grp = item % a.groups;
+                const int br = item / a.groups;
+                const int r = br % a.R, b = br / a.R;
+                const int cb0 = grp * NCB, nh = min(NCB, a.ncb - cb0);
+                const int qx = (r % a.n_win) * a.wr, qy = (r / a.n_win) * a.hr;
+                if (!(alive = mbar_wait(&empty_q[qs], qph ^ 1, a.err))) break;
+                mbar_arrive_expect_tx(&full_q[qs], (uint32_t)(nh * TILE));
+                for (int cb = 0; cb < nh; ++cb)
+                    tma_load_4d(sQ + (size_t)(qs * NCB + cb) * TILE, &tq, (cb0 + cb) * 64, qx, qy, b, &full_q[qs]);
+                if (++qs == a.qslots) {
+                    qs = 0;
+                    qph ^= 1;
+                }
+                for (int j = 0; j < a.topk; ++j) {
+                    const int s = sidx[i * a.topk + j];
+                    const bool ok = s >= 0 && s < a.R;
+                    if (!(alive = mbar_wait(&empty_kv[kvs], kvph ^ 1, a.err))) break;
+                    kv_ok[kvs] = ok;
+                    if (ok) {
+                        const int sx = (s % a.n_win) * a.wr, sy = (s / a.n_win) * a.hr;
+                        mbar_arrive_expect_tx(&full_kv[kvs], (uint32_t)(2 * nh * TILE));
+                        uint8_t *kt = sKV + (size_t)kvs * 2 * NCB * TILE;
+                        for (int cb = 0; cb < nh; ++cb) {
+                            tma_load_4d(kt + cb * TILE, &tk, (cb0 + cb) * 64, sx, sy, b, &full_kv[kvs]);
+                            tma_load_4d(kt + (NCB + cb) * TILE, &tv, (cb0 + cb) * 64, sx, sy, b, &full_kv[kvs]);
+                        }
+                    } else {
+                        flag_error(a.err, kErrIndex);
+                        mbar_arrive_expect_tx(&full_kv[kvs], 0);
+                    }
+                    if (++kvs == a.kvslots) {
+                        kvs = 0;
+                        kvph ^= 1;
+                    }
+                }
+            }
         }
-        mbar_arrive_expect_tx(bar, (uint32_t)(2 * ncb_here * TILE));
-        const int sx = (s % a.n_win) * a.wr, sy = (s / a.n_win) * a.hr;
-        uint8_t *kt = sKV + (size_t)slot * 2 * NCB * TILE;
-        uint8_t *vt = kt + NCB * TILE;
-        for (int cb = 0; cb < ncb_here; ++cb) {
-            tma_load_4d(kt + cb * TILE, &tk, (cb0 + cb) * 64, sx, sy, b, bar);
-            tma_load_4d(vt + cb * TILE, &tv, (cb0 + cb) * 64, sx, sy, b, bar);
-        }
-    };
-
-    if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(&bars[0], (uint32_t)(ncb_here * TILE));
-        for (int cb = 0; cb < ncb_here; ++cb) tma_load_4d(sQ + cb * TILE, &tq, (cb0 + cb) * 64, qx, qy, b, &bars[0]);
-        const int first = min(a.nstage, a.topk);
-        for (int j = 0; j < first; ++j) issue_stage(j);
+        return;
     }
 
+    // ----------------------------------------------------------------- consumer warps
     const int rt = warp % RT, hb = (warp / RT) & 1, cbl = warp / (2 * RT);
-    const bool active = cbl < ncb_here;
-    const uint32_t qtile = smem_u32(sQ + cbl * TILE);
+    const int consumers = a.ncw * 32;
+    int qs = 0, kvs = 0, os = 0;
+    uint32_t qph = 0, kvph = 0;
+    bool alive = true;
+    for (int item = begin; item < end; ++item) {
+        const int grp = item % a.groups;
+        const int br = item / a.groups;
+        const int r = br % a.R, b = br / a.R;
+        const int cb0 = grp * NCB, nh = min(NCB, a.ncb - cb0);
+        const int qx = (r % a.n_win) * a.wr, qy = (r / a.n_win) * a.hr;
+        const bool active = cbl < nh;
 
-    uint32_t qf[2][4];
-    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-    float o[4][4];
+        uint32_t qf[2][4];
+        if (alive) alive = mbar_wait(&full_q[qs], qph, a.err);
+        if (alive && active) {
+            const uint32_t qtile = smem_u32(sQ + (size_t)(qs * NCB + cbl) * TILE);
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-
-    bool alive = mbar_wait(&bars[0], 0, a.err);
-    if (alive && active) {
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks)
-            ldmatrix_x4(qtile + sw128(rt * 16 + (lane & 15), hb * 4 + ks * 2 + (lane >> 4)), qf[ks][0], qf[ks][1],
-                        qf[ks][2], qf[ks][3]);
-    }
-
-    for (int j = 0; j < a.topk; ++j) {
-        const int slot = j % a.nstage;
-        if (alive) alive = mbar_wait(&bars[1 + slot], (uint32_t)((j / a.nstage) & 1), a.err);
-        if (alive && active && stage_ok[slot]) {
-            const uint32_t ktile = smem_u32(sKV + (size_t)slot * 2 * NCB * TILE + cbl * TILE);
-            const uint32_t vtile = ktile + NCB * TILE;
-            float sc[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-                uint32_t b0, b1, b2, b3;
-                ldmatrix_x4(ktile + sw128(nt * 8 + (lane & 7), hb * 4 + (lane >> 3)), b0, b1, b2, b3);
-                mma_bf16_16816(sc[nt], qf[0], b0, b1);
-                mma_bf16_16816(sc[nt], qf[1], b2, b3);
-            }
-            float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
-                mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
-            }
-            const float mn0 = fmaxf(m[0], quad_max(mx0) * a.scale_log2);
-            const float mn1 = fmaxf(m[1], quad_max(mx1) * a.scale_log2);
-            rescale(o, l, exp2f(m[0] - mn0), exp2f(m[1] - mn1));
-            m[0] = mn0;
-            m[1] = mn1;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                sc[nt][0] = exp2f(fmaf(sc[nt][0], a.scale_log2, -mn0));
-                sc[nt][1] = exp2f(fmaf(sc[nt][1], a.scale_log2, -mn0));
-                sc[nt][2] = exp2f(fmaf(sc[nt][2], a.scale_log2, -mn1));
-                sc[nt][3] = exp2f(fmaf(sc[nt][3], a.scale_log2, -mn1));
-                l[0] += sc[nt][0] + sc[nt][1];
-                l[1] += sc[nt][2] + sc[nt][3];
-            }
-            pv_product<RT>(o, sc, vtile, 0, hb, lane);
+            for (int ks = 0; ks < 2; ++ks)
+                ldmatrix_x4(qtile + sw128(rt * 16 + (lane & 15), hb * 4 + ks * 2 + (lane >> 4)), qf[ks][0], qf[ks][1],
+                            qf[ks][2], qf[ks][3]);
         }
-        if (j + a.nstage < a.topk) {
-            __syncthreads();  // every warp is done with this slot
-            if (threadIdx.x == 0 && alive) issue_stage(j + a.nstage);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_q[qs]);
+        if (++qs == a.qslots) {
+            qs = 0;
+            qph ^= 1;
         }
-    }
 
-    __syncthreads();  // the query tiles are free: stage the output there
-    if (alive && active) stage_output(qtile, o, l, rt * 16, hb, lane);
-    fence_async_shared();
-    __syncthreads();
-    if (threadIdx.x == 0 && alive) {
-        for (int cb = 0; cb < ncb_here; ++cb) tma_store_4d(&tout, sQ + cb * TILE, (cb0 + cb) * 64, qx, qy, b);
-        tma_store_commit();
-        tma_store_wait_read();
+        float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+        float o[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+        for (int j = 0; j < a.topk; ++j) {
+            if (alive) alive = mbar_wait(&full_kv[kvs], kvph, a.err);
+            if (alive && active && kv_ok[kvs]) {
+                const uint32_t ktile = smem_u32(sKV + (size_t)(kvs * 2 * NCB + cbl) * TILE);
+                attend_region<NT>(o, m, l, qf, ktile, ktile + NCB * TILE, hb, lane, a.scale_log2);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty_kv[kvs]);
+            if (++kvs == a.kvslots) {
+                kvs = 0;
+                kvph ^= 1;
+            }
+        }
+
+        // epilogue: output slot `os` was last stored two items ago; let that store finish reading
+        if (warp == 0 && lane == 0) tma_store_wait_read_n<1>();
+        named_barrier(1, consumers);
+        if (alive && active) stage_output(smem_u32(sO + (size_t)(os * NCB + cbl) * TILE), o, l, rt * 16, hb, lane);
+        fence_async_shared();
+        named_barrier(1, consumers);
+        if (warp == 0 && lane == 0 && alive) {
+            for (int cb = 0; cb < nh; ++cb)
+                tma_store_4d(&tout, sO + (size_t)(os * NCB + cb) * TILE, (cb0 + cb) * 64, qx, qy, b);
+            tma_store_commit();
+        }
+        os ^= 1;
     }
+    if (warp == 0 && lane == 0) tma_store_wait_read_n<0>();
 }
 
 bool gather_mma_supports(const Geometry &g)
@@ -278,20 +372,20 @@ void gather_mma_box(const Geometry &g, int box[4])
 
 template <int RS>
 static cudaError_t launch_gather_rs(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                    const CUtensorMap &tout, const GatherArgs &a, int threads, size_t smem,
-                                    long long blocks, cudaStream_t stream)
+                                    const CUtensorMap &tout, const GatherArgs &a, int grid, size_t smem,
+                                    cudaStream_t stream)
 {
     static_assert(RS % 16 == 0 && RS <= 64, "tokens per region");
     static int granted[64] = {0};
     cudaError_t e = ensure_smem_limit(attend_gather_mma_kernel<RS>, smem, granted);
     if (e != cudaSuccess) return e;
-    attend_gather_mma_kernel<RS><<<(unsigned)blocks, threads, smem, stream>>>(tq, tk, tv, tout, a);
+    attend_gather_mma_kernel<RS><<<grid, (a.ncw + 1) * 32, smem, stream>>>(tq, tk, tv, tout, a);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                     const CUtensorMap &tout, const int32_t *idx, const Geometry &g, unsigned *err,
-                                     cudaStream_t stream)
+                                     const CUtensorMap &tout, const int32_t *idx, const Geometry &g, int num_sms,
+                                     unsigned *err, cudaStream_t stream)
 {
     GatherArgs a;
     a.idx = idx;
@@ -308,18 +402,31 @@ cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &t
     if (ncb_per_cta > a.ncb) ncb_per_cta = a.ncb;
     a.ncb_per_cta = ncb_per_cta;
     a.groups = (a.ncb + ncb_per_cta - 1) / ncb_per_cta;
-    a.nstage = g.topk < 4 ? g.topk : 4;
+    a.ncw = ncb_per_cta * 2 * rt;
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)g.hd));
-    const int threads = ncb_per_cta * 2 * rt * 32;
-    const size_t tile = (size_t)g.rs * kRowBytes;
-    const size_t smem = 1024 + tile * ncb_per_cta * (1 + 2 * (size_t)a.nstage) + 8 * (1 + a.nstage) + 4 * a.nstage;
-    const long long blocks = (long long)g.B * g.R * a.groups;
-    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const long long nitems = (long long)g.B * g.R * a.groups;
+    if (nitems > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    a.nitems = (int)nitems;
+    // Two CTAs per SM: ~111 KB of shared memory each for the rings.
+    const size_t tile = (size_t)g.rs * kRowBytes * ncb_per_cta;  // one slot of one tensor
+    const size_t budget = 111 * 1024;
+    a.qslots = g.topk <= 2 ? 3 : 2;
+    long long kv = (long long)((budget - (a.qslots + 2) * tile) / (2 * tile));
+    if (kv > 8) kv = 8;
+    if (kv < 2) kv = 2;
+    a.kvslots = (int)kv;
+    a.idx_chunk = g.topk >= 32 ? 1 : 32 / g.topk;
+    const size_t smem = 1024 + tile * (a.qslots + 2 * a.kvslots + 2) + 16 * (a.qslots + a.kvslots) +
+                        4 * a.kvslots + 4 * (size_t)a.idx_chunk * g.topk;
+    int grid = 2 * num_sms;
+    if (grid > a.nitems) grid = a.nitems;
+    a.per_cta = (a.nitems + grid - 1) / grid;
+    grid = (a.nitems + a.per_cta - 1) / a.per_cta;
     switch (g.rs) {
-    case 16: return launch_gather_rs<16>(tq, tk, tv, tout, a, threads, smem, blocks, stream);
-    case 32: return launch_gather_rs<32>(tq, tk, tv, tout, a, threads, smem, blocks, stream);
-    case 48: return launch_gather_rs<48>(tq, tk, tv, tout, a, threads, smem, blocks, stream);
-    case 64: return launch_gather_rs<64>(tq, tk, tv, tout, a, threads, smem, blocks, stream);
+    case 16: return launch_gather_rs<16>(tq, tk, tv, tout, a, grid, smem, stream);
+    case 32: return launch_gather_rs<32>(tq, tk, tv, tout, a, grid, smem, stream);
+    case 48: return launch_gather_rs<48>(tq, tk, tv, tout, a, grid, smem, stream);
+    case 64: return launch_gather_rs<64>(tq, tk, tv, tout, a, grid, smem, stream);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -43,6 +43,17 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(f
 template <typename T> struct Vec16;
 template <> struct Vec16<float> {
     static constexpr int N = 4;
+    __device__ __forceinline__ static uint4 load_raw(const float *p)
+    {
+        return __ldg(reinterpret_cast<const uint4 *>(p));
+    }
+    __device__ __forceinline__ static void accumulate(const uint4 &v, float *acc)
+    {
+        acc[0] += __uint_as_float(v.x);
+        acc[1] += __uint_as_float(v.y);
+        acc[2] += __uint_as_float(v.z);
+        acc[3] += __uint_as_float(v.w);
+    }
     __device__ __forceinline__ static void load(const float *p, float *f)
     {
         const float4 v = __ldg(reinterpret_cast<const float4 *>(p));
@@ -51,6 +62,19 @@ template <> struct Vec16<float> {
 };
 template <> struct Vec16<__nv_bfloat16> {
     static constexpr int N = 8;
+    __device__ __forceinline__ static uint4 load_raw(const __nv_bfloat16 *p)
+    {
+        return __ldg(reinterpret_cast<const uint4 *>(p));
+    }
+    __device__ __forceinline__ static void accumulate(const uint4 &v, float *acc)
+    {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            acc[2 * i] += __uint_as_float(w[i] << 16);
+            acc[2 * i + 1] += __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
     __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float *f)
     {
         const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p));
@@ -189,6 +213,41 @@ __device__ __forceinline__ void mma_bf16_16816(float *d, const uint32_t *a, uint
         "{%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// 2^x on the MUFU unit (ex2.approx, denormal results flushed to zero).
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Drops the low 16 bits of x: the value whose bf16 encoding is x's upper half.
+__device__ __forceinline__ float bf16_trunc(float x) { return __uint_as_float(__float_as_uint(x) & 0xffff0000u); }
+
+// Packs the upper halves of two floats (already bf16-exact, see bf16_trunc) into bf16x2:
+// one byte permute on the integer pipe, no conversion instruction.
+__device__ __forceinline__ uint32_t pack_bf16x2_trunc(float lo, float hi)
+{
+    return __byte_perm(__float_as_uint(lo), __float_as_uint(hi), 0x7632);
+}
+
+// Named barrier among `threads` threads (a multiple of 32) with id `id` (1..15).
+__device__ __forceinline__ void named_barrier(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Waits until at most N committed bulk stores still read shared memory.
+template <int N> __device__ __forceinline__ void tma_store_wait_read_n()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)

@@ -42,7 +42,7 @@ bool dense_mma_supports(const Geometry &g);
 // Boxes (channels, x, y, images) of the gather kernel: one region, 64 channels, for all four maps.
 void gather_mma_box(const Geometry &g, int box[4]);
 cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                     const CUtensorMap &tout, const int32_t *idx, const Geometry &g,
+                                     const CUtensorMap &tout, const int32_t *idx, const Geometry &g, int num_sms,
                                      unsigned *err, cudaStream_t stream);
 
 // Boxes of the dense kernel: q and out (64, W, rows_per_split, 1); k and v (64, W, H, 1).

@@ -22,12 +22,14 @@ namespace bra {
 // The summation order is the same for every region, so regions with equal content get
 // bit-identical means (exact affinity ties stay exact).
 template <typename T>
-__global__ void __launch_bounds__(512) region_means_kernel(const T *__restrict__ q, const T *__restrict__ k,
+__global__ void __launch_bounds__(256, 4) region_means_kernel(const T *__restrict__ q, const T *__restrict__ k,
                                                            float *__restrict__ qm, float *__restrict__ km, int H,
                                                            int W, int C, int n_win, int rx_per_cta, int n_chunks)
 {
-    extern __shared__ float part[];  // [rx_per_cta * wr][C]
+    extern __shared__ float4 part4[];  // [rx_per_cta * wr][C] floats
+    float *part = reinterpret_cast<float *>(part4);
     constexpr int V = Vec16<T>::N;
+    constexpr int ROWS = 8;  // loads in flight per thread
     const int hr = H / n_win, wr = W / n_win, R = n_win * n_win;
     const int chunk = blockIdx.x % n_chunks;
     const int band = blockIdx.x / n_chunks;
@@ -48,25 +50,19 @@ __global__ void __launch_bounds__(512) region_means_kernel(const T *__restrict__
 #pragma unroll
         for (int i = 0; i < V; ++i) acc[i] = 0.f;
         const T *ptr = base + (int64_t)p * V;
-        int yy = 0;
-        for (; yy + 4 <= hr; yy += 4) {
-            float f[4][V];
+        for (int y0 = 0; y0 < hr; y0 += ROWS) {
+            const int n = min(ROWS, hr - y0);
+            uint4 raw[ROWS];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) Vec16<T>::load(ptr + (int64_t)(yy + u) * row_stride, f[u]);
+            for (int u = 0; u < ROWS; ++u)
+                if (u < n) raw[u] = Vec16<T>::load_raw(ptr + (int64_t)(y0 + u) * row_stride);
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-                for (int i = 0; i < V; ++i) acc[i] += f[u][i];
+            for (int u = 0; u < ROWS; ++u)
+                if (u < n) Vec16<T>::accumulate(raw[u], acc);
         }
-        for (; yy < hr; ++yy) {
-            float f[V];
-            Vec16<T>::load(ptr + (int64_t)yy * row_stride, f);
+        float4 *dst = reinterpret_cast<float4 *>(part + (p / vpt) * C + (p % vpt) * V);
 #pragma unroll
-            for (int i = 0; i < V; ++i) acc[i] += f[i];
-        }
-        float *dst = part + (p / vpt) * C + (p % vpt) * V;
-#pragma unroll
-        for (int i = 0; i < V; ++i) dst[i] = acc[i];
+        for (int i = 0; i < V / 4; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
     }
     __syncthreads();
 
@@ -90,60 +86,84 @@ __device__ __forceinline__ unsigned long long routing_key(float a, int s)
     return ((unsigned long long)f << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)s);
 }
 
-// One warp per affinity row (blockIdx.x = image b * row blocks + row block). keys: P (power of two >= R)
-// entries per warp in shared memory, sorted descending by a warp-wide bitonic network.
-__global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ qm, const float *__restrict__ km,
-                                                         int32_t *__restrict__ idx, int R, int C, int topk, int P,
-                                                         float scale)
+// Dot product of two fp32 rows of length C (a multiple of 4) with four interleaved partial
+// sums, combined in a fixed order: the same arithmetic for every row pair, so equal rows
+// give equal results.
+__device__ __forceinline__ float dot_rows(const float *__restrict__ a, const float *__restrict__ b, int C)
 {
-    extern __shared__ unsigned long long keys[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row_blocks = (R + (blockDim.x >> 5) - 1) / (blockDim.x >> 5);
-    const int b = blockIdx.x / row_blocks;
-    const int r = (blockIdx.x % row_blocks) * (blockDim.x >> 5) + warp;
-    if (r >= R) return;
-    unsigned long long *kw = keys + (size_t)warp * P;
-    const float *qrow = qm + ((int64_t)b * R + r) * C;
-
-    for (int s = lane; s < P; s += 32) {
-        unsigned long long key = 0ull;
-        if (s < R) {
-            const float *krow = km + ((int64_t)b * R + s) * C;
-            float dot = 0.f;
-            for (int c = 0; c < C; c += 4) {
-                const float4 qa = __ldg(reinterpret_cast<const float4 *>(qrow + c));
-                const float4 ka = __ldg(reinterpret_cast<const float4 *>(krow + c));
-                dot = fmaf(qa.x, ka.x, dot);
-                dot = fmaf(qa.y, ka.y, dot);
-                dot = fmaf(qa.z, ka.z, dot);
-                dot = fmaf(qa.w, ka.w, dot);
-            }
-            key = routing_key(dot * scale, s);
-        }
-        kw[s] = key;
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    for (int c = 0; c < C; c += 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(a + c);
+        const float4 y = *reinterpret_cast<const float4 *>(b + c);
+        s0 = fmaf(x.x, y.x, s0);
+        s1 = fmaf(x.y, y.y, s1);
+        s2 = fmaf(x.z, y.z, s2);
+        s3 = fmaf(x.w, y.w, s3);
     }
-    __syncwarp();
+    return (s0 + s1) + (s2 + s3);
+}
 
-    // bitonic sort, descending
-    for (int size = 2; size <= P; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int i = lane; i < P; i += 32) {
-                const int partner = i ^ stride;
-                if (partner > i) {
-                    const unsigned long long a = kw[i], c = kw[partner];
-                    const bool descending = (i & size) == 0;
-                    if (descending ? (a < c) : (a > c)) {
-                        kw[i] = c;
-                        kw[partner] = a;
+// One CTA per (image, block of `rows` affinity rows); each warp handles rows in turn. The
+// image's key means (and this block's query means) are staged in shared memory when
+// `staged` (rows padded to C + 4 floats: lanes reading different rows hit different banks),
+// otherwise read through L1. Per row, lane s computes A[r, s], the keys go to the warp's
+// slice of shared memory, and a bitonic network sorts them descending.
+__global__ void __launch_bounds__(256, 1) route_topk_kernel(const float *__restrict__ qm, const float *__restrict__ km,
+                                                         int32_t *__restrict__ idx, int R, int C, int topk, int P,
+                                                         int rows, int staged, float scale)
+{
+    extern __shared__ unsigned long long keys[];  // [warps][P], then staged means
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    const int row_blocks = (R + rows - 1) / rows;
+    const int b = blockIdx.x / row_blocks;
+    const int r0 = (blockIdx.x % row_blocks) * rows;
+    const int nrows = min(rows, R - r0);
+    const int stride = C + 4;
+    float *skm = reinterpret_cast<float *>(keys + (size_t)nwarps * P);
+    float *sqm = skm + (size_t)R * stride;
+    const float *gkm = km + (int64_t)b * R * C;
+    const float *gqm = qm + ((int64_t)b * R + r0) * C;
+    if (staged) {
+        for (int e = threadIdx.x; e < R * (C / 4); e += blockDim.x) {
+            const int s = e / (C / 4), c = (e % (C / 4)) * 4;
+            *reinterpret_cast<float4 *>(skm + s * stride + c) = __ldg(reinterpret_cast<const float4 *>(gkm + s * C + c));
+        }
+        for (int e = threadIdx.x; e < nrows * (C / 4); e += blockDim.x) {
+            const int s = e / (C / 4), c = (e % (C / 4)) * 4;
+            *reinterpret_cast<float4 *>(sqm + s * stride + c) = __ldg(reinterpret_cast<const float4 *>(gqm + s * C + c));
+        }
+        __syncthreads();
+    }
+    unsigned long long *kw = keys + (size_t)warp * P;
+    for (int i = warp; i < nrows; i += nwarps) {
+        const int r = r0 + i;
+        const float *qrow = staged ? sqm + i * stride : gqm + i * C;
+        for (int s = lane; s < P; s += 32) {
+            unsigned long long key = 0ull;
+            if (s < R) key = routing_key(dot_rows(qrow, staged ? skm + s * stride : gkm + s * C, C) * scale, s);
+            kw[s] = key;
+        }
+        __syncwarp();
+        for (int size = 2; size <= P; size <<= 1) {
+            for (int st = size >> 1; st > 0; st >>= 1) {
+                for (int e = lane; e < P; e += 32) {
+                    const int partner = e ^ st;
+                    if (partner > e) {
+                        const unsigned long long x = kw[e], y = kw[partner];
+                        const bool descending = (e & size) == 0;
+                        if (descending ? (x < y) : (x > y)) {
+                            kw[e] = y;
+                            kw[partner] = x;
+                        }
                     }
                 }
+                __syncwarp();
             }
-            __syncwarp();
         }
+        int32_t *out = idx + ((int64_t)b * R + r) * topk;
+        for (int j = lane; j < topk; j += 32) out[j] = (int32_t)(0xFFFFFFFFu - (uint32_t)(kw[j] & 0xFFFFFFFFull));
+        __syncwarp();
     }
-
-    int32_t *out = idx + ((int64_t)b * R + r) * topk;
-    for (int j = lane; j < topk; j += 32) out[j] = (int32_t)(0xFFFFFFFFu - (uint32_t)(kw[j] & 0xFFFFFFFFull));
 }
 
 cudaError_t launch_region_means(const void *q, const void *k, float *qm, float *km, const Geometry &g, bool bf16,
@@ -163,7 +183,7 @@ cudaError_t launch_region_means(const void *q, const void *k, float *qm, float *
     const int n_chunks = (g.n_win + rx_per_cta - 1) / rx_per_cta;
     const int nvec = rx_per_cta * g.wr * (g.C / V);
     int threads = ((nvec + 31) / 32) * 32;
-    threads = threads < 64 ? 64 : (threads > 512 ? 512 : threads);
+    threads = threads < 64 ? 64 : (threads > 256 ? 256 : threads);
     const dim3 grid((unsigned)((long long)g.B * g.n_win * n_chunks), 2);
     if (bf16)
         region_means_kernel<__nv_bfloat16><<<grid, threads, smem, stream>>>(
@@ -179,11 +199,26 @@ cudaError_t launch_route_topk(const float *qm, const float *km, int32_t *idx, co
     int P = 1;
     while (P < g.R) P <<= 1;
     if (P < 32) P = 32;
-    int warps = 8;
-    while (warps > 1 && (size_t)warps * P * 8 > 48 * 1024) --warps;
-    const dim3 grid((unsigned)((long long)((g.R + warps - 1) / warps) * g.B));
+    const int warps = 8;
+    const int rows = 16;
+    const size_t key_bytes = (size_t)warps * P * 8;
+    const size_t stage_bytes = (size_t)(g.R + rows) * (g.C + 4) * sizeof(float);
+    const int staged = key_bytes + stage_bytes <= 160 * 1024;
+    const size_t smem = key_bytes + (staged ? stage_bytes : 0);
+    static int granted[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if ((int)smem > granted[dev]) {
+        e = cudaFuncSetAttribute(route_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        granted[dev] = (int)smem;
+    }
+    const long long blocks = (long long)((g.R + rows - 1) / rows) * g.B;
     const float scale = (float)(1.0 / sqrt((double)g.C));
-    route_topk_kernel<<<grid, warps * 32, (size_t)warps * P * 8, stream>>>(qm, km, idx, g.R, g.C, g.topk, P, scale);
+    route_topk_kernel<<<(unsigned)blocks, warps * 32, smem, stream>>>(qm, km, idx, g.R, g.C, g.topk, P, rows, staged,
+                                                                      scale);
     return cudaGetLastError();
 }
 
