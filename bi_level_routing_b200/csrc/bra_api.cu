@@ -208,6 +208,22 @@ bra_status attend_impl(const void *q, const void *k, const void *v, const int32_
 
 }  // namespace
 
+namespace bra {
+
+void set_last_error(const std::string &msg) { g_last_error = msg; }
+
+bra_status check_route_args(const void *q, const void *k, const int32_t *idx, int B, int H, int W, int C, int n_win,
+                            int topk, bra_dtype dtype, Geometry *g)
+{
+    bra_status s = check_shape(B, H, W, C, 1, n_win, topk, dtype, g);
+    if (s != BRA_OK || B == 0) return s;
+    if (!q || !k || !idx) return BRA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(idx, 4)) return BRA_ERR_INVALID_ARG;
+    return BRA_OK;
+}
+
+}  // namespace bra
+
 extern "C" {
 
 bra_status bra_route(const void *q, const void *k, int32_t *idx, int B, int H, int W, int C, int n_win, int topk,

@@ -5,6 +5,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <string>
+
+#include "bra.h"
+
 namespace bra {
 
 // Bits of the sticky device error word.
@@ -16,6 +20,13 @@ struct Geometry {
     int B, H, W, C, heads, n_win, topk;
     int R, hr, wr, rs, hd, N;
 };
+
+// Sets the message bra_last_error_message returns on this thread.
+void set_last_error(const std::string &msg);
+
+// The argument checks of bra_route (shape, NULL pointers, alignment); fills g.
+bra_status check_route_args(const void *q, const void *k, const int32_t *idx, int B, int H, int W, int C, int n_win,
+                            int topk, bra_dtype dtype, Geometry *g);
 
 // Region means of q and k (fp32, [B, R, C] each) into qm and km.
 cudaError_t launch_region_means(const void *q, const void *k, float *qm, float *km, const Geometry &g,

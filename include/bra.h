@@ -98,6 +98,20 @@ bra_status bra_attend(const void *q, const void *k, const void *v, const int32_t
 bra_status bra_forward(const void *q, const void *k, const void *v, int32_t *idx, void *out, int B, int H,
                        int W, int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream);
 
+/* Steps 1-4 exactly like bra_route (same kernels, same idx), for callers that cannot
+   allocate device memory when they call: for example a process that hands all of HBM to its
+   own allocator at start-up, or a latency-critical loop that must not take allocator locks or
+   risk an out-of-memory error mid-step. It allocates nothing: the fp32 scratch for the
+   region means (2 * B * n_win^2 * C * 4 bytes) lives in a fixed 8 MiB device array inside
+   the library (held by every GPU that loads it until the process exits), and a call that
+   needs more returns BRA_ERR_UNSUPPORTED, with the sizes in bra_last_error_message(),
+   before anything runs. The first call on each device finds that array's device address
+   (cudaGetSymbolAddress), so make it before any stream capture. All calls on a device share
+   the array; calls whose kernels overlap on the GPU race on it, so order them on one stream.
+   The paper has no counterpart to this entry point: it is a deployment variant. */
+bra_status bra_route_noalloc(const void *q, const void *k, int32_t *idx, int B, int H, int W, int C, int n_win,
+                             int topk, bra_dtype dtype, void *stream);
+
 /* bra_forward on HOST buffers: copies q, k, v (host, [B, H, W, C]) to device scratch from
    the library's pool, runs the forward pass on `stream`, copies idx and out back to the
    host buffers and synchronises `stream` before returning. Page-locked host memory gives

@@ -1,0 +1,55 @@
+"""bra_route_noalloc: routing with no device allocation, checked against bra_route.
+
+Callers that cannot allocate device memory mid-run use bra_route_noalloc instead of
+bra_route: a process that hands all of HBM to its own allocator at start-up, or a
+latency-critical loop that must not take allocator locks or risk an out-of-memory error.
+Its scratch is a fixed array inside the library, shared by every call, so this test makes
+two calls in a row on different shapes and checks that each returns exactly bra_route's
+indices (the same kernels run, so the routing must be bit-identical). It sits in a file of
+its own, collected last.
+"""
+import ctypes
+
+import pytest
+import torch
+
+import bi_level_routing_b200 as bra
+from bi_level_routing_b200 import api
+from bi_level_routing_b200.workloads import WORKLOADS
+from parity import make
+
+pytestmark = pytest.mark.gpu
+
+
+def _lib():
+    L = api.lib()
+    vp, I = ctypes.c_void_p, ctypes.c_int
+    L.bra_route_noalloc.argtypes = [vp, vp, vp, I, I, I, I, I, I, I, vp]
+    L.bra_route_noalloc.restype = I
+    return L
+
+
+def _route_noalloc(L, q, k, idx, n_win, topk):
+    B, H, W, C = q.shape
+    return L.bra_route_noalloc(q.data_ptr(), k.data_ptr(), idx.data_ptr(), B, H, W, C, n_win, topk,
+                               api.DTYPES[q.dtype], torch.cuda.current_stream().cuda_stream)
+
+
+def test_no_alloc_route_matches_bra_route_on_two_calls_in_a_row():
+    L = _lib()
+    for w in (WORKLOADS["stage1"].with_(B=16), WORKLOADS["highres"].with_(B=2)):
+        _, (q, k, _) = make(w)
+        ref = bra.route(q, k, w.n_win, w.topk)
+        idx = torch.full_like(ref, -7)
+        assert _route_noalloc(L, q, k, idx, w.n_win, w.topk) == 0, L.bra_last_error_message()
+        torch.cuda.synchronize()
+        assert torch.equal(idx, ref), f"{w.name}: bra_route_noalloc differs from bra_route"
+
+
+def test_no_alloc_route_rejects_sizes_beyond_its_scratch():
+    L = _lib()
+    w = WORKLOADS["stage4"]  # 2 * 64 * 49 * 512 * 4 bytes = 12.8 MB > 8 MiB
+    fake = 0x10000  # rejected before any use
+    status = L.bra_route_noalloc(fake, fake, fake, w.B, w.H, w.W, w.C, w.n_win, w.topk, 1, None)
+    assert status == 2  # BRA_ERR_UNSUPPORTED
+    assert b"bytes of scratch" in L.bra_last_error_message()
