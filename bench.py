@@ -34,7 +34,8 @@ sys.path.insert(0, ROOT)
 METRIC = "BRA forward tokens/s on 1 B200 (device-timed) and % of roofline"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = {"attend_gather_mma": "bi_level_routing_b200/csrc/bra_attend_mma.cu",
+KERNEL_SOURCES = {"attend_gather_umma": "bi_level_routing_b200/csrc/bra_attend_umma.cu",
+                  "attend_gather_mma": "bi_level_routing_b200/csrc/bra_attend_mma.cu",
                   "attend_dense_mma": "bi_level_routing_b200/csrc/bra_attend_mma.cu",
                   "attend_simt": "bi_level_routing_b200/csrc/bra_attend_simt.cu"}
 

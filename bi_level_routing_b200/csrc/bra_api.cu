@@ -112,8 +112,8 @@ bra_status check_shape(int B, int H, int W, int C, int heads, int n_win, int top
     g->rs = g->hr * g->wr;
     g->hd = C / heads;
     g->N = H * W;
-    // The means kernel keeps one region column's partial sums (wr x C fp32) in 48 KB.
-    if ((long long)g->wr * C * 4 > 48 * 1024) return BRA_ERR_UNSUPPORTED;
+    // The means kernel holds one region's row segment (wr tokens x C channels) in registers.
+    if ((long long)g->wr * C * elem > 16LL * bra::kMaxMeansVectors) return BRA_ERR_UNSUPPORTED;
     return BRA_OK;
 }
 
@@ -123,14 +123,17 @@ int choose_attend_kernel(const bra::Geometry &g, bra_dtype dtype)
     const bool simt_ok = g.hd <= bra::kSimtMaxHeadDim;
     const bool gather_ok = bf16 && bra::gather_mma_supports(g);
     const bool dense_ok = bf16 && bra::dense_mma_supports(g);
+    const bool umma_ok = bf16 && bra::gather_umma_supports(g);
     switch (g_forced_kernel.load()) {
     case BRA_ATTEND_SIMT: return simt_ok ? BRA_ATTEND_SIMT : -1;
     case BRA_ATTEND_GATHER_MMA: return gather_ok ? BRA_ATTEND_GATHER_MMA : -1;
     case BRA_ATTEND_DENSE_MMA: return dense_ok ? BRA_ATTEND_DENSE_MMA : -1;
+    case BRA_ATTEND_GATHER_UMMA: return umma_ok ? BRA_ATTEND_GATHER_UMMA : -1;
     default: break;
     }
     // Dense attention over the whole image wastes at most 4x the routed work here.
     if (dense_ok && 4LL * g.topk * g.rs >= g.N) return BRA_ATTEND_DENSE_MMA;
+    if (umma_ok) return BRA_ATTEND_GATHER_UMMA;
     if (gather_ok) return BRA_ATTEND_GATHER_MMA;
     if (dense_ok) return BRA_ATTEND_DENSE_MMA;
     return simt_ok ? BRA_ATTEND_SIMT : -1;
@@ -184,6 +187,12 @@ bra_status attend_impl(const void *q, const void *k, const void *v, const int32_
     cudaError_t e = cudaSuccess;
     if (kernel == BRA_ATTEND_SIMT) {
         e = bra::launch_attend_simt(q, k, v, idx, out, g, dtype == BRA_BF16, st->error_word, stream);
+    } else if (kernel == BRA_ATTEND_GATHER_UMMA) {
+        CUtensorMap tq, tk, tv;
+        if ((s = encode_map(&tq, q, g, g.wr, g.hr)) != BRA_OK) return s;
+        if ((s = encode_map(&tk, k, g, g.wr, g.hr)) != BRA_OK) return s;
+        if ((s = encode_map(&tv, v, g, g.wr, g.hr)) != BRA_OK) return s;
+        e = bra::launch_attend_gather_umma(tq, tk, tv, idx, out, g, st->num_sms, st->error_word, stream);
     } else if (kernel == BRA_ATTEND_GATHER_MMA) {
         CUtensorMap tq, tk, tv, to;
         int box[4];
@@ -192,7 +201,7 @@ bra_status attend_impl(const void *q, const void *k, const void *v, const int32_
         if ((s = encode_map(&tk, k, g, box[1], box[2])) != BRA_OK) return s;
         if ((s = encode_map(&tv, v, g, box[1], box[2])) != BRA_OK) return s;
         if ((s = encode_map(&to, out, g, box[1], box[2])) != BRA_OK) return s;
-        e = bra::launch_attend_gather_mma(tq, tk, tv, to, idx, g, st->num_sms, st->error_word, stream);
+        e = bra::launch_attend_gather_mma(tq, tk, tv, to, idx, out, g, st->num_sms, st->error_word, stream);
     } else {
         const int rows = bra::dense_mma_rows_per_split(g, st->num_sms);
         CUtensorMap tq, tk, tv, to;
@@ -308,7 +317,7 @@ bra_status bra_forward_host(const void *q, const void *k, const void *v, int32_t
 
 bra_status bra_set_attend_kernel(bra_attend_kernel kernel)
 {
-    if (kernel < BRA_ATTEND_AUTO || kernel > BRA_ATTEND_DENSE_MMA) return BRA_ERR_INVALID_ARG;
+    if (kernel < BRA_ATTEND_AUTO || kernel > BRA_ATTEND_GATHER_UMMA) return BRA_ERR_INVALID_ARG;
     g_forced_kernel.store(kernel);
     return BRA_OK;
 }

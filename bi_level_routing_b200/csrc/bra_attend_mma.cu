@@ -106,7 +106,7 @@ __device__ __forceinline__ void stage_output(uint32_t tile, const float (&o)[4][
                                              int hb, int lane)
 {
     const float l0 = quad_sum(l[0]), l1 = quad_sum(l[1]);
-    const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+    const float inv0 = l0 > 0.f ? __fdividef(1.f, l0) : 0.f, inv1 = l1 > 0.f ? __fdividef(1.f, l1) : 0.f;
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
@@ -118,6 +118,8 @@ __device__ __forceinline__ void stage_output(uint32_t tile, const float (&o)[4][
 struct GatherArgs {
     const int32_t *idx;
     unsigned *err;
+    __nv_bfloat16 *out;   // [B, H, W, C]
+    int H, W, C;
     int n_win, topk, R, hr, wr;
     int ncb;          // 64-channel blocks in C
     int ncb_per_cta;  // channel blocks one work item covers (NCB)
@@ -129,20 +131,42 @@ struct GatherArgs {
     float scale_log2;
 };
 
+// Per-lane byte offsets of the ldmatrix rows inside 128-byte-swizzled tiles. Every row a lane
+// addresses has the same (row & 7), so the swizzle XOR depends on the lane only and the
+// offsets of later 8-row groups are compile-time constants (+1024 per 8 rows).
+struct LaneOffsets {
+    uint32_t q[2];   // Q tile, 16-row tile rt, k-steps 0 and 1 of head hb
+    uint32_t k;      // K tile, keys (lane & 7) + 8 nt, channels of head hb
+    uint32_t v[2];   // V tile (transposed loads), keys + 16 kk, channel pairs np = 0, 1
+};
+
+__device__ __forceinline__ LaneOffsets lane_offsets(int rt, int hb, int lane)
+{
+    LaneOffsets o;
+    const int x = lane & 7;
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) o.q[ks] = sw128(rt * 16 + (lane & 15), hb * 4 + ks * 2 + (lane >> 4));
+    o.k = (uint32_t)x * 128u + ((uint32_t)((hb * 4 + (lane >> 3)) ^ x) << 4);
+#pragma unroll
+    for (int np = 0; np < 2; ++np)
+        o.v[np] = (uint32_t)(x + ((lane >> 3) & 1) * 8) * 128u + ((uint32_t)((hb * 4 + np * 2 + (lane >> 4)) ^ x) << 4);
+    return o;
+}
+
 // S = Q K^T for one 16-row tile of one head against one routed region (NT 8-key n-tiles),
 // online-softmax update of (m, l, o), then O += P V. P is rounded down to bf16 (the low
 // half of the fp32 bits dropped) and the row sums accumulate exactly those values, so the
 // normalisation matches the weights used.
 template <int NT>
 __device__ __forceinline__ void attend_region(float (&o)[4][4], float (&m)[2], float (&l)[2], const uint32_t (&qf)[2][4],
-                                              uint32_t ktile, uint32_t vtile, int hb, int lane, float scale_log2)
+                                              uint32_t ktile, uint32_t vtile, const LaneOffsets &off, float scale_log2)
 {
     float sc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
         uint32_t b0, b1, b2, b3;
-        ldmatrix_x4(ktile + sw128(nt * 8 + (lane & 7), hb * 4 + (lane >> 3)), b0, b1, b2, b3);
+        ldmatrix_x4(ktile + off.k + nt * 1024, b0, b1, b2, b3);
         mma_bf16_16816(sc[nt], qf[0], b0, b1);
         mma_bf16_16816(sc[nt], qf[1], b2, b3);
     }
@@ -176,13 +200,18 @@ __device__ __forceinline__ void attend_region(float (&o)[4][4], float (&m)[2], f
 #pragma unroll
         for (int np = 0; np < 2; ++np) {
             uint32_t b0, b1, b2, b3;
-            const int row = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-            ldmatrix_x4_trans(vtile + sw128(row, hb * 4 + np * 2 + (lane >> 4)), b0, b1, b2, b3);
+            ldmatrix_x4_trans(vtile + off.v[np] + kk * 2048, b0, b1, b2, b3);
             mma_bf16_16816(o[2 * np], pa, b0, b1);
             mma_bf16_16816(o[2 * np + 1], pa, b2, b3);
         }
     }
 }
+
+// Item coordinates the producer publishes with each query slot: image, the query region's
+// top-left token (x, y), first channel block and number of channel blocks.
+struct ItemInfo {
+    int b, qx, qy, cb;
+};
 
 // Persistent, warp-specialised gather attention. Each CTA owns a contiguous run of work
 // items (image, query region, group of NCB 64-channel blocks), in image order.
@@ -212,13 +241,13 @@ __global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_
     const int NCB = a.ncb_per_cta;
     uint8_t *sQ = smem;
     uint8_t *sKV = sQ + (size_t)a.qslots * NCB * TILE;
-    uint8_t *sO = sKV + (size_t)a.kvslots * 2 * NCB * TILE;
-    uint64_t *full_q = reinterpret_cast<uint64_t *>(sO + (size_t)2 * NCB * TILE);
+    uint64_t *full_q = reinterpret_cast<uint64_t *>(sKV + (size_t)a.kvslots * 2 * NCB * TILE);
     uint64_t *empty_q = full_q + a.qslots;
     uint64_t *full_kv = empty_q + a.qslots;
     uint64_t *empty_kv = full_kv + a.kvslots;
     int *kv_ok = reinterpret_cast<int *>(empty_kv + a.kvslots);
-    int *sidx = kv_ok + a.kvslots;
+    ItemInfo *qinfo = reinterpret_cast<ItemInfo *>(kv_ok + a.kvslots);
+    int *sidx = reinterpret_cast<int *>(qinfo + a.qslots);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int begin = blockIdx.x * a.per_cta;
@@ -259,6 +288,7 @@ __global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_
                 const int cb0 = grp * NCB, nh = min(NCB, a.ncb - cb0);
                 const int qx = (r % a.n_win) * a.wr, qy = (r / a.n_win) * a.hr;
                 if (!(alive = mbar_wait(&empty_q[qs], qph ^ 1, a.err))) break;
+                qinfo[qs] = ItemInfo{b, qx, qy, (cb0 << 8) | nh};
                 mbar_arrive_expect_tx(&full_q[qs], (uint32_t)(nh * TILE));
                 for (int cb = 0; cb < nh; ++cb)
                     tma_load_4d(sQ + (size_t)(qs * NCB + cb) * TILE, &tq, (cb0 + cb) * 64, qx, qy, b, &full_q[qs]);
@@ -295,26 +325,28 @@ __global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_
 
     // ----------------------------------------------------------------- consumer warps
     const int rt = warp % RT, hb = (warp / RT) & 1, cbl = warp / (2 * RT);
-    const int consumers = a.ncw * 32;
-    int qs = 0, kvs = 0, os = 0;
+    const LaneOffsets off = lane_offsets(rt, hb, lane);
+    // element offsets, inside the region's first token, of this lane's two output rows
+    // (rows g and g + 8 of the 16-row tile), channel pair 2t of head hb
+    int row_off[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int ri = rt * 16 + (lane >> 2) + 8 * h;
+        row_off[h] = ((ri / a.wr) * a.W + ri % a.wr) * a.C + hb * 32 + 2 * (lane & 3);
+    }
+    int qs = 0, kvs = 0;
     uint32_t qph = 0, kvph = 0;
     bool alive = true;
     for (int item = begin; item < end; ++item) {
-        const int grp = item % a.groups;
-        const int br = item / a.groups;
-        const int r = br % a.R, b = br / a.R;
-        const int cb0 = grp * NCB, nh = min(NCB, a.ncb - cb0);
-        const int qx = (r % a.n_win) * a.wr, qy = (r / a.n_win) * a.hr;
-        const bool active = cbl < nh;
-
         uint32_t qf[2][4];
         if (alive) alive = mbar_wait(&full_q[qs], qph, a.err);
+        const ItemInfo info = qinfo[qs];
+        const int cb0 = info.cb >> 8, nh = info.cb & 0xff;
+        const bool active = cbl < nh;
         if (alive && active) {
             const uint32_t qtile = smem_u32(sQ + (size_t)(qs * NCB + cbl) * TILE);
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks)
-                ldmatrix_x4(qtile + sw128(rt * 16 + (lane & 15), hb * 4 + ks * 2 + (lane >> 4)), qf[ks][0], qf[ks][1],
-                            qf[ks][2], qf[ks][3]);
+            ldmatrix_x4(qtile + off.q[0], qf[0][0], qf[0][1], qf[0][2], qf[0][3]);
+            ldmatrix_x4(qtile + off.q[1], qf[1][0], qf[1][1], qf[1][2], qf[1][3]);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_q[qs]);
@@ -331,7 +363,7 @@ __global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_
             if (alive) alive = mbar_wait(&full_kv[kvs], kvph, a.err);
             if (alive && active && kv_ok[kvs]) {
                 const uint32_t ktile = smem_u32(sKV + (size_t)(kvs * 2 * NCB + cbl) * TILE);
-                attend_region<NT>(o, m, l, qf, ktile, ktile + NCB * TILE, hb, lane, a.scale_log2);
+                attend_region<NT>(o, m, l, qf, ktile, ktile + NCB * TILE, off, a.scale_log2);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty_kv[kvs]);
@@ -341,25 +373,24 @@ __global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_
             }
         }
 
-        // epilogue: output slot `os` was last stored two items ago; let that store finish reading
-        if (warp == 0 && lane == 0) tma_store_wait_read_n<1>();
-        named_barrier(1, consumers);
-        if (alive && active) stage_output(smem_u32(sO + (size_t)(os * NCB + cbl) * TILE), o, l, rt * 16, hb, lane);
-        fence_async_shared();
-        named_barrier(1, consumers);
-        if (warp == 0 && lane == 0 && alive) {
-            for (int cb = 0; cb < nh; ++cb)
-                tma_store_4d(&tout, sO + (size_t)(os * NCB + cb) * TILE, (cb0 + cb) * 64, qx, qy, b);
-            tma_store_commit();
+        // epilogue: normalise and store this warp's 16 x 32 output straight to global memory
+        if (alive && active) {
+            const float l0 = quad_sum(l[0]), l1 = quad_sum(l[1]);
+            const float inv0 = l0 > 0.f ? __fdividef(1.f, l0) : 0.f, inv1 = l1 > 0.f ? __fdividef(1.f, l1) : 0.f;
+            __nv_bfloat16 *dst = a.out + (((int64_t)info.b * a.H + info.qy) * a.W + info.qx) * a.C + (cb0 + cbl) * 64;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                *reinterpret_cast<uint32_t *>(dst + row_off[0] + nt * 8) = pack_bf16x2(o[nt][0] * inv0, o[nt][1] * inv0);
+                *reinterpret_cast<uint32_t *>(dst + row_off[1] + nt * 8) = pack_bf16x2(o[nt][2] * inv1, o[nt][3] * inv1);
+            }
         }
-        os ^= 1;
     }
-    if (warp == 0 && lane == 0) tma_store_wait_read_n<0>();
 }
 
 bool gather_mma_supports(const Geometry &g)
 {
-    return g.hd == 32 && g.C % 64 == 0 && g.rs % 16 == 0 && g.rs <= 64 && g.wr <= 256 && g.hr <= 256;
+    return g.hd == 32 && g.C % 64 == 0 && g.rs % 16 == 0 && g.rs <= 64 && g.wr <= 256 && g.hr <= 256 &&
+           (long long)g.hr * g.W * g.C < (1LL << 31);
 }
 
 void gather_mma_box(const Geometry &g, int box[4])
@@ -384,12 +415,16 @@ static cudaError_t launch_gather_rs(const CUtensorMap &tq, const CUtensorMap &tk
 }
 
 cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                     const CUtensorMap &tout, const int32_t *idx, const Geometry &g, int num_sms,
-                                     unsigned *err, cudaStream_t stream)
+                                     const CUtensorMap &tout, const int32_t *idx, void *out, const Geometry &g,
+                                     int num_sms, unsigned *err, cudaStream_t stream)
 {
     GatherArgs a;
     a.idx = idx;
     a.err = err;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.H = g.H;
+    a.W = g.W;
+    a.C = g.C;
     a.n_win = g.n_win;
     a.topk = g.topk;
     a.R = g.R;
@@ -410,14 +445,14 @@ cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &t
     // Two CTAs per SM: ~111 KB of shared memory each for the rings.
     const size_t tile = (size_t)g.rs * kRowBytes * ncb_per_cta;  // one slot of one tensor
     const size_t budget = 111 * 1024;
-    a.qslots = g.topk <= 2 ? 3 : 2;
-    long long kv = (long long)((budget - (a.qslots + 2) * tile) / (2 * tile));
+    a.qslots = g.topk <= 2 ? 4 : 2;
+    long long kv = (long long)((budget - a.qslots * tile) / (2 * tile));
     if (kv > 8) kv = 8;
     if (kv < 2) kv = 2;
     a.kvslots = (int)kv;
     a.idx_chunk = g.topk >= 32 ? 1 : 32 / g.topk;
-    const size_t smem = 1024 + tile * (a.qslots + 2 * a.kvslots + 2) + 16 * (a.qslots + a.kvslots) +
-                        4 * a.kvslots + 4 * (size_t)a.idx_chunk * g.topk;
+    const size_t smem = 1024 + tile * (a.qslots + 2 * a.kvslots) + 16 * (a.qslots + a.kvslots) + 4 * a.kvslots +
+                        sizeof(ItemInfo) * a.qslots + 4 * (size_t)a.idx_chunk * g.topk;
     int grid = 2 * num_sms;
     if (grid > a.nitems) grid = a.nitems;
     a.per_cta = (a.nitems + grid - 1) / grid;

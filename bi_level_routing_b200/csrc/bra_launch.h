@@ -28,7 +28,9 @@ void set_last_error(const std::string &msg);
 bra_status check_route_args(const void *q, const void *k, const int32_t *idx, int B, int H, int W, int C, int n_win,
                             int topk, bra_dtype dtype, Geometry *g);
 
-// Region means of q and k (fp32, [B, R, C] each) into qm and km.
+// Region means of q and k (fp32, [B, R, C] each) into qm and km. One region row segment
+// (wr tokens x C channels) may hold at most kMaxMeansVectors 16-byte vectors.
+constexpr int kMaxMeansVectors = 2048;
 cudaError_t launch_region_means(const void *q, const void *k, float *qm, float *km, const Geometry &g,
                                 bool bf16, int num_sms, cudaStream_t stream);
 
@@ -53,8 +55,15 @@ bool dense_mma_supports(const Geometry &g);
 // Boxes (channels, x, y, images) of the gather kernel: one region, 64 channels, for all four maps.
 void gather_mma_box(const Geometry &g, int box[4]);
 cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                     const CUtensorMap &tout, const int32_t *idx, const Geometry &g, int num_sms,
-                                     unsigned *err, cudaStream_t stream);
+                                     const CUtensorMap &tout, const int32_t *idx, void *out, const Geometry &g,
+                                     int num_sms, unsigned *err, cudaStream_t stream);
+
+// tcgen05 gather attention for 64-token regions (bf16, hd == 32, C % 64 == 0). Maps: q, k, v
+// with box (64, wr, hr, 1).
+bool gather_umma_supports(const Geometry &g);
+cudaError_t launch_attend_gather_umma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                      const int32_t *idx, void *out, const Geometry &g, int num_sms, unsigned *err,
+                                      cudaStream_t stream);
 
 // Boxes of the dense kernel: q and out (64, W, rows_per_split, 1); k and v (64, W, H, 1).
 int dense_mma_rows_per_split(const Geometry &g, int num_sms);

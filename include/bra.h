@@ -77,8 +77,11 @@ typedef enum {
     BRA_ATTEND_SIMT = 1,      /* any dtype, hd <= 128: one thread per (query, head), CUDA cores */
     BRA_ATTEND_GATHER_MMA = 2,/* bf16, hd == 32, C % 64 == 0, rs % 16 == 0, rs <= 64: per-region
                                  tiles staged by TMA, tensor-core QK^T and PV */
-    BRA_ATTEND_DENSE_MMA = 3  /* bf16, hd == 32, C % 64 == 0, R <= 64, H*W <= 256: the image's
+    BRA_ATTEND_DENSE_MMA = 3, /* bf16, hd == 32, C % 64 == 0, R <= 64, H*W <= 256: the image's
                                  K/V staged once, masked by the routing multiplicities */
+    BRA_ATTEND_GATHER_UMMA = 4/* bf16, hd == 32, C % 64 == 0, rs == 64: per-region tiles staged by
+                                 TMA, QK^T and PV on the tcgen05 tensor cores with TMEM
+                                 accumulators, one softmax thread per query row */
 } bra_attend_kernel;
 
 /* Steps 1-4: idx[b, r, :] = routing index of region r of image b.

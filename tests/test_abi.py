@@ -86,8 +86,8 @@ def test_unsupported_sizes(L):
 
 def test_kernel_selection_per_workload(L):
     assert L.bra_set_attend_kernel(0) == OK
-    want = {"tiny_f32": "simt", "stage1": "gather_mma", "stage2": "gather_mma", "stage3": "dense_mma",
-            "stage4": "dense_mma", "highres": "gather_mma"}
+    want = {"tiny_f32": "simt", "stage1": "gather_umma", "stage2": "gather_mma", "stage3": "dense_mma",
+            "stage4": "dense_mma", "highres": "gather_umma"}
     import torch
     for name, kernel in want.items():
         w = WORKLOADS[name]
@@ -98,6 +98,9 @@ def test_kernel_selection_per_workload(L):
 def test_forcing_a_kernel(L):
     try:
         assert L.bra_set_attend_kernel(9) == INVALID
+        assert L.bra_set_attend_kernel(4) == OK
+        assert L.bra_selected_attend_kernel(64, 56, 56, 64, 2, 7, 1, 1) == 4
+        assert L.bra_selected_attend_kernel(64, 28, 28, 128, 4, 7, 4, 1) == -1  # 16-token regions
         assert L.bra_set_attend_kernel(1) == OK
         assert L.bra_selected_attend_kernel(64, 56, 56, 64, 2, 7, 1, 1) == 1
         assert L.bra_set_attend_kernel(3) == OK

@@ -75,7 +75,7 @@ def _small(spec, values="region_offset", seed=1234):
 def _kernels_for(w):
     dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
     out = []
-    for kname in ("simt", "gather_mma", "dense_mma"):
+    for kname in ("simt", "gather_mma", "dense_mma", "gather_umma"):
         bra.set_attend_kernel(kname)
         if bra.selected_attend_kernel(w.B, w.H, w.W, w.C, w.heads, w.n_win, w.topk, dt) == kname:
             out.append(kname)
