@@ -15,9 +15,9 @@
 //                        into TMEM lanes {0-15, 32-47, 64-79, 96-111} columns 0-63, head 1 into
 //                        the same columns at lane offset 16 (an M = 64 accumulator fills 16
 //                        lanes of each 32-lane quadrant);
-//      O_h = P_h V      (M = 64, N = 64 channels of V, K = 64 keys), P_h from shared memory;
-//                        head 0 at columns 64-127, head 1 at columns 32-95 of its lanes, so
-//                        that both heads' own 32 output channels land in columns 64-95.
+//      O_h = P_h V_h    (M = 64, N = 32 channels of head h, K = 64 keys), P_h from shared
+//                        memory, V_h = head h's channels of the V tile (MN-major); both heads'
+//                        products land in the same 32 columns, at their own lanes.
 //    tcgen05.commit signals each product on an mbarrier and frees the query / KV slots.
 //  * warps 2-5, softmax: thread t of warp w owns query row 16 (w % 4) + (t % 16) of head t / 16,
 //    i.e. TMEM lane 32 (w % 4) + t. Per region it loads its 64 scores, updates the running max
@@ -35,9 +35,9 @@ namespace {
 
 constexpr int kRows = 64;                 // tokens per region = M of every MMA
 constexpr int kTile = kRows * 128;        // 64 rows x 64 bf16 channels, 128-byte swizzled rows
-constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kTmemCols = 256;  // S buffers at 0 and 64, O buffers at 128 and 192
 constexpr uint32_t kIdescS = umma_idesc_bf16(64, 64, false);  // Q K^T: B = K tile, K-major
-constexpr uint32_t kIdescPV = umma_idesc_bf16(64, 64, true);  // P V: B = V tile, MN-major
+constexpr uint32_t kIdescPV = umma_idesc_bf16(64, 32, true);  // P V_h: B = head h's 32 channels of V, MN-major
 
 struct UmmaArgs {
     const int32_t *idx;
@@ -64,16 +64,17 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem;
     uint8_t *sKV = sQ + (size_t)a.qslots * kTile;
-    uint8_t *sP = sKV + (size_t)a.kvslots * 2 * kTile;  // P tiles of heads 0 and 1
-    uint64_t *q_full = reinterpret_cast<uint64_t *>(sP + 2 * kTile);
+    uint8_t *sP = sKV + (size_t)a.kvslots * 2 * kTile;  // [2 buffers][2 heads] P tiles
+    uint64_t *q_full = reinterpret_cast<uint64_t *>(sP + 4 * kTile);
     uint64_t *q_empty = q_full + a.qslots;
     uint64_t *kv_full = q_empty + a.qslots;
     uint64_t *kv_empty = kv_full + a.kvslots;
-    uint64_t *s_full = kv_empty + a.kvslots;
-    uint64_t *p_full = s_full + 1;
-    uint64_t *o_full = p_full + 1;
-    uint64_t *o_free = o_full + 1;
-    uint64_t *drain = o_free + 1;
+    uint64_t *s_full = kv_empty + a.kvslots;  // [2] per buffer
+    uint64_t *s_free = s_full + 2;
+    uint64_t *p_full = s_free + 2;
+    uint64_t *o_full = p_full + 2;
+    uint64_t *o_free = o_full + 2;
+    uint64_t *drain = o_free + 2;
     int *kv_ok = reinterpret_cast<int *>(drain + 1);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(kv_ok + a.kvslots);
     int *sidx = reinterpret_cast<int *>(tmem_slot + 1);
@@ -91,10 +92,13 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
             mbar_init(&kv_full[i], 1);
             mbar_init(&kv_empty[i], 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(p_full, 4);
-        mbar_init(o_full, 1);
-        mbar_init(o_free, 4);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_free[i], 4);
+            mbar_init(&p_full[i], 4);
+            mbar_init(&o_full[i], 1);
+            mbar_init(&o_free[i], 4);
+        }
         mbar_init(drain, 1);
         mbar_fence_init();
     }
@@ -158,63 +162,83 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------- MMA issuer
+        // Units u = (item, routed region j) in CTA order. S(u) goes to TMEM buffer u & 1 as soon
+        // as the softmax has loaded S(u - 2); PV(u - 1) follows once its P is written and the
+        // softmax has loaded O(u - 3). So S(u + 1) and PV(u - 1) run while the softmax works
+        // on unit u.
         if (lane == 0) {
-            int qs = 0, kvs = 0;
-            uint32_t qph = 0, kvph = 0, pph = 0, fph = 0;
-            bool alive = true, first_pv = true;
-            const uint32_t p_base = smem_u32(sP);
-            for (int item = begin; item < end && alive; ++item) {
-                if (!(alive = mbar_wait(&q_full[qs], qph, a.err))) break;
-                tcgen05_after_sync();
-                const uint32_t qa = smem_u32(sQ + (size_t)qs * kTile);
-                for (int j = 0; j < a.topk; ++j) {
-                    if (!(alive = mbar_wait(&kv_full[kvs], kvph, a.err))) break;
+            const int units = (end - begin) * a.topk;
+            int qs = 0;
+            uint32_t qph = 0;
+            bool alive = true, ok_prev = false;
+            int kvs_prev = 0;
+            // Descriptors of the tile bases; an offset of x bytes inside a tile is + (x >> 4).
+            const uint64_t dq0 = umma_desc_sw128(smem_u32(sQ));
+            const uint64_t dkv0 = umma_desc_sw128(smem_u32(sKV));
+            const uint64_t dp0 = umma_desc_sw128(smem_u32(sP));
+            constexpr uint64_t kTileStep = kTile >> 4;
+            uint64_t dq = dq0;
+            for (int u = 0; u <= units && alive; ++u) {
+                bool ok = false;
+                const int kvs = u % a.kvslots;
+                if (u < units) {
+                    const int j = u % a.topk;
+                    if (j == 0) {
+                        if (!(alive = mbar_wait(&q_full[qs], qph, a.err))) break;
+                        dq = dq0 + (uint64_t)qs * kTileStep;
+                    }
+                    if (!(alive = mbar_wait(&kv_full[kvs], (uint32_t)((u / a.kvslots) & 1), a.err))) break;
+                    const int b = u & 1;
+                    if (u >= 2 && !(alive = mbar_wait(&s_free[b], (uint32_t)(((u >> 1) & 1) ^ 1), a.err))) break;
                     tcgen05_after_sync();
-                    const bool ok = kv_ok[kvs] != 0;
-                    const uint32_t ka = smem_u32(sKV + (size_t)kvs * 2 * kTile), va = ka + kTile;
+                    ok = kv_ok[kvs] != 0;
                     if (ok) {
-#pragma unroll
-                        for (int h = 0; h < 2; ++h)
-#pragma unroll
-                            for (int ks = 0; ks < 2; ++ks)
-                                umma_bf16(tmem + ((uint32_t)(16 * h) << 16),
-                                          umma_desc_sw128(qa + h * 64 + ks * 32),
-                                          umma_desc_sw128(ka + h * 64 + ks * 32), kIdescS, (uint32_t)ks);
-                        umma_commit(s_full);
+                        const uint64_t dk = dkv0 + (uint64_t)(2 * kvs) * kTileStep;
+                        const uint32_t ds = tmem + 64 * b;
+                        // S_h = Q_h K_h^T: head h's 32 channels start 64 h bytes into each row
+                        umma_bf16(ds, dq + 0, dk + 0, kIdescS, 0u);
+                        umma_bf16(ds, dq + 2, dk + 2, kIdescS, 1u);
+                        umma_bf16(ds + (16u << 16), dq + 4, dk + 4, kIdescS, 0u);
+                        umma_bf16(ds + (16u << 16), dq + 6, dk + 6, kIdescS, 1u);
+                        umma_commit(&s_full[b]);
                     } else {
-                        mbar_arrive(s_full);
+                        mbar_arrive(&s_full[b]);
                     }
-                    if (j == a.topk - 1) umma_commit(&q_empty[qs]);
-                    if (!(alive = mbar_wait(p_full, pph, a.err))) break;
-                    pph ^= 1;
-                    if (!first_pv) {
-                        if (!(alive = mbar_wait(o_free, fph, a.err))) break;
-                        fph ^= 1;
-                    }
-                    first_pv = false;
-                    tcgen05_after_sync();
-                    if (ok) {
-#pragma unroll
-                        for (int h = 0; h < 2; ++h)
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                umma_bf16(tmem + ((uint32_t)(16 * h) << 16) + (h ? 32u : 64u),
-                                          umma_desc_sw128(p_base + h * kTile + kk * 32),
-                                          umma_desc_sw128(va + kk * 2048), kIdescPV, (uint32_t)kk);
-                        umma_commit(o_full);
-                    } else {
-                        mbar_arrive(o_full);
-                    }
-                    umma_commit(&kv_empty[kvs]);
-                    if (++kvs == a.kvslots) {
-                        kvs = 0;
-                        kvph ^= 1;
+                    if (j == a.topk - 1) {
+                        umma_commit(&q_empty[qs]);
+                        if (++qs == a.qslots) {
+                            qs = 0;
+                            qph ^= 1;
+                        }
                     }
                 }
-                if (++qs == a.qslots) {
-                    qs = 0;
-                    qph ^= 1;
+                if (u >= 1) {
+                    const int v = u - 1, bv = v & 1;
+                    if (!(alive = mbar_wait(&p_full[bv], (uint32_t)((v >> 1) & 1), a.err))) break;
+                    if (v >= 2 && !(alive = mbar_wait(&o_free[bv], (uint32_t)(((v >> 1) & 1) ^ 1), a.err))) break;
+                    tcgen05_after_sync();
+                    if (ok_prev) {
+                        const uint64_t dv = dkv0 + (uint64_t)(2 * kvs_prev + 1) * kTileStep;
+                        const uint64_t dp = dp0 + (uint64_t)(2 * bv) * kTileStep;
+                        const uint32_t d0 = tmem + 128 + 64 * bv;
+                        // O_h = P_h V_h: A = P tile of head h (K = 64 keys, 32 bytes per 16-key
+                        // step), B = head h's 32 channels of V (MN-major, 64 h bytes into each
+                        // row; the next 16 keys are 16 rows = 2048 bytes on)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(d0, dp + 2 * kk, dv + 128 * kk, kIdescPV, (uint32_t)kk);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(d0 + (16u << 16), dp + kTileStep + 2 * kk, dv + 4 + 128 * kk, kIdescPV,
+                                      (uint32_t)kk);
+                        umma_commit(&o_full[bv]);
+                    } else {
+                        mbar_arrive(&o_full[bv]);
+                    }
+                    umma_commit(&kv_empty[kvs_prev]);
                 }
+                ok_prev = ok;
+                kvs_prev = kvs;
             }
             // every commit above arrives once the MMAs before it are done; wait for the last
             // one so that no arrival lands after this CTA has left
@@ -223,47 +247,72 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
         }
     } else {
         // ------------------------------------------------------------- softmax warpgroup
+        // Per unit u: load S(u), update the running max / sum of its item, write P(u); then fold
+        // in PV(u - 1): added to the accumulator (kept relative to the max of the previous
+        // unit) when it belongs to the same item, else it completes the previous item, which
+        // is normalised and stored.
         const int q = warp & 3;  // the TMEM lane quadrant this warp may access
         const int h = lane >> 4;
         const int row = 16 * q + (lane & 15);
-        const uint32_t t_s = tmem + ((uint32_t)(32 * q) << 16);
-        const uint32_t t_o = t_s + 64;
+        const uint32_t t_lane = tmem + ((uint32_t)(32 * q) << 16);
         const int out_row = ((row / a.wr) * a.W + row % a.wr) * a.C + h * 32;
-        uint8_t *prow = sP + h * kTile + row * 128;
-        uint32_t sph = 0, oph = 0;
-        bool alive = true;
-        for (int item = begin; item < end; ++item) {
-            const int cb = item % a.ncb;
-            const int br = item / a.ncb;
-            const int r = br % a.R, b = br / a.R;
-            const int32_t *routed = a.idx + (int64_t)br * a.topk;
-            float m = -INFINITY, l = 0.f;
-            float o[32];
+        const int units = (end - begin) * a.topk;
+        bool alive = true, ok_prev = false;
+        float m = -INFINITY, l = 0.f, l_prev = 0.f, corr = 1.f;
+        float o[32];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = 0.f;
-            int s_next = routed[0];
-            for (int j = 0; j < a.topk; ++j) {
+        for (int c = 0; c < 32; ++c) o[c] = 0.f;
+        __nv_bfloat16 *dst = nullptr, *dst_prev = nullptr;
+        // routing index of the next unit, loaded one unit ahead
+        int s_next = units > 0 ? a.idx[(int64_t)(begin / a.ncb) * a.topk] : 0;
+        for (int u = 0; u <= units; ++u) {
+            bool ok = false;
+            bool item_start = false;
+            if (u < units) {
+                const int item = begin + u / a.topk, j = u % a.topk;
                 const int s = s_next;
-                if (j + 1 < a.topk) s_next = routed[j + 1];
-                const bool ok = s >= 0 && s < a.R;
-                if (alive) alive = mbar_wait(s_full, sph, a.err);
-                sph ^= 1;
+                if (u + 1 < units) {
+                    const int item_n = begin + (u + 1) / a.topk, j_n = (u + 1) % a.topk;
+                    s_next = a.idx[(int64_t)(item_n / a.ncb) * a.topk + j_n];
+                }
+                ok = s >= 0 && s < a.R;
+                if (j == 0) {
+                    item_start = true;
+                    const int cb = item % a.ncb;
+                    const int br = item / a.ncb;
+                    const int r = br % a.R, bimg = br / a.R;
+                    const int qx = (r % a.n_win) * a.wr, qy = (r / a.n_win) * a.hr;
+                    dst_prev = dst;
+                    dst = a.out + (((int64_t)bimg * a.H + qy) * a.W + qx) * a.C + cb * 64 + out_row;
+                    l_prev = l;
+                    m = -INFINITY;
+                    l = 0.f;
+                }
+                const int b = u & 1;
+                if (alive) alive = mbar_wait(&s_full[b], (uint32_t)((u >> 1) & 1), a.err);
                 tcgen05_after_sync();
+                corr = 1.f;
                 if (alive && ok) {
                     uint32_t v0[32], v1[32];
-                    tmem_ld_32x32(t_s, v0);
-                    tmem_ld_32x32(t_s + 32, v1);
+                    tmem_ld_32x32(t_lane + 64 * b, v0);
+                    tmem_ld_32x32(t_lane + 64 * b + 32, v1);
                     tmem_wait_ld();
-                    float mx = -INFINITY;
+                    tcgen05_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s_free[b]);
+                    // row max with four independent chains
+                    float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fmaxf(__uint_as_float(v0[c]), __uint_as_float(v1[c])));
+                    for (int c = 0; c < 32; c += 2) {
+                        mx4[(c >> 1) & 3] = fmaxf(mx4[(c >> 1) & 3], fmaxf(__uint_as_float(v0[c]), __uint_as_float(v0[c + 1])));
+                        mx4[(c >> 1) & 3] = fmaxf(mx4[(c >> 1) & 3], fmaxf(__uint_as_float(v1[c]), __uint_as_float(v1[c + 1])));
+                    }
+                    const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
                     const float mn = fmaxf(m, mx * a.scale_log2);
-                    const float corr = fast_exp2(m - mn);
+                    corr = fast_exp2(m - mn);
                     m = mn;
-                    l *= corr;
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] *= corr;
-                    // probabilities, packed to bf16 pairs and written as 8 swizzled 16-byte chunks
+                    uint8_t *prow = sP + (2 * b + h) * kTile + row * 128;
+                    float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) {
                         uint32_t w[4];
@@ -274,42 +323,60 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
                             const float x1 = __uint_as_float(c + 1 < 32 ? v0[c + 1] : v1[c + 1 - 32]);
                             const float p0 = bf16_trunc(fast_exp2(fmaf(x0, a.scale_log2, -mn)));
                             const float p1 = bf16_trunc(fast_exp2(fmaf(x1, a.scale_log2, -mn)));
-                            l += p0 + p1;
+                            ls[e] += p0 + p1;
                             w[e] = pack_bf16x2_trunc(p0, p1);
                         }
                         *reinterpret_cast<uint4 *>(prow + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
+                    l = l * corr + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+                } else {
+                    tcgen05_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s_free[b]);
                 }
                 fence_async_shared();
                 tcgen05_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(p_full);
-                if (alive) alive = mbar_wait(o_full, oph, a.err);
-                oph ^= 1;
+                if (lane == 0) mbar_arrive(&p_full[b]);
+            }
+            if (u >= 1) {
+                const int v = u - 1, bv = v & 1;
+                if (alive) alive = mbar_wait(&o_full[bv], (uint32_t)((v >> 1) & 1), a.err);
                 tcgen05_after_sync();
-                if (alive && ok) {
-                    uint32_t pv[32];
-                    tmem_ld_32x32(t_o, pv);
+                if (alive && ok_prev) {
+                    // this thread's 32 output channels (both heads' products sit in the same columns)
+                    uint32_t w0[32];
+                    tmem_ld_32x32(t_lane + 128 + 64 * bv, w0);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] += __uint_as_float(pv[c]);
+                    for (int c = 0; c < 32; ++c) o[c] += __uint_as_float(w0[c]);
                 }
                 tcgen05_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(o_free);
-            }
-            if (alive) {
-                const float inv = l > 0.f ? __fdividef(1.f, l) : 0.f;
-                const int qx = (r % a.n_win) * a.wr, qy = (r / a.n_win) * a.hr;
-                __nv_bfloat16 *dst = a.out + (((int64_t)b * a.H + qy) * a.W + qx) * a.C + cb * 64 + out_row;
+                if (lane == 0) mbar_arrive(&o_free[bv]);
+                if (u == units || item_start) {
+                    // PV(u - 1) was the last region of the previous item: normalise and store it
+                    const float lf = (u == units) ? l : l_prev;
+                    __nv_bfloat16 *out = (u == units) ? dst : dst_prev;
+                    const float inv = lf > 0.f ? __fdividef(1.f, lf) : 0.f;
+                    if (alive) {
 #pragma unroll
-                for (int v = 0; v < 4; ++v)
-                    *reinterpret_cast<uint4 *>(dst + 8 * v) =
-                        make_uint4(pack_bf16x2(o[8 * v] * inv, o[8 * v + 1] * inv),
-                                   pack_bf16x2(o[8 * v + 2] * inv, o[8 * v + 3] * inv),
-                                   pack_bf16x2(o[8 * v + 4] * inv, o[8 * v + 5] * inv),
-                                   pack_bf16x2(o[8 * v + 6] * inv, o[8 * v + 7] * inv));
+                        for (int x = 0; x < 4; ++x)
+                            *reinterpret_cast<uint4 *>(out + 8 * x) =
+                                make_uint4(pack_bf16x2(o[8 * x] * inv, o[8 * x + 1] * inv),
+                                           pack_bf16x2(o[8 * x + 2] * inv, o[8 * x + 3] * inv),
+                                           pack_bf16x2(o[8 * x + 4] * inv, o[8 * x + 5] * inv),
+                                           pack_bf16x2(o[8 * x + 6] * inv, o[8 * x + 7] * inv));
+                    }
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = 0.f;
+                } else {
+                    // same item: bring the accumulator to the max of unit u
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] *= corr;
+                }
             }
+            ok_prev = ok;
         }
     }
 
@@ -346,10 +413,10 @@ cudaError_t launch_attend_gather_umma(const CUtensorMap &tq, const CUtensorMap &
     const long long nitems = (long long)g.B * g.R * a.ncb;
     if (nitems > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     a.nitems = (int)nitems;
-    a.qslots = 2;
-    a.kvslots = 2;
+    a.qslots = 3;
+    a.kvslots = 3;
     a.idx_chunk = g.topk >= 32 ? 1 : 32 / g.topk;
-    const size_t smem = 1024 + (size_t)kTile * (a.qslots + 2 * a.kvslots + 2) + 8 * (2 * a.qslots + 2 * a.kvslots + 5) +
+    const size_t smem = 1024 + (size_t)kTile * (a.qslots + 2 * a.kvslots + 4) + 8 * (2 * a.qslots + 2 * a.kvslots + 11) +
                         4 * a.kvslots + 4 + 4 * (size_t)a.idx_chunk * g.topk;
     int grid = 2 * num_sms;
     if (grid > a.nitems) grid = a.nitems;

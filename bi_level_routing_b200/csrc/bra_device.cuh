@@ -14,6 +14,8 @@ namespace bra {
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// Longest hardware suspension of one mbarrier try (a hint, in nanoseconds).
+constexpr uint32_t kWaitSuspendNs = 100000u;
 
 __device__ __forceinline__ unsigned long long global_timer_ns()
 {
@@ -119,16 +121,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitSuspendNs)
         : "memory");
     return done != 0;
 }
 
 // Waits for phase `parity` of `bar` to complete; gives up after kWaitLimitNs, flags
-// kErrTimeout and returns false.
+// kErrTimeout and returns false. Each try suspends the thread in hardware (up to
+// kWaitSuspendNs) until the phase completes, so waiting costs no issue slots.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned *err)
 {
     if (mbar_try_wait(bar, parity)) return true;
