@@ -331,7 +331,8 @@ def main():
                                              f"(> 2x the {l2 / 2**20:.0f} MiB L2)",
                        "launch": launch, "parallelism": f"dp{world} (images split, no collective)"},
             "roofline": roofline,
-            "gpu_launches": K * bra.kernels_per_call("bra_forward", w.B),
+            "gpu_launches": K * bra.kernels_per_call("bra_forward", w.B, w.H, w.W, w.C, w.heads, w.n_win, w.topk,
+                                                     torch.bfloat16 if w.dtype == "bf16" else torch.float32),
             "clocks": sampler.summary()}
 
     # ---- end to end through the host entry point (pinned buffers, copies inside the timed region)

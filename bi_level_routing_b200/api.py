@@ -50,7 +50,7 @@ def lib() -> ctypes.CDLL:
     L.bra_check_device_error.argtypes = [vp]
     L.bra_route_scratch_bytes.argtypes = [I, I, I, I, I]
     L.bra_route_scratch_bytes.restype = ctypes.c_size_t
-    L.bra_kernels_per_call.argtypes = [ctypes.c_char_p, I]
+    L.bra_kernels_per_call.argtypes = [ctypes.c_char_p, I, I, I, I, I, I, I, I]
     L.bra_status_string.argtypes = [I]
     L.bra_status_string.restype = ctypes.c_char_p
     L.bra_last_error_message.restype = ctypes.c_char_p
@@ -182,8 +182,8 @@ def selected_attend_kernel(B, H, W, C, heads, n_win, topk, dtype) -> str | None:
     return {v: k for k, v in ATTEND_KERNELS.items()}.get(code)
 
 
-def kernels_per_call(entry_point: str, B: int) -> int:
-    return lib().bra_kernels_per_call(entry_point.encode(), B)
+def kernels_per_call(entry_point: str, B, H, W, C, heads, n_win, topk, dtype) -> int:
+    return lib().bra_kernels_per_call(entry_point.encode(), B, H, W, C, heads, n_win, topk, DTYPES[dtype])
 
 
 def route_scratch_bytes(B, H, W, C, n_win) -> int:

@@ -112,7 +112,7 @@ bra_status check_shape(int B, int H, int W, int C, int heads, int n_win, int top
     g->rs = g->hr * g->wr;
     g->hd = C / heads;
     g->N = H * W;
-    // The means kernel holds one region's row segment (wr tokens x C channels) in registers.
+    // The means kernel holds one region's row segment (wr tokens x C channels) in shared memory.
     if ((long long)g->wr * C * elem > 16LL * bra::kMaxMeansVectors) return BRA_ERR_UNSUPPORTED;
     return BRA_OK;
 }
@@ -351,12 +351,18 @@ size_t bra_route_scratch_bytes(int B, int H, int W, int C, int n_win)
     return (size_t)2 * B * n_win * n_win * C * sizeof(float);
 }
 
-int bra_kernels_per_call(const char *entry_point, int B)
+int bra_kernels_per_call(const char *entry_point, int B, int H, int W, int C, int heads, int n_win, int topk,
+                         bra_dtype dtype)
 {
     if (!entry_point || B <= 0) return 0;
-    if (!std::strcmp(entry_point, "bra_route")) return 2;
-    if (!std::strcmp(entry_point, "bra_attend")) return 1;
-    if (!std::strcmp(entry_point, "bra_forward") || !std::strcmp(entry_point, "bra_forward_host")) return 3;
+    bra::Geometry g;
+    if (check_shape(B, H, W, C, heads, n_win, topk, dtype, &g) != BRA_OK) return 0;
+    const int route = 2;
+    const int attend = choose_attend_kernel(g, dtype) < 0 ? 0 : 1;
+    if (!std::strcmp(entry_point, "bra_route")) return route;
+    if (!std::strcmp(entry_point, "bra_attend")) return attend;
+    if (!std::strcmp(entry_point, "bra_forward") || !std::strcmp(entry_point, "bra_forward_host"))
+        return attend ? route + attend : 0;
     return 0;
 }
 

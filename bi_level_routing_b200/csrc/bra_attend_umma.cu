@@ -10,21 +10,23 @@
 //  * warp 0 lane 0, producer: TMA loads of the query tile (64 tokens x 64 channels) into a
 //    ring of query slots and, per routed region, of its K and V tiles into a ring of KV
 //    slots (128-byte swizzle, no multicast), as in the mma.sync gather kernel;
-//  * warp 1: allocates 128 TMEM columns; its lane 0 issues every MMA. Per routed region:
+//  * warp 1: allocates 256 TMEM columns (two S buffers at columns 0 and 64, two O buffers at
+//    128 and 192); its lane 0 issues every MMA. Per routed region:
 //      S_h = Q_h K_h^T  (M = 64 query rows, N = 64 keys, K = 32 channels of head h), head 0
-//                        into TMEM lanes {0-15, 32-47, 64-79, 96-111} columns 0-63, head 1 into
-//                        the same columns at lane offset 16 (an M = 64 accumulator fills 16
-//                        lanes of each 32-lane quadrant);
-//      O_h = P_h V_h    (M = 64, N = 32 channels of head h, K = 64 keys), P_h from shared
-//                        memory, V_h = head h's channels of the V tile (MN-major); both heads'
-//                        products land in the same 32 columns, at their own lanes.
+//                        into TMEM lanes {0-15, 32-47, 64-79, 96-111}, head 1 into the same
+//                        columns at lane offset 16 (an M = 64 accumulator fills 16 lanes of
+//                        each 32-lane quadrant);
+//      O = P V          (M = 128: the P rows of both heads, read from TMEM, N = 64 channels,
+//                        K = 64 keys; V MN-major from shared memory); row p of O in TMEM lane
+//                        p, of which the owner of that lane keeps its own head's 32 channels.
 //    tcgen05.commit signals each product on an mbarrier and frees the query / KV slots.
 //  * warps 2-5, softmax: thread t of warp w owns query row 16 (w % 4) + (t % 16) of head t / 16,
 //    i.e. TMEM lane 32 (w % 4) + t. Per region it loads its 64 scores, updates the running max
 //    and sum (exp2 with a log2(e) pre-scale), writes its 64 probabilities (rounded down to bf16,
-//    the sum taken over exactly those values) into the P tile, then adds the region's PV
-//    product into 32 fp32 registers (rescaled by the max correction). After the last region
-//    it normalises and stores its 32 output channels (64 contiguous bytes).
+//    the sum taken over exactly those values) as 32 bf16 pairs over the first 32 columns of
+//    its scores (P row = its TMEM lane), then adds the region's PV product into 32 fp32
+//    registers (rescaled by the max correction). After the last region it normalises and
+//    stores its 32 output channels (64 contiguous bytes).
 // Every wait is bounded (kErrTimeout); no thread leaves before the TMEM is released.
 #include "bra_device.cuh"
 #include "bra_launch.h"
@@ -37,7 +39,7 @@ constexpr int kRows = 64;                 // tokens per region = M of every MMA
 constexpr int kTile = kRows * 128;        // 64 rows x 64 bf16 channels, 128-byte swizzled rows
 constexpr uint32_t kTmemCols = 256;  // S buffers at 0 and 64, O buffers at 128 and 192
 constexpr uint32_t kIdescS = umma_idesc_bf16(64, 64, false);  // Q K^T: B = K tile, K-major
-constexpr uint32_t kIdescPV = umma_idesc_bf16(64, 32, true);  // P V_h: B = head h's 32 channels of V, MN-major
+constexpr uint32_t kIdescPV = umma_idesc_bf16(128, 64, true);  // P V: A = both heads' P rows, B = V, MN-major
 
 struct UmmaArgs {
     const int32_t *idx;
@@ -64,14 +66,12 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem;
     uint8_t *sKV = sQ + (size_t)a.qslots * kTile;
-    uint8_t *sP = sKV + (size_t)a.kvslots * 2 * kTile;  // [2 buffers][2 heads] P tiles
-    uint64_t *q_full = reinterpret_cast<uint64_t *>(sP + 4 * kTile);
+    uint64_t *q_full = reinterpret_cast<uint64_t *>(sKV + (size_t)a.kvslots * 2 * kTile);
     uint64_t *q_empty = q_full + a.qslots;
     uint64_t *kv_full = q_empty + a.qslots;
     uint64_t *kv_empty = kv_full + a.kvslots;
     uint64_t *s_full = kv_empty + a.kvslots;  // [2] per buffer
-    uint64_t *s_free = s_full + 2;
-    uint64_t *p_full = s_free + 2;
+    uint64_t *p_full = s_full + 2;
     uint64_t *o_full = p_full + 2;
     uint64_t *o_free = o_full + 2;
     uint64_t *drain = o_free + 2;
@@ -94,7 +94,6 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_free[i], 4);
             mbar_init(&p_full[i], 4);
             mbar_init(&o_full[i], 1);
             mbar_init(&o_free[i], 4);
@@ -162,10 +161,11 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------- MMA issuer
-        // Units u = (item, routed region j) in CTA order. S(u) goes to TMEM buffer u & 1 as soon
-        // as the softmax has loaded S(u - 2); PV(u - 1) follows once its P is written and the
-        // softmax has loaded O(u - 3). So S(u + 1) and PV(u - 1) run while the softmax works
-        // on unit u.
+        // Units u = (item, routed region j) in CTA order. S(u) goes to TMEM buffer u & 1, where
+        // the softmax overwrites its first 32 columns with P(u); PV(u - 1) follows once P(u - 1)
+        // is written and the softmax has loaded O(u - 3). S(u) is issued after PV(u - 2), which
+        // read the P that S(u) overwrites: the MMAs of this thread run in issue order. So
+        // S(u + 1) and PV(u - 1) run while the softmax works on unit u.
         if (lane == 0) {
             const int units = (end - begin) * a.topk;
             int qs = 0;
@@ -175,7 +175,6 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
             // Descriptors of the tile bases; an offset of x bytes inside a tile is + (x >> 4).
             const uint64_t dq0 = umma_desc_sw128(smem_u32(sQ));
             const uint64_t dkv0 = umma_desc_sw128(smem_u32(sKV));
-            const uint64_t dp0 = umma_desc_sw128(smem_u32(sP));
             constexpr uint64_t kTileStep = kTile >> 4;
             uint64_t dq = dq0;
             for (int u = 0; u <= units && alive; ++u) {
@@ -189,7 +188,6 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
                     }
                     if (!(alive = mbar_wait(&kv_full[kvs], (uint32_t)((u / a.kvslots) & 1), a.err))) break;
                     const int b = u & 1;
-                    if (u >= 2 && !(alive = mbar_wait(&s_free[b], (uint32_t)(((u >> 1) & 1) ^ 1), a.err))) break;
                     tcgen05_after_sync();
                     ok = kv_ok[kvs] != 0;
                     if (ok) {
@@ -219,18 +217,15 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
                     tcgen05_after_sync();
                     if (ok_prev) {
                         const uint64_t dv = dkv0 + (uint64_t)(2 * kvs_prev + 1) * kTileStep;
-                        const uint64_t dp = dp0 + (uint64_t)(2 * bv) * kTileStep;
+                        const uint32_t pa = tmem + 64 * bv;
                         const uint32_t d0 = tmem + 128 + 64 * bv;
-                        // O_h = P_h V_h: A = P tile of head h (K = 64 keys, 32 bytes per 16-key
-                        // step), B = head h's 32 channels of V (MN-major, 64 h bytes into each
-                        // row; the next 16 keys are 16 rows = 2048 bytes on)
+                        // O = P V: A = the 128 P rows of both heads in TMEM (K = 64 keys, 8
+                        // columns per 16-key step), B = all 64 channels of V (MN-major; the next
+                        // 16 keys are 16 rows = 2048 bytes on). Row p of O lands in TMEM lane p;
+                        // its thread keeps the 32 channels of its own head.
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            umma_bf16(d0, dp + 2 * kk, dv + 128 * kk, kIdescPV, (uint32_t)kk);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_bf16(d0 + (16u << 16), dp + kTileStep + 2 * kk, dv + 4 + 128 * kk, kIdescPV,
-                                      (uint32_t)kk);
+                            umma_bf16_ts(d0, pa + 8 * kk, dv + 128 * kk, kIdescPV, (uint32_t)kk);
                         umma_commit(&o_full[bv]);
                     } else {
                         mbar_arrive(&o_full[bv]);
@@ -263,31 +258,60 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
 #pragma unroll
         for (int c = 0; c < 32; ++c) o[c] = 0.f;
         __nv_bfloat16 *dst = nullptr, *dst_prev = nullptr;
-        // routing index of the next unit, loaded one unit ahead
-        int s_next = units > 0 ? a.idx[(int64_t)(begin / a.ncb) * a.topk] : 0;
+        // Routing indices run three units ahead of use, loaded with a volatile load at a fixed
+        // place in the loop: the L2 latency under full HBM load is close to a microsecond.
+        // (pb, pc, pj) = (image * R + region, channel block, routed slot) of the next load.
+        int pb = begin / a.ncb, pc = begin % a.ncb, pj = 0;
+        int sq[3] = {0, 0, 0};
+        auto next_index = [&](int uu) -> int {
+            int v = 0;
+            if (uu < units) {
+                v = ld_nc_volatile(a.idx + (int64_t)pb * a.topk + pj);
+                if (++pj == a.topk) {
+                    pj = 0;
+                    if (++pc == a.ncb) {
+                        pc = 0;
+                        ++pb;
+                    }
+                }
+            }
+            return v;
+        };
+#pragma unroll
+        for (int i = 0; i < 3; ++i) sq[i] = next_index(i);
+        // ib, ic: image and channel block of the next item; rx, ry: column and row of its region
+        const int ir = (begin / a.ncb) % a.R;
+        int ic = begin % a.ncb, ib = (begin / a.ncb) / a.R;
+        int rx = ir % a.n_win, ry = ir / a.n_win;
+        int j = 0;  // routed slot of unit u
         for (int u = 0; u <= units; ++u) {
             bool ok = false;
             bool item_start = false;
             if (u < units) {
-                const int item = begin + u / a.topk, j = u % a.topk;
-                const int s = s_next;
-                if (u + 1 < units) {
-                    const int item_n = begin + (u + 1) / a.topk, j_n = (u + 1) % a.topk;
-                    s_next = a.idx[(int64_t)(item_n / a.ncb) * a.topk + j_n];
-                }
+                const int s = sq[0];
+                sq[0] = sq[1];
+                sq[1] = sq[2];
+                sq[2] = next_index(u + 3);
                 ok = s >= 0 && s < a.R;
                 if (j == 0) {
                     item_start = true;
-                    const int cb = item % a.ncb;
-                    const int br = item / a.ncb;
-                    const int r = br % a.R, bimg = br / a.R;
-                    const int qx = (r % a.n_win) * a.wr, qy = (r / a.n_win) * a.hr;
                     dst_prev = dst;
-                    dst = a.out + (((int64_t)bimg * a.H + qy) * a.W + qx) * a.C + cb * 64 + out_row;
+                    dst = a.out + (((int64_t)ib * a.H + ry * a.hr) * a.W + rx * a.wr) * a.C + ic * 64 + out_row;
+                    if (++ic == a.ncb) {
+                        ic = 0;
+                        if (++rx == a.n_win) {
+                            rx = 0;
+                            if (++ry == a.n_win) {
+                                ry = 0;
+                                ++ib;
+                            }
+                        }
+                    }
                     l_prev = l;
                     m = -INFINITY;
                     l = 0.f;
                 }
+                if (++j == a.topk) j = 0;
                 const int b = u & 1;
                 if (alive) alive = mbar_wait(&s_full[b], (uint32_t)((u >> 1) & 1), a.err);
                 tcgen05_after_sync();
@@ -297,9 +321,6 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
                     tmem_ld_32x32(t_lane + 64 * b, v0);
                     tmem_ld_32x32(t_lane + 64 * b + 32, v1);
                     tmem_wait_ld();
-                    tcgen05_before_sync();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&s_free[b]);
                     // row max with four independent chains
                     float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -311,30 +332,24 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
                     const float mn = fmaxf(m, mx * a.scale_log2);
                     corr = fast_exp2(m - mn);
                     m = mn;
-                    uint8_t *prow = sP + (2 * b + h) * kTile + row * 128;
+                    // P row 32 q + lane (this thread's TMEM lane) over the first 32 columns of
+                    // S: column j holds the bf16 pair of keys 2 j, 2 j + 1
                     float ls[4] = {0.f, 0.f, 0.f, 0.f};
+                    uint32_t pw[32];
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int c = ch * 8 + 2 * e;
-                            const float x0 = __uint_as_float(c < 32 ? v0[c] : v1[c - 32]);
-                            const float x1 = __uint_as_float(c + 1 < 32 ? v0[c + 1] : v1[c + 1 - 32]);
-                            const float p0 = bf16_trunc(fast_exp2(fmaf(x0, a.scale_log2, -mn)));
-                            const float p1 = bf16_trunc(fast_exp2(fmaf(x1, a.scale_log2, -mn)));
-                            ls[e] += p0 + p1;
-                            w[e] = pack_bf16x2_trunc(p0, p1);
-                        }
-                        *reinterpret_cast<uint4 *>(prow + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                    for (int j = 0; j < 32; ++j) {
+                        const int c = 2 * j;
+                        const float x0 = __uint_as_float(c < 32 ? v0[c] : v1[c - 32]);
+                        const float x1 = __uint_as_float(c + 1 < 32 ? v0[c + 1] : v1[c + 1 - 32]);
+                        const float p0 = bf16_trunc(fast_exp2(fmaf(x0, a.scale_log2, -mn)));
+                        const float p1 = bf16_trunc(fast_exp2(fmaf(x1, a.scale_log2, -mn)));
+                        ls[j & 3] += p0 + p1;
+                        pw[j] = pack_bf16x2_trunc(p0, p1);
                     }
+                    tmem_st_32x32(t_lane + 64 * b, pw);
+                    tmem_wait_st();
                     l = l * corr + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
-                } else {
-                    tcgen05_before_sync();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&s_free[b]);
                 }
-                fence_async_shared();
                 tcgen05_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_full[b]);
@@ -344,12 +359,14 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
                 if (alive) alive = mbar_wait(&o_full[bv], (uint32_t)((v >> 1) & 1), a.err);
                 tcgen05_after_sync();
                 if (alive && ok_prev) {
-                    // this thread's 32 output channels (both heads' products sit in the same columns)
-                    uint32_t w0[32];
+                    // this thread's 32 output channels: columns 32 h of its O row (the column
+                    // address of a TMEM load is the same for the whole warp, so both halves)
+                    uint32_t w0[32], w1[32];
                     tmem_ld_32x32(t_lane + 128 + 64 * bv, w0);
+                    tmem_ld_32x32(t_lane + 128 + 64 * bv + 32, w1);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] += __uint_as_float(w0[c]);
+                    for (int c = 0; c < 32; ++c) o[c] += __uint_as_float(h ? w1[c] : w0[c]);
                 }
                 tcgen05_before_sync();
                 __syncwarp();
@@ -414,9 +431,9 @@ cudaError_t launch_attend_gather_umma(const CUtensorMap &tq, const CUtensorMap &
     if (nitems > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     a.nitems = (int)nitems;
     a.qslots = 3;
-    a.kvslots = 3;
+    a.kvslots = 5;
     a.idx_chunk = g.topk >= 32 ? 1 : 32 / g.topk;
-    const size_t smem = 1024 + (size_t)kTile * (a.qslots + 2 * a.kvslots + 4) + 8 * (2 * a.qslots + 2 * a.kvslots + 11) +
+    const size_t smem = 1024 + (size_t)kTile * (a.qslots + 2 * a.kvslots) + 8 * (2 * a.qslots + 2 * a.kvslots + 9) +
                         4 * a.kvslots + 4 + 4 * (size_t)a.idx_chunk * g.topk;
     int grid = 2 * num_sms;
     if (grid > a.nitems) grid = a.nitems;

@@ -34,6 +34,7 @@ constexpr int kMaxMeansVectors = 2048;
 cudaError_t launch_region_means(const void *q, const void *k, float *qm, float *km, const Geometry &g,
                                 bool bf16, int num_sms, cudaStream_t stream);
 
+
 // Affinity rows and top-k: idx[b, r, :] from qm, km.
 cudaError_t launch_route_topk(const float *qm, const float *km, int32_t *idx, const Geometry &g,
                               cudaStream_t stream);

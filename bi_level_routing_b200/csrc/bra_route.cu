@@ -4,13 +4,13 @@
 // tokens (step 1), the affinity A = C^-1/2 qm km^T between regions (step 2) and, per row,
 // the indices of the topk largest affinities (step 3).
 //
-// Kernel 1 streams q and k once from HBM and writes fp32 means [B, R, C] to scratch: one small
-// CTA per (image, region), each thread with all its 16-byte row loads in flight at once.
-// Kernel 2 computes affinity rows,
-// one warp per row, and selects the top-k in registers: rounds of warp argmax for a small k,
-// a shuffle bitonic network otherwise. Keys are 64-bit (order-preserving float bits, then the
-// complement of the region index), which gives affinity-descending order, ties to the lower
-// region and NaN after every number, deterministically.
+// The means kernel streams q and k once from HBM and writes fp32 means [B, R, C] to scratch:
+// a group of threads per (image, region), each thread with its 16-byte row loads in flight at
+// once. The routing kernel computes affinity rows, several rows per warp pass, and selects the
+// top-k in registers: rounds of warp argmax for a small k, a shuffle bitonic network otherwise. Keys are 64-bit
+// (order-preserving float bits, then the complement of the region index), which gives
+// affinity-descending order, ties to the lower region and NaN after every number,
+// deterministically.
 #include "bra_device.cuh"
 #include "bra_launch.h"
 
@@ -18,67 +18,79 @@ namespace bra {
 
 // ============================================================================ region means
 
-// One CTA per (image, region), for q and k together. Thread t owns the 16-byte vectors
-// v = t, t + blockDim, ... of one region row (token column v / (C / V), V channels), and for
-// each it issues the loads of all hr rows of q and of k at once (up to 2 x 8 in flight), then
-// sums them in row order. The CTA then sums each channel over the wr columns in order and
-// divides by rs. The arithmetic is the same for every region, so regions with equal content
-// get bit-identical means.
+// Arguments of the means kernel.
+struct MeansArgs {
+    const void *q, *k;
+    float *qm, *km;
+    int B, H, W, C, n_win, hr, wr, R;
+    int slots;  // threads per region: the row segment's vectors rounded up to a warp, <= 256
+    int rpc;    // regions per CTA (256 / slots)
+};
+
+constexpr int kMeansThreads = 256;
+constexpr int kMeansMaxRegions = kMeansThreads / 32;
+
+// The means of the regions i0 .. i0 + nreg - 1 (flat index b * R + r), q and k together. A
+// region row segment is nvec = wr C / V 16-byte vectors; thread t of group g = t / slots owns
+// the vectors v = t % slots, t % slots + slots, ... of region i0 + g and, eight region rows at
+// a time, issues the loads of those rows of q and of k at once (16 in flight), then sums them
+// in row order. The CTA then sums each channel over the wr columns in order and divides by
+// rs: the arithmetic is the same for every region, so regions with equal content get
+// bit-identical means.
 template <typename T>
-__global__ void __launch_bounds__(256) region_means_kernel(const T *__restrict__ q, const T *__restrict__ k,
-                                                           float *__restrict__ qm, float *__restrict__ km, int H,
-                                                           int W, int C, int n_win)
+__device__ __forceinline__ void region_means_block(const MeansArgs &a, float *part, long long i0, int nreg)
 {
     constexpr int V = Vec16<T>::N;
     constexpr int ROWS = 8;
-    extern __shared__ float4 part4[];  // [2][wr][C] floats
-    float *part = reinterpret_cast<float *>(part4);
-    const int hr = H / n_win, wr = W / n_win, R = n_win * n_win;
-    const int r = blockIdx.x % R;
-    const int64_t b = blockIdx.x / R;
-    const int ry = r / n_win, rx = r % n_win;
+    const int C = a.C;
     const int vpt = C / V;
-    const int nvec = wr * vpt;
-    const int64_t row_stride = (int64_t)W * C;
-    const int64_t base = ((b * H + (int64_t)ry * hr) * W + (int64_t)rx * wr) * C;
-
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-        float aq[V], ak[V];
+    const int nvec = a.wr * vpt;
+    const int grp = threadIdx.x / a.slots;
+    if (grp < nreg) {
+        const long long flat = i0 + grp;
+        const int64_t b = flat / a.R;
+        const int r = (int)(flat % a.R);
+        const int ry = r / a.n_win, rx = r % a.n_win;
+        const int64_t row_stride = (int64_t)a.W * C;
+        const int64_t base = ((b * a.H + (int64_t)ry * a.hr) * a.W + (int64_t)rx * a.wr) * C;
+        for (int v = threadIdx.x % a.slots; v < nvec; v += a.slots) {
+            float aq[V], ak[V];
 #pragma unroll
-        for (int i = 0; i < V; ++i) aq[i] = ak[i] = 0.f;
-        const T *pq = q + base + (int64_t)v * V;
-        const T *pk = k + base + (int64_t)v * V;
-        for (int y0 = 0; y0 < hr; y0 += ROWS) {
-            const int n = min(ROWS, hr - y0);
-            uint4 rq[ROWS], rk[ROWS];
+            for (int i = 0; i < V; ++i) aq[i] = ak[i] = 0.f;
+            const T *pq = static_cast<const T *>(a.q) + base + (int64_t)v * V;
+            const T *pk = static_cast<const T *>(a.k) + base + (int64_t)v * V;
+            for (int y0 = 0; y0 < a.hr; y0 += ROWS) {
+                const int n = min(ROWS, a.hr - y0);
+                uint4 rq[ROWS], rk[ROWS];
 #pragma unroll
-            for (int u = 0; u < ROWS; ++u)
-                if (u < n) {
-                    rq[u] = Vec16<T>::load_raw(pq + (int64_t)(y0 + u) * row_stride);
-                    rk[u] = Vec16<T>::load_raw(pk + (int64_t)(y0 + u) * row_stride);
-                }
+                for (int u = 0; u < ROWS; ++u)
+                    if (u < n) {
+                        rq[u] = Vec16<T>::load_raw(pq + (int64_t)(y0 + u) * row_stride);
+                        rk[u] = Vec16<T>::load_raw(pk + (int64_t)(y0 + u) * row_stride);
+                    }
 #pragma unroll
-            for (int u = 0; u < ROWS; ++u)
-                if (u < n) {
-                    Vec16<T>::accumulate(rq[u], aq);
-                    Vec16<T>::accumulate(rk[u], ak);
-                }
-        }
-        float4 *dq = reinterpret_cast<float4 *>(part + (size_t)(v / vpt) * C + (v % vpt) * V);
-        float4 *dk = reinterpret_cast<float4 *>(part + (size_t)(wr + v / vpt) * C + (v % vpt) * V);
+                for (int u = 0; u < ROWS; ++u)
+                    if (u < n) {
+                        Vec16<T>::accumulate(rq[u], aq);
+                        Vec16<T>::accumulate(rk[u], ak);
+                    }
+            }
+            float4 *dq = reinterpret_cast<float4 *>(part + ((size_t)(2 * grp) * a.wr + v / vpt) * C + (v % vpt) * V);
+            float4 *dk = reinterpret_cast<float4 *>(part + ((size_t)(2 * grp + 1) * a.wr + v / vpt) * C + (v % vpt) * V);
 #pragma unroll
-        for (int j = 0; j < V / 4; ++j) {
-            dq[j] = make_float4(aq[4 * j], aq[4 * j + 1], aq[4 * j + 2], aq[4 * j + 3]);
-            dk[j] = make_float4(ak[4 * j], ak[4 * j + 1], ak[4 * j + 2], ak[4 * j + 3]);
+            for (int j = 0; j < V / 4; ++j) {
+                dq[j] = make_float4(aq[4 * j], aq[4 * j + 1], aq[4 * j + 2], aq[4 * j + 3]);
+                dk[j] = make_float4(ak[4 * j], ak[4 * j + 1], ak[4 * j + 2], ak[4 * j + 3]);
+            }
         }
     }
     __syncthreads();
-    const float rs = (float)(hr * wr);
-    for (int e = threadIdx.x; e < 2 * C; e += blockDim.x) {
-        const int t = e / C, c = e % C;
+    const float rs = (float)(a.hr * a.wr);
+    for (int e = threadIdx.x; e < nreg * 2 * C; e += blockDim.x) {
+        const int g = e / (2 * C), t = (e / C) & 1, c = e % C;
         float s = 0.f;
-        for (int xx = 0; xx < wr; ++xx) s += part[(size_t)(t * wr + xx) * C + c];
-        (t ? km : qm)[(b * R + r) * C + c] = s / rs;
+        for (int xx = 0; xx < a.wr; ++xx) s += part[((size_t)(2 * g + t) * a.wr + xx) * C + c];
+        (t ? a.km : a.qm)[(i0 + g) * C + c] = s / rs;
     }
 }
 
@@ -127,10 +139,160 @@ __device__ __forceinline__ unsigned long long warp_max_key(unsigned long long x)
     return x;
 }
 
-// One CTA per (image, block of `rows` rows), one warp per row at a time. Lane l holds the keys
-// of regions s = e * 32 + l, e < E (P = 32 E >= R). The image's key means (and the block's
-// query means) are staged in shared memory when STAGED, rows padded to C + 4 floats so that
-// lanes reading different rows hit different banks; otherwise they are read through L1.
+// Selects the topk largest of a warp's keys (lane l holds the keys of positions e * 32 + l,
+// e < E) and writes their regions to out[0 .. topk): rounds of warp argmax (ROUNDS) or a
+// shuffle bitonic network over position p = e * 32 + lane.
+template <int E, bool ROUNDS>
+__device__ __forceinline__ void select_topk(unsigned long long (&key)[E], int topk, int32_t *out, int lane)
+{
+    if (ROUNDS) {
+        // topk rounds of warp argmax; the winner's key is unique (it holds the region)
+        for (int j = 0; j < topk; ++j) {
+            unsigned long long best = key[0];
+#pragma unroll
+            for (int e = 1; e < E; ++e) best = key[e] > best ? key[e] : best;
+            best = warp_max_key(best);
+            if (lane == 0) out[j] = key_region(best);
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                if (key[e] == best) key[e] = 0ull;
+        }
+    } else {
+#pragma unroll
+        for (int size = 2; size <= 32 * E; size <<= 1) {
+#pragma unroll
+            for (int st = size >> 1; st > 0; st >>= 1) {
+                if (st >= 32) {
+#pragma unroll
+                    for (int e = 0; e < E; ++e) {
+                        const int e2 = e ^ (st >> 5);
+                        if (e2 > e) {
+                            const bool desc = (((e * 32 + lane) & size) == 0);
+                            const unsigned long long x = key[e], y = key[e2];
+                            if (desc ? (x < y) : (x > y)) {
+                                key[e] = y;
+                                key[e2] = x;
+                            }
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < E; ++e) {
+                        const unsigned long long other = __shfl_xor_sync(0xffffffffu, key[e], st);
+                        const bool desc = (((e * 32 + lane) & size) == 0);
+                        const bool lower = (lane & st) == 0;
+                        const bool keep_max = (lower == desc);
+                        key[e] = keep_max ? (other > key[e] ? other : key[e]) : (other < key[e] ? other : key[e]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int p = e * 32 + lane;
+            if (p < topk) out[p] = key_region(key[e]);
+        }
+    }
+}
+
+// Rows per warp pass of route_rows: NR rows x E keys x 4 partial sums stay in registers.
+template <int E>
+struct RowsPerPass {
+    static constexpr int value = E <= 2 ? 2 : 1;
+};
+
+// Routing rows i < nr (nr <= NR) of one image, by one warp: query mean row i at
+// qrows + i * qstride, key mean row s at kbase + s * kstride. Lane l computes the affinities of
+// regions s = e * 32 + l, e < E (R <= 32 E), for all NR rows at once: every pair (row, s) is
+// the dot product of dot_rows, four interleaved partial sums over the channels in order,
+// combined as (s0 + s1) + (s2 + s3), times C^-1/2; the NR x E products only run side by side,
+// so that each 16-byte key load serves NR rows and the loads of consecutive channel steps
+// overlap. Every routing kernel goes through this function, so the index is the same bits
+// whichever kernel computed it.
+template <int E, int NR, bool ROUNDS>
+__device__ __forceinline__ void route_rows(const float *qrows, int qstride, int nr, const float *kbase, int kstride,
+                                           int R, int C, int topk, float scale, int32_t *out, int lane)
+{
+    float acc[NR][E][4];
+#pragma unroll
+    for (int i = 0; i < NR; ++i)
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][e][j] = 0.f;
+    int krow[E], qrow[NR];  // element offsets of the rows
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int s = e * 32 + lane;
+        krow[e] = (s < R ? s : 0) * kstride;  // lanes past R compute a discarded key
+    }
+#pragma unroll
+    for (int i = 0; i < NR; ++i) qrow[i] = (i < nr ? i : 0) * qstride;
+#pragma unroll 4
+    for (int c = 0; c < C; c += 4) {
+        float4 y[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) y[e] = *reinterpret_cast<const float4 *>(kbase + krow[e] + c);
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+            const float4 x = *reinterpret_cast<const float4 *>(qrows + qrow[i] + c);
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                acc[i][e][0] = fmaf(x.x, y[e].x, acc[i][e][0]);
+                acc[i][e][1] = fmaf(x.y, y[e].y, acc[i][e][1]);
+                acc[i][e][2] = fmaf(x.z, y[e].z, acc[i][e][2]);
+                acc[i][e][3] = fmaf(x.w, y[e].w, acc[i][e][3]);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NR; ++i) {
+        if (i >= nr) break;
+        unsigned long long key[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int s = e * 32 + lane;
+            const float d = (acc[i][e][0] + acc[i][e][1]) + (acc[i][e][2] + acc[i][e][3]);
+            key[e] = s < R ? routing_key(d * scale, s) : 0ull;
+        }
+        select_topk<E, ROUNDS>(key, topk, out + (size_t)i * topk, lane);
+    }
+}
+
+// Copies rows0 fp32 rows of length C (a multiple of 4) from src0 and then rows1 rows from src1
+// (row stride C) to consecutive rows of dst (row stride dst_stride), all threads of the CTA,
+// eight 16-byte loads in flight per thread. With L2 set, the loads bypass L1 (ld.global.cg):
+// the rows were written by other CTAs of this grid.
+template <bool L2>
+__device__ __forceinline__ void stage_rows(const float *__restrict__ src0, int rows0, const float *__restrict__ src1,
+                                           int rows1, float *dst, int C, int dst_stride)
+{
+    const int c4 = C / 4;
+    const int n0 = rows0 * c4;
+    const int total = (rows0 + rows1) * c4;
+    for (int e0 = threadIdx.x; e0 < total; e0 += 8 * blockDim.x) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = e0 + u * blockDim.x;
+            if (e < total) {
+                const float *src = e < n0 ? src0 + (size_t)(e / c4) * C : src1 + (size_t)((e - n0) / c4) * C;
+                const float4 *p = reinterpret_cast<const float4 *>(src + (e % c4) * 4);
+                v[u] = L2 ? __ldcg(p) : __ldg(p);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = e0 + u * blockDim.x;
+            if (e < total) *reinterpret_cast<float4 *>(dst + (size_t)(e / c4) * dst_stride + (e % c4) * 4) = v[u];
+        }
+    }
+}
+
+// One CTA per (image, block of `rows` rows), one warp per row at a time. The image's key means
+// (and the block's query means) are staged in shared memory when STAGED, rows padded to C + 4
+// floats so that lanes reading different rows hit different banks; otherwise they are read
+// through L1.
 template <int E, bool STAGED, bool ROUNDS>
 __global__ void __launch_bounds__(256, 2) route_topk_kernel(const float *__restrict__ qm, const float *__restrict__ km,
                                                          int32_t *__restrict__ idx, int R, int C, int topk, int rows,
@@ -143,99 +305,20 @@ __global__ void __launch_bounds__(256, 2) route_topk_kernel(const float *__restr
     const int r0 = (blockIdx.x % row_blocks) * rows;
     const int nrows = min(rows, R - r0);
     const int stride = STAGED ? C + 4 : C;
-    const float *gkm = km + (int64_t)b * R * C;
-    const float *gqm = qm + ((int64_t)b * R + r0) * C;
-    const float *kbase = gkm, *qbase = gqm;
+    const float *kbase = km + (int64_t)b * R * C;
+    const float *qbase = qm + ((int64_t)b * R + r0) * C;
     if (STAGED) {
-        // copy the key means and this block's query means into padded rows, four 16-byte
-        // loads in flight per thread
         float *skm = reinterpret_cast<float *>(smem4);
         float *sqm = skm + (size_t)R * stride;
-        const int c4 = C / 4;
-        const int total = (R + nrows) * c4;
-        for (int e0 = threadIdx.x; e0 < total; e0 += 4 * blockDim.x) {
-            float4 v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = e0 + u * blockDim.x;
-                if (e < total) {
-                    const int s = e / c4, c = (e % c4) * 4;
-                    v[u] = __ldg(reinterpret_cast<const float4 *>(s < R ? gkm + s * C + c : gqm + (s - R) * C + c));
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = e0 + u * blockDim.x;
-                if (e < total) {
-                    const int s = e / c4, c = (e % c4) * 4;
-                    *reinterpret_cast<float4 *>((s < R ? skm + s * stride : sqm + (s - R) * stride) + c) = v[u];
-                }
-            }
-        }
+        stage_rows<false>(kbase, R, qbase, nrows, skm, C, stride);
         __syncthreads();
         kbase = skm;
         qbase = sqm;
     }
-    for (int i = warp; i < nrows; i += nwarps) {
-        const int r = r0 + i;
-        const float *qrow = qbase + (size_t)i * stride;
-        unsigned long long key[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const int s = e * 32 + lane;
-            key[e] = s < R ? routing_key(dot_rows(qrow, kbase + (size_t)s * stride, C) * scale, s) : 0ull;
-        }
-        int32_t *out = idx + ((int64_t)b * R + r) * topk;
-        if (ROUNDS) {
-            // topk rounds of warp argmax; the winner's key is unique (it holds the region)
-            for (int j = 0; j < topk; ++j) {
-                unsigned long long best = key[0];
-#pragma unroll
-                for (int e = 1; e < E; ++e) best = key[e] > best ? key[e] : best;
-                best = warp_max_key(best);
-                if (lane == 0) out[j] = key_region(best);
-#pragma unroll
-                for (int e = 0; e < E; ++e)
-                    if (key[e] == best) key[e] = 0ull;
-            }
-        } else {
-            // bitonic network, descending, over position p = e * 32 + lane
-#pragma unroll
-            for (int size = 2; size <= 32 * E; size <<= 1) {
-#pragma unroll
-                for (int st = size >> 1; st > 0; st >>= 1) {
-                    if (st >= 32) {
-#pragma unroll
-                        for (int e = 0; e < E; ++e) {
-                            const int e2 = e ^ (st >> 5);
-                            if (e2 > e) {
-                                const bool desc = (((e * 32 + lane) & size) == 0);
-                                const unsigned long long x = key[e], y = key[e2];
-                                if (desc ? (x < y) : (x > y)) {
-                                    key[e] = y;
-                                    key[e2] = x;
-                                }
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < E; ++e) {
-                            const unsigned long long other = __shfl_xor_sync(0xffffffffu, key[e], st);
-                            const bool desc = (((e * 32 + lane) & size) == 0);
-                            const bool lower = (lane & st) == 0;
-                            const bool keep_max = (lower == desc);
-                            key[e] = keep_max ? (other > key[e] ? other : key[e]) : (other < key[e] ? other : key[e]);
-                        }
-                    }
-                }
-            }
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const int p = e * 32 + lane;
-                if (p < topk) out[p] = key_region(key[e]);
-            }
-        }
-    }
+    constexpr int NR = RowsPerPass<E>::value;
+    for (int i = warp * NR; i < nrows; i += nwarps * NR)
+        route_rows<E, NR, ROUNDS>(qbase + (size_t)i * stride, stride, min(NR, nrows - i), kbase, stride, R, C, topk,
+                                  scale, idx + ((int64_t)b * R + r0 + i) * topk, lane);
 }
 
 // Wide rows (R > 256): one warp per row, keys in shared memory, bitonic network there.
@@ -274,6 +357,18 @@ __global__ void __launch_bounds__(256) route_topk_wide_kernel(const float *__res
     for (int j = lane; j < topk; j += 32) out[j] = key_region(kw[j]);
 }
 
+// ============================================================================ means kernels
+
+// Means only.
+template <typename T>
+__global__ void __launch_bounds__(kMeansThreads, 2) region_means_kernel(const MeansArgs a)
+{
+    extern __shared__ float4 smem4[];
+    const long long i0 = (long long)blockIdx.x * a.rpc;
+    const int nreg = (int)min((long long)a.rpc, (long long)a.B * a.R - i0);
+    region_means_block<T>(a, reinterpret_cast<float *>(smem4), i0, nreg);
+}
+
 // ============================================================================ launchers
 
 template <typename Kernel>
@@ -289,28 +384,61 @@ static cudaError_t raise_smem_limit(Kernel kernel, size_t bytes, int (&granted)[
     return e;
 }
 
+// Regions per CTA of the means kernels: one group of `slots` threads (the region row segment's
+// vectors, rounded up to a warp) per region, as many as fit in 256 threads.
+static MeansArgs means_args(const void *q, const void *k, float *qm, float *km, const Geometry &g, bool bf16)
+{
+    MeansArgs a;
+    a.q = q;
+    a.k = k;
+    a.qm = qm;
+    a.km = km;
+    a.B = g.B;
+    a.H = g.H;
+    a.W = g.W;
+    a.C = g.C;
+    a.n_win = g.n_win;
+    a.hr = g.hr;
+    a.wr = g.wr;
+    a.R = g.R;
+    const int V = bf16 ? 8 : 4;
+    const int nvec = g.wr * (g.C / V);
+    a.slots = nvec >= kMeansThreads ? kMeansThreads : (nvec + 31) / 32 * 32;
+    a.rpc = kMeansThreads / a.slots;
+    return a;
+}
+
+static size_t means_part_bytes(const MeansArgs &a) { return (size_t)a.rpc * 2 * a.wr * a.C * sizeof(float); }
+
+static long long means_blocks(const MeansArgs &a) { return ((long long)a.B * a.R + a.rpc - 1) / a.rpc; }
+
+// topk rounds of argmax cost about topk * (E + 20) instructions; the bitonic network
+// log2(P) (log2(P) + 1) / 2 stages of about 8 E.
+static bool topk_by_rounds(int E, int topk)
+{
+    int lg = 5;
+    while ((1 << lg) < 32 * E) ++lg;
+    const long long stages = (long long)lg * (lg + 1) / 2;
+    return (long long)topk * (E + 20) <= stages * E * 8;
+}
+
 cudaError_t launch_region_means(const void *q, const void *k, float *qm, float *km, const Geometry &g, bool bf16,
                                 int num_sms, cudaStream_t stream)
 {
     (void)num_sms;
-    const int V = bf16 ? 8 : 4;
-    const long long nvec = (long long)g.wr * (g.C / V);
-    if (nvec > kMaxMeansVectors) return cudaErrorInvalidConfiguration;  // validated earlier
-    int threads = (int)(((nvec + 31) / 32) * 32);
-    if (threads > 256) threads = 256;
-    const size_t smem = (size_t)2 * g.wr * g.C * sizeof(float);
+    const MeansArgs a = means_args(q, k, qm, km, g, bf16);
+    if ((long long)a.wr * (g.C / (bf16 ? 8 : 4)) > kMaxMeansVectors) return cudaErrorInvalidConfiguration;
+    const size_t smem = means_part_bytes(a);
     static int granted[2][64] = {{0}};
     cudaError_t e = bf16 ? raise_smem_limit(region_means_kernel<__nv_bfloat16>, smem, granted[0])
                          : raise_smem_limit(region_means_kernel<float>, smem, granted[1]);
     if (e != cudaSuccess) return e;
-    const long long blocks = (long long)g.B * g.R;
+    const long long blocks = means_blocks(a);
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     if (bf16)
-        region_means_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, smem, stream>>>(
-            (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, qm, km, g.H, g.W, g.C, g.n_win);
+        region_means_kernel<__nv_bfloat16><<<(unsigned)blocks, kMeansThreads, smem, stream>>>(a);
     else
-        region_means_kernel<float><<<(unsigned)blocks, threads, smem, stream>>>((const float *)q, (const float *)k, qm,
-                                                                               km, g.H, g.W, g.C, g.n_win);
+        region_means_kernel<float><<<(unsigned)blocks, kMeansThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -331,12 +459,7 @@ template <int E>
 static cudaError_t launch_topk_e(const float *qm, const float *km, int32_t *idx, const Geometry &g, cudaStream_t stream)
 {
     const float scale = (float)(1.0 / sqrt((double)g.C));
-    // topk rounds of argmax cost about topk * (E + 20) instructions; the bitonic network
-    // log2(P) (log2(P) + 1) / 2 stages of about 8 E.
-    int lg = 5;
-    while ((1 << lg) < 32 * E) ++lg;
-    const long long stages = (long long)lg * (lg + 1) / 2;
-    const int rounds = (long long)g.topk * (E + 20) <= stages * E * 8 ? 1 : 0;
+    const bool rounds = topk_by_rounds(E, g.topk);
     const int rows = g.R <= 64 ? (g.C >= 256 ? 16 : 8) : 16;
     const size_t stage_bytes = (size_t)(g.R + rows) * (g.C + 4) * sizeof(float);
     if (stage_bytes <= 100 * 1024)

@@ -135,12 +135,14 @@ int bra_selected_attend_kernel(int B, int H, int W, int C, int heads, int n_win,
    BRA_OK, BRA_ERR_INDEX (an idx entry outside [0, R) was skipped) or BRA_ERR_TIMEOUT. */
 bra_status bra_check_device_error(void *stream);
 
-/* Bytes of scratch bra_route / bra_forward take from the pool for these sizes. */
+/* Bytes of scratch bra_route / bra_forward take from the pool for these sizes (fp32 means). */
 size_t bra_route_scratch_bytes(int B, int H, int W, int C, int n_win);
 
-/* Number of kernels one bra_route, bra_attend or bra_forward call launches (for launch
-   accounting); 0 for a call that would launch nothing. */
-int bra_kernels_per_call(const char *entry_point, int B);
+/* Number of library kernels one call of `entry_point` ("bra_route", "bra_attend",
+   "bra_forward", "bra_forward_host") launches with these arguments, for launch accounting
+   (memset and copy nodes not counted); 0 for a call that would launch nothing or be rejected. */
+int bra_kernels_per_call(const char *entry_point, int B, int H, int W, int C, int heads, int n_win, int topk,
+                         bra_dtype dtype);
 
 /* Static strings: the name of a status, and the last CUDA error message of this thread. */
 const char *bra_status_string(bra_status status);

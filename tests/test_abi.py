@@ -76,7 +76,7 @@ def test_empty_batch_is_a_no_op(L):
     assert _route(L, B=0, q=0, k=0, idx=0) == OK
     assert _attend(L, B=0, q=0, k=0, v=0, idx=0, out=0) == OK
     assert _forward(L, B=0, q=0, k=0, v=0, idx=0, out=0) == OK
-    assert L.bra_kernels_per_call(b"bra_forward", 0) == 0
+    assert L.bra_kernels_per_call(b"bra_forward", 0, 28, 28, 64, 2, 7, 4, 1) == 0
 
 
 def test_unsupported_sizes(L):
@@ -114,7 +114,12 @@ def test_forcing_a_kernel(L):
 
 def test_scratch_and_launch_accounting(L):
     assert L.bra_route_scratch_bytes(64, 56, 56, 64, 7) == 2 * 64 * 49 * 64 * 4
-    assert L.bra_kernels_per_call(b"bra_route", 2) == 2
-    assert L.bra_kernels_per_call(b"bra_attend", 2) == 1
-    assert L.bra_kernels_per_call(b"bra_forward", 2) == 3
-    assert L.bra_kernels_per_call(b"nonsense", 2) == 0
+    stage1 = (64, 56, 56, 64, 2, 7, 1, 1)
+    highres = (8, 128, 128, 64, 2, 16, 4, 1)
+    assert L.bra_kernels_per_call(b"bra_route", *stage1) == 2  # means, then affinity + top-k
+    assert L.bra_kernels_per_call(b"bra_route", *highres) == 2
+    assert L.bra_kernels_per_call(b"bra_attend", *stage1) == 1
+    assert L.bra_kernels_per_call(b"bra_forward", *stage1) == 3
+    assert L.bra_kernels_per_call(b"bra_forward", *highres) == 3
+    assert L.bra_kernels_per_call(b"bra_forward", 1, 30, 28, 64, 2, 7, 4, 1) == 0  # rejected
+    assert L.bra_kernels_per_call(b"nonsense", *stage1) == 0
