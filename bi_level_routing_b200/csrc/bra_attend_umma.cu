@@ -22,11 +22,10 @@
 //    tcgen05.commit signals each product on an mbarrier and frees the query / KV slots.
 //  * warps 2-5, softmax: thread t of warp w owns query row 16 (w % 4) + (t % 16) of head t / 16,
 //    i.e. TMEM lane 32 (w % 4) + t. Per region it loads its 64 scores, updates the running max
-//    and sum (exp2 with a log2(e) pre-scale), writes its 64 probabilities (rounded down to bf16,
-//    the sum taken over exactly those values) as 32 bf16 pairs over the first 32 columns of
-//    its scores (P row = its TMEM lane), then adds the region's PV product into 32 fp32
-//    registers (rescaled by the max correction). After the last region it normalises and
-//    stores its 32 output channels (64 contiguous bytes).
+//    and sum (exp2 with a log2(e) pre-scale; packed fp32 pairs), writes its 64 probabilities
+//    rounded to bf16 as 32 pairs over the first 32 columns of its scores (P row = its TMEM
+//    lane), then folds the region's PV product into 32 fp32 registers (o = o * correction +
+//    PV). After the last region it normalises and stores its 32 output channels (64 bytes).
 // Every wait is bounded (kErrTimeout); no thread leaves before the TMEM is released.
 #include "bra_device.cuh"
 #include "bra_launch.h"
@@ -284,9 +283,11 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
         int ic = begin % a.ncb, ib = (begin / a.ncb) / a.R;
         int rx = ir % a.n_win, ry = ir / a.n_win;
         int j = 0;  // routed slot of unit u
+        bool start_prev = false;  // unit u - 1 opened its item
         for (int u = 0; u <= units; ++u) {
             bool ok = false;
             bool item_start = false;
+            const float corr_prev = corr;  // max correction of unit u - 1
             if (u < units) {
                 const int s = sq[0];
                 sq[0] = sq[1];
@@ -321,34 +322,38 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
                     tmem_ld_32x32(t_lane + 64 * b, v0);
                     tmem_ld_32x32(t_lane + 64 * b + 32, v1);
                     tmem_wait_ld();
-                    // row max with four independent chains
+                    // row max: four chains of three-input max
                     float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
                     for (int c = 0; c < 32; c += 2) {
-                        mx4[(c >> 1) & 3] = fmaxf(mx4[(c >> 1) & 3], fmaxf(__uint_as_float(v0[c]), __uint_as_float(v0[c + 1])));
-                        mx4[(c >> 1) & 3] = fmaxf(mx4[(c >> 1) & 3], fmaxf(__uint_as_float(v1[c]), __uint_as_float(v1[c + 1])));
+                        mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(v0[c]), __uint_as_float(v0[c + 1]));
+                        mx4[((c >> 1) + 2) & 3] =
+                            fmax3(mx4[((c >> 1) + 2) & 3], __uint_as_float(v1[c]), __uint_as_float(v1[c + 1]));
                     }
                     const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
                     const float mn = fmaxf(m, mx * a.scale_log2);
                     corr = fast_exp2(m - mn);
                     m = mn;
                     // P row 32 q + lane (this thread's TMEM lane) over the first 32 columns of
-                    // S: column j holds the bf16 pair of keys 2 j, 2 j + 1
-                    float ls[4] = {0.f, 0.f, 0.f, 0.f};
+                    // S: column j holds keys 2 j, 2 j + 1 rounded to bf16; the row sum is taken
+                    // over the fp32 probabilities. Scale-and-shift, sums: packed fp32 pairs.
+                    const float2 sc = make_float2(a.scale_log2, a.scale_log2), nm = make_float2(-mn, -mn);
+                    float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                    make_float2(0.f, 0.f)};
                     uint32_t pw[32];
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const int c = 2 * j;
-                        const float x0 = __uint_as_float(c < 32 ? v0[c] : v1[c - 32]);
-                        const float x1 = __uint_as_float(c + 1 < 32 ? v0[c + 1] : v1[c + 1 - 32]);
-                        const float p0 = bf16_trunc(fast_exp2(fmaf(x0, a.scale_log2, -mn)));
-                        const float p1 = bf16_trunc(fast_exp2(fmaf(x1, a.scale_log2, -mn)));
-                        ls[j & 3] += p0 + p1;
-                        pw[j] = pack_bf16x2_trunc(p0, p1);
+                        const float x0 = __uint_as_float(j < 16 ? v0[2 * j] : v1[2 * j - 32]);
+                        const float x1 = __uint_as_float(j < 16 ? v0[2 * j + 1] : v1[2 * j + 1 - 32]);
+                        const float2 t = __ffma2_rn(make_float2(x0, x1), sc, nm);
+                        const float2 pr = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+                        ls[j & 3] = __fadd2_rn(ls[j & 3], pr);
+                        pw[j] = pack_bf16x2(pr.x, pr.y);
                     }
                     tmem_st_32x32(t_lane + 64 * b, pw);
                     tmem_wait_st();
-                    l = l * corr + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+                    const float2 lsum = __fadd2_rn(__fadd2_rn(ls[0], ls[1]), __fadd2_rn(ls[2], ls[3]));
+                    l = l * corr + (lsum.x + lsum.y);
                 }
                 tcgen05_before_sync();
                 __syncwarp();
@@ -360,13 +365,33 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
                 tcgen05_after_sync();
                 if (alive && ok_prev) {
                     // this thread's 32 output channels: columns 32 h of its O row (the column
-                    // address of a TMEM load is the same for the whole warp, so both halves)
+                    // address of a TMEM load is the same for the whole warp, so both halves).
+                    // The accumulator holds the item's earlier units relative to the max before
+                    // unit v: o = o * corr(v) + PV(v), or o = PV(v) when v opened the item.
                     uint32_t w0[32], w1[32];
                     tmem_ld_32x32(t_lane + 128 + 64 * bv, w0);
                     tmem_ld_32x32(t_lane + 128 + 64 * bv + 32, w1);
                     tmem_wait_ld();
+                    if (start_prev) {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] += __uint_as_float(h ? w1[c] : w0[c]);
+                        for (int c = 0; c < 32; ++c) o[c] = __uint_as_float(h ? w1[c] : w0[c]);
+                    } else {
+                        const float2 cv = make_float2(corr_prev, corr_prev);
+#pragma unroll
+                        for (int c = 0; c < 32; c += 2) {
+                            const float2 r = __ffma2_rn(make_float2(o[c], o[c + 1]), cv,
+                                                        make_float2(__uint_as_float(h ? w1[c] : w0[c]),
+                                                                    __uint_as_float(h ? w1[c + 1] : w0[c + 1])));
+                            o[c] = r.x;
+                            o[c + 1] = r.y;
+                        }
+                    }
+                } else if (start_prev) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = 0.f;  // a skipped first unit adds nothing
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] *= corr_prev;
                 }
                 tcgen05_before_sync();
                 __syncwarp();
@@ -377,22 +402,20 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
                     __nv_bfloat16 *out = (u == units) ? dst : dst_prev;
                     const float inv = lf > 0.f ? __fdividef(1.f, lf) : 0.f;
                     if (alive) {
+                        const float2 iv = make_float2(inv, inv);
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int c = 0; c < 32; c += 2) {
+                            const float2 r = __fmul2_rn(make_float2(o[c], o[c + 1]), iv);
+                            pk[c / 2] = pack_bf16x2(r.x, r.y);
+                        }
 #pragma unroll
                         for (int x = 0; x < 4; ++x)
-                            *reinterpret_cast<uint4 *>(out + 8 * x) =
-                                make_uint4(pack_bf16x2(o[8 * x] * inv, o[8 * x + 1] * inv),
-                                           pack_bf16x2(o[8 * x + 2] * inv, o[8 * x + 3] * inv),
-                                           pack_bf16x2(o[8 * x + 4] * inv, o[8 * x + 5] * inv),
-                                           pack_bf16x2(o[8 * x + 6] * inv, o[8 * x + 7] * inv));
+                            *reinterpret_cast<uint4 *>(out + 8 * x) = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
                     }
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] = 0.f;
-                } else {
-                    // same item: bring the accumulator to the max of unit u
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] *= corr;
                 }
             }
+            start_prev = item_start;
             ok_prev = ok;
         }
     }

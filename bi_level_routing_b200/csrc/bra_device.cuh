@@ -255,6 +255,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2_trunc(float lo, float hi)
     return __byte_perm(__float_as_uint(lo), __float_as_uint(hi), 0x7632);
 }
 
+// max(a, b, c) in one instruction (sm_100 three-input max; a NaN operand is ignored like fmaxf).
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // Named barrier among `threads` threads (a multiple of 32) with id `id` (1..15).
 __device__ __forceinline__ void named_barrier(int id, int threads)
 {
@@ -311,14 +319,16 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
 }
 
 // D[tmem] = A[tmem] * B[smem] (+ D when accumulate != 0), issued by one thread. A is M rows
-// (TMEM lane = row) of K-major bf16 pairs, one pair per 32-bit column.
+// (TMEM lane = row) of K-major bf16 pairs, one pair per 32-bit column. Lane l of D (l < 128) is
+// left untouched when bit l % 32 of `disabled_lanes` is set (the same mask for every 32-lane
+// quadrant).
 __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                             uint32_t accumulate)
+                                             uint32_t accumulate, uint32_t disabled_lanes = 0u)
 {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u)
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(disabled_lanes)
         : "memory");
 }
 

@@ -460,7 +460,8 @@ static cudaError_t launch_topk_e(const float *qm, const float *km, int32_t *idx,
 {
     const float scale = (float)(1.0 / sqrt((double)g.C));
     const bool rounds = topk_by_rounds(E, g.topk);
-    const int rows = g.R <= 64 ? (g.C >= 256 ? 16 : 8) : 16;
+    // one pass of route_rows per warp: every warp of the CTA busy, the image's key means staged once
+    const int rows = 8 * RowsPerPass<E>::value;
     const size_t stage_bytes = (size_t)(g.R + rows) * (g.C + 4) * sizeof(float);
     if (stage_bytes <= 100 * 1024)
         return rounds ? launch_topk_typed<E, true, true>(qm, km, idx, g, rows, scale, stage_bytes, stream)
