@@ -137,7 +137,8 @@ class ClockSampler:
 
 
 def cpu_baseline(w, inp, seconds: float):
-    """The oracle's forward pass, as it stands, on the first images of the batch."""
+    """The oracle's forward pass, as it stands, on the first images of the batch (the whole batch,
+    repeated, when one pass over it takes less than `seconds`)."""
     import oracle
     orc = oracle.default()
     q, k, v = inp["q"], inp["k"], inp["v"]
@@ -145,13 +146,20 @@ def cpu_baseline(w, inp, seconds: float):
     orc.forward(q[:1], k[:1], v[:1], w.n_win, w.topk, w.heads)
     t1 = time.perf_counter() - t0
     n = int(max(1, min(w.B, math.floor(seconds / max(t1, 1e-6)))))
+    reps = 1
     if n > 1:
         t0 = time.perf_counter()
         orc.forward(q[:n], k[:n], v[:n], w.n_win, w.topk, w.heads)
         t1 = time.perf_counter() - t0
-    return {"value": n * w.N / t1, "unit": UNIT, "cores": orc.max_threads(), "kind": "oracle",
+    if n == w.B and t1 < seconds:
+        reps = int(max(1, min(100, math.floor(seconds / max(t1, 1e-6)))))
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            orc.forward(q, k, v, w.n_win, w.topk, w.heads)
+        t1 = time.perf_counter() - t0
+    return {"value": reps * n * w.N / t1, "unit": UNIT, "cores": orc.max_threads(), "kind": "oracle",
             "sample": f"oracle forward (route + attend, float64) on the first {n} of {w.B} images "
-                      f"({n * w.N} query tokens), {t1:.2f} s"}
+                      f"({n * w.N} query tokens) x {reps}, {t1:.2f} s"}
 
 
 def run_reference(args, w, rank):
