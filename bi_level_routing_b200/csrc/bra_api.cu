@@ -162,6 +162,11 @@ bra_status route_impl(const void *q, const void *k, int32_t *idx, const bra::Geo
     DeviceState *st = nullptr;
     bra_status s = device_state(&st);
     if (s != BRA_OK) return s;
+    if (g.rs == 1 && g.R <= 256) {
+        // one-token regions: the means are the tokens, no scratch and no means kernel
+        const cudaError_t e = bra::launch_route_topk_tokens(q, k, idx, g, dtype == BRA_BF16, stream);
+        return e == cudaSuccess ? BRA_OK : cuda_fail(e, "routing kernel");
+    }
     const size_t bytes = (size_t)2 * g.B * g.R * g.C * sizeof(float);
     void *scratch = nullptr;
     cudaError_t e = cudaMallocFromPoolAsync(&scratch, bytes, st->pool, stream);
@@ -348,6 +353,7 @@ bra_status bra_check_device_error(void *stream)
 size_t bra_route_scratch_bytes(int B, int H, int W, int C, int n_win)
 {
     if (B <= 0 || H <= 0 || W <= 0 || C <= 0 || n_win <= 0) return 0;
+    if (H == n_win && W == n_win && n_win * n_win <= 256) return 0;  // one-token regions: no means
     return (size_t)2 * B * n_win * n_win * C * sizeof(float);
 }
 
@@ -357,7 +363,7 @@ int bra_kernels_per_call(const char *entry_point, int B, int H, int W, int C, in
     if (!entry_point || B <= 0) return 0;
     bra::Geometry g;
     if (check_shape(B, H, W, C, heads, n_win, topk, dtype, &g) != BRA_OK) return 0;
-    const int route = 2;
+    const int route = (g.rs == 1 && g.R <= 256) ? 1 : 2;
     const int attend = choose_attend_kernel(g, dtype) < 0 ? 0 : 1;
     if (!std::strcmp(entry_point, "bra_route")) return route;
     if (!std::strcmp(entry_point, "bra_attend")) return attend;

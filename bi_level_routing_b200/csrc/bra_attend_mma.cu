@@ -492,8 +492,8 @@ __global__ void __launch_bounds__(256) attend_dense_mma_kernel(const __grid_cons
     uint8_t *sK = sQ + (size_t)nqpad * kRowBytes;
     uint8_t *sV = sK + (size_t)a.npad * kRowBytes;
     float *lw = reinterpret_cast<float *>(sV + (size_t)a.npad * kRowBytes);  // [R][R] log2(multiplicity)
-    uint8_t *cnt = reinterpret_cast<uint8_t *>(lw + a.R * a.R);                // [R][R]
-    uint8_t *reg = cnt + a.R * a.R;                                            // [npad] region of each key
+    int *cnt = reinterpret_cast<int *>(lw + a.R * a.R);                        // [R][R]
+    uint8_t *reg = reinterpret_cast<uint8_t *>(cnt + a.R * a.R);               // [npad] region of each key
     uint64_t *bar = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(reg + a.npad) + 7) & ~uintptr_t(7));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -528,14 +528,14 @@ __global__ void __launch_bounds__(256) attend_dense_mma_kernel(const __grid_cons
         reg[t] = t < a.N ? (uint8_t)(((t / a.W) / a.hr) * a.n_win + (t % a.W) / a.wr) : 0;
     for (int e = threadIdx.x; e < a.R * a.R; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
-    for (int r = threadIdx.x; r < a.R; r += blockDim.x)
-        for (int j = 0; j < a.topk; ++j) {
-            const int s = routed[r * a.topk + j];
-            if (s >= 0 && s < a.R)
-                ++cnt[r * a.R + s];
-            else if (cb == 0 && split == 0)
-                flag_error(a.err, kErrIndex);
-        }
+    // multiplicity of every routed region, one thread per idx entry (all loads in flight)
+    for (int e = threadIdx.x; e < a.R * a.topk; e += blockDim.x) {
+        const int s = routed[e];
+        if (s >= 0 && s < a.R)
+            atomicAdd(&cnt[(e / a.topk) * a.R + s], 1);
+        else if (cb == 0 && split == 0)
+            flag_error(a.err, kErrIndex);
+    }
     __syncthreads();
     for (int e = threadIdx.x; e < a.R * a.R; e += blockDim.x) lw[e] = cnt[e] ? log2f((float)cnt[e]) : -INFINITY;
     __syncthreads();
@@ -641,7 +641,7 @@ static size_t dense_smem_bytes(const Geometry &g, int rows_per_split)
 {
     const int nq = rows_per_split * g.W, nqpad = (nq + 15) & ~15;
     const int npad = (g.N + 15) & ~15;
-    return 1024 + (size_t)(nqpad + 2 * npad) * kRowBytes + (size_t)g.R * g.R * 5 + npad + 16;
+    return 1024 + (size_t)(nqpad + 2 * npad) * kRowBytes + (size_t)g.R * g.R * 8 + npad + 16;
 }
 
 cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,

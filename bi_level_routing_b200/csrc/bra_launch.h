@@ -35,6 +35,11 @@ cudaError_t launch_region_means(const void *q, const void *k, float *qm, float *
                                 bool bf16, int num_sms, cudaStream_t stream);
 
 
+// Affinity rows and top-k straight from q and k when a region is one token (rs == 1, R <= 256):
+// the means are the tokens, widened exactly to fp32, so the index is the same as from the means.
+cudaError_t launch_route_topk_tokens(const void *q, const void *k, int32_t *idx, const Geometry &g, bool bf16,
+                                     cudaStream_t stream);
+
 // Affinity rows and top-k: idx[b, r, :] from qm, km.
 cudaError_t launch_route_topk(const float *qm, const float *km, int32_t *idx, const Geometry &g,
                               cudaStream_t stream);

@@ -94,6 +94,54 @@ __device__ __forceinline__ void region_means_block(const MeansArgs &a, float *pa
     }
 }
 
+// Small regions (rs <= 16): one thread per (region, 16-byte vector of channels) sums the
+// region's rs tokens of q and of k in token order (row by row), eight tokens' loads in flight
+// at a time, and writes the V means of each. No shared memory, no barrier.
+template <typename T>
+__device__ __forceinline__ void region_means_flat(const MeansArgs &a, long long gid)
+{
+    constexpr int V = Vec16<T>::N;
+    constexpr int ROWS = 8;
+    const int vpt = a.C / V;
+    const long long flat = gid / vpt;
+    const int v = (int)(gid % vpt);
+    const int64_t b = flat / a.R;
+    const int r = (int)(flat % a.R);
+    const int ry = r / a.n_win, rx = r % a.n_win;
+    const int64_t base = ((b * a.H + (int64_t)ry * a.hr) * a.W + (int64_t)rx * a.wr) * a.C + (int64_t)v * V;
+    const int rs = a.hr * a.wr;
+    const T *pq = static_cast<const T *>(a.q) + base;
+    const T *pk = static_cast<const T *>(a.k) + base;
+    float aq[V], ak[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) aq[i] = ak[i] = 0.f;
+    for (int t0 = 0; t0 < rs; t0 += ROWS) {
+        uint4 rq[ROWS], rk[ROWS];
+#pragma unroll
+        for (int u = 0; u < ROWS; ++u)
+            if (t0 + u < rs) {
+                const int t = t0 + u;
+                const int64_t off = ((int64_t)(t / a.wr) * a.W + t % a.wr) * a.C;
+                rq[u] = Vec16<T>::load_raw(pq + off);
+                rk[u] = Vec16<T>::load_raw(pk + off);
+            }
+#pragma unroll
+        for (int u = 0; u < ROWS; ++u)
+            if (t0 + u < rs) {
+                Vec16<T>::accumulate(rq[u], aq);
+                Vec16<T>::accumulate(rk[u], ak);
+            }
+    }
+    const float inv_n = (float)rs;
+    float4 *dq = reinterpret_cast<float4 *>(a.qm + flat * a.C + v * V);
+    float4 *dk = reinterpret_cast<float4 *>(a.km + flat * a.C + v * V);
+#pragma unroll
+    for (int j = 0; j < V / 4; ++j) {
+        dq[j] = make_float4(aq[4 * j] / inv_n, aq[4 * j + 1] / inv_n, aq[4 * j + 2] / inv_n, aq[4 * j + 3] / inv_n);
+        dk[j] = make_float4(ak[4 * j] / inv_n, ak[4 * j + 1] / inv_n, ak[4 * j + 2] / inv_n, ak[4 * j + 3] / inv_n);
+    }
+}
+
 // ============================================================================ affinity + top-k
 
 // Order-preserving 64-bit key: larger affinity -> larger key; equal affinities -> the lower
@@ -195,31 +243,23 @@ __device__ __forceinline__ void select_topk(unsigned long long (&key)[E], int to
     }
 }
 
-// Rows per warp pass of route_rows: NR rows x E keys x 4 partial sums stay in registers.
+// Rows per warp pass of affinity_accumulate: NR rows x E keys x 4 partial sums stay in registers.
 template <int E>
 struct RowsPerPass {
     static constexpr int value = E <= 2 ? 2 : 1;
 };
 
-// Routing rows i < nr (nr <= NR) of one image, by one warp: query mean row i at
-// qrows + i * qstride, key mean row s at kbase + s * kstride. Lane l computes the affinities of
-// regions s = e * 32 + l, e < E (R <= 32 E), for all NR rows at once: every pair (row, s) is
-// the dot product of dot_rows, four interleaved partial sums over the channels in order,
-// combined as (s0 + s1) + (s2 + s3), times C^-1/2; the NR x E products only run side by side,
-// so that each 16-byte key load serves NR rows and the loads of consecutive channel steps
-// overlap. Every routing kernel goes through this function, so the index is the same bits
-// whichever kernel computed it.
-template <int E, int NR, bool ROUNDS>
-__device__ __forceinline__ void route_rows(const float *qrows, int qstride, int nr, const float *kbase, int kstride,
-                                           int R, int C, int topk, float scale, int32_t *out, int lane)
+// Routing rows i < nr (nr <= NR) of one image, by one warp, over channels [0, cn) of the rows
+// given: query mean row i at qrows + i * qstride, key mean row s at kbase + s * kstride. Lane l
+// accumulates the affinities of regions s = e * 32 + l, e < E (R <= 32 E), for all NR rows at
+// once: every pair (row, s) is the dot product of dot_rows, four interleaved partial sums over
+// the channels in order, so that calls over consecutive channel windows continue the same sum;
+// the NR x E products only run side by side, so that each 16-byte key load serves NR rows and
+// the loads of consecutive channel steps overlap.
+template <int E, int NR>
+__device__ __forceinline__ void affinity_accumulate(float (&acc)[NR][E][4], const float *qrows, int qstride, int nr,
+                                                    const float *kbase, int kstride, int R, int cn, int lane)
 {
-    float acc[NR][E][4];
-#pragma unroll
-    for (int i = 0; i < NR; ++i)
-#pragma unroll
-        for (int e = 0; e < E; ++e)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][e][j] = 0.f;
     int krow[E], qrow[NR];  // element offsets of the rows
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -228,8 +268,9 @@ __device__ __forceinline__ void route_rows(const float *qrows, int qstride, int 
     }
 #pragma unroll
     for (int i = 0; i < NR; ++i) qrow[i] = (i < nr ? i : 0) * qstride;
-#pragma unroll 4
-    for (int c = 0; c < C; c += 4) {
+    constexpr int kUnroll = E >= 8 ? 2 : 4;  // keeps the E x kUnroll key loads in registers
+#pragma unroll kUnroll
+    for (int c = 0; c < cn; c += 4) {
         float4 y[E];
 #pragma unroll
         for (int e = 0; e < E; ++e) y[e] = *reinterpret_cast<const float4 *>(kbase + krow[e] + c);
@@ -245,6 +286,16 @@ __device__ __forceinline__ void route_rows(const float *qrows, int qstride, int 
             }
         }
     }
+}
+
+// The affinities of rows i < nr from their partial sums, combined as (s0 + s1) + (s2 + s3), times
+// C^-1/2, and their top-k, written to out + i * topk. Every routing kernel goes through
+// affinity_accumulate and this function, so the index is the same bits whichever kernel
+// computed it.
+template <int E, int NR, bool ROUNDS>
+__device__ __forceinline__ void affinity_select(const float (&acc)[NR][E][4], int nr, int R, int topk, float scale,
+                                                int32_t *out, int lane)
+{
 #pragma unroll
     for (int i = 0; i < NR; ++i) {
         if (i >= nr) break;
@@ -259,66 +310,95 @@ __device__ __forceinline__ void route_rows(const float *qrows, int qstride, int 
     }
 }
 
-// Copies rows0 fp32 rows of length C (a multiple of 4) from src0 and then rows1 rows from src1
-// (row stride C) to consecutive rows of dst (row stride dst_stride), all threads of the CTA,
-// eight 16-byte loads in flight per thread. With L2 set, the loads bypass L1 (ld.global.cg):
-// the rows were written by other CTAs of this grid.
-template <bool L2>
-__device__ __forceinline__ void stage_rows(const float *__restrict__ src0, int rows0, const float *__restrict__ src1,
-                                           int rows1, float *dst, int C, int dst_stride)
+// 16 bytes of S elements as fp32 (bf16 widens exactly).
+__device__ __forceinline__ void store_as_f32(float *d, uint4 v, float)
 {
-    const int c4 = C / 4;
-    const int n0 = rows0 * c4;
-    const int total = (rows0 + rows1) * c4;
+    *reinterpret_cast<float4 *>(d) = make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
+                                                 __uint_as_float(v.w));
+}
+__device__ __forceinline__ void store_as_f32(float *d, uint4 v, __nv_bfloat16)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float f[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+    *reinterpret_cast<float4 *>(d) = make_float4(f[0], f[1], f[2], f[3]);
+    *reinterpret_cast<float4 *>(d + 4) = make_float4(f[4], f[5], f[6], f[7]);
+}
+
+// Copies channels [c0, c0 + cn) (multiples of 16 bytes of S) of rows0 rows from src0 and then of
+// rows1 rows from src1 (row stride C elements) as fp32 to consecutive rows of dst (row stride
+// dst_stride), all threads of the CTA, eight 16-byte loads in flight per thread. With L2 set,
+// the loads bypass L1 (ld.global.cg): the rows were written by other CTAs of this grid.
+template <bool L2, typename S>
+__device__ __forceinline__ void stage_rows(const S *__restrict__ src0, int rows0, const S *__restrict__ src1, int rows1,
+                                           float *dst, int C, int c0, int cn, int dst_stride)
+{
+    constexpr int V = 16 / sizeof(S);
+    const int cv = cn / V;
+    const int n0 = rows0 * cv;
+    const int total = (rows0 + rows1) * cv;
     for (int e0 = threadIdx.x; e0 < total; e0 += 8 * blockDim.x) {
-        float4 v[8];
+        uint4 v[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int e = e0 + u * blockDim.x;
             if (e < total) {
-                const float *src = e < n0 ? src0 + (size_t)(e / c4) * C : src1 + (size_t)((e - n0) / c4) * C;
-                const float4 *p = reinterpret_cast<const float4 *>(src + (e % c4) * 4);
+                const S *src = e < n0 ? src0 + (size_t)(e / cv) * C : src1 + (size_t)((e - n0) / cv) * C;
+                const uint4 *p = reinterpret_cast<const uint4 *>(src + c0 + (e % cv) * V);
                 v[u] = L2 ? __ldcg(p) : __ldg(p);
             }
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int e = e0 + u * blockDim.x;
-            if (e < total) *reinterpret_cast<float4 *>(dst + (size_t)(e / c4) * dst_stride + (e % c4) * 4) = v[u];
+            if (e < total) store_as_f32(dst + (size_t)(e / cv) * dst_stride + (e % cv) * V, v[u], S());
         }
     }
 }
 
-// One CTA per (image, block of `rows` rows), one warp per row at a time. The image's key means
-// (and the block's query means) are staged in shared memory when STAGED, rows padded to C + 4
-// floats so that lanes reading different rows hit different banks; otherwise they are read
-// through L1.
-template <int E, bool STAGED, bool ROUNDS>
-__global__ void __launch_bounds__(256, 2) route_topk_kernel(const float *__restrict__ qm, const float *__restrict__ km,
+// One CTA per (image, block of `rows` = 8 NR rows), NR rows per warp. The image's key means and
+// the block's query means (fp32 means, or the bf16 / fp32 tokens themselves when a region is one
+// token) are staged in shared memory as fp32 a window of `chunk` channels at a time
+// (the whole row when it fits), rows padded to chunk + 4 floats so that lanes reading different
+// rows hit different banks; the partial sums carry over from window to window.
+template <int E, bool ROUNDS, typename S>
+__global__ void __launch_bounds__(256, 2) route_topk_kernel(const S *__restrict__ qm, const S *__restrict__ km,
                                                          int32_t *__restrict__ idx, int R, int C, int topk, int rows,
-                                                         float scale)
+                                                         int chunk, float scale)
 {
     extern __shared__ float4 smem4[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    constexpr int NR = RowsPerPass<E>::value;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row_blocks = (R + rows - 1) / rows;
     const int b = blockIdx.x / row_blocks;
     const int r0 = (blockIdx.x % row_blocks) * rows;
     const int nrows = min(rows, R - r0);
-    const int stride = STAGED ? C + 4 : C;
-    const float *kbase = km + (int64_t)b * R * C;
-    const float *qbase = qm + ((int64_t)b * R + r0) * C;
-    if (STAGED) {
-        float *skm = reinterpret_cast<float *>(smem4);
-        float *sqm = skm + (size_t)R * stride;
-        stage_rows<false>(kbase, R, qbase, nrows, skm, C, stride);
+    const int stride = chunk + 4;
+    const S *gkm = km + (int64_t)b * R * C;
+    const S *gqm = qm + ((int64_t)b * R + r0) * C;
+    float *skm = reinterpret_cast<float *>(smem4);
+    float *sqm = skm + (size_t)R * stride;
+    const int i0 = warp * NR;  // this warp's first row in the block
+    const int nr = min(NR, nrows - i0);
+    float acc[NR][E][4];
+#pragma unroll
+    for (int i = 0; i < NR; ++i)
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][e][j] = 0.f;
+    for (int c0 = 0; c0 < C; c0 += chunk) {
+        const int cn = min(chunk, C - c0);
+        if (c0 > 0) __syncthreads();  // the previous window is no longer read
+        stage_rows<false, S>(gkm, R, gqm, nrows, skm, C, c0, cn, stride);
         __syncthreads();
-        kbase = skm;
-        qbase = sqm;
+        if (nr > 0) affinity_accumulate<E, NR>(acc, sqm + (size_t)i0 * stride, stride, nr, skm, stride, R, cn, lane);
     }
-    constexpr int NR = RowsPerPass<E>::value;
-    for (int i = warp * NR; i < nrows; i += nwarps * NR)
-        route_rows<E, NR, ROUNDS>(qbase + (size_t)i * stride, stride, min(NR, nrows - i), kbase, stride, R, C, topk,
-                                  scale, idx + ((int64_t)b * R + r0 + i) * topk, lane);
+    if (nr > 0) affinity_select<E, NR, ROUNDS>(acc, nr, R, topk, scale, idx + ((int64_t)b * R + r0 + i0) * topk, lane);
 }
 
 // Wide rows (R > 256): one warp per row, keys in shared memory, bitonic network there.
@@ -359,7 +439,7 @@ __global__ void __launch_bounds__(256) route_topk_wide_kernel(const float *__res
 
 // ============================================================================ means kernels
 
-// Means only.
+// Means of rs > 16 regions: several regions per CTA.
 template <typename T>
 __global__ void __launch_bounds__(kMeansThreads, 2) region_means_kernel(const MeansArgs a)
 {
@@ -367,6 +447,14 @@ __global__ void __launch_bounds__(kMeansThreads, 2) region_means_kernel(const Me
     const long long i0 = (long long)blockIdx.x * a.rpc;
     const int nreg = (int)min((long long)a.rpc, (long long)a.B * a.R - i0);
     region_means_block<T>(a, reinterpret_cast<float *>(smem4), i0, nreg);
+}
+
+// Means of rs <= 16 regions: one thread per (region, 16-byte vector).
+template <typename T>
+__global__ void __launch_bounds__(kMeansThreads) region_means_flat_kernel(const MeansArgs a, long long total)
+{
+    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid < total) region_means_flat<T>(a, gid);
 }
 
 // ============================================================================ launchers
@@ -428,6 +516,16 @@ cudaError_t launch_region_means(const void *q, const void *k, float *qm, float *
     (void)num_sms;
     const MeansArgs a = means_args(q, k, qm, km, g, bf16);
     if ((long long)a.wr * (g.C / (bf16 ? 8 : 4)) > kMaxMeansVectors) return cudaErrorInvalidConfiguration;
+    if (g.rs <= 16) {
+        const long long total = (long long)g.B * g.R * (g.C / (bf16 ? 8 : 4));
+        const long long blocks = (total + kMeansThreads - 1) / kMeansThreads;
+        if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+        if (bf16)
+            region_means_flat_kernel<__nv_bfloat16><<<(unsigned)blocks, kMeansThreads, 0, stream>>>(a, total);
+        else
+            region_means_flat_kernel<float><<<(unsigned)blocks, kMeansThreads, 0, stream>>>(a, total);
+        return cudaGetLastError();
+    }
     const size_t smem = means_part_bytes(a);
     static int granted[2][64] = {{0}};
     cudaError_t e = bf16 ? raise_smem_limit(region_means_kernel<__nv_bfloat16>, smem, granted[0])
@@ -442,40 +540,61 @@ cudaError_t launch_region_means(const void *q, const void *k, float *qm, float *
     return cudaGetLastError();
 }
 
-template <int E, bool STAGED, bool ROUNDS>
-static cudaError_t launch_topk_typed(const float *qm, const float *km, int32_t *idx, const Geometry &g, int rows,
+template <int E, bool ROUNDS, typename S>
+static cudaError_t launch_topk_typed(const S *qm, const S *km, int32_t *idx, const Geometry &g, int rows, int chunk,
                                      float scale, size_t smem, cudaStream_t stream)
 {
     static int granted[64] = {0};
-    cudaError_t e = raise_smem_limit(route_topk_kernel<E, STAGED, ROUNDS>, smem, granted);
+    cudaError_t e = raise_smem_limit(route_topk_kernel<E, ROUNDS, S>, smem, granted);
     if (e != cudaSuccess) return e;
     const long long blocks = (long long)((g.R + rows - 1) / rows) * g.B;
-    route_topk_kernel<E, STAGED, ROUNDS><<<(unsigned)blocks, 256, smem, stream>>>(qm, km, idx, g.R, g.C, g.topk, rows,
-                                                                                  scale);
+    route_topk_kernel<E, ROUNDS, S><<<(unsigned)blocks, 256, smem, stream>>>(qm, km, idx, g.R, g.C, g.topk, rows, chunk,
+                                                                             scale);
     return cudaGetLastError();
 }
 
-template <int E>
-static cudaError_t launch_topk_e(const float *qm, const float *km, int32_t *idx, const Geometry &g, cudaStream_t stream)
+template <int E, typename S>
+static cudaError_t launch_topk_e(const S *qm, const S *km, int32_t *idx, const Geometry &g, cudaStream_t stream)
 {
     const float scale = (float)(1.0 / sqrt((double)g.C));
     const bool rounds = topk_by_rounds(E, g.topk);
-    // one pass of route_rows per warp: every warp of the CTA busy, the image's key means staged once
+    // one pass of the row routine per warp: every warp of the CTA busy, the image's key means
+    // staged once per channel window; the window is the whole row when the staged rows fit in
+    // 100 KB, else the widest multiple of 32 channels that does (a row stride of 4 mod 32 words
+    // keeps the lanes' 16-byte key loads free of bank conflicts)
     const int rows = 8 * RowsPerPass<E>::value;
-    const size_t stage_bytes = (size_t)(g.R + rows) * (g.C + 4) * sizeof(float);
-    if (stage_bytes <= 100 * 1024)
-        return rounds ? launch_topk_typed<E, true, true>(qm, km, idx, g, rows, scale, stage_bytes, stream)
-                      : launch_topk_typed<E, true, false>(qm, km, idx, g, rows, scale, stage_bytes, stream);
-    return rounds ? launch_topk_typed<E, false, true>(qm, km, idx, g, rows, scale, 0, stream)
-                  : launch_topk_typed<E, false, false>(qm, km, idx, g, rows, scale, 0, stream);
+    const long long per_col = (long long)(g.R + rows) * sizeof(float);
+    int chunk = g.C;
+    if (per_col * (chunk + 4) > 100 * 1024) {
+        chunk = (int)((100 * 1024) / per_col - 4) / 32 * 32;
+        if (chunk < 32) return cudaErrorInvalidConfiguration;  // R is at most 256 here
+    }
+    const size_t smem = (size_t)per_col * (chunk + 4);
+    return rounds ? launch_topk_typed<E, true, S>(qm, km, idx, g, rows, chunk, scale, smem, stream)
+                  : launch_topk_typed<E, false, S>(qm, km, idx, g, rows, chunk, scale, smem, stream);
+}
+
+template <typename S>
+static cudaError_t launch_topk_any(const S *qm, const S *km, int32_t *idx, const Geometry &g, cudaStream_t stream)
+{
+    if (g.R <= 32) return launch_topk_e<1, S>(qm, km, idx, g, stream);
+    if (g.R <= 64) return launch_topk_e<2, S>(qm, km, idx, g, stream);
+    if (g.R <= 128) return launch_topk_e<4, S>(qm, km, idx, g, stream);
+    return launch_topk_e<8, S>(qm, km, idx, g, stream);
+}
+
+cudaError_t launch_route_topk_tokens(const void *q, const void *k, int32_t *idx, const Geometry &g, bool bf16,
+                                     cudaStream_t stream)
+{
+    if (g.rs != 1 || g.R > 256) return cudaErrorInvalidConfiguration;
+    return bf16 ? launch_topk_any<__nv_bfloat16>(static_cast<const __nv_bfloat16 *>(q),
+                                                 static_cast<const __nv_bfloat16 *>(k), idx, g, stream)
+                : launch_topk_any<float>(static_cast<const float *>(q), static_cast<const float *>(k), idx, g, stream);
 }
 
 cudaError_t launch_route_topk(const float *qm, const float *km, int32_t *idx, const Geometry &g, cudaStream_t stream)
 {
-    if (g.R <= 32) return launch_topk_e<1>(qm, km, idx, g, stream);
-    if (g.R <= 64) return launch_topk_e<2>(qm, km, idx, g, stream);
-    if (g.R <= 128) return launch_topk_e<4>(qm, km, idx, g, stream);
-    if (g.R <= 256) return launch_topk_e<8>(qm, km, idx, g, stream);
+    if (g.R <= 256) return launch_topk_any<float>(qm, km, idx, g, stream);
     int P = 512;
     while (P < g.R) P <<= 1;
     int warps = (int)((48 * 1024) / ((size_t)P * 8));

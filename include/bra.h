@@ -135,7 +135,8 @@ int bra_selected_attend_kernel(int B, int H, int W, int C, int heads, int n_win,
    BRA_OK, BRA_ERR_INDEX (an idx entry outside [0, R) was skipped) or BRA_ERR_TIMEOUT. */
 bra_status bra_check_device_error(void *stream);
 
-/* Bytes of scratch bra_route / bra_forward take from the pool for these sizes (fp32 means). */
+/* Bytes of scratch bra_route / bra_forward take from the pool for these sizes (fp32 means; 0 when
+   every region is one token and R <= 256, where routing reads q and k directly). */
 size_t bra_route_scratch_bytes(int B, int H, int W, int C, int n_win);
 
 /* Number of library kernels one call of `entry_point` ("bra_route", "bra_attend",

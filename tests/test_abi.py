@@ -122,4 +122,8 @@ def test_scratch_and_launch_accounting(L):
     assert L.bra_kernels_per_call(b"bra_forward", *stage1) == 3
     assert L.bra_kernels_per_call(b"bra_forward", *highres) == 3
     assert L.bra_kernels_per_call(b"bra_forward", 1, 30, 28, 64, 2, 7, 4, 1) == 0  # rejected
+    stage4 = (64, 7, 7, 512, 16, 7, 49, 1)  # one-token regions: routing reads q and k directly
+    assert L.bra_kernels_per_call(b"bra_route", *stage4) == 1
+    assert L.bra_kernels_per_call(b"bra_forward", *stage4) == 2
+    assert L.bra_route_scratch_bytes(64, 7, 7, 512, 7) == 0
     assert L.bra_kernels_per_call(b"nonsense", *stage1) == 0
