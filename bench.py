@@ -53,6 +53,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     ap.add_argument("--soak-seconds", type=float, default=1.0,
                     help="identical untimed steps before the timed region, while clocks are sampled")
+    ap.add_argument("--repeats", type=int, default=5, help="timed runs of K steps; the median is reported")
     return ap.parse_args()
 
 
@@ -244,15 +245,27 @@ def main():
     torch.cuda.synchronize()
 
 
-    # ---- the timed region: K steps, each [event, route, event, attend], captured as ONE CUDA
-    # graph (timing events as external event-record nodes) so that host launch overhead does
-    # not pace the GPU; eager launches if capture is refused.
+    # ---- the timed region: K steps [route, attend], captured as ONE CUDA graph with a timing
+    # event (an external event-record node) before the first and after the last, so that host
+    # launch overhead does not pace the GPU and consecutive kernels keep their programmatic
+    # (overlapping) launches; eager launches if capture is refused. A second graph of the same
+    # steps with an event around every route and every attention call gives the breakdown.
     K = args.steps
+    ev_start = torch.cuda.Event(enable_timing=True, external=True)
+    ev_stop = torch.cuda.Event(enable_timing=True, external=True)
     ev_route = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(K)]
     ev_attend = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(K)]
     ev_end = torch.cuda.Event(enable_timing=True, external=True)
 
     def record_steps():
+        ev_start.record()
+        for i in range(K):
+            s = sets[i % nsets]
+            route(s)
+            attend(s)
+        ev_stop.record()
+
+    def record_breakdown():
         for i in range(K):
             s = sets[i % nsets]
             ev_route[i].record()
@@ -262,21 +275,26 @@ def main():
         ev_end.record()
 
     launch = "cuda_graph (all K steps in one graph)"
-    graph = None
+    graph = graph_bd = None
     if not args.eager:
         try:
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph):
                 record_steps()
+            graph_bd = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph_bd):
+                record_breakdown()
         except Exception as e:  # capture refused: time eager launches
-            graph = None
+            graph = graph_bd = None
             launch = f"eager (graph capture failed: {type(e).__name__}: {e})"
             torch.cuda.synchronize()
     if graph is None and launch.startswith("cuda_graph"):
         launch = "eager"
     run_steps = graph.replay if graph is not None else record_steps
+    run_breakdown = graph_bd.replay if graph_bd is not None else record_breakdown
 
     run_steps()  # untimed: the first replay also uploads the graph
+    run_breakdown()
     torch.cuda.synchronize()
 
     # ---- clock samples over a soak of identical steps around the timed region
@@ -286,17 +304,25 @@ def main():
         while time.perf_counter() - t_soak < args.soak_seconds:
             run_steps()
             torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
+        runs = []
+        for _ in range(max(1, args.repeats)):
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            run_steps()  # K timed steps
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            runs.append(ev_start.elapsed_time(ev_stop))
+        repeat_ms = list(runs)
+        total_ms = sorted(runs)[len(runs) // 2]  # the median run
+        # the per-kernel breakdown, from the graph with events around every call
+        run_breakdown()
         torch.cuda.synchronize()
-        run_steps()  # the timed K steps
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        total_ms = ev_route[0].elapsed_time(ev_end)
         attend_ms = [ev_attend[i].elapsed_time(ev_route[i + 1] if i + 1 < K else ev_end) for i in range(K)]
         route_ms = [ev_route[i].elapsed_time(ev_attend[i]) for i in range(K)]
+        breakdown_ms = ev_route[0].elapsed_time(ev_end)
         t_tail = time.perf_counter()
         while time.perf_counter() - t_tail < min(0.5, args.soak_seconds):
             run_steps()
@@ -306,6 +332,37 @@ def main():
         t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
+
+    # ---- secondary: warm L2, every step on the same buffer set (one graph of K steps)
+    warm = None
+    if graph is not None:
+        ev_w0 = torch.cuda.Event(enable_timing=True, external=True)
+        ev_w1 = torch.cuda.Event(enable_timing=True, external=True)
+        try:
+            gw = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gw):
+                ev_w0.record()
+                for _ in range(K):
+                    route(sets[0])
+                    attend(sets[0])
+                ev_w1.record()
+            gw.replay()
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            gw.replay()
+            torch.cuda.synchronize()
+            warm_ms = ev_w0.elapsed_time(ev_w1)
+            if world > 1:
+                t = torch.tensor([warm_ms], device=dev, dtype=torch.float64)
+                dist.all_reduce(t, op=dist.ReduceOp.MAX)
+                warm_ms = float(t.item())
+            warm = {"value": w.tokens * world * K / (warm_ms / 1e3), "unit": UNIT, "ms_per_step": warm_ms / K,
+                    "note": "secondary: one buffer set for every step, inputs warm in L2"}
+            del gw
+        except Exception as e:  # capture refused: no warm number
+            warm = {"unavailable": f"{type(e).__name__}: {e}"}
+            torch.cuda.synchronize()
 
     tokens = w.tokens * world
     value = tokens * K / (total_ms / 1e3)
@@ -330,6 +387,7 @@ def main():
                 "algorithmic_bytes_per_launch": attend_bytes, "mean_launch_us": mean_attend * 1e3,
                 "route_kernels_mean_us": mean_route * 1e3,
                 "step_roofline_us": roof_step_ms * 1e3, "step_frac": roof_step_ms / ms_per_step,
+                "breakdown_ms_per_step": breakdown_ms / K,
                 "step_frac_vs_8tbs": (w.unique_bytes() / 8e12 * 1e3) / ms_per_step}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -341,7 +399,11 @@ def main():
             "roofline": roofline,
             "gpu_launches": K * bra.kernels_per_call("bra_forward", w.B, w.H, w.W, w.C, w.heads, w.n_win, w.topk,
                                                      torch.bfloat16 if w.dtype == "bf16" else torch.float32),
-            "clocks": sampler.summary()}
+            "clocks": sampler.summary(),
+            "repeats": {"runs": len(repeat_ms), "ms_per_step": [r / K for r in repeat_ms],
+                        "reported": "median run"}}
+    if warm is not None:
+        line["warm_l2"] = warm
 
     # ---- end to end through the host entry point (pinned buffers, copies inside the timed region)
     if not args.no_e2e:
@@ -373,7 +435,7 @@ def main():
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_seconds)
 
-    del graph
+    del graph, graph_bd
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

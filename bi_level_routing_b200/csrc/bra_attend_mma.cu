@@ -252,6 +252,7 @@ __global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int begin = blockIdx.x * a.per_cta;
     const int end = min(a.nitems, begin + a.per_cta);
+    grid_dependency_wait();
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.qslots; ++i) {
@@ -410,8 +411,8 @@ static cudaError_t launch_gather_rs(const CUtensorMap &tq, const CUtensorMap &tk
     static int granted[64] = {0};
     cudaError_t e = ensure_smem_limit(attend_gather_mma_kernel<RS>, smem, granted);
     if (e != cudaSuccess) return e;
-    attend_gather_mma_kernel<RS><<<grid, (a.ncw + 1) * 32, smem, stream>>>(tq, tk, tv, tout, a);
-    return cudaGetLastError();
+    return launch_pdl(attend_gather_mma_kernel<RS>, dim3(grid), dim3((a.ncw + 1) * 32), smem, stream, tq, tk, tv, tout,
+                      a);
 }
 
 cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
@@ -505,6 +506,7 @@ __global__ void __launch_bounds__(256) attend_dense_mma_kernel(const __grid_cons
     const int b = (int)(item / a.ncb);
     const int y0 = split * a.rows_per_split;
     const int32_t *routed = a.idx + (int64_t)b * a.R * a.topk;
+    grid_dependency_wait();
 
     if (threadIdx.x == 0) {
         mbar_init(bar, 1);
@@ -670,8 +672,7 @@ cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk
     static int granted[64] = {0};
     cudaError_t e = ensure_smem_limit(attend_dense_mma_kernel, smem, granted);
     if (e != cudaSuccess) return e;
-    attend_dense_mma_kernel<<<(unsigned)blocks, 256, smem, stream>>>(tq, tk, tv, tout, a);
-    return cudaGetLastError();
+    return launch_pdl(attend_dense_mma_kernel, dim3((unsigned)blocks), dim3(256), smem, stream, tq, tk, tv, tout, a);
 }
 
 }  // namespace bra

@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(128) attend_simt_kernel(const T *__restrict__ 
                                                           T *__restrict__ out, int H, int W, int C, int heads,
                                                           int n_win, int topk, float scale_log2, unsigned *err)
 {
+    grid_dependency_wait();
     const int hd = C / heads;
     const int hr = H / n_win, wr = W / n_win, rs = hr * wr, R = n_win * n_win;
     const int64_t blk = blockIdx.x;
@@ -90,15 +91,13 @@ static cudaError_t launch_simt_typed(const void *q, const void *k, const void *v
     const T *tq = (const T *)q, *tk = (const T *)k, *tv = (const T *)v;
     T *to = (T *)out;
     if (g.hd <= 32)
-        attend_simt_kernel<T, 32><<<grid, threads, 0, stream>>>(tq, tk, tv, idx, to, g.H, g.W, g.C, g.heads, g.n_win,
-                                                                g.topk, scale_log2, err);
-    else if (g.hd <= 64)
-        attend_simt_kernel<T, 64><<<grid, threads, 0, stream>>>(tq, tk, tv, idx, to, g.H, g.W, g.C, g.heads, g.n_win,
-                                                                g.topk, scale_log2, err);
-    else
-        attend_simt_kernel<T, 128><<<grid, threads, 0, stream>>>(tq, tk, tv, idx, to, g.H, g.W, g.C, g.heads,
-                                                                 g.n_win, g.topk, scale_log2, err);
-    return cudaGetLastError();
+        return launch_pdl(attend_simt_kernel<T, 32>, grid, dim3(threads), 0, stream, tq, tk, tv, idx, to, g.H, g.W, g.C,
+                          g.heads, g.n_win, g.topk, scale_log2, err);
+    if (g.hd <= 64)
+        return launch_pdl(attend_simt_kernel<T, 64>, grid, dim3(threads), 0, stream, tq, tk, tv, idx, to, g.H, g.W, g.C,
+                          g.heads, g.n_win, g.topk, scale_log2, err);
+    return launch_pdl(attend_simt_kernel<T, 128>, grid, dim3(threads), 0, stream, tq, tk, tv, idx, to, g.H, g.W, g.C,
+                      g.heads, g.n_win, g.topk, scale_log2, err);
 }
 
 cudaError_t launch_attend_simt(const void *q, const void *k, const void *v, const int32_t *idx, void *out,

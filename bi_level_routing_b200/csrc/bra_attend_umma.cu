@@ -108,6 +108,7 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
     __syncthreads();
     tcgen05_after_sync();
     const uint32_t tmem = *tmem_slot;
+    grid_dependency_wait();  // the barriers and the TMEM are set up while the previous kernel drains
 
     if (warp == 0) {
         // ------------------------------------------------------------- producer (TMA)
@@ -472,8 +473,7 @@ cudaError_t launch_attend_gather_umma(const CUtensorMap &tq, const CUtensorMap &
         if (e != cudaSuccess) return e;
         granted[dev] = (int)smem;
     }
-    attend_gather_umma_kernel<<<grid, 192, smem, stream>>>(tq, tk, tv, a);
-    return cudaGetLastError();
+    return launch_pdl(attend_gather_umma_kernel, dim3(grid), dim3(192), smem, stream, tq, tk, tv, a);
 }
 
 }  // namespace bra

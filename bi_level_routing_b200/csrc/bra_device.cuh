@@ -29,6 +29,14 @@ __device__ __forceinline__ void flag_error(unsigned *err, unsigned bit)
     if (err) atomicOr(err, bit);
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+
+// Waits until the kernel launched before this one on the stream has completed and its writes
+// are visible (the launch allowed this grid to start while that kernel drained); returns at
+// once when there is no such dependency. Every kernel of the library calls it before its first
+// global access that may depend on an earlier kernel.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- element loads
 
 // A 32-bit load through the read-only path that the compiler keeps where it is written (to

@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <string>
+#include <utility>
 
 #include "bra.h"
 
@@ -20,6 +21,27 @@ struct Geometry {
     int B, H, W, C, heads, n_win, topk;
     int R, hr, wr, rs, hd, N;
 };
+
+// Launches `kernel` on `stream` with programmatic stream serialization: the grid may be
+// scheduled as soon as the previous kernel's blocks have exited, and waits in
+// grid_dependency_wait() for that kernel's completion before its dependent reads, so the launch
+// latency and the prologue overlap the previous kernel's drain.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Sets the message bra_last_error_message returns on this thread.
 void set_last_error(const std::string &msg);

@@ -94,51 +94,63 @@ __device__ __forceinline__ void region_means_block(const MeansArgs &a, float *pa
     }
 }
 
-// Small regions (rs <= 16): one thread per (region, 16-byte vector of channels) sums the
-// region's rs tokens of q and of k in token order (row by row), eight tokens' loads in flight
-// at a time, and writes the V means of each. No shared memory, no barrier.
+// Small regions (rs <= 16): `lanes` consecutive threads per (region, 16-byte vector of
+// channels), thread j summing region rows j, j + lanes, ... in order (all their tokens' loads in
+// flight at once), then a butterfly over the lanes adds the row sums in a fixed order. lanes is
+// hr when hr is a power of two up to 8, else 1. No shared memory, no barrier.
 template <typename T>
-__device__ __forceinline__ void region_means_flat(const MeansArgs &a, long long gid)
+__device__ __forceinline__ void region_means_flat(const MeansArgs &a, long long gid, int lanes, bool write)
 {
     constexpr int V = Vec16<T>::N;
-    constexpr int ROWS = 8;
+    constexpr int TOK = 4;  // tokens whose loads are in flight together
     const int vpt = a.C / V;
-    const long long flat = gid / vpt;
-    const int v = (int)(gid % vpt);
+    const int j = (int)(gid % lanes);
+    const long long item = gid / lanes;
+    const long long flat = item / vpt;
+    const int v = (int)(item % vpt);
     const int64_t b = flat / a.R;
     const int r = (int)(flat % a.R);
     const int ry = r / a.n_win, rx = r % a.n_win;
     const int64_t base = ((b * a.H + (int64_t)ry * a.hr) * a.W + (int64_t)rx * a.wr) * a.C + (int64_t)v * V;
-    const int rs = a.hr * a.wr;
     const T *pq = static_cast<const T *>(a.q) + base;
     const T *pk = static_cast<const T *>(a.k) + base;
+    const int per = (a.hr / lanes) * a.wr;  // tokens of this thread: its rows, row by row
     float aq[V], ak[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) aq[i] = ak[i] = 0.f;
-    for (int t0 = 0; t0 < rs; t0 += ROWS) {
-        uint4 rq[ROWS], rk[ROWS];
+    for (int t0 = 0; t0 < per; t0 += TOK) {
+        uint4 rq[TOK], rk[TOK];
 #pragma unroll
-        for (int u = 0; u < ROWS; ++u)
-            if (t0 + u < rs) {
+        for (int u = 0; u < TOK; ++u)
+            if (t0 + u < per) {
                 const int t = t0 + u;
-                const int64_t off = ((int64_t)(t / a.wr) * a.W + t % a.wr) * a.C;
+                const int y = j + (t / a.wr) * lanes, x = t % a.wr;
+                const int64_t off = ((int64_t)y * a.W + x) * a.C;
                 rq[u] = Vec16<T>::load_raw(pq + off);
                 rk[u] = Vec16<T>::load_raw(pk + off);
             }
 #pragma unroll
-        for (int u = 0; u < ROWS; ++u)
-            if (t0 + u < rs) {
+        for (int u = 0; u < TOK; ++u)
+            if (t0 + u < per) {
                 Vec16<T>::accumulate(rq[u], aq);
                 Vec16<T>::accumulate(rk[u], ak);
             }
     }
-    const float inv_n = (float)rs;
+    for (int off = 1; off < lanes; off <<= 1) {
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            aq[i] += __shfl_xor_sync(0xffffffffu, aq[i], off);
+            ak[i] += __shfl_xor_sync(0xffffffffu, ak[i], off);
+        }
+    }
+    if (j != 0 || !write) return;
+    const float n = (float)(a.hr * a.wr);
     float4 *dq = reinterpret_cast<float4 *>(a.qm + flat * a.C + v * V);
     float4 *dk = reinterpret_cast<float4 *>(a.km + flat * a.C + v * V);
 #pragma unroll
-    for (int j = 0; j < V / 4; ++j) {
-        dq[j] = make_float4(aq[4 * j] / inv_n, aq[4 * j + 1] / inv_n, aq[4 * j + 2] / inv_n, aq[4 * j + 3] / inv_n);
-        dk[j] = make_float4(ak[4 * j] / inv_n, ak[4 * j + 1] / inv_n, ak[4 * j + 2] / inv_n, ak[4 * j + 3] / inv_n);
+    for (int i = 0; i < V / 4; ++i) {
+        dq[i] = make_float4(aq[4 * i] / n, aq[4 * i + 1] / n, aq[4 * i + 2] / n, aq[4 * i + 3] / n);
+        dk[i] = make_float4(ak[4 * i] / n, ak[4 * i + 1] / n, ak[4 * i + 2] / n, ak[4 * i + 3] / n);
     }
 }
 
@@ -371,6 +383,7 @@ __global__ void __launch_bounds__(256, 2) route_topk_kernel(const S *__restrict_
                                                          int chunk, float scale)
 {
     extern __shared__ float4 smem4[];
+    grid_dependency_wait();
     constexpr int NR = RowsPerPass<E>::value;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row_blocks = (R + rows - 1) / rows;
@@ -407,6 +420,7 @@ __global__ void __launch_bounds__(256) route_topk_wide_kernel(const float *__res
                                                               int R, int C, int topk, int P, float scale)
 {
     extern __shared__ unsigned long long keys[];
+    grid_dependency_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
     const int row_blocks = (R + nwarps - 1) / nwarps;
     const int b = blockIdx.x / row_blocks;
@@ -444,17 +458,23 @@ template <typename T>
 __global__ void __launch_bounds__(kMeansThreads, 2) region_means_kernel(const MeansArgs a)
 {
     extern __shared__ float4 smem4[];
+    grid_dependency_wait();
     const long long i0 = (long long)blockIdx.x * a.rpc;
     const int nreg = (int)min((long long)a.rpc, (long long)a.B * a.R - i0);
     region_means_block<T>(a, reinterpret_cast<float *>(smem4), i0, nreg);
 }
 
-// Means of rs <= 16 regions: one thread per (region, 16-byte vector).
+// Means of rs <= 16 regions: `lanes` threads per (region, 16-byte vector). total is a multiple
+// of 32 (threads past the last region read region 0 and write nothing), so whole warps take part
+// in the butterfly.
 template <typename T>
-__global__ void __launch_bounds__(kMeansThreads) region_means_flat_kernel(const MeansArgs a, long long total)
+__global__ void __launch_bounds__(kMeansThreads, 3) region_means_flat_kernel(const MeansArgs a, long long total,
+                                                                         long long real, int lanes)
 {
+    grid_dependency_wait();
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid < total) region_means_flat<T>(a, gid);
+    if (gid >= total) return;
+    region_means_flat<T>(a, gid < real ? gid : gid % lanes, lanes, gid < real);
 }
 
 // ============================================================================ launchers
@@ -517,14 +537,16 @@ cudaError_t launch_region_means(const void *q, const void *k, float *qm, float *
     const MeansArgs a = means_args(q, k, qm, km, g, bf16);
     if ((long long)a.wr * (g.C / (bf16 ? 8 : 4)) > kMaxMeansVectors) return cudaErrorInvalidConfiguration;
     if (g.rs <= 16) {
-        const long long total = (long long)g.B * g.R * (g.C / (bf16 ? 8 : 4));
+        const int lanes = (g.hr == 2 || g.hr == 4 || g.hr == 8) ? g.hr : 1;
+        const long long real = (long long)g.B * g.R * (g.C / (bf16 ? 8 : 4)) * lanes;
+        const long long total = (real + 31) / 32 * 32;
         const long long blocks = (total + kMeansThreads - 1) / kMeansThreads;
         if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
         if (bf16)
-            region_means_flat_kernel<__nv_bfloat16><<<(unsigned)blocks, kMeansThreads, 0, stream>>>(a, total);
-        else
-            region_means_flat_kernel<float><<<(unsigned)blocks, kMeansThreads, 0, stream>>>(a, total);
-        return cudaGetLastError();
+            return launch_pdl(region_means_flat_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3(kMeansThreads), 0,
+                              stream, a, total, real, lanes);
+        return launch_pdl(region_means_flat_kernel<float>, dim3((unsigned)blocks), dim3(kMeansThreads), 0, stream, a,
+                          total, real, lanes);
     }
     const size_t smem = means_part_bytes(a);
     static int granted[2][64] = {{0}};
@@ -534,10 +556,9 @@ cudaError_t launch_region_means(const void *q, const void *k, float *qm, float *
     const long long blocks = means_blocks(a);
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     if (bf16)
-        region_means_kernel<__nv_bfloat16><<<(unsigned)blocks, kMeansThreads, smem, stream>>>(a);
-    else
-        region_means_kernel<float><<<(unsigned)blocks, kMeansThreads, smem, stream>>>(a);
-    return cudaGetLastError();
+        return launch_pdl(region_means_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3(kMeansThreads), smem, stream,
+                          a);
+    return launch_pdl(region_means_kernel<float>, dim3((unsigned)blocks), dim3(kMeansThreads), smem, stream, a);
 }
 
 template <int E, bool ROUNDS, typename S>
@@ -548,9 +569,8 @@ static cudaError_t launch_topk_typed(const S *qm, const S *km, int32_t *idx, con
     cudaError_t e = raise_smem_limit(route_topk_kernel<E, ROUNDS, S>, smem, granted);
     if (e != cudaSuccess) return e;
     const long long blocks = (long long)((g.R + rows - 1) / rows) * g.B;
-    route_topk_kernel<E, ROUNDS, S><<<(unsigned)blocks, 256, smem, stream>>>(qm, km, idx, g.R, g.C, g.topk, rows, chunk,
-                                                                             scale);
-    return cudaGetLastError();
+    return launch_pdl(route_topk_kernel<E, ROUNDS, S>, dim3((unsigned)blocks), dim3(256), smem, stream, qm, km, idx, g.R,
+                      g.C, g.topk, rows, chunk, scale);
 }
 
 template <int E, typename S>
@@ -601,9 +621,8 @@ cudaError_t launch_route_topk(const float *qm, const float *km, int32_t *idx, co
     if (warps > 8) warps = 8;
     const long long blocks = (long long)((g.R + warps - 1) / warps) * g.B;
     const float scale = (float)(1.0 / sqrt((double)g.C));
-    route_topk_wide_kernel<<<(unsigned)blocks, warps * 32, (size_t)warps * P * 8, stream>>>(qm, km, idx, g.R, g.C,
-                                                                                             g.topk, P, scale);
-    return cudaGetLastError();
+    return launch_pdl(route_topk_wide_kernel, dim3((unsigned)blocks), dim3(warps * 32), (size_t)warps * P * 8, stream, qm,
+                      km, idx, g.R, g.C, g.topk, P, scale);
 }
 
 }  // namespace bra
