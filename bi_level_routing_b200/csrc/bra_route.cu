@@ -350,19 +350,34 @@ __device__ __forceinline__ void stage_rows(const S *__restrict__ src0, int rows0
                                            float *dst, int C, int c0, int cn, int dst_stride)
 {
     constexpr int V = 16 / sizeof(S);
-    const int cv = cn / V;
-    const int n0 = rows0 * cv;
-    const int total = (rows0 + rows1) * cv;
+    const int cv = cn / V;  // 16-byte vectors per row window
+    const int nrows = rows0 + rows1;
+    auto load = [&](int row, int col) -> uint4 {
+        const S *src = row < rows0 ? src0 + (size_t)row * C : src1 + (size_t)(row - rows0) * C;
+        const uint4 *p = reinterpret_cast<const uint4 *>(src + c0 + col * V);
+        return L2 ? __ldcg(p) : __ldg(p);
+    };
+    if (blockDim.x % cv == 0) {
+        // each thread keeps one column and steps through the rows: no division per element
+        const int col = threadIdx.x % cv, step = blockDim.x / cv;
+        for (int r0 = threadIdx.x / cv; r0 < nrows; r0 += 8 * step) {
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (r0 + u * step < nrows) v[u] = load(r0 + u * step, col);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (r0 + u * step < nrows) store_as_f32(dst + (size_t)(r0 + u * step) * dst_stride + col * V, v[u], S());
+        }
+        return;
+    }
+    const int total = nrows * cv;
     for (int e0 = threadIdx.x; e0 < total; e0 += 8 * blockDim.x) {
         uint4 v[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int e = e0 + u * blockDim.x;
-            if (e < total) {
-                const S *src = e < n0 ? src0 + (size_t)(e / cv) * C : src1 + (size_t)((e - n0) / cv) * C;
-                const uint4 *p = reinterpret_cast<const uint4 *>(src + c0 + (e % cv) * V);
-                v[u] = L2 ? __ldcg(p) : __ldg(p);
-            }
+            if (e < total) v[u] = load(e / cv, e % cv);
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -580,14 +595,16 @@ static cudaError_t launch_topk_e(const S *qm, const S *km, int32_t *idx, const G
     const bool rounds = topk_by_rounds(E, g.topk);
     // one pass of the row routine per warp: every warp of the CTA busy, the image's key means
     // staged once per channel window; the window is the whole row when the staged rows fit in
-    // 100 KB, else the widest multiple of 32 channels that does (a row stride of 4 mod 32 words
-    // keeps the lanes' 16-byte key loads free of bank conflicts)
+    // 100 KB, else the widest power-of-two multiple of 32 channels that does (a row stride of
+    // 4 mod 32 words keeps the lanes' 16-byte key loads free of bank conflicts, and the window's
+    // 16-byte vectors divide the CTA, which keeps the staging free of divisions)
     const int rows = 8 * RowsPerPass<E>::value;
     const long long per_col = (long long)(g.R + rows) * sizeof(float);
     int chunk = g.C;
     if (per_col * (chunk + 4) > 100 * 1024) {
-        chunk = (int)((100 * 1024) / per_col - 4) / 32 * 32;
-        if (chunk < 32) return cudaErrorInvalidConfiguration;  // R is at most 256 here
+        chunk = 32;
+        while (chunk * 2 < g.C && per_col * (chunk * 2 + 4) <= 100 * 1024) chunk *= 2;
+        if (per_col * (chunk + 4) > 100 * 1024) return cudaErrorInvalidConfiguration;  // R is at most 256 here
     }
     const size_t smem = (size_t)per_col * (chunk + 4);
     return rounds ? launch_topk_typed<E, true, S>(qm, km, idx, g, rows, chunk, scale, smem, stream)
