@@ -94,63 +94,68 @@ __device__ __forceinline__ void region_means_block(const MeansArgs &a, float *pa
     }
 }
 
-// Small regions (rs <= 16): `lanes` consecutive threads per (region, 16-byte vector of
-// channels), thread j summing region rows j, j + lanes, ... in order (all their tokens' loads in
-// flight at once), then a butterfly over the lanes adds the row sums in a fixed order. lanes is
-// hr when hr is a power of two up to 8, else 1. No shared memory, no barrier.
+// Small regions (rs <= 16): one CTA per region. `lanes` consecutive threads per 16-byte vector
+// of channels (lanes = hr when hr is 2, 4 or 8, else 1); thread j of a vector sums region rows
+// j, j + lanes, ... token by token in order, with up to 4 tokens' loads of q and of k in flight,
+// then a butterfly over the lanes adds the row sums in a fixed order. No shared memory, no
+// barrier, and no division per token.
 template <typename T>
-__device__ __forceinline__ void region_means_flat(const MeansArgs &a, long long gid, int lanes, bool write)
+__device__ __forceinline__ void region_means_small(const MeansArgs &a, int64_t b, int r, int lshift)
 {
     constexpr int V = Vec16<T>::N;
-    constexpr int TOK = 4;  // tokens whose loads are in flight together
+    constexpr int TOK = 4;
+    const int lanes = 1 << lshift;
+    const int j = threadIdx.x & (lanes - 1);
     const int vpt = a.C / V;
-    const int j = (int)(gid % lanes);
-    const long long item = gid / lanes;
-    const long long flat = item / vpt;
-    const int v = (int)(item % vpt);
-    const int64_t b = flat / a.R;
-    const int r = (int)(flat % a.R);
     const int ry = r / a.n_win, rx = r % a.n_win;
-    const int64_t base = ((b * a.H + (int64_t)ry * a.hr) * a.W + (int64_t)rx * a.wr) * a.C + (int64_t)v * V;
-    const T *pq = static_cast<const T *>(a.q) + base;
-    const T *pk = static_cast<const T *>(a.k) + base;
-    const int per = (a.hr / lanes) * a.wr;  // tokens of this thread: its rows, row by row
-    float aq[V], ak[V];
-#pragma unroll
-    for (int i = 0; i < V; ++i) aq[i] = ak[i] = 0.f;
-    for (int t0 = 0; t0 < per; t0 += TOK) {
-        uint4 rq[TOK], rk[TOK];
-#pragma unroll
-        for (int u = 0; u < TOK; ++u)
-            if (t0 + u < per) {
-                const int t = t0 + u;
-                const int y = j + (t / a.wr) * lanes, x = t % a.wr;
-                const int64_t off = ((int64_t)y * a.W + x) * a.C;
-                rq[u] = Vec16<T>::load_raw(pq + off);
-                rk[u] = Vec16<T>::load_raw(pk + off);
-            }
-#pragma unroll
-        for (int u = 0; u < TOK; ++u)
-            if (t0 + u < per) {
-                Vec16<T>::accumulate(rq[u], aq);
-                Vec16<T>::accumulate(rk[u], ak);
-            }
-    }
-    for (int off = 1; off < lanes; off <<= 1) {
-#pragma unroll
-        for (int i = 0; i < V; ++i) {
-            aq[i] += __shfl_xor_sync(0xffffffffu, aq[i], off);
-            ak[i] += __shfl_xor_sync(0xffffffffu, ak[i], off);
-        }
-    }
-    if (j != 0 || !write) return;
+    const int64_t base = ((b * a.H + (int64_t)ry * a.hr) * a.W + (int64_t)rx * a.wr) * a.C;
+    const int64_t row_stride = (int64_t)a.W * a.C;
     const float n = (float)(a.hr * a.wr);
-    float4 *dq = reinterpret_cast<float4 *>(a.qm + flat * a.C + v * V);
-    float4 *dk = reinterpret_cast<float4 *>(a.km + flat * a.C + v * V);
+    const int step = blockDim.x >> lshift;
+    // the same trip count for every lane of a warp, so that all of them take part in the
+    // butterfly; a lane past the last vector loads and stores nothing
+    for (int v0 = 0; v0 < vpt; v0 += step) {
+        const int v = v0 + (threadIdx.x >> lshift);
+        const bool live = v < vpt;
+        const T *pq = static_cast<const T *>(a.q) + base + (int64_t)(live ? v : 0) * V;
+        const T *pk = static_cast<const T *>(a.k) + base + (int64_t)(live ? v : 0) * V;
+        float aq[V], ak[V];
 #pragma unroll
-    for (int i = 0; i < V / 4; ++i) {
-        dq[i] = make_float4(aq[4 * i] / n, aq[4 * i + 1] / n, aq[4 * i + 2] / n, aq[4 * i + 3] / n);
-        dk[i] = make_float4(ak[4 * i] / n, ak[4 * i + 1] / n, ak[4 * i + 2] / n, ak[4 * i + 3] / n);
+        for (int i = 0; i < V; ++i) aq[i] = ak[i] = 0.f;
+        for (int y = j; live && y < a.hr; y += lanes) {
+            const T *rq0 = pq + (int64_t)y * row_stride, *rk0 = pk + (int64_t)y * row_stride;
+            for (int x0 = 0; x0 < a.wr; x0 += TOK) {
+                uint4 rq[TOK], rk[TOK];
+#pragma unroll
+                for (int u = 0; u < TOK; ++u)
+                    if (x0 + u < a.wr) {
+                        rq[u] = Vec16<T>::load_raw(rq0 + (int64_t)(x0 + u) * a.C);
+                        rk[u] = Vec16<T>::load_raw(rk0 + (int64_t)(x0 + u) * a.C);
+                    }
+#pragma unroll
+                for (int u = 0; u < TOK; ++u)
+                    if (x0 + u < a.wr) {
+                        Vec16<T>::accumulate(rq[u], aq);
+                        Vec16<T>::accumulate(rk[u], ak);
+                    }
+            }
+        }
+        for (int off = 1; off < lanes; off <<= 1) {
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                aq[i] += __shfl_xor_sync(0xffffffffu, aq[i], off);
+                ak[i] += __shfl_xor_sync(0xffffffffu, ak[i], off);
+            }
+        }
+        if (live && j == 0) {
+            float4 *dq = reinterpret_cast<float4 *>(a.qm + (b * a.R + r) * a.C + v * V);
+            float4 *dk = reinterpret_cast<float4 *>(a.km + (b * a.R + r) * a.C + v * V);
+#pragma unroll
+            for (int i = 0; i < V / 4; ++i) {
+                dq[i] = make_float4(aq[4 * i] / n, aq[4 * i + 1] / n, aq[4 * i + 2] / n, aq[4 * i + 3] / n);
+                dk[i] = make_float4(ak[4 * i] / n, ak[4 * i + 1] / n, ak[4 * i + 2] / n, ak[4 * i + 3] / n);
+            }
+        }
     }
 }
 
@@ -479,17 +484,13 @@ __global__ void __launch_bounds__(kMeansThreads, 2) region_means_kernel(const Me
     region_means_block<T>(a, reinterpret_cast<float *>(smem4), i0, nreg);
 }
 
-// Means of rs <= 16 regions: `lanes` threads per (region, 16-byte vector). total is a multiple
-// of 32 (threads past the last region read region 0 and write nothing), so whole warps take part
-// in the butterfly.
+// Means of rs <= 16 regions: one CTA per region, a multiple of 32 threads (every warp whole for
+// the butterfly).
 template <typename T>
-__global__ void __launch_bounds__(kMeansThreads, 3) region_means_flat_kernel(const MeansArgs a, long long total,
-                                                                         long long real, int lanes)
+__global__ void __launch_bounds__(256) region_means_small_kernel(const MeansArgs a, int lshift)
 {
     grid_dependency_wait();
-    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= total) return;
-    region_means_flat<T>(a, gid < real ? gid : gid % lanes, lanes, gid < real);
+    region_means_small<T>(a, blockIdx.x / a.R, blockIdx.x % a.R, lshift);
 }
 
 // ============================================================================ launchers
@@ -552,16 +553,17 @@ cudaError_t launch_region_means(const void *q, const void *k, float *qm, float *
     const MeansArgs a = means_args(q, k, qm, km, g, bf16);
     if ((long long)a.wr * (g.C / (bf16 ? 8 : 4)) > kMaxMeansVectors) return cudaErrorInvalidConfiguration;
     if (g.rs <= 16) {
-        const int lanes = (g.hr == 2 || g.hr == 4 || g.hr == 8) ? g.hr : 1;
-        const long long real = (long long)g.B * g.R * (g.C / (bf16 ? 8 : 4)) * lanes;
-        const long long total = (real + 31) / 32 * 32;
-        const long long blocks = (total + kMeansThreads - 1) / kMeansThreads;
+        const int lshift = g.hr == 8 ? 3 : (g.hr == 4 ? 2 : (g.hr == 2 ? 1 : 0));
+        long long threads = ((long long)(g.C / (bf16 ? 8 : 4)) << lshift);
+        threads = (threads + 31) / 32 * 32;
+        if (threads > 256) threads = 256;
+        const long long blocks = (long long)g.B * g.R;
         if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
         if (bf16)
-            return launch_pdl(region_means_flat_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3(kMeansThreads), 0,
-                              stream, a, total, real, lanes);
-        return launch_pdl(region_means_flat_kernel<float>, dim3((unsigned)blocks), dim3(kMeansThreads), 0, stream, a,
-                          total, real, lanes);
+            return launch_pdl(region_means_small_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3((unsigned)threads),
+                              0, stream, a, lshift);
+        return launch_pdl(region_means_small_kernel<float>, dim3((unsigned)blocks), dim3((unsigned)threads), 0, stream, a,
+                          lshift);
     }
     const size_t smem = means_part_bytes(a);
     static int granted[2][64] = {{0}};
