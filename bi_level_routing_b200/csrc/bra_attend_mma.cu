@@ -539,7 +539,10 @@ __global__ void __launch_bounds__(256) attend_dense_mma_kernel(const __grid_cons
             flag_error(a.err, kErrIndex);
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < a.R * a.R; e += blockDim.x) lw[e] = cnt[e] ? log2f((float)cnt[e]) : -INFINITY;
+    for (int e = threadIdx.x; e < a.R * a.R; e += blockDim.x) {
+        const int c = cnt[e];
+        lw[e] = c == 1 ? 0.f : (c ? log2f((float)c) : -INFINITY);  // log2(1) = 0 exactly: skip the call
+    }
     __syncthreads();
 
     const bool alive = mbar_wait(bar, 0, a.err);

@@ -53,3 +53,18 @@ def test_no_alloc_route_rejects_sizes_beyond_its_scratch():
     status = L.bra_route_noalloc(fake, fake, fake, w.B, w.H, w.W, w.C, w.n_win, w.topk, 1, None)
     assert status == 2  # BRA_ERR_UNSUPPORTED
     assert b"bytes of scratch" in L.bra_last_error_message()
+
+
+def test_one_token_regions_route_the_same_from_the_tokens():
+    """For one-token regions bra_route reads q and k directly (their means are the tokens, widened
+    exactly to fp32); bra_route_noalloc still runs the means kernel. The indices must agree bit
+    for bit, bf16 and fp32."""
+    L = _lib()
+    for w in (WORKLOADS["stage4"].with_(B=8), WORKLOADS["stage4"].with_(B=3, dtype="f32")):
+        _, (q, k, _) = make(w)
+        ref = bra.route(q, k, w.n_win, w.topk)
+        idx = torch.full_like(ref, -7)
+        assert _route_noalloc(L, q, k, idx, w.n_win, w.topk) == 0, L.bra_last_error_message()
+        torch.cuda.synchronize()
+        assert torch.equal(idx, ref), f"{w.name} {w.dtype}: the token path differs from the means path"
+
