@@ -1,15 +1,17 @@
-"""Benchmark of the BRA forward pass (bra_forward = bra_route + bra_attend) on B200.
+"""Benchmark of the BRA forward pass (bra_forward) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload stage1] [--impl ours|reference]
 
-A step is one pass of the whole hot path (region means, affinity + top-k, gather-attention)
-over one batch of the workload. Inputs are seeded synthetic data of the workload's shape,
-resident in HBM before timing starts; the step rotates through enough input/output buffer
-sets (copies of the batch, rolled along the image axis) that the set it reads was evicted
-from L2 by the others. The K timed steps are captured as one CUDA graph (eager launches if
-capture is refused), with timing events recorded as graph nodes on the launching stream
-around every route and every attention call. With N > 1 (torchrun), each rank runs its own
-batch (weak scaling, no data-path collective) and the time is the max over ranks.
+A step is one bra_forward call: the whole hot path (region means, affinity + top-k,
+gather-attention) over one batch of the workload. Inputs are seeded synthetic data of the
+workload's shape, resident in HBM before timing starts; the step rotates through enough
+input/output buffer sets (copies of the batch, rolled along the image axis) that the set it
+reads was evicted from L2 by the others. The K timed steps are captured as one CUDA graph
+(eager launches if capture is refused) with a timing event before the first and after the
+last, on the launching stream; the median of several such runs is reported. A second graph of
+bra_route then bra_attend, with an event around every call, gives the per-kernel breakdown.
+With N > 1 (torchrun), each rank runs its own batch (weak scaling, no data-path collective)
+and the time is the max over ranks.
 
 Prints one JSON line on rank 0. `--impl reference` times the CPU oracle on the host cores
 instead (a bounded sample of the same workload per step).
@@ -238,18 +240,24 @@ def main():
         q, k, v, out, idx = s
         bra.attend(q, k, v, idx, w.heads, w.n_win, out=out)
 
+    def forward(s):
+        q, k, v, out, idx = s
+        bra.forward(q, k, v, w.n_win, w.topk, w.heads, out=out, idx=idx)
+
     # eager warm-up (also initialises the library's per-device state before any capture)
     for i in range(max(3, args.warmup)):
+        forward(sets[i % nsets])
         route(sets[i % nsets])
         attend(sets[i % nsets])
     torch.cuda.synchronize()
 
 
-    # ---- the timed region: K steps [route, attend], captured as ONE CUDA graph with a timing
+    # ---- the timed region: K steps of bra_forward, captured as ONE CUDA graph with a timing
     # event (an external event-record node) before the first and after the last, so that host
     # launch overhead does not pace the GPU and consecutive kernels keep their programmatic
-    # (overlapping) launches; eager launches if capture is refused. A second graph of the same
-    # steps with an event around every route and every attention call gives the breakdown.
+    # (overlapping) launches; eager launches if capture is refused. A second graph of K steps
+    # of bra_route then bra_attend, with an event around every call, gives the breakdown (the
+    # attention kernel's duration; in bra_forward the same kernel may also do the routing).
     K = args.steps
     ev_start = torch.cuda.Event(enable_timing=True, external=True)
     ev_stop = torch.cuda.Event(enable_timing=True, external=True)
@@ -260,9 +268,7 @@ def main():
     def record_steps():
         ev_start.record()
         for i in range(K):
-            s = sets[i % nsets]
-            route(s)
-            attend(s)
+            forward(sets[i % nsets])
         ev_stop.record()
 
     def record_breakdown():
@@ -343,8 +349,7 @@ def main():
             with torch.cuda.graph(gw):
                 ev_w0.record()
                 for _ in range(K):
-                    route(sets[0])
-                    attend(sets[0])
+                    forward(sets[0])
                 ev_w1.record()
             gw.replay()
             torch.cuda.synchronize()

@@ -57,6 +57,16 @@ cudaError_t launch_region_means(const void *q, const void *k, float *qm, float *
                                 bool bf16, int num_sms, cudaStream_t stream);
 
 
+// topk rounds of argmax cost about topk * (E + 20) instructions; the bitonic network
+// log2(P) (log2(P) + 1) / 2 stages of about 8 E.
+inline bool topk_by_rounds(int E, int topk)
+{
+    int lg = 5;
+    while ((1 << lg) < 32 * E) ++lg;
+    const long long stages = (long long)lg * (lg + 1) / 2;
+    return (long long)topk * (E + 20) <= stages * E * 8;
+}
+
 // Affinity rows and top-k straight from q and k when a region is one token (rs == 1, R <= 256):
 // the means are the tokens, widened exactly to fp32, so the index is the same as from the means.
 cudaError_t launch_route_topk_tokens(const void *q, const void *k, int32_t *idx, const Geometry &g, bool bf16,

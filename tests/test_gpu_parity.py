@@ -64,6 +64,9 @@ SMALL = [
     ("tiny_f32", 1, 28, 28, 64, 2, 7, 4, "f32"),
     ("max_regions_bf16", 1, 32, 32, 8, 1, 32, 7, "bf16"),
     ("topk_all_256_bf16", 1, 16, 16, 32, 1, 16, 256, "bf16"),
+    # 64-token regions, 64 channels (the tcgen05 kernel) with topk > 1
+    ("rs64_c64_bf16", 3, 32, 32, 64, 2, 4, 3, "bf16"),
+    ("stage1_topk4_bf16", 2, 56, 56, 64, 2, 7, 4, "bf16"),
 ]
 
 
