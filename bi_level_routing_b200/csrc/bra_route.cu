@@ -48,13 +48,13 @@ __device__ __forceinline__ void region_means_block(const MeansArgs &a, float *pa
     const int nvec = a.wr * vpt;
     const int grp = threadIdx.x / a.slots;
     if (grp < nreg) {
-        const long long flat = i0 + grp;
-        const int64_t b = flat / a.R;
-        const int r = (int)(flat % a.R);
+        const int flat = (int)i0 + grp;  // B * R < 2^31 (checked by the launcher)
+        const int b = flat / a.R;
+        const int r = flat - b * a.R;
         const int ry = r / a.n_win, rx = r % a.n_win;
         const int64_t row_stride = (int64_t)a.W * C;
-        const int64_t base = ((b * a.H + (int64_t)ry * a.hr) * a.W + (int64_t)rx * a.wr) * C;
-        for (int v = threadIdx.x % a.slots; v < nvec; v += a.slots) {
+        const int64_t base = (((int64_t)b * a.H + (int64_t)ry * a.hr) * a.W + (int64_t)rx * a.wr) * C;
+        for (int v = threadIdx.x - grp * a.slots; v < nvec; v += a.slots) {
             float aq[V], ak[V];
 #pragma unroll
             for (int i = 0; i < V; ++i) aq[i] = ak[i] = 0.f;
@@ -88,7 +88,7 @@ __device__ __forceinline__ void region_means_block(const MeansArgs &a, float *pa
     __syncthreads();
     const float rs = (float)(a.hr * a.wr);
     for (int e = threadIdx.x; e < nreg * 2 * C; e += blockDim.x) {
-        const int g = e / (2 * C), t = (e / C) & 1, c = e % C;
+        const int qc = e / C, g = qc >> 1, t = qc & 1, c = e - qc * C;
         float s = 0.f;
         for (int xx = 0; xx < a.wr; ++xx) s += part[((size_t)(2 * g + t) * a.wr + xx) * C + c];
         (t ? a.km : a.qm)[(i0 + g) * C + c] = s / rs;
@@ -330,6 +330,7 @@ cudaError_t launch_region_means(const void *q, const void *k, float *qm, float *
     (void)num_sms;
     const MeansArgs a = means_args(q, k, qm, km, g, bf16);
     if ((long long)a.wr * (g.C / (bf16 ? 8 : 4)) > kMaxMeansVectors) return cudaErrorInvalidConfiguration;
+    if ((long long)g.B * g.R > 0x7fffffffLL) return cudaErrorInvalidConfiguration;  // 32-bit region index
     if (g.rs <= 16) {
         const int lshift = g.hr == 8 ? 3 : (g.hr == 4 ? 2 : (g.hr == 2 ? 1 : 0));
         long long threads = ((long long)(g.C / (bf16 ? 8 : 4)) << lshift);
