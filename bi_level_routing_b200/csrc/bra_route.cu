@@ -10,7 +10,8 @@
 // top-k in registers: rounds of warp argmax for a small k, a shuffle bitonic network otherwise. Keys are 64-bit
 // (order-preserving float bits, then the complement of the region index), which gives
 // affinity-descending order, ties to the lower region and NaN after every number,
-// deterministically.
+// deterministically. One-token regions skip the means: the routing kernels read q and k
+// themselves, and in bf16 (up to 64 regions) a tensor-core kernel forms the dot products.
 #include "bra_device.cuh"
 #include "bra_launch.h"
 #include "bra_routing.cuh"
@@ -401,10 +402,110 @@ static cudaError_t launch_topk_any(const S *qm, const S *km, int32_t *idx, const
     return launch_topk_e<8, S>(qm, km, idx, g, stream);
 }
 
+// One-token regions in bf16 (rs = 1, R <= 64, C % 32 == 0): the means are the tokens, and the
+// product of two bf16 values is exact in fp32, so the affinities are fp32 sums of exact products
+// whichever unit forms them. Here the tensor cores form them: one CTA per (image, 16 query
+// rows); warp w takes the 32-channel chunks w, w + 8, ... and computes the 16 x 64 tile of
+// partial dot products with mma.sync m16n8k16 (bf16 in, fp32 accumulate) straight from 16-byte
+// global loads, every load of the warp in flight at once. Within a chunk, lane (g, c) loads
+// channels 8 c .. 8 c + 7 of query rows g and g + 8 and of key g of each 8-key tile; the MMA's
+// k slots take these channels in the same permuted order for A and B, which a sum over
+// channels does not see. The eight partial tiles are added in warp order in shared memory, then
+// warp w selects the top-k of rows 2 w and 2 w + 1 as every routing kernel does.
+template <bool ROUNDS>
+__global__ void __launch_bounds__(256, 2) route_tokens_mma_kernel(const __nv_bfloat16 *__restrict__ q,
+                                                               const __nv_bfloat16 *__restrict__ k,
+                                                               int32_t *__restrict__ idx, int R, int C, int topk,
+                                                               float scale)
+{
+    constexpr int kWarps = 8, kPad = 68;  // row stride of a partial tile (floats)
+    __shared__ float part[kWarps][16][kPad];
+    grid_dependency_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int row_blocks = (R + 15) >> 4;
+    const int b = blockIdx.x / row_blocks;
+    const int r0 = (blockIdx.x - b * row_blocks) * 16;
+    const int ntiles = (R + 7) >> 3;
+    const __nv_bfloat16 *qb = q + (int64_t)b * R * C;
+    const __nv_bfloat16 *kb = k + (int64_t)b * R * C;
+    // offsets inside the image (R * C < 2^31, checked by the launcher); rows and keys past R
+    // read row R - 1, and their results are never selected
+    const int ra = min(r0 + g, R - 1) * C + 8 * c, rb = min(r0 + g + 8, R - 1) * C + 8 * c;
+    int kr[8];
+#pragma unroll
+    for (int n = 0; n < 8; ++n) kr[n] = min(8 * n + g, R - 1) * C + 8 * c;
+    float acc[8][4];
+#pragma unroll
+    for (int n = 0; n < 8; ++n)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[n][j] = 0.f;
+    for (int col = 32 * warp; col < C; col += 32 * kWarps) {
+        const uint4 xa = __ldg(reinterpret_cast<const uint4 *>(qb + ra + col));
+        const uint4 xb = __ldg(reinterpret_cast<const uint4 *>(qb + rb + col));
+        uint4 y[8];
+#pragma unroll
+        for (int n = 0; n < 8; ++n)
+            if (n < ntiles) y[n] = __ldg(reinterpret_cast<const uint4 *>(kb + kr[n] + col));
+        const uint32_t a0[4] = {xa.x, xb.x, xa.y, xb.y};  // k slots 2c, 2c+1 | 2c+8, 2c+9: channels 8c..8c+3
+        const uint32_t a1[4] = {xa.z, xb.z, xa.w, xb.w};  // channels 8c+4 .. 8c+7
+#pragma unroll
+        for (int n = 0; n < 8; ++n)
+            if (n < ntiles) {
+                mma_bf16_16816(acc[n], a0, y[n].x, y[n].y);
+                mma_bf16_16816(acc[n], a1, y[n].z, y[n].w);
+            }
+    }
+    // acc[n][0..1]: row g, keys 8 n + 2 c, + 1; acc[n][2..3]: row g + 8, the same keys
+#pragma unroll
+    for (int n = 0; n < 8; ++n)
+        if (n < ntiles) {
+            *reinterpret_cast<float2 *>(&part[warp][g][8 * n + 2 * c]) = make_float2(acc[n][0], acc[n][1]);
+            *reinterpret_cast<float2 *>(&part[warp][g + 8][8 * n + 2 * c]) = make_float2(acc[n][2], acc[n][3]);
+        }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int rr = 2 * warp + i;
+        if (r0 + rr >= R) break;
+        unsigned long long key[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int s = 32 * e + lane;
+            float d = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) d += (s < 8 * ntiles) ? part[w][rr][s] : 0.f;
+            key[e] = s < R ? routing_key(d * scale, s) : 0ull;
+        }
+        select_topk<2, ROUNDS>(key, topk, idx + ((int64_t)b * R + r0 + rr) * topk, lane);
+    }
+}
+
+bool route_tokens_mma_supports(const Geometry &g, bool bf16)
+{
+    return bf16 && g.rs == 1 && g.R <= 64 && g.C % 32 == 0 && (long long)g.R * g.C < (1LL << 31);
+}
+
+static cudaError_t launch_route_tokens_mma(const __nv_bfloat16 *q, const __nv_bfloat16 *k, int32_t *idx,
+                                           const Geometry &g, cudaStream_t stream)
+{
+    const long long blocks = (long long)g.B * ((g.R + 15) / 16);
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const float scale = (float)(1.0 / sqrt((double)g.C));
+    if (topk_by_rounds(2, g.topk))
+        return launch_pdl(route_tokens_mma_kernel<true>, dim3((unsigned)blocks), dim3(256), 0, stream, q, k, idx, g.R,
+                          g.C, g.topk, scale);
+    return launch_pdl(route_tokens_mma_kernel<false>, dim3((unsigned)blocks), dim3(256), 0, stream, q, k, idx, g.R,
+                      g.C, g.topk, scale);
+}
+
 cudaError_t launch_route_topk_tokens(const void *q, const void *k, int32_t *idx, const Geometry &g, bool bf16,
                                      cudaStream_t stream)
 {
     if (g.rs != 1 || g.R > 256) return cudaErrorInvalidConfiguration;
+    if (route_tokens_mma_supports(g, bf16))
+        return launch_route_tokens_mma(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), idx,
+                                       g, stream);
     return bf16 ? launch_topk_any<__nv_bfloat16>(static_cast<const __nv_bfloat16 *>(q),
                                                  static_cast<const __nv_bfloat16 *>(k), idx, g, stream)
                 : launch_topk_any<float>(static_cast<const float *>(q), static_cast<const float *>(k), idx, g, stream);

@@ -13,10 +13,12 @@
 // The scratch is g_route_scratch below: kNoAllocScratchBytes (8 MiB) of fp32 space for the
 // query and key region means, 2 * B * R * C floats. Every GPU that loads this library
 // holds that array until the process exits. Calls that need more are rejected with
-// BRA_ERR_UNSUPPORTED before anything runs. All calls on a device share the one array and
-// it keeps the last call's contents; the kernels overwrite every element they read, so
-// nothing needs clearing between calls. Two calls whose kernels overlap on the GPU (two
-// streams, or two host threads) race on the array: order them on one stream.
+// BRA_ERR_UNSUPPORTED before anything runs. One-token regions (R <= 256) need no scratch:
+// their means are the tokens, and routing reads q and k directly, as in bra_route. All calls
+// on a device share the one array and it keeps the last call's contents; the kernels
+// overwrite every element they read, so nothing needs clearing between calls. Two calls
+// whose kernels overlap on the GPU (two streams, or two host threads) race on the array:
+// order them on one stream.
 #include <cstdio>
 #include <mutex>
 
@@ -90,6 +92,16 @@ bra_status bra_route_noalloc(const void *q, const void *k, int32_t *idx, int B, 
     bra::Geometry g;
     bra_status s = bra::check_route_args(q, k, idx, B, H, W, C, n_win, topk, dtype, &g);
     if (s != BRA_OK || B == 0) return s;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (g.rs == 1 && g.R <= 256) {
+        // one-token regions: the means are the tokens; the same kernels as bra_route, no scratch
+        const cudaError_t e = bra::launch_route_topk_tokens(q, k, idx, g, dtype == BRA_BF16, cs);
+        if (e != cudaSuccess) {
+            bra::set_last_error(std::string("routing kernel: ") + cudaGetErrorString(e));
+            return BRA_ERR_CUDA;
+        }
+        return BRA_OK;
+    }
     const size_t need = (size_t)2 * g.B * g.R * g.C * sizeof(float);
     if (need > kNoAllocScratchBytes) {
         char msg[200];
@@ -104,7 +116,6 @@ bra_status bra_route_noalloc(const void *q, const void *k, int32_t *idx, int B, 
     if ((s = noalloc_setup(&st)) != BRA_OK) return s;
     float *qm = st->scratch;
     float *km = qm + (size_t)g.B * g.R * g.C;
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
     cudaError_t e = bra::launch_region_means(q, k, qm, km, g, dtype == BRA_BF16, st->num_sms, cs);
     if (e == cudaSuccess) e = bra::launch_route_topk(qm, km, idx, g, cs);
     if (e != cudaSuccess) {

@@ -1,7 +1,9 @@
 // bra_routing.cuh -- device routines of the routing step: the 64-bit routing keys, the warp
 // top-k selection, the affinity rows (several rows x several keys per lane) and the staging of
 // mean rows into padded shared-memory rows. Every routing kernel is built from these, so the
-// routing index is the same bits whichever of them computed it.
+// routing index is the same bits whichever of them computed it. The one exception is the
+// tensor-core kernel for one-token bf16 regions, whose sums run in another order; it serves
+// every call of that shape, through either routing entry point.
 #pragma once
 
 #include "bra_device.cuh"

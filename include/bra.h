@@ -108,7 +108,8 @@ bra_status bra_forward(const void *q, const void *k, const void *v, int32_t *idx
    region means (2 * B * n_win^2 * C * 4 bytes) lives in a fixed 8 MiB device array inside
    the library (held by every GPU that loads it until the process exits), and a call that
    needs more returns BRA_ERR_UNSUPPORTED, with the sizes in bra_last_error_message(),
-   before anything runs. The first call on each device finds that array's device address
+   before anything runs. One-token regions (n_win = H = W, n_win^2 <= 256) need no scratch,
+   as in bra_route. The first call on each device finds that array's device address
    (cudaGetSymbolAddress), so make it before any stream capture. All calls on a device share
    the array; calls whose kernels overlap on the GPU race on it, so order them on one stream.
    The paper has no counterpart to this entry point: it is a deployment variant. */

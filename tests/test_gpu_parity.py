@@ -67,6 +67,11 @@ SMALL = [
     # 64-token regions, 64 channels (the tcgen05 kernel) with topk > 1
     ("rs64_c64_bf16", 3, 32, 32, 64, 2, 4, 3, "bf16"),
     ("stage1_topk4_bf16", 2, 56, 56, 64, 2, 7, 4, "bf16"),
+    # one-token regions in bf16 (the tensor-core routing kernel): ragged key tiles and row
+    # blocks with a full sort, one 32-channel chunk, argmax rounds over 512 channels
+    ("rs1_r25_c96_bf16", 3, 5, 5, 96, 3, 5, 25, "bf16"),
+    ("rs1_r64_c32_bf16", 2, 8, 8, 32, 1, 8, 64, "bf16"),
+    ("rs1_r49_c512_topk3_bf16", 2, 7, 7, 512, 16, 7, 3, "bf16"),
 ]
 
 
@@ -172,6 +177,35 @@ def test_route_exact_ties_go_to_the_lower_region():
         for r in range(w.R):
             row = list(gidx[b, r])
             assert row.index(1) < row.index(6) < row.index(12)
+
+
+def test_route_exact_ties_one_token_regions():
+    """One-token regions (routed on the tensor cores in bf16): keys that are copies of one another
+    give exactly equal affinities in every row, and the lower region ranks first."""
+    w = Workload("ties1", 2, 7, 7, 512, 16, 7, 49, "bf16", "iid", 4324)
+    inp = make_inputs(w)
+    for t in ("k_bits", "k"):  # regions (1,2)=9 and (4,2)=30 copy region (0,3)=3
+        inp[t][:, 1, 2, :] = inp[t][:, 0, 3, :]
+        inp[t][:, 4, 2, :] = inp[t][:, 0, 3, :]
+    q, k, _ = device_tensors(inp, w)
+    gidx = bra.route(q, k, w.n_win, w.topk).cpu().numpy()
+    check_routing(gidx, inp["q"], inp["k"], w.n_win, w.topk)
+    for b in range(w.B):
+        for r in range(w.R):
+            row = list(gidx[b, r])
+            i3, i9, i30 = row.index(3), row.index(9), row.index(30)
+            assert i9 == i3 + 1 and i30 == i3 + 2, (b, r, row)
+
+
+def test_route_nan_ranks_last_one_token_regions():
+    w = Workload("nan1", 1, 7, 7, 64, 2, 7, 49, "bf16", "iid", 4325)
+    inp = make_inputs(w)
+    inp["k"][0, 2, 3, 5] = np.nan  # token (2,3) = region 17: column 17 is NaN in every row
+    inp["k_bits"][0, 2, 3, 5] = 0x7FC0
+    q, k, _ = device_tensors(inp, w)
+    gidx = bra.route(q, k, w.n_win, w.topk).cpu().numpy()
+    assert np.all(gidx[0, :, -1] == 17)
+    check_routing(gidx, inp["q"], inp["k"], w.n_win, w.topk)
 
 
 def test_route_nan_ranks_last():

@@ -5,8 +5,8 @@ bra_route: a process that hands all of HBM to its own allocator at start-up, or 
 latency-critical loop that must not take allocator locks or risk an out-of-memory error.
 Its scratch is a fixed array inside the library, shared by every call, so this test makes
 two calls in a row on different shapes and checks that each returns exactly bra_route's
-indices (the same kernels run, so the routing must be bit-identical). It sits in a file of
-its own, collected last.
+indices (the same kernels run, so the routing must be bit-identical). One-token regions need
+no scratch at all. It sits in a file of its own, collected last.
 """
 import ctypes
 
@@ -48,23 +48,26 @@ def test_no_alloc_route_matches_bra_route_on_two_calls_in_a_row():
 
 def test_no_alloc_route_rejects_sizes_beyond_its_scratch():
     L = _lib()
-    w = WORKLOADS["stage4"]  # 2 * 64 * 49 * 512 * 4 bytes = 12.8 MB > 8 MiB
+    # four-token regions, so the means need scratch: 2 * 128 * 49 * 256 * 4 bytes = 12.8 MB > 8 MiB
+    w = WORKLOADS["stage3"].with_(B=128)
+    assert w.H // w.n_win * (w.W // w.n_win) > 1
     fake = 0x10000  # rejected before any use
     status = L.bra_route_noalloc(fake, fake, fake, w.B, w.H, w.W, w.C, w.n_win, w.topk, 1, None)
     assert status == 2  # BRA_ERR_UNSUPPORTED
     assert b"bytes of scratch" in L.bra_last_error_message()
 
 
-def test_one_token_regions_route_the_same_from_the_tokens():
-    """For one-token regions bra_route reads q and k directly (their means are the tokens, widened
-    exactly to fp32); bra_route_noalloc still runs the means kernel. The indices must agree bit
-    for bit, bf16 and fp32."""
+def test_one_token_regions_route_from_the_tokens_without_scratch():
+    """For one-token regions the means are the tokens, so both entry points route from q and k
+    directly and need no scratch: the full stage4 batch, whose fp32 means would not fit the fixed
+    scratch, routes too. The indices must equal bra_route's bit for bit, bf16 (tensor-core
+    kernel) and fp32 (CUDA-core kernel)."""
     L = _lib()
-    for w in (WORKLOADS["stage4"].with_(B=8), WORKLOADS["stage4"].with_(B=3, dtype="f32")):
+    for w in (WORKLOADS["stage4"], WORKLOADS["stage4"].with_(B=3, dtype="f32")):
+        assert w.H == w.n_win and w.W == w.n_win
         _, (q, k, _) = make(w)
         ref = bra.route(q, k, w.n_win, w.topk)
         idx = torch.full_like(ref, -7)
         assert _route_noalloc(L, q, k, idx, w.n_win, w.topk) == 0, L.bra_last_error_message()
         torch.cuda.synchronize()
-        assert torch.equal(idx, ref), f"{w.name} {w.dtype}: the token path differs from the means path"
-
+        assert torch.equal(idx, ref), f"{w.name} {w.dtype}: bra_route_noalloc differs from bra_route"
