@@ -479,7 +479,10 @@ struct DenseArgs {
     float scale_log2;
 };
 
-__global__ void __launch_bounds__(256) attend_dense_mma_kernel(const __grid_constant__ CUtensorMap tq,
+// MIN_CTAS: CTAs per SM the registers are budgeted for (2, or 3 when three CTAs' shared memory
+// fits on an SM).
+template <int MIN_CTAS>
+__global__ void __launch_bounds__(256, MIN_CTAS) attend_dense_mma_kernel(const __grid_constant__ CUtensorMap tq,
                                                                const __grid_constant__ CUtensorMap tk,
                                                                const __grid_constant__ CUtensorMap tv,
                                                                const __grid_constant__ CUtensorMap tout,
@@ -492,9 +495,10 @@ __global__ void __launch_bounds__(256) attend_dense_mma_kernel(const __grid_cons
     uint8_t *sQ = smem;
     uint8_t *sK = sQ + (size_t)nqpad * kRowBytes;
     uint8_t *sV = sK + (size_t)a.npad * kRowBytes;
-    float *lw = reinterpret_cast<float *>(sV + (size_t)a.npad * kRowBytes);  // [R][R] log2(multiplicity)
-    int *cnt = reinterpret_cast<int *>(lw + a.R * a.R);                        // [R][R]
-    uint8_t *reg = reinterpret_cast<uint8_t *>(cnt + a.R * a.R);               // [npad] region of each key
+    // [R][R]: the multiplicity of each (query region, key region) pair, then, in place, its log2
+    int *cnt = reinterpret_cast<int *>(sV + (size_t)a.npad * kRowBytes);
+    float *lw = reinterpret_cast<float *>(cnt);
+    uint8_t *reg = reinterpret_cast<uint8_t *>(cnt + a.R * a.R);  // [npad] region of each key
     uint64_t *bar = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(reg + a.npad) + 7) & ~uintptr_t(7));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -530,13 +534,16 @@ __global__ void __launch_bounds__(256) attend_dense_mma_kernel(const __grid_cons
         reg[t] = t < a.N ? (uint8_t)(((t / a.W) / a.hr) * a.n_win + (t % a.W) / a.wr) : 0;
     for (int e = threadIdx.x; e < a.R * a.R; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
-    // multiplicity of every routed region, one thread per idx entry (all loads in flight)
-    for (int e = threadIdx.x; e < a.R * a.topk; e += blockDim.x) {
-        const int s = routed[e];
-        if (s >= 0 && s < a.R)
-            atomicAdd(&cnt[(e / a.topk) * a.R + s], 1);
-        else if (cb == 0 && split == 0)
-            flag_error(a.err, kErrIndex);
+    // multiplicity of every routed region: warp w takes query regions w, w + 8, ..., a lane per
+    // idx entry of the row (all loads of a row in flight)
+    for (int r = warp; r < a.R; r += nwarps) {
+        for (int j = lane; j < a.topk; j += 32) {
+            const int s = routed[r * a.topk + j];
+            if (s >= 0 && s < a.R)
+                atomicAdd(&cnt[r * a.R + s], 1);
+            else if (cb == 0 && split == 0)
+                flag_error(a.err, kErrIndex);
+        }
     }
     __syncthreads();
     for (int e = threadIdx.x; e < a.R * a.R; e += blockDim.x) {
@@ -595,15 +602,15 @@ __global__ void __launch_bounds__(256) attend_dense_mma_kernel(const __grid_cons
             const float mn0 = fmaxf(m[0], quad_max(mx0)), mn1 = fmaxf(m[1], quad_max(mx1));
             // a row with no unmasked key so far keeps m = -inf: nothing to rescale, p = 0
             const float base0 = mn0 == -INFINITY ? 0.f : mn0, base1 = mn1 == -INFINITY ? 0.f : mn1;
-            rescale(o, l, mn0 == -INFINITY ? 1.f : exp2f(m[0] - mn0), mn1 == -INFINITY ? 1.f : exp2f(m[1] - mn1));
+            rescale(o, l, mn0 == -INFINITY ? 1.f : fast_exp2(m[0] - mn0), mn1 == -INFINITY ? 1.f : fast_exp2(m[1] - mn1));
             m[0] = mn0;
             m[1] = mn1;
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
-                sc[nt][0] = exp2f(sc[nt][0] - base0);
-                sc[nt][1] = exp2f(sc[nt][1] - base0);
-                sc[nt][2] = exp2f(sc[nt][2] - base1);
-                sc[nt][3] = exp2f(sc[nt][3] - base1);
+                sc[nt][0] = fast_exp2(sc[nt][0] - base0);
+                sc[nt][1] = fast_exp2(sc[nt][1] - base0);
+                sc[nt][2] = fast_exp2(sc[nt][2] - base1);
+                sc[nt][3] = fast_exp2(sc[nt][3] - base1);
                 l[0] += sc[nt][0] + sc[nt][1];
                 l[1] += sc[nt][2] + sc[nt][3];
             }
@@ -646,7 +653,7 @@ static size_t dense_smem_bytes(const Geometry &g, int rows_per_split)
 {
     const int nq = rows_per_split * g.W, nqpad = (nq + 15) & ~15;
     const int npad = (g.N + 15) & ~15;
-    return 1024 + (size_t)(nqpad + 2 * npad) * kRowBytes + (size_t)g.R * g.R * 8 + npad + 16;
+    return 1024 + (size_t)(nqpad + 2 * npad) * kRowBytes + (size_t)g.R * g.R * 4 + npad + 16;
 }
 
 cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
@@ -672,10 +679,18 @@ cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk
     const size_t smem = dense_smem_bytes(g, rows_per_split);
     const long long blocks = (long long)g.B * a.ncb * a.nsplit;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    // three CTAs per SM when their shared memory fits (227 KB per SM, 1 KB reserved per CTA)
+    if (3 * (smem + 1024) <= 227 * 1024) {
+        static int granted3[64] = {0};
+        cudaError_t e = ensure_smem_limit(attend_dense_mma_kernel<3>, smem, granted3);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(attend_dense_mma_kernel<3>, dim3((unsigned)blocks), dim3(256), smem, stream, tq, tk, tv, tout,
+                          a);
+    }
     static int granted[64] = {0};
-    cudaError_t e = ensure_smem_limit(attend_dense_mma_kernel, smem, granted);
+    cudaError_t e = ensure_smem_limit(attend_dense_mma_kernel<2>, smem, granted);
     if (e != cudaSuccess) return e;
-    return launch_pdl(attend_dense_mma_kernel, dim3((unsigned)blocks), dim3(256), smem, stream, tq, tk, tv, tout, a);
+    return launch_pdl(attend_dense_mma_kernel<2>, dim3((unsigned)blocks), dim3(256), smem, stream, tq, tk, tv, tout, a);
 }
 
 }  // namespace bra

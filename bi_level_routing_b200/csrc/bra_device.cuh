@@ -245,6 +245,33 @@ __device__ __forceinline__ void mma_bf16_16816(float *d, const uint32_t *a, uint
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D(16x8, fp32) += A(16x8, tf32, row) * B(8x8, tf32, col)
+__device__ __forceinline__ void mma_tf32_1688(float *d, const uint32_t *a, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// x rounded to tf32 (10 explicit mantissa bits, to nearest, ties away from zero), as fp32 bits.
+__device__ __forceinline__ uint32_t to_tf32(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// x = hi + lo + e with hi, lo tf32 and |e| <= 2^-22 |x|: hi = tf32(x), lo = tf32(x - hi) (x - hi
+// is exact in fp32). For an infinite or NaN x, lo = 0 and hi carries the value.
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo)
+{
+    hi = to_tf32(x);
+    const float r = x - __uint_as_float(hi);
+    lo = to_tf32(r == r ? r : 0.f);
+}
+
 // 2^x on the MUFU unit (ex2.approx, denormal results flushed to zero).
 __device__ __forceinline__ float fast_exp2(float x)
 {

@@ -12,6 +12,8 @@
 // affinity-descending order, ties to the lower region and NaN after every number,
 // deterministically. One-token regions skip the means: the routing kernels read q and k
 // themselves, and in bf16 (up to 64 regions) a tensor-core kernel forms the dot products.
+#include <type_traits>
+
 #include "bra_device.cuh"
 #include "bra_launch.h"
 #include "bra_routing.cuh"
@@ -30,7 +32,6 @@ struct MeansArgs {
 };
 
 constexpr int kMeansThreads = 256;
-constexpr int kMeansMaxRegions = kMeansThreads / 32;
 
 // The means of the regions i0 .. i0 + nreg - 1 (flat index b * R + r), q and k together. A
 // region row segment is nvec = wr C / V 16-byte vectors; thread t of group g = t / slots owns
@@ -393,33 +394,80 @@ static cudaError_t launch_topk_e(const S *qm, const S *km, int32_t *idx, const G
                   : launch_topk_typed<E, false, S>(qm, km, idx, g, rows, chunk, scale, smem, stream);
 }
 
+static cudaError_t launch_route_tf32x3(const float *qm, const float *km, int32_t *idx, const Geometry &g,
+                                       cudaStream_t stream);
+bool route_tf32x3_supports(const Geometry &g);
+
 template <typename S>
 static cudaError_t launch_topk_any(const S *qm, const S *km, int32_t *idx, const Geometry &g, cudaStream_t stream)
 {
+    if constexpr (std::is_same<S, float>::value)
+        if (route_tf32x3_supports(g)) return launch_route_tf32x3(qm, km, idx, g, stream);
     if (g.R <= 32) return launch_topk_e<1, S>(qm, km, idx, g, stream);
     if (g.R <= 64) return launch_topk_e<2, S>(qm, km, idx, g, stream);
     if (g.R <= 128) return launch_topk_e<4, S>(qm, km, idx, g, stream);
     return launch_topk_e<8, S>(qm, km, idx, g, stream);
 }
 
-// One-token regions in bf16 (rs = 1, R <= 64, C % 32 == 0): the means are the tokens, and the
-// product of two bf16 values is exact in fp32, so the affinities are fp32 sums of exact products
-// whichever unit forms them. Here the tensor cores form them: one CTA per (image, 16 query
-// rows); warp w takes the 32-channel chunks w, w + 8, ... and computes the 16 x 64 tile of
-// partial dot products with mma.sync m16n8k16 (bf16 in, fp32 accumulate) straight from 16-byte
-// global loads, every load of the warp in flight at once. Within a chunk, lane (g, c) loads
-// channels 8 c .. 8 c + 7 of query rows g and g + 8 and of key g of each 8-key tile; the MMA's
-// k slots take these channels in the same permuted order for A and B, which a sum over
-// channels does not see. The eight partial tiles are added in warp order in shared memory, then
-// warp w selects the top-k of rows 2 w and 2 w + 1 as every routing kernel does.
+// Tensor-core routing for up to 64 regions. One CTA per (image, 16 query rows); warp w takes
+// channel chunks w, w + 8, ... and accumulates the 16 x 64 tile of partial dot products of its
+// chunks with mma.sync, straight from 16-byte global loads, every load of the warp in flight at
+// once. Within a chunk, lane (g, c) loads the same channel window of query rows g and g + 8 and
+// of key g of each 8-key tile; the MMA's k slots take those channels in the same permuted order
+// for A and B, which a sum over channels does not see. The eight partial tiles are then added
+// in warp order in shared memory and warp w selects the top-k of rows 2 w and 2 w + 1 as every
+// routing kernel does.
+//  * bf16 one-token regions (route_tokens_mma_kernel): the means are the tokens, and a product
+//    of two bf16 values is exact in fp32, so m16n8k16 bf16 MMAs with fp32 accumulation form the
+//    same sums of exact products as fp32 FMAs would (32-channel chunks, 8 channels per lane).
+//  * fp32 means or tokens (route_tf32x3_kernel): each value is split into two tf32 parts,
+//    x = hi + lo with |x - hi - lo| <= 2^-22 |x|, and m16n8k8 tf32 MMAs add lo*hi, hi*lo and
+//    hi*hi (smallest first; lo*lo, below 2^-22 of the product, is left out). Every product is
+//    exact in fp32, so an affinity is off by at most about 1e-6 of the sum of its terms'
+//    magnitudes plus fp32 accumulation, and equal inputs give equal affinities (16-channel
+//    chunks, 4 channels per lane).
+constexpr int kRouteWarps = 8, kPartPad = 68;  // row stride of a partial tile (floats)
+
+// acc[n][0..1]: row g, keys 8 n + 2 c, + 1; acc[n][2..3]: row g + 8, the same keys
+__device__ __forceinline__ void store_partials(float (*part)[16][kPartPad], const float (&acc)[8][4], int ntiles,
+                                               int warp, int g, int c)
+{
+#pragma unroll
+    for (int n = 0; n < 8; ++n)
+        if (n < ntiles) {
+            *reinterpret_cast<float2 *>(&part[warp][g][8 * n + 2 * c]) = make_float2(acc[n][0], acc[n][1]);
+            *reinterpret_cast<float2 *>(&part[warp][g + 8][8 * n + 2 * c]) = make_float2(acc[n][2], acc[n][3]);
+        }
+}
+
+template <bool ROUNDS>
+__device__ __forceinline__ void select_from_partials(float (*part)[16][kPartPad], int R, int r0, int ntiles,
+                                                     int topk, float scale, int32_t *idx_image, int warp, int lane)
+{
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int rr = 2 * warp + i;
+        if (r0 + rr >= R) break;
+        unsigned long long key[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int s = 32 * e + lane;
+            float d = 0.f;
+#pragma unroll
+            for (int w = 0; w < kRouteWarps; ++w) d += (s < 8 * ntiles) ? part[w][rr][s] : 0.f;
+            key[e] = s < R ? routing_key(d * scale, s) : 0ull;
+        }
+        select_topk<2, ROUNDS>(key, topk, idx_image + (int64_t)(r0 + rr) * topk, lane);
+    }
+}
+
 template <bool ROUNDS>
 __global__ void __launch_bounds__(256, 2) route_tokens_mma_kernel(const __nv_bfloat16 *__restrict__ q,
-                                                               const __nv_bfloat16 *__restrict__ k,
-                                                               int32_t *__restrict__ idx, int R, int C, int topk,
-                                                               float scale)
+                                                                  const __nv_bfloat16 *__restrict__ k,
+                                                                  int32_t *__restrict__ idx, int R, int C, int topk,
+                                                                  float scale)
 {
-    constexpr int kWarps = 8, kPad = 68;  // row stride of a partial tile (floats)
-    __shared__ float part[kWarps][16][kPad];
+    __shared__ float part[kRouteWarps][16][kPartPad];
     grid_dependency_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
@@ -440,7 +488,7 @@ __global__ void __launch_bounds__(256, 2) route_tokens_mma_kernel(const __nv_bfl
     for (int n = 0; n < 8; ++n)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[n][j] = 0.f;
-    for (int col = 32 * warp; col < C; col += 32 * kWarps) {
+    for (int col = 32 * warp; col < C; col += 32 * kRouteWarps) {
         const uint4 xa = __ldg(reinterpret_cast<const uint4 *>(qb + ra + col));
         const uint4 xb = __ldg(reinterpret_cast<const uint4 *>(qb + rb + col));
         uint4 y[8];
@@ -456,29 +504,90 @@ __global__ void __launch_bounds__(256, 2) route_tokens_mma_kernel(const __nv_bfl
                 mma_bf16_16816(acc[n], a1, y[n].z, y[n].w);
             }
     }
-    // acc[n][0..1]: row g, keys 8 n + 2 c, + 1; acc[n][2..3]: row g + 8, the same keys
+    store_partials(part, acc, ntiles, warp, g, c);
+    __syncthreads();
+    select_from_partials<ROUNDS>(part, R, r0, ntiles, topk, scale, idx + (int64_t)b * R * topk, warp, lane);
+}
+
+template <bool ROUNDS>
+__global__ void __launch_bounds__(256, 2) route_tf32x3_kernel(const float *__restrict__ qm,
+                                                              const float *__restrict__ km,
+                                                              int32_t *__restrict__ idx, int R, int C, int topk,
+                                                              float scale)
+{
+    __shared__ float part[kRouteWarps][16][kPartPad];
+    grid_dependency_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int row_blocks = (R + 15) >> 4;
+    const int b = blockIdx.x / row_blocks;
+    const int r0 = (blockIdx.x - b * row_blocks) * 16;
+    const int ntiles = (R + 7) >> 3;
+    const float *qb = qm + (int64_t)b * R * C;
+    const float *kb = km + (int64_t)b * R * C;
+    const int ra = min(r0 + g, R - 1) * C + 4 * c, rb = min(r0 + g + 8, R - 1) * C + 4 * c;
+    int kr[8];
+#pragma unroll
+    for (int n = 0; n < 8; ++n) kr[n] = min(8 * n + g, R - 1) * C + 4 * c;
+    float acc[8][4];
 #pragma unroll
     for (int n = 0; n < 8; ++n)
-        if (n < ntiles) {
-            *reinterpret_cast<float2 *>(&part[warp][g][8 * n + 2 * c]) = make_float2(acc[n][0], acc[n][1]);
-            *reinterpret_cast<float2 *>(&part[warp][g + 8][8 * n + 2 * c]) = make_float2(acc[n][2], acc[n][3]);
-        }
-    __syncthreads();
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int rr = 2 * warp + i;
-        if (r0 + rr >= R) break;
-        unsigned long long key[2];
+        for (int j = 0; j < 4; ++j) acc[n][j] = 0.f;
+    for (int col = 16 * warp; col < C; col += 16 * kRouteWarps) {
+        const float4 xa = __ldg(reinterpret_cast<const float4 *>(qb + ra + col));
+        const float4 xb = __ldg(reinterpret_cast<const float4 *>(qb + rb + col));
+        float4 y[8];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int s = 32 * e + lane;
-            float d = 0.f;
+        for (int n = 0; n < 8; ++n)
+            if (n < ntiles) y[n] = __ldg(reinterpret_cast<const float4 *>(kb + kr[n] + col));
+        // MMA m of the chunk: k slot c <- channel 4c + 2m, k slot c + 4 <- channel 4c + 2m + 1
+        uint32_t ah[2][4], al[2][4];
+        split_tf32(xa.x, ah[0][0], al[0][0]);
+        split_tf32(xb.x, ah[0][1], al[0][1]);
+        split_tf32(xa.y, ah[0][2], al[0][2]);
+        split_tf32(xb.y, ah[0][3], al[0][3]);
+        split_tf32(xa.z, ah[1][0], al[1][0]);
+        split_tf32(xb.z, ah[1][1], al[1][1]);
+        split_tf32(xa.w, ah[1][2], al[1][2]);
+        split_tf32(xb.w, ah[1][3], al[1][3]);
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) d += (s < 8 * ntiles) ? part[w][rr][s] : 0.f;
-            key[e] = s < R ? routing_key(d * scale, s) : 0ull;
-        }
-        select_topk<2, ROUNDS>(key, topk, idx + ((int64_t)b * R + r0 + rr) * topk, lane);
+        for (int n = 0; n < 8; ++n)
+            if (n < ntiles) {
+                uint32_t bh[4], bl[4];
+                split_tf32(y[n].x, bh[0], bl[0]);
+                split_tf32(y[n].y, bh[1], bl[1]);
+                split_tf32(y[n].z, bh[2], bl[2]);
+                split_tf32(y[n].w, bh[3], bl[3]);
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    mma_tf32_1688(acc[n], al[m], bh[2 * m], bh[2 * m + 1]);
+                    mma_tf32_1688(acc[n], ah[m], bl[2 * m], bl[2 * m + 1]);
+                    mma_tf32_1688(acc[n], ah[m], bh[2 * m], bh[2 * m + 1]);
+                }
+            }
     }
+    store_partials(part, acc, ntiles, warp, g, c);
+    __syncthreads();
+    select_from_partials<ROUNDS>(part, R, r0, ntiles, topk, scale, idx + (int64_t)b * R * topk, warp, lane);
+}
+
+bool route_tf32x3_supports(const Geometry &g)
+{
+    return g.R <= 64 && g.C % 16 == 0 && (long long)g.R * g.C < (1LL << 31);
+}
+
+static cudaError_t launch_route_tf32x3(const float *qm, const float *km, int32_t *idx, const Geometry &g,
+                                       cudaStream_t stream)
+{
+    const long long blocks = (long long)g.B * ((g.R + 15) / 16);
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const float scale = (float)(1.0 / sqrt((double)g.C));
+    if (topk_by_rounds(2, g.topk))
+        return launch_pdl(route_tf32x3_kernel<true>, dim3((unsigned)blocks), dim3(256), 0, stream, qm, km, idx, g.R,
+                          g.C, g.topk, scale);
+    return launch_pdl(route_tf32x3_kernel<false>, dim3((unsigned)blocks), dim3(256), 0, stream, qm, km, idx, g.R, g.C,
+                      g.topk, scale);
 }
 
 bool route_tokens_mma_supports(const Geometry &g, bool bf16)
