@@ -396,6 +396,106 @@ static cudaError_t launch_topk_e(const S *qm, const S *km, int32_t *idx, const G
 
 static cudaError_t launch_route_tf32x3(const float *qm, const float *km, int32_t *idx, const Geometry &g,
                                        cudaStream_t stream);
+// 3xTF32 routing for 64 < R <= 256 (E = 4 or 8 keys per lane in the selection): one CTA per
+// (image, 16 query rows); the 8-key tiles are dealt to the warps (warp w takes tiles w, w + 8,
+// w + 16, w + 24), and each warp forms whole dot products of its tiles over all channels, in
+// 16-channel chunks with the same split, permutation and MMA order as route_tf32x3_kernel. The
+// 16 x R tile goes to shared memory, then warp w selects the top-k of rows 2 w and 2 w + 1.
+template <int E, bool ROUNDS>
+__global__ void __launch_bounds__(256, 2) route_tf32x3_wide_kernel(const float *__restrict__ qm,
+                                                                   const float *__restrict__ km,
+                                                                   int32_t *__restrict__ idx, int R, int C, int topk,
+                                                                   float scale)
+{
+    constexpr int kStride = 32 * E + 4;
+    __shared__ float aff[16][kStride];
+    grid_dependency_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int row_blocks = (R + 15) >> 4;
+    const int b = blockIdx.x / row_blocks;
+    const int r0 = (blockIdx.x - b * row_blocks) * 16;
+    const int ntiles = (R + 7) >> 3;
+    const float *qb = qm + (int64_t)b * R * C;
+    const float *kb = km + (int64_t)b * R * C;
+    const int ra = min(r0 + g, R - 1) * C + 4 * c, rb = min(r0 + g + 8, R - 1) * C + 4 * c;
+    constexpr int T = E / 2;  // tiles per warp: 32 E / 8 keys over 8 warps
+    int kr[T];
+#pragma unroll
+    for (int i = 0; i < T; ++i) kr[i] = min(8 * (warp + 8 * i) + g, R - 1) * C + 4 * c;
+    float acc[T][4];
+#pragma unroll
+    for (int i = 0; i < T; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int col = 0; col < C; col += 16) {
+        const float4 xa = __ldg(reinterpret_cast<const float4 *>(qb + ra + col));
+        const float4 xb = __ldg(reinterpret_cast<const float4 *>(qb + rb + col));
+        float4 y[T];
+#pragma unroll
+        for (int i = 0; i < T; ++i)
+            if (warp + 8 * i < ntiles) y[i] = __ldg(reinterpret_cast<const float4 *>(kb + kr[i] + col));
+        uint32_t ah[2][4], al[2][4];
+        split_tf32(xa.x, ah[0][0], al[0][0]);
+        split_tf32(xb.x, ah[0][1], al[0][1]);
+        split_tf32(xa.y, ah[0][2], al[0][2]);
+        split_tf32(xb.y, ah[0][3], al[0][3]);
+        split_tf32(xa.z, ah[1][0], al[1][0]);
+        split_tf32(xb.z, ah[1][1], al[1][1]);
+        split_tf32(xa.w, ah[1][2], al[1][2]);
+        split_tf32(xb.w, ah[1][3], al[1][3]);
+#pragma unroll
+        for (int i = 0; i < T; ++i)
+            if (warp + 8 * i < ntiles) {
+                uint32_t bh[4], bl[4];
+                split_tf32(y[i].x, bh[0], bl[0]);
+                split_tf32(y[i].y, bh[1], bl[1]);
+                split_tf32(y[i].z, bh[2], bl[2]);
+                split_tf32(y[i].w, bh[3], bl[3]);
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    mma_tf32_1688(acc[i], al[m], bh[2 * m], bh[2 * m + 1]);
+                    mma_tf32_1688(acc[i], ah[m], bl[2 * m], bl[2 * m + 1]);
+                    mma_tf32_1688(acc[i], ah[m], bh[2 * m], bh[2 * m + 1]);
+                }
+            }
+    }
+#pragma unroll
+    for (int i = 0; i < T; ++i)
+        if (warp + 8 * i < ntiles) {
+            const int s0 = 8 * (warp + 8 * i) + 2 * c;
+            *reinterpret_cast<float2 *>(&aff[g][s0]) = make_float2(acc[i][0], acc[i][1]);
+            *reinterpret_cast<float2 *>(&aff[g + 8][s0]) = make_float2(acc[i][2], acc[i][3]);
+        }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int rr = 2 * warp + i;
+        if (r0 + rr >= R) break;
+        unsigned long long key[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int s = 32 * e + lane;
+            key[e] = s < R ? routing_key(aff[rr][s] * scale, s) : 0ull;
+        }
+        select_topk<E, ROUNDS>(key, topk, idx + ((int64_t)b * R + r0 + rr) * topk, lane);
+    }
+}
+
+template <int E>
+static cudaError_t launch_route_tf32x3_wide(const float *qm, const float *km, int32_t *idx, const Geometry &g,
+                                            cudaStream_t stream)
+{
+    const long long blocks = (long long)g.B * ((g.R + 15) / 16);
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const float scale = (float)(1.0 / sqrt((double)g.C));
+    if (topk_by_rounds(E, g.topk))
+        return launch_pdl(route_tf32x3_wide_kernel<E, true>, dim3((unsigned)blocks), dim3(256), 0, stream, qm, km, idx,
+                          g.R, g.C, g.topk, scale);
+    return launch_pdl(route_tf32x3_wide_kernel<E, false>, dim3((unsigned)blocks), dim3(256), 0, stream, qm, km, idx,
+                      g.R, g.C, g.topk, scale);
+}
+
 bool route_tf32x3_supports(const Geometry &g);
 
 template <typename S>
@@ -574,7 +674,7 @@ __global__ void __launch_bounds__(256, 2) route_tf32x3_kernel(const float *__res
 
 bool route_tf32x3_supports(const Geometry &g)
 {
-    return g.R <= 64 && g.C % 16 == 0 && (long long)g.R * g.C < (1LL << 31);
+    return g.R <= 256 && g.C % 16 == 0 && (long long)g.R * g.C < (1LL << 31);
 }
 
 static cudaError_t launch_route_tf32x3(const float *qm, const float *km, int32_t *idx, const Geometry &g,
@@ -582,6 +682,8 @@ static cudaError_t launch_route_tf32x3(const float *qm, const float *km, int32_t
 {
     const long long blocks = (long long)g.B * ((g.R + 15) / 16);
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    if (g.R > 128) return launch_route_tf32x3_wide<8>(qm, km, idx, g, stream);
+    if (g.R > 64) return launch_route_tf32x3_wide<4>(qm, km, idx, g, stream);
     const float scale = (float)(1.0 / sqrt((double)g.C));
     if (topk_by_rounds(2, g.topk))
         return launch_pdl(route_tf32x3_kernel<true>, dim3((unsigned)blocks), dim3(256), 0, stream, qm, km, idx, g.R,

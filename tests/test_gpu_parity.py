@@ -72,6 +72,9 @@ SMALL = [
     ("rs1_r25_c96_bf16", 3, 5, 5, 96, 3, 5, 25, "bf16"),
     ("rs1_r64_c32_bf16", 2, 8, 8, 32, 1, 8, 64, "bf16"),
     ("rs1_r49_c512_topk3_bf16", 2, 7, 7, 512, 16, 7, 3, "bf16"),
+    # 64 < R <= 256 with fp32 means (the key-split 3xTF32 routing kernel): E = 4 and E = 8
+    ("r100_rs4_f32", 2, 20, 20, 32, 1, 10, 7, "f32"),
+    ("r144_rs4_bf16", 2, 24, 24, 64, 2, 12, 20, "bf16"),
 ]
 
 
