@@ -156,6 +156,25 @@ bra_status encode_map(CUtensorMap *map, const void *base, const bra::Geometry &g
     return BRA_OK;
 }
 
+// 5-D bf16 tensor map of a [B, H, W, C] array viewed as (channel in its 64-channel block, x, y,
+// channel block, image), 128-byte swizzle, box (64, bw, bh, nblk, 1): the nblk channel blocks
+// of a box land in shared memory one after the other, each as its own (bh x bw)-row tile.
+bra_status encode_map_blocks(CUtensorMap *map, const void *base, const bra::Geometry &g, int bw, int bh, int nblk)
+{
+    cuuint64_t dims[5] = {64u, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)(g.C / 64), (cuuint64_t)g.B};
+    cuuint64_t strides[4] = {(cuuint64_t)g.C * 2, (cuuint64_t)g.W * g.C * 2, 128u, (cuuint64_t)g.H * g.W * g.C * 2};
+    cuuint32_t box[5] = {64u, (cuuint32_t)bw, (cuuint32_t)bh, (cuuint32_t)nblk, 1u};
+    cuuint32_t elem_strides[5] = {1u, 1u, 1u, 1u, 1u};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box,
+                          elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_error = "cuTensorMapEncodeTiled (5-D) failed with CUresult " + std::to_string((int)r);
+        return BRA_ERR_CUDA;
+    }
+    return BRA_OK;
+}
+
 bra_status route_impl(const void *q, const void *k, int32_t *idx, const bra::Geometry &g, bra_dtype dtype,
                       cudaStream_t stream)
 {
@@ -200,11 +219,11 @@ bra_status attend_impl(const void *q, const void *k, const void *v, const int32_
         e = bra::launch_attend_gather_umma(tq, tk, tv, idx, out, g, st->num_sms, st->error_word, stream);
     } else if (kernel == BRA_ATTEND_GATHER_MMA) {
         CUtensorMap tq, tk, tv, to;
-        int box[4];
+        int box[5];
         bra::gather_mma_box(g, box);
-        if ((s = encode_map(&tq, q, g, box[1], box[2])) != BRA_OK) return s;
-        if ((s = encode_map(&tk, k, g, box[1], box[2])) != BRA_OK) return s;
-        if ((s = encode_map(&tv, v, g, box[1], box[2])) != BRA_OK) return s;
+        if ((s = encode_map_blocks(&tq, q, g, box[1], box[2], box[3])) != BRA_OK) return s;
+        if ((s = encode_map_blocks(&tk, k, g, box[1], box[2], box[3])) != BRA_OK) return s;
+        if ((s = encode_map_blocks(&tv, v, g, box[1], box[2], box[3])) != BRA_OK) return s;
         if ((s = encode_map(&to, out, g, box[1], box[2])) != BRA_OK) return s;
         e = bra::launch_attend_gather_mma(tq, tk, tv, to, idx, out, g, st->num_sms, st->error_word, stream);
     } else {

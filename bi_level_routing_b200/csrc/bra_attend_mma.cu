@@ -290,9 +290,10 @@ __global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_
                 const int qx = (r % a.n_win) * a.wr, qy = (r / a.n_win) * a.hr;
                 if (!(alive = mbar_wait(&empty_q[qs], qph ^ 1, a.err))) break;
                 qinfo[qs] = ItemInfo{b, qx, qy, (cb0 << 8) | nh};
-                mbar_arrive_expect_tx(&full_q[qs], (uint32_t)(nh * TILE));
-                for (int cb = 0; cb < nh; ++cb)
-                    tma_load_4d(sQ + (size_t)(qs * NCB + cb) * TILE, &tq, (cb0 + cb) * 64, qx, qy, b, &full_q[qs]);
+                // one box brings all NCB channel-block tiles (blocks past C are zero-filled and
+                // counted like the others)
+                mbar_arrive_expect_tx(&full_q[qs], (uint32_t)(NCB * TILE));
+                tma_load_5d(sQ + (size_t)qs * NCB * TILE, &tq, 0, qx, qy, cb0, b, &full_q[qs]);
                 if (++qs == a.qslots) {
                     qs = 0;
                     qph ^= 1;
@@ -304,12 +305,10 @@ __global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_
                     kv_ok[kvs] = ok;
                     if (ok) {
                         const int sx = (s % a.n_win) * a.wr, sy = (s / a.n_win) * a.hr;
-                        mbar_arrive_expect_tx(&full_kv[kvs], (uint32_t)(2 * nh * TILE));
+                        mbar_arrive_expect_tx(&full_kv[kvs], (uint32_t)(2 * NCB * TILE));
                         uint8_t *kt = sKV + (size_t)kvs * 2 * NCB * TILE;
-                        for (int cb = 0; cb < nh; ++cb) {
-                            tma_load_4d(kt + cb * TILE, &tk, (cb0 + cb) * 64, sx, sy, b, &full_kv[kvs]);
-                            tma_load_4d(kt + (NCB + cb) * TILE, &tv, (cb0 + cb) * 64, sx, sy, b, &full_kv[kvs]);
-                        }
+                        tma_load_5d(kt, &tk, 0, sx, sy, cb0, b, &full_kv[kvs]);
+                        tma_load_5d(kt + NCB * TILE, &tv, 0, sx, sy, cb0, b, &full_kv[kvs]);
                     } else {
                         flag_error(a.err, kErrIndex);
                         mbar_arrive_expect_tx(&full_kv[kvs], 0);
@@ -394,12 +393,23 @@ bool gather_mma_supports(const Geometry &g)
            (long long)g.hr * g.W * g.C < (1LL << 31);
 }
 
-void gather_mma_box(const Geometry &g, int box[4])
+// 64-channel blocks per work item: eight consumer warps of 16 rows x 1 head at most.
+static int gather_blocks_per_item(const Geometry &g)
+{
+    const int rt = g.rs / 16;
+    int n = 8 / (2 * rt);
+    if (n < 1) n = 1;
+    if (n > g.C / 64) n = g.C / 64;
+    return n;
+}
+
+void gather_mma_box(const Geometry &g, int box[5])
 {
     box[0] = 64;
     box[1] = g.wr;
     box[2] = g.hr;
-    box[3] = 1;
+    box[3] = gather_blocks_per_item(g);
+    box[4] = 1;
 }
 
 template <int RS>
@@ -433,9 +443,7 @@ cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &t
     a.wr = g.wr;
     a.ncb = g.C / 64;
     const int rt = g.rs / 16;
-    int ncb_per_cta = 8 / (2 * rt);
-    if (ncb_per_cta < 1) ncb_per_cta = 1;
-    if (ncb_per_cta > a.ncb) ncb_per_cta = a.ncb;
+    const int ncb_per_cta = gather_blocks_per_item(g);
     a.ncb_per_cta = ncb_per_cta;
     a.groups = (a.ncb + ncb_per_cta - 1) / ncb_per_cta;
     a.ncw = ncb_per_cta * 2 * rt;

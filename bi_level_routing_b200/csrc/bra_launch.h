@@ -85,13 +85,16 @@ cudaError_t launch_attend_simt(const void *q, const void *k, const void *v, cons
                                const Geometry &g, bool bf16, unsigned *err, cudaStream_t stream);
 
 // Tensor-core attention kernels (bf16, hd == 32, C % 64 == 0). The tensor maps describe
-// q, k, v, out as 4-D (C, W, H, B) bf16 tensors, 128-byte swizzle; box sizes as each
-// launcher's `*_boxes` function states.
+// q, k, v, out as 4-D (C, W, H, B) bf16 tensors, 128-byte swizzle (except the gather kernel's
+// q, k and v maps, 5-D, below); box sizes as each launcher's comment states.
 bool gather_mma_supports(const Geometry &g);
 bool dense_mma_supports(const Geometry &g);
 
-// Boxes (channels, x, y, images) of the gather kernel: one region, 64 channels, for all four maps.
-void gather_mma_box(const Geometry &g, int box[4]);
+// Box of the gather kernel's q, k and v maps: (64 channels, wr, hr, NCB channel blocks, 1 image)
+// on the 5-D view (channel in block, x, y, channel block, image) of [B, H, W, C], so that one
+// TMA load brings a region's NCB 64-channel tiles, one after the other. Its out map is 4-D,
+// box (64, wr, hr, 1).
+void gather_mma_box(const Geometry &g, int box[5]);
 cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                      const CUtensorMap &tout, const int32_t *idx, void *out, const Geometry &g,
                                      int num_sms, unsigned *err, cudaStream_t stream);
