@@ -39,6 +39,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 KERNEL_SOURCES = {"attend_gather_umma": "bi_level_routing_b200/csrc/bra_attend_umma.cu",
                   "attend_gather_mma": "bi_level_routing_b200/csrc/bra_attend_mma.cu",
                   "attend_dense_mma": "bi_level_routing_b200/csrc/bra_attend_mma.cu",
+                  "attend_region_mma": "bi_level_routing_b200/csrc/bra_attend_region.cu",
                   "attend_simt": "bi_level_routing_b200/csrc/bra_attend_simt.cu"}
 
 

@@ -19,7 +19,7 @@ HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))
 STATUS = {0: "BRA_OK", 1: "BRA_ERR_INVALID_ARG", 2: "BRA_ERR_UNSUPPORTED", 3: "BRA_ERR_CUDA",
           4: "BRA_ERR_INDEX", 5: "BRA_ERR_TIMEOUT"}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
-ATTEND_KERNELS = {"auto": 0, "simt": 1, "gather_mma": 2, "dense_mma": 3, "gather_umma": 4}
+ATTEND_KERNELS = {"auto": 0, "simt": 1, "gather_mma": 2, "dense_mma": 3, "gather_umma": 4, "region_mma": 5}
 
 _lib = None
 

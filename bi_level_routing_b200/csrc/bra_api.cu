@@ -124,13 +124,17 @@ int choose_attend_kernel(const bra::Geometry &g, bra_dtype dtype)
     const bool gather_ok = bf16 && bra::gather_mma_supports(g);
     const bool dense_ok = bf16 && bra::dense_mma_supports(g);
     const bool umma_ok = bf16 && bra::gather_umma_supports(g);
+    const bool region_ok = bf16 && bra::region_mma_supports(g);
     switch (g_forced_kernel.load()) {
     case BRA_ATTEND_SIMT: return simt_ok ? BRA_ATTEND_SIMT : -1;
     case BRA_ATTEND_GATHER_MMA: return gather_ok ? BRA_ATTEND_GATHER_MMA : -1;
     case BRA_ATTEND_DENSE_MMA: return dense_ok ? BRA_ATTEND_DENSE_MMA : -1;
     case BRA_ATTEND_GATHER_UMMA: return umma_ok ? BRA_ATTEND_GATHER_UMMA : -1;
+    case BRA_ATTEND_REGION_MMA: return region_ok ? BRA_ATTEND_REGION_MMA : -1;
     default: break;
     }
+    // 4-token regions: tiles of 4 tokens x 4 heads over the routed keys only
+    if (region_ok) return BRA_ATTEND_REGION_MMA;
     // Dense attention over the whole image wastes at most 4x the routed work here.
     if (dense_ok && 4LL * g.topk * g.rs >= g.N) return BRA_ATTEND_DENSE_MMA;
     if (umma_ok) return BRA_ATTEND_GATHER_UMMA;
@@ -217,6 +221,12 @@ bra_status attend_impl(const void *q, const void *k, const void *v, const int32_
         if ((s = encode_map(&tk, k, g, g.wr, g.hr)) != BRA_OK) return s;
         if ((s = encode_map(&tv, v, g, g.wr, g.hr)) != BRA_OK) return s;
         e = bra::launch_attend_gather_umma(tq, tk, tv, idx, out, g, st->num_sms, st->error_word, stream);
+    } else if (kernel == BRA_ATTEND_REGION_MMA) {
+        CUtensorMap tq, tk, tv;
+        if ((s = encode_map_blocks(&tq, q, g, g.W, g.H, 2)) != BRA_OK) return s;
+        if ((s = encode_map_blocks(&tk, k, g, g.W, g.H, 2)) != BRA_OK) return s;
+        if ((s = encode_map_blocks(&tv, v, g, g.W, g.H, 2)) != BRA_OK) return s;
+        e = bra::launch_attend_region_mma(tq, tk, tv, idx, out, g, st->num_sms, st->error_word, stream);
     } else if (kernel == BRA_ATTEND_GATHER_MMA) {
         CUtensorMap tq, tk, tv, to;
         int box[5];
@@ -341,7 +351,7 @@ bra_status bra_forward_host(const void *q, const void *k, const void *v, int32_t
 
 bra_status bra_set_attend_kernel(bra_attend_kernel kernel)
 {
-    if (kernel < BRA_ATTEND_AUTO || kernel > BRA_ATTEND_GATHER_UMMA) return BRA_ERR_INVALID_ARG;
+    if (kernel < BRA_ATTEND_AUTO || kernel > BRA_ATTEND_REGION_MMA) return BRA_ERR_INVALID_ARG;
     g_forced_kernel.store(kernel);
     return BRA_OK;
 }

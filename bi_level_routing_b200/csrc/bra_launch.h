@@ -90,6 +90,13 @@ cudaError_t launch_attend_simt(const void *q, const void *k, const void *v, cons
 bool gather_mma_supports(const Geometry &g);
 bool dense_mma_supports(const Geometry &g);
 
+// Stacked-head gather attention for 4-token regions (bf16, hd == 32, C % 128 == 0, N <= 256,
+// topk <= 64). Maps: q, k, v as 5-D views, box (64, W, H, 2, 1).
+bool region_mma_supports(const Geometry &g);
+cudaError_t launch_attend_region_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                     const int32_t *idx, void *out, const Geometry &g, int num_sms, unsigned *err,
+                                     cudaStream_t stream);
+
 // Box of the gather kernel's q, k and v maps: (64 channels, wr, hr, NCB channel blocks, 1 image)
 // on the 5-D view (channel in block, x, y, channel block, image) of [B, H, W, C], so that one
 // TMA load brings a region's NCB 64-channel tiles, one after the other. Its out map is 4-D,

@@ -79,9 +79,13 @@ typedef enum {
                                  tiles staged by TMA, tensor-core QK^T and PV */
     BRA_ATTEND_DENSE_MMA = 3, /* bf16, hd == 32, C % 64 == 0, R <= 64, H*W <= 256: the image's
                                  K/V staged once, masked by the routing multiplicities */
-    BRA_ATTEND_GATHER_UMMA = 4/* bf16, hd == 32, C % 64 == 0, rs == 64: per-region tiles staged by
-                                 TMA, QK^T and PV on the tcgen05 tensor cores with TMEM
+    BRA_ATTEND_GATHER_UMMA = 4,/* bf16, hd == 32, C % 64 == 0, rs == 64: per-region tiles staged
+                                 by TMA, QK^T and PV on the tcgen05 tensor cores with TMEM
                                  accumulators, one softmax thread per query row */
+    BRA_ATTEND_REGION_MMA = 5 /* bf16, hd == 32, C % 128 == 0, rs == 4, H*W <= 256, topk <= 64:
+                                 the image's q, k, v for 4 heads staged once; tiles of 4 tokens
+                                 x 4 heads of one region, routed keys gathered from shared
+                                 memory */
 } bra_attend_kernel;
 
 /* Steps 1-4: idx[b, r, :] = routing index of region r of image b.

@@ -86,7 +86,7 @@ def test_unsupported_sizes(L):
 
 def test_kernel_selection_per_workload(L):
     assert L.bra_set_attend_kernel(0) == OK
-    want = {"tiny_f32": "simt", "stage1": "gather_umma", "stage2": "gather_mma", "stage3": "dense_mma",
+    want = {"tiny_f32": "simt", "stage1": "gather_umma", "stage2": "gather_mma", "stage3": "region_mma",
             "stage4": "dense_mma", "highres": "gather_umma"}
     import torch
     for name, kernel in want.items():

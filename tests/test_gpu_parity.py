@@ -75,6 +75,10 @@ SMALL = [
     # 64 < R <= 256 with fp32 means (the key-split 3xTF32 routing kernel): E = 4 and E = 8
     ("r100_rs4_f32", 2, 20, 20, 32, 1, 10, 7, "f32"),
     ("r144_rs4_bf16", 2, 24, 24, 64, 2, 12, 20, "bf16"),
+    # 4-token regions in bf16 (the stacked-head kernel): 1 x 4 regions with padded keys, and
+    # 160 routed keys in three chunks of the online softmax
+    ("rs4_1x4_c128_bf16", 2, 4, 16, 128, 4, 4, 3, "bf16"),
+    ("rs4_topk40_c256_bf16", 1, 16, 16, 256, 8, 8, 40, "bf16"),
 ]
 
 
@@ -86,7 +90,7 @@ def _small(spec, values="region_offset", seed=1234):
 def _kernels_for(w):
     dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
     out = []
-    for kname in ("simt", "gather_mma", "dense_mma", "gather_umma"):
+    for kname in ("simt", "gather_mma", "dense_mma", "gather_umma", "region_mma"):
         bra.set_attend_kernel(kname)
         if bra.selected_attend_kernel(w.B, w.H, w.W, w.C, w.heads, w.n_win, w.topk, dt) == kname:
             out.append(kname)
