@@ -18,8 +18,8 @@
 //
 // One CTA per (image, group of 4 heads = 128 channels, split of the query regions): one TMA
 // load per tensor stages the image's q, k and v for those channels in shared memory (5-D box:
-// two 64-channel tiles of H x W rows, 128-byte swizzle); warp w then takes query regions
-// w, w + 16, ... (of its split). Per region it gathers the routed keys straight from shared
+// two 64-channel tiles of H x W rows, 128-byte swizzle); warp w of 12 then takes query regions
+// w, w + 12, ... (of its split). Per region it gathers the routed keys straight from shared
 // memory: ldmatrix reads rows at per-lane addresses, so key j of the tile is token j % 4 of
 // region idx[b, r, j / 4] wherever it sits. Keys go in chunks of 64 with an online softmax.
 // Every wait is bounded (kErrTimeout).
@@ -30,13 +30,14 @@ namespace bra {
 
 namespace {
 
-constexpr int kRegionWarps = 16;
+constexpr int kRegionWarps = 12;
 
 struct RegionArgs {
     const int32_t *idx;
     unsigned *err;
     __nv_bfloat16 *out;
     int H, W, C, n_win, topk, R, hr, wr, N;
+    int wshift;   // log2(wr)
     int ngroups;  // C / 128
     int nsplit;   // CTAs per (image, group); query regions are dealt among them
     int keys;     // 4 topk rounded up to a multiple of 16
@@ -65,9 +66,6 @@ __device__ __forceinline__ float quad_sum_f(float x)
     x += __shfl_xor_sync(0xffffffffu, x, 1);
     return x + __shfl_xor_sync(0xffffffffu, x, 2);
 }
-
-// row offset of token t (0..3) of a region from the region's first token
-__device__ __forceinline__ int token_offset(int t, int wr, int W) { return (t / wr) * W + t % wr; }
 
 }  // namespace
 
@@ -123,6 +121,8 @@ __global__ void __launch_bounds__(32 * kRegionWarps, 1) attend_region_mma_kernel
     const int hA = g >> 2, hB = 2 + (g >> 2);  // heads of this lane's rows g and g + 8
     const uint32_t qbase = smem_u32(sQ), kbase = smem_u32(sK), vbase = smem_u32(sV);
     const int n_keys = 4 * a.topk;
+    // row offset of token t of a region from its first token (wr = 1 << wshift is 1, 2 or 4)
+    auto toff = [&](int t) -> int { return (t >> a.wshift) * a.W + (t & (a.wr - 1)); };
     // address of channel c (0..127, even) of staged row n: channel block c / 64, 16-byte chunk
     auto addr = [&](uint32_t base, int n, int c) -> uint32_t {
         return base + sw128((c >> 6) * a.N + n, (c & 63) >> 3) + (c & 7) * 2;
@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(32 * kRegionWarps, 1) attend_region_mma_kernel
     for (int r = split + a.nsplit * warp; alive && r < a.R; r += a.nsplit * kRegionWarps) {
         // Q of this lane's rows: token g % 4 of region r, heads hA (row g) and hB (row g + 8);
         // per head two 16-channel k steps, each a low and a high pair of channels
-        const int qrow = row0[r] + token_offset(g & 3, a.wr, a.W);
+        const int qrow = row0[r] + toff(g & 3);
         uint32_t qa[2][2], qb[2][2];
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
@@ -141,6 +141,9 @@ __global__ void __launch_bounds__(32 * kRegionWarps, 1) attend_region_mma_kernel
             qb[ks][1] = ld_shared_u32(addr(qbase, qrow, 32 * hB + 16 * ks + 2 * t4 + 8));
         }
         const int *ridx = sidx + r * a.topk;
+        // bit j: routed region j of this row is in range (topk <= 64)
+        const uint32_t ok_lo = __ballot_sync(0xffffffffu, lane < a.topk && ridx[lane] >= 0);
+        const uint32_t ok_hi = __ballot_sync(0xffffffffu, lane + 32 < a.topk && ridx[lane + 32] >= 0);
         float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
         float oA[4][2], oB[4][2];  // row g: head hA's 32 channels; row g + 8: head hB's
 #pragma unroll
@@ -150,14 +153,23 @@ __global__ void __launch_bounds__(32 * kRegionWarps, 1) attend_region_mma_kernel
             const int nk = min(64, a.keys - kc);  // a multiple of 16
             // S = Q K^T for the chunk's 8-key tiles: per head, the 8 tiles' ldmatrix first, then
             // their MMAs side by side (independent accumulators)
+            // staged row of keys kc + lane and kc + 32 + lane (-1: padding or a skipped region);
+            // the ldmatrix rows of K and V come from these by shuffles
+            int kra, krb;
+            {
+                const int k0 = kc + lane, k1 = kc + 32 + lane;
+                const int s0 = k0 < n_keys ? ridx[k0 >> 2] : -1, s1 = k1 < n_keys ? ridx[k1 >> 2] : -1;
+                kra = s0 >= 0 ? row0[s0] + toff(k0 & 3) : -1;
+                krb = s1 >= 0 ? row0[s1] + toff(k1 & 3) : -1;
+            }
             float sc[8][4];
             int krow[8];
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-                const int kr = kc + nt * 8 + (lane & 7);  // this lane's ldmatrix row: key kr
-                const int sr = kr < n_keys ? ridx[kr >> 2] : -1;
-                krow[nt] = sr >= 0 ? row0[sr] + token_offset(kr & 3, a.wr, a.W) : 0;
+                // this lane's ldmatrix row: key kc + 8 nt + (lane & 7); masked keys read row 0
+                const int kr = __shfl_sync(0xffffffffu, nt < 4 ? kra : krb, (8 * nt + (lane & 7)) & 31);
+                krow[nt] = kr >= 0 ? kr : 0;
             }
 #pragma unroll
             for (int hk = 0; hk < 4; ++hk) {
@@ -183,8 +195,8 @@ __global__ void __launch_bounds__(32 * kRegionWarps, 1) attend_region_mma_kernel
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 // keys kc + 8 nt + 2 t4 and + 1 lie in one region: both valid or both not
-                const int kk = kc + nt * 8 + 2 * t4;
-                const bool ok = nt * 8 < nk && kk < n_keys && ridx[kk >> 2] >= 0;
+                const int kk = kc + nt * 8 + 2 * t4, j = kk >> 2;
+                const bool ok = nt * 8 < nk && kk < n_keys && (((j < 32 ? ok_lo >> j : ok_hi >> (j - 32)) & 1u) != 0);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) sc[nt][j] = ok ? sc[nt][j] * a.scale_log2 : -INFINITY;
             }
@@ -229,9 +241,7 @@ __global__ void __launch_bounds__(32 * kRegionWarps, 1) attend_region_mma_kernel
                 pa[kk][1] = pack_bf16x2(sc[2 * kk][2], sc[2 * kk][3]);
                 pa[kk][2] = pack_bf16x2(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
                 pa[kk][3] = pack_bf16x2(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
-                const int kr = kc + 16 * kk + (lane & 15);
-                const int sr = kr < n_keys ? ridx[kr >> 2] : -1;
-                vrow[kk] = sr >= 0 ? row0[sr] + token_offset(kr & 3, a.wr, a.W) : -1;
+                vrow[kk] = __shfl_sync(0xffffffffu, kk < 2 ? kra : krb, (16 * kk + (lane & 15)) & 31);
             }
             // two 16-channel pairs at a time: four independent accumulators per key step
 #pragma unroll
@@ -307,6 +317,7 @@ cudaError_t launch_attend_region_mma(const CUtensorMap &tq, const CUtensorMap &t
     a.hr = g.hr;
     a.wr = g.wr;
     a.N = g.N;
+    a.wshift = g.wr == 4 ? 2 : (g.wr == 2 ? 1 : 0);  // rs = 4: wr is 1, 2 or 4
     a.ngroups = g.C / 128;
     a.keys = (4 * g.topk + 15) & ~15;
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)g.hd));
