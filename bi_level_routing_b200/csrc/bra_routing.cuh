@@ -1,9 +1,10 @@
 // bra_routing.cuh -- device routines of the routing step: the 64-bit routing keys, the warp
 // top-k selection, the affinity rows (several rows x several keys per lane) and the staging of
-// mean rows into padded shared-memory rows. Every routing kernel is built from these, so the
-// routing index is the same bits whichever of them computed it. The one exception is the
-// tensor-core kernel for one-token bf16 regions, whose sums run in another order; it serves
-// every call of that shape, through either routing entry point.
+// mean rows into padded shared-memory rows. The CUDA-core routing kernels are built from these
+// and sum in one order, so they give the same bits. The tensor-core routing kernels (bf16 MMAs
+// for one-token regions, 3xTF32 for fp32 inputs) use the keys and the selection from here with
+// their sums in another order; each serves every call of its shapes, through either routing
+// entry point, so the index of a shape never depends on the entry point.
 #pragma once
 
 #include "bra_device.cuh"
@@ -139,8 +140,8 @@ __device__ __forceinline__ void affinity_accumulate(float (&acc)[NR][E][4], cons
 }
 
 // The affinities of rows i < nr from their partial sums, combined as (s0 + s1) + (s2 + s3), times
-// C^-1/2, and their top-k, written to out + i * topk. Every routing kernel goes through
-// affinity_accumulate and this function, so the index is the same bits whichever kernel
+// C^-1/2, and their top-k, written to out + i * topk. The CUDA-core routing kernels go through
+// affinity_accumulate and this function, so their index is the same bits whichever of them
 // computed it.
 template <int E, int NR, bool ROUNDS>
 __device__ __forceinline__ void affinity_select(const float (&acc)[NR][E][4], int nr, int R, int topk, float scale,

@@ -108,6 +108,12 @@ def test_forcing_a_kernel(L):
         assert L.bra_selected_attend_kernel(64, 14, 14, 256, 8, 7, 16, 1) == 3
         assert L.bra_set_attend_kernel(2) == OK
         assert L.bra_selected_attend_kernel(1, 28, 28, 64, 2, 7, 4, 0) == -1  # fp32 has no tensor-core kernel
+        assert L.bra_set_attend_kernel(6) == INVALID
+        assert L.bra_set_attend_kernel(5) == OK
+        assert L.bra_selected_attend_kernel(64, 14, 14, 256, 8, 7, 16, 1) == 5  # 4-token regions
+        assert L.bra_selected_attend_kernel(64, 14, 14, 64, 2, 7, 16, 1) == -1  # C % 128 != 0
+        assert L.bra_selected_attend_kernel(64, 28, 28, 128, 4, 7, 4, 1) == -1  # 16-token regions
+        assert L.bra_selected_attend_kernel(4, 28, 28, 128, 4, 14, 4, 1) == -1  # 784 tokens > 256
     finally:
         L.bra_set_attend_kernel(0)
 
