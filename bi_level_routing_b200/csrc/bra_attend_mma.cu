@@ -7,7 +7,7 @@
 // for the PV product; out is rounded to bf16.
 //
 // Two kernels, both with K/V staged in shared memory by TMA (cp.async.bulk.tensor, 128-byte
-// swizzle, no multicast) and the gathered K/V never written to HBM:
+// swizzle, each CTA loading its own tiles) and the gathered K/V never written to HBM:
 //
 // * gather: one CTA per (image, query region, group of 64-channel blocks). The query tile and,
 //   per routed region, its K and V tiles (rs tokens x 64 channels each) arrive by TMA on

@@ -9,7 +9,7 @@
 // One work item = (image, query region, 64-channel block = 2 heads). Per CTA, 6 warps:
 //  * warp 0 lane 0, producer: TMA loads of the query tile (64 tokens x 64 channels) into a
 //    ring of query slots and, per routed region, of its K and V tiles into a ring of KV
-//    slots (128-byte swizzle, no multicast), as in the mma.sync gather kernel;
+//    slots (128-byte swizzle, each CTA loading its own tiles), as in the mma.sync gather kernel;
 //  * warp 1: allocates 256 TMEM columns (two S buffers at columns 0 and 64, two O buffers at
 //    128 and 192); its lane 0 issues every MMA. Per routed region:
 //      S_h = Q_h K_h^T  (M = 64 query rows, N = 64 keys, K = 32 channels of head h), head 0

@@ -169,7 +169,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 4-D tiled load of one box into shared memory, completing on `bar` (no multicast).
+// 4-D tiled load of one box into shared memory, completing on `bar`; only this CTA receives it.
 __device__ __forceinline__ void tma_load_5d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, int c3, int c4,
                                             uint64_t *bar)
 {
@@ -191,7 +191,7 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, i
 }
 
 // Contiguous bulk copy global -> shared of `bytes` (a multiple of 16, both addresses 16-byte
-// aligned), completing on `bar` (no multicast).
+// aligned), completing on `bar`; only this CTA receives it.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
 {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
