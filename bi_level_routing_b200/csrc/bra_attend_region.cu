@@ -151,8 +151,6 @@ __global__ void __launch_bounds__(32 * kRegionWarps, 1) attend_region_mma_kernel
 
         for (int kc = 0; kc < a.keys; kc += 64) {
             const int nk = min(64, a.keys - kc);  // a multiple of 16
-            // S = Q K^T for the chunk's 8-key tiles: per head, the 8 tiles' ldmatrix first, then
-            // their MMAs side by side (independent accumulators)
             // staged row of keys kc + lane and kc + 32 + lane (-1: padding or a skipped region);
             // the ldmatrix rows of K and V come from these by shuffles
             int kra, krb;
@@ -171,6 +169,8 @@ __global__ void __launch_bounds__(32 * kRegionWarps, 1) attend_region_mma_kernel
                 const int kr = __shfl_sync(0xffffffffu, nt < 4 ? kra : krb, (8 * nt + (lane & 7)) & 31);
                 krow[nt] = kr >= 0 ? kr : 0;
             }
+            // S = Q K^T for the chunk's 8-key tiles: per head, four tiles' ldmatrix first, then
+            // their MMAs side by side (independent accumulators)
 #pragma unroll
             for (int hk = 0; hk < 4; ++hk) {
 #pragma unroll
