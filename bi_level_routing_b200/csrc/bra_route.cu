@@ -518,8 +518,9 @@ static cudaError_t launch_topk_any(const S *qm, const S *km, int32_t *idx, const
 // in warp order in shared memory and warp w selects the top-k of rows 2 w and 2 w + 1 as every
 // routing kernel does.
 //  * bf16 one-token regions (route_tokens_mma_kernel): the means are the tokens, and a product
-//    of two bf16 values is exact in fp32, so m16n8k16 bf16 MMAs with fp32 accumulation form the
-//    same sums of exact products as fp32 FMAs would (32-channel chunks, 8 channels per lane).
+//    of two bf16 values is exact in fp32, so m16n8k16 bf16 MMAs with fp32 accumulation add the
+//    same exact products an fp32 FMA path would, in another order (32-channel chunks, 8
+//    channels per lane).
 //  * fp32 means or tokens (route_tf32x3_kernel): each value is split into two tf32 parts,
 //    x = hi + lo with |x - hi - lo| <= 2^-22 |x|, and m16n8k8 tf32 MMAs add lo*hi, hi*lo and
 //    hi*hi (smallest first; lo*lo, below 2^-22 of the product, is left out). Every product is
