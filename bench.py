@@ -13,8 +13,10 @@ bra_route then bra_attend, with an event around every call, gives the per-kernel
 With N > 1 (torchrun), each rank runs its own batch (weak scaling, no data-path collective)
 and the time is the max over ranks.
 
-Prints one JSON line on rank 0. `--impl reference` times the CPU oracle on the host cores
-instead (a bounded sample of the same workload per step).
+The headline workload (--workload, stage1 by default) gives the line's top-level fields; every
+named workload is also timed the same way and reported under "per_config" (skip with
+--no-per-config). Prints one JSON line on rank 0. `--impl reference` times the CPU oracle on
+the host cores instead (a bounded sample of the same workload per step).
 """
 from __future__ import annotations
 
@@ -43,7 +45,7 @@ KERNEL_SOURCES = {"attend_gather_umma": "bi_level_routing_b200/csrc/bra_attend_u
                   "attend_simt": "bi_level_routing_b200/csrc/bra_attend_simt.cu"}
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
@@ -52,12 +54,15 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="time the headline workload only")
     ap.add_argument("--eager", action="store_true", help="do not capture CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--cpu-seconds-per-config", type=float, default=2.0,
+                    help="target CPU time of the oracle sample of each per_config workload")
     ap.add_argument("--soak-seconds", type=float, default=1.0,
                     help="identical untimed steps before the timed region, while clocks are sampled")
     ap.add_argument("--repeats", type=int, default=5, help="timed runs of K steps; the median is reported")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def peaks():
@@ -82,7 +87,7 @@ def recorded_traffic(kernel: str, workload: str):
     with open(path) as f:
         table = json.load(f)
     rec = table.get(kernel, {}).get(workload)
-    if not rec or rec.get("source_sha256") != source_sha(KERNEL_SOURCES[kernel]):
+    if not rec or kernel not in KERNEL_SOURCES or rec.get("source_sha256") != source_sha(KERNEL_SOURCES[kernel]):
         return None
     return rec.get("bytes_per_launch")
 
@@ -97,6 +102,7 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.lines = []
 
     def __enter__(self):
         try:
@@ -116,28 +122,31 @@ class ClockSampler:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
-        else:
-            self.lines = []
 
     def summary(self):
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return summarize_clocks(self.lines)
+
+
+def summarize_clocks(lines):
+    """Median SM clock, max clock and the throttle reasons seen, from nvidia-smi csv lines."""
+    sm, smax, reasons = [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for ln in lines:
+        parts = [p.strip() for p in ln.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            smax.append(float(parts[2]))
+        except ValueError:
+            continue
+        for name, val in zip(names, parts[5:9]):
+            if val.lower() == "active":
+                reasons.add(name)
+    if not sm:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+            "samples": len(sm)}
 
 
 def cpu_baseline(w, inp, seconds: float):
@@ -193,28 +202,39 @@ def run_reference(args, w, rank):
     print(json.dumps(line), flush=True)
 
 
-def main():
-    args = parse_args()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    from bi_level_routing_b200.workloads import WORKLOADS, make_inputs
-    w = WORKLOADS[args.workload]
-    if args.impl == "reference":
-        run_reference(args, w, rank)
-        return
+def step_roofline_us(w, pk) -> float:
+    """max(unique q/k/v/out bytes at HBM bandwidth, routed attention flops at the bf16 peak)."""
+    return max(w.unique_bytes() / (float(pk["hbm_gbs"]) * 1e9),
+               w.attention_flops() / (float(pk["bf16_tflops"]) * 1e12)) * 1e6
 
+
+def roofline_record(w, pk, pk_kind, step_us, kernel, kernel_us, route_us, breakdown_us):
+    """The step against its roofline (frac) and the dominant kernel's own figures (kernel_*)."""
+    hbm = float(pk["hbm_gbs"])
+    roof_us = step_roofline_us(w, pk)
+    achieved = w.unique_bytes() / (step_us * 1e-6) / 1e9
+    kernel_achieved = w.unique_bytes() / (kernel_us * 1e-6) / 1e9
+    return {"bound": "hbm", "scope": "bra_forward step (every kernel of the call)",
+            "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+            "traffic": None,
+            "peak_source": f"{pk_kind} hbm_gbs (MEASURED_PEAKS.json)" if pk_kind == "measured" else "fallback",
+            "algorithmic_bytes_per_step": w.unique_bytes(), "step_roofline_us": roof_us, "step_us": step_us,
+            "step_frac_vs_8tbs": (w.unique_bytes() / 8e12 * 1e6) / step_us,
+            "dominant_kernel": {"name": kernel, "mean_launch_us": kernel_us, "achieved": kernel_achieved,
+                                "unit": "GB/s", "kernel_frac": kernel_achieved / hbm,
+                                "algorithmic_bytes_per_launch": w.unique_bytes(),
+                                "traffic": recorded_traffic(kernel, w.name)},
+            "route_kernels_mean_us": route_us, "breakdown_us_per_step": breakdown_us}
+
+
+def measure(w, args, dev, world, rank, with_warm=True):
+    """Times K steps of bra_forward on workload w (L2-cold rotation; one graph per run, median of
+    the runs), the breakdown of route / attend, and clocks during a soak around the runs."""
     import torch
     import torch.distributed as dist
     import bi_level_routing_b200 as bra
+    from bi_level_routing_b200.workloads import make_inputs
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-
-    # ---- inputs: one seeded batch per rank, resident in HBM; rotation sets are rolled copies
     inp = make_inputs(w, seed=w.seed + 1000 * rank)
     if w.dtype == "bf16":
         host = [torch.from_numpy(inp[n + "_bits"].view(np.int16)).view(torch.bfloat16) for n in "qkv"]
@@ -231,19 +251,17 @@ def main():
         out = torch.empty_like(q)
         idx = torch.empty((w.B, w.R, w.topk), dtype=torch.int32, device=dev)
         sets.append((q, k, v, out, idx))
+    del base
     torch.cuda.synchronize()
 
     def route(s):
-        q, k, v, out, idx = s
-        bra.route(q, k, w.n_win, w.topk, idx=idx)
+        bra.route(s[0], s[1], w.n_win, w.topk, idx=s[4])
 
     def attend(s):
-        q, k, v, out, idx = s
-        bra.attend(q, k, v, idx, w.heads, w.n_win, out=out)
+        bra.attend(s[0], s[1], s[2], s[4], w.heads, w.n_win, out=s[3])
 
     def forward(s):
-        q, k, v, out, idx = s
-        bra.forward(q, k, v, w.n_win, w.topk, w.heads, out=out, idx=idx)
+        bra.forward(s[0], s[1], s[2], w.n_win, w.topk, w.heads, out=s[3], idx=s[4])
 
     # eager warm-up (also initialises the library's per-device state before any capture)
     for i in range(max(3, args.warmup)):
@@ -252,13 +270,11 @@ def main():
         attend(sets[i % nsets])
     torch.cuda.synchronize()
 
-
-    # ---- the timed region: K steps of bra_forward, captured as ONE CUDA graph with a timing
-    # event (an external event-record node) before the first and after the last, so that host
-    # launch overhead does not pace the GPU and consecutive kernels keep their programmatic
-    # (overlapping) launches; eager launches if capture is refused. A second graph of K steps
-    # of bra_route then bra_attend, with an event around every call, gives the breakdown (the
-    # attention kernel's duration; in bra_forward the same kernel may also do the routing).
+    # The timed region: K steps of bra_forward captured as ONE CUDA graph with a timing event
+    # (an external event-record node) before the first and after the last, so that host launch
+    # overhead does not pace the GPU and consecutive kernels keep their programmatic
+    # (overlapping) launches; eager launches if capture is refused. A second graph of K steps of
+    # bra_route then bra_attend, with an event around every call, gives the breakdown.
     K = args.steps
     ev_start = torch.cuda.Event(enable_timing=True, external=True)
     ev_stop = torch.cuda.Event(enable_timing=True, external=True)
@@ -304,8 +320,7 @@ def main():
     run_breakdown()
     torch.cuda.synchronize()
 
-    # ---- clock samples over a soak of identical steps around the timed region
-    sampler = ClockSampler(local_rank)
+    sampler = ClockSampler(dev.index)
     with sampler:
         t_soak = time.perf_counter()
         while time.perf_counter() - t_soak < args.soak_seconds:
@@ -322,9 +337,7 @@ def main():
                 dist.barrier()
             torch.cuda.synchronize()
             runs.append(ev_start.elapsed_time(ev_stop))
-        repeat_ms = list(runs)
         total_ms = sorted(runs)[len(runs) // 2]  # the median run
-        # the per-kernel breakdown, from the graph with events around every call
         run_breakdown()
         torch.cuda.synchronize()
         attend_ms = [ev_attend[i].elapsed_time(ev_route[i + 1] if i + 1 < K else ev_end) for i in range(K)]
@@ -340,9 +353,8 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
 
-    # ---- secondary: warm L2, every step on the same buffer set (one graph of K steps)
     warm = None
-    if graph is not None:
+    if with_warm and graph is not None:
         ev_w0 = torch.cuda.Event(enable_timing=True, external=True)
         ev_w1 = torch.cuda.Event(enable_timing=True, external=True)
         try:
@@ -370,78 +382,117 @@ def main():
             warm = {"unavailable": f"{type(e).__name__}: {e}"}
             torch.cuda.synchronize()
 
-    tokens = w.tokens * world
-    value = tokens * K / (total_ms / 1e3)
-    ms_per_step = total_ms / K
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    kernel = "attend_" + str(bra.selected_attend_kernel(w.B, w.H, w.W, w.C, w.heads, w.n_win, w.topk, dt))
+    res = {"total_ms": total_ms, "ms_per_step": total_ms / K, "repeat_ms_per_step": [r / K for r in runs],
+           "attend_us": statistics.mean(attend_ms) * 1e3, "route_us": statistics.mean(route_ms) * 1e3,
+           "breakdown_us": breakdown_ms / K * 1e3, "kernel": kernel, "launch": launch, "warm": warm,
+           "clocks": sampler.summary(), "nsets": nsets, "set_bytes": set_bytes, "l2": l2,
+           "launches_per_step": bra.kernels_per_call("bra_forward", w.B, w.H, w.W, w.C, w.heads, w.n_win, w.topk, dt),
+           "host": host, "inp": inp}
+    del graph, graph_bd, sets
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
 
-    # ---- roofline of the dominant kernel
+
+def e2e_record(w, host, dev, world, K):
+    """bra_forward_host on pinned host buffers: copies in and out inside the timed region."""
+    import torch
+    import torch.distributed as dist
+    import bi_level_routing_b200 as bra
+    hq, hk, hv = (t.pin_memory() for t in host)
+    hout = torch.empty_like(hq).pin_memory()
+    hidx = torch.empty((w.B, w.R, w.topk), dtype=torch.int32).pin_memory()
+    for _ in range(2):
+        bra.forward_host(hq, hk, hv, w.n_win, w.topk, w.heads, out=hout, idx=hidx)
+    ke = max(3, min(20, K))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(ke):
+        bra.forward_host(hq, hk, hv, w.n_win, w.topk, w.heads, out=hout, idx=hidx)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    return {"value": w.tokens * world * ke / (e2e_ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": 3 * w.B * w.N * w.C * w.elem_bytes,
+            "d2h_bytes_per_step": w.B * w.N * w.C * w.elem_bytes + w.B * w.R * w.topk * 4,
+            "steps": ke, "entry_point": "bra_forward_host"}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from bi_level_routing_b200.workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
     pk, pk_kind = peaks()
-    hbm = float(pk["hbm_gbs"])
-    kernel = bra.selected_attend_kernel(w.B, w.H, w.W, w.C, w.heads, w.n_win, w.topk,
-                                        torch.bfloat16 if w.dtype == "bf16" else torch.float32)
-    kname = "attend_" + kernel
-    mean_attend = statistics.mean(attend_ms)
-    mean_route = statistics.mean(route_ms)
-    attend_bytes = w.unique_bytes()  # q, k, v read once, out written once
-    achieved = attend_bytes / (mean_attend / 1e3) / 1e9
-    traffic = recorded_traffic(kname, w.name)
-    roof_step_ms = max(w.unique_bytes() / (hbm * 1e9),
-                       w.attention_flops() / (float(pk["bf16_tflops"]) * 1e12)) * 1e3
-    roofline = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": traffic,
-                "peak_source": f"{pk_kind} hbm_gbs (MEASURED_PEAKS.json)" if pk_kind == "measured" else "fallback",
-                "algorithmic_bytes_per_launch": attend_bytes, "mean_launch_us": mean_attend * 1e3,
-                "route_kernels_mean_us": mean_route * 1e3,
-                "step_roofline_us": roof_step_ms * 1e3, "step_frac": roof_step_ms / ms_per_step,
-                "breakdown_ms_per_step": breakdown_ms / K,
-                "step_frac_vs_8tbs": (w.unique_bytes() / 8e12 * 1e3) / ms_per_step}
-
+    K = args.steps
+    m = measure(w, args, dev, world, rank)
+    tokens = w.tokens * world
+    value = tokens * K / (m["total_ms"] / 1e3)
+    step_us = m["ms_per_step"] * 1e3
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
-            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic",
-            "config": {**w.describe(), "l2": f"rotating {nsets} buffer sets of {set_bytes / 1e6:.1f} MB "
-                                             f"(> 2x the {l2 / 2**20:.0f} MiB L2)",
-                       "launch": launch, "parallelism": f"dp{world} (images split, no collective)"},
-            "roofline": roofline,
-            "gpu_launches": K * bra.kernels_per_call("bra_forward", w.B, w.H, w.W, w.C, w.heads, w.n_win, w.topk,
-                                                     torch.bfloat16 if w.dtype == "bf16" else torch.float32),
-            "clocks": sampler.summary(),
-            "repeats": {"runs": len(repeat_ms), "ms_per_step": [r / K for r in repeat_ms],
+            "config": {**w.describe(), "l2": f"rotating {m['nsets']} buffer sets of {m['set_bytes'] / 1e6:.1f} MB "
+                                             f"(> 2x the {m['l2'] / 2**20:.0f} MiB L2)",
+                       "launch": m["launch"], "parallelism": f"dp{world} (images split, no collective)"},
+            "roofline": roofline_record(w, pk, pk_kind, step_us, m["kernel"], m["attend_us"], m["route_us"],
+                                        m["breakdown_us"]),
+            "gpu_launches": K * m["launches_per_step"],
+            "clocks": m["clocks"],
+            "repeats": {"runs": len(m["repeat_ms_per_step"]), "ms_per_step": m["repeat_ms_per_step"],
                         "reported": "median run"}}
-    if warm is not None:
-        line["warm_l2"] = warm
-
-    # ---- end to end through the host entry point (pinned buffers, copies inside the timed region)
+    if m["warm"] is not None:
+        line["warm_l2"] = m["warm"]
     if not args.no_e2e:
-        hq, hk, hv = (t.pin_memory() for t in host)
-        hout = torch.empty_like(hq).pin_memory()
-        hidx = torch.empty((w.B, w.R, w.topk), dtype=torch.int32).pin_memory()
-        for _ in range(2):
-            bra.forward_host(hq, hk, hv, w.n_win, w.topk, w.heads, out=hout, idx=hidx)
-        ke = max(3, min(20, K))
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        e0.record()
-        for _ in range(ke):
-            bra.forward_host(hq, hk, hv, w.n_win, w.topk, w.heads, out=hout, idx=hidx)
-        e1.record()
-        torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        line["e2e"] = {"value": tokens * ke / (e2e_ms / 1e3), "unit": UNIT,
-                       "h2d_bytes_per_step": 3 * w.B * w.N * w.C * w.elem_bytes,
-                       "d2h_bytes_per_step": w.B * w.N * w.C * w.elem_bytes + w.B * w.R * w.topk * 4,
-                       "steps": ke, "entry_point": "bra_forward_host"}
-
+        line["e2e"] = e2e_record(w, m["host"], dev, world, K)
     if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(w, m["inp"], args.cpu_seconds)
 
-    del graph, graph_bd
+    # ---- every named workload, timed the same way (the headline's own entry repeats its numbers)
+    if not args.no_per_config:
+        per = {}
+        for name, wc in WORKLOADS.items():
+            mc = m if name == w.name else measure(wc, args, dev, world, rank, with_warm=False)
+            sus = mc["ms_per_step"] * 1e3
+            roof = roofline_record(wc, pk, pk_kind, sus, mc["kernel"], mc["attend_us"], mc["route_us"],
+                                   mc["breakdown_us"])
+            entry = {"value": wc.tokens * world / (sus * 1e-6), "unit": UNIT, "step_us": sus,
+                     "step_roofline_us": roof["step_roofline_us"], "step_frac": roof["frac"],
+                     "dominant_kernel": roof["dominant_kernel"], "route_us": mc["route_us"],
+                     "breakdown_us_per_step": mc["breakdown_us"], "gpu_launches_per_step": mc["launches_per_step"],
+                     "dtype": wc.dtype, "clocks": mc["clocks"], "config": wc.describe()}
+            if rank == 0 and not args.no_cpu_baseline:
+                entry["cpu_baseline"] = (line["cpu_baseline"] if name == w.name
+                                         else cpu_baseline(wc, mc["inp"], args.cpu_seconds_per_config))
+            per[name] = entry
+            if mc is not m:
+                del mc
+        line["per_config"] = per
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -5,5 +5,5 @@ The compute lives in ``libbra.so`` (hand-written CUDA behind a C ABI, declared i
 on first use and a missing library raises: there is no CPU fallback.
 """
 from .api import (BraError, attend, check_device_error, forward, forward_host, kernels_per_call,  # noqa: F401
-                  route, route_scratch_bytes, selected_attend_kernel, set_attend_kernel)
+                  route, route_scratch_bytes, selected_attend_kernel, set_attend_kernel, set_max_ctas)
 from .workloads import HEADLINE, WORKLOADS, Workload, make_inputs  # noqa: F401

@@ -46,6 +46,7 @@ def lib() -> ctypes.CDLL:
     L.bra_forward.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, I, I, I, I, vp]
     L.bra_forward_host.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, I, I, I, I, vp]
     L.bra_set_attend_kernel.argtypes = [I]
+    L.bra_set_max_ctas.argtypes = [I]
     L.bra_selected_attend_kernel.argtypes = [I, I, I, I, I, I, I, I]
     L.bra_check_device_error.argtypes = [vp]
     L.bra_route_scratch_bytes.argtypes = [I, I, I, I, I]
@@ -54,7 +55,7 @@ def lib() -> ctypes.CDLL:
     L.bra_status_string.argtypes = [I]
     L.bra_status_string.restype = ctypes.c_char_p
     L.bra_last_error_message.restype = ctypes.c_char_p
-    for name in ("bra_route", "bra_attend", "bra_forward", "bra_forward_host", "bra_set_attend_kernel",
+    for name in ("bra_route", "bra_attend", "bra_forward", "bra_forward_host", "bra_set_attend_kernel", "bra_set_max_ctas",
                  "bra_selected_attend_kernel", "bra_check_device_error", "bra_kernels_per_call"):
         getattr(L, name).restype = I
     _lib = L
@@ -175,6 +176,11 @@ def check_device_error(device=None) -> int:
 def set_attend_kernel(name: str):
     """Force one attention kernel ("simt", "gather_mma", "dense_mma", "gather_umma") or release ("auto")."""
     _check(lib().bra_set_attend_kernel(ATTEND_KERNELS[name]), "bra_set_attend_kernel")
+
+
+def set_max_ctas(n: int):
+    """Cap the persistent attention kernels' grid at n CTAs (0 = no cap); the result does not change."""
+    _check(lib().bra_set_max_ctas(int(n)), "bra_set_max_ctas")
 
 
 def selected_attend_kernel(B, H, W, C, heads, n_win, topk, dtype) -> str | None:

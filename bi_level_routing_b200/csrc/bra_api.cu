@@ -20,7 +20,7 @@ __device__ unsigned g_device_error;
 constexpr int kMaxDevices = 64;
 
 struct DeviceState {
-    bool ready = false;
+    std::atomic<bool> ready{false};  // set (release) after every other field
     unsigned *error_word = nullptr;
     cudaMemPool_t pool = nullptr;
     int num_sms = 0;
@@ -30,6 +30,7 @@ std::mutex g_mutex;
 DeviceState g_devices[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::atomic<int> g_forced_kernel{BRA_ATTEND_AUTO};
+std::atomic<int> g_max_ctas{0};
 thread_local std::string g_last_error;
 
 bra_status cuda_fail(cudaError_t e, const char *what)
@@ -49,9 +50,9 @@ bra_status device_state(DeviceState **out)
         return BRA_ERR_UNSUPPORTED;
     }
     DeviceState &st = g_devices[dev];
-    if (!st.ready) {
+    if (!st.ready.load(std::memory_order_acquire)) {
         std::lock_guard<std::mutex> lock(g_mutex);
-        if (!st.ready) {
+        if (!st.ready.load(std::memory_order_relaxed)) {
             void *p = nullptr;
             if ((e = cudaGetSymbolAddress(&p, g_device_error)) != cudaSuccess)
                 return cuda_fail(e, "cudaGetSymbolAddress(error word)");
@@ -77,7 +78,7 @@ bra_status device_state(DeviceState **out)
                 }
                 g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
             }
-            st.ready = true;
+            st.ready.store(true, std::memory_order_release);
         }
     }
     *out = &st;
@@ -179,8 +180,11 @@ bra_status encode_map_blocks(CUtensorMap *map, const void *base, const bra::Geom
     return BRA_OK;
 }
 
+// The routing step. `workspace` (may be NULL): caller memory of `ws_bytes` bytes, 16-byte
+// aligned, that nothing reads until the stream passes this call; the fp32 means go there when
+// they fit, else into scratch from the pool.
 bra_status route_impl(const void *q, const void *k, int32_t *idx, const bra::Geometry &g, bra_dtype dtype,
-                      cudaStream_t stream)
+                      cudaStream_t stream, void *workspace = nullptr, size_t ws_bytes = 0)
 {
     DeviceState *st = nullptr;
     bra_status s = device_state(&st);
@@ -191,21 +195,26 @@ bra_status route_impl(const void *q, const void *k, int32_t *idx, const bra::Geo
         return e == cudaSuccess ? BRA_OK : cuda_fail(e, "routing kernel");
     }
     const size_t bytes = (size_t)2 * g.B * g.R * g.C * sizeof(float);
-    void *scratch = nullptr;
-    cudaError_t e = cudaMallocFromPoolAsync(&scratch, bytes, st->pool, stream);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync(route scratch)");
+    const bool in_workspace = workspace && bytes <= ws_bytes;
+    void *scratch = in_workspace ? workspace : nullptr;
+    cudaError_t e = cudaSuccess;
+    if (!in_workspace && (e = cudaMallocFromPoolAsync(&scratch, bytes, st->pool, stream)) != cudaSuccess)
+        return cuda_fail(e, "cudaMallocFromPoolAsync(route scratch)");
     float *qm = static_cast<float *>(scratch);
     float *km = qm + (size_t)g.B * g.R * g.C;
     e = bra::launch_region_means(q, k, qm, km, g, dtype == BRA_BF16, st->num_sms, stream);
     if (e == cudaSuccess) e = bra::launch_route_topk(qm, km, idx, g, stream);
-    cudaError_t f = cudaFreeAsync(scratch, stream);
+    cudaError_t f = in_workspace ? cudaSuccess : cudaFreeAsync(scratch, stream);
     if (e != cudaSuccess) return cuda_fail(e, "routing kernels");
     if (f != cudaSuccess) return cuda_fail(f, "cudaFreeAsync(route scratch)");
     return BRA_OK;
 }
 
+// inputs_ready: the kernel launched just before on `stream` is this library's routing kernel,
+// which has already waited for the producers of q, k and v, so the attention kernel may read
+// them before it waits for its predecessor (only idx comes from that kernel).
 bra_status attend_impl(const void *q, const void *k, const void *v, const int32_t *idx, void *out,
-                       const bra::Geometry &g, bra_dtype dtype, cudaStream_t stream)
+                       const bra::Geometry &g, bra_dtype dtype, cudaStream_t stream, bool inputs_ready = false)
 {
     const int kernel = choose_attend_kernel(g, dtype);
     if (kernel < 0) return BRA_ERR_UNSUPPORTED;
@@ -226,7 +235,7 @@ bra_status attend_impl(const void *q, const void *k, const void *v, const int32_
         if ((s = encode_map_blocks(&tq, q, g, g.W, g.H, 2)) != BRA_OK) return s;
         if ((s = encode_map_blocks(&tk, k, g, g.W, g.H, 2)) != BRA_OK) return s;
         if ((s = encode_map_blocks(&tv, v, g, g.W, g.H, 2)) != BRA_OK) return s;
-        e = bra::launch_attend_region_mma(tq, tk, tv, idx, out, g, st->num_sms, st->error_word, stream);
+        e = bra::launch_attend_region_mma(tq, tk, tv, idx, out, g, st->num_sms, st->error_word, inputs_ready, stream);
     } else if (kernel == BRA_ATTEND_GATHER_MMA) {
         CUtensorMap tq, tk, tv, to;
         int box[5];
@@ -243,7 +252,7 @@ bra_status attend_impl(const void *q, const void *k, const void *v, const int32_
         if ((s = encode_map(&tk, k, g, g.W, g.H)) != BRA_OK) return s;
         if ((s = encode_map(&tv, v, g, g.W, g.H)) != BRA_OK) return s;
         if ((s = encode_map(&to, out, g, g.W, rows)) != BRA_OK) return s;
-        e = bra::launch_attend_dense_mma(tq, tk, tv, to, idx, g, rows, st->error_word, stream);
+        e = bra::launch_attend_dense_mma(tq, tk, tv, to, idx, g, rows, st->error_word, inputs_ready, stream);
     }
     if (e != cudaSuccess) return cuda_fail(e, "attention kernel");
     return BRA_OK;
@@ -254,6 +263,15 @@ bra_status attend_impl(const void *q, const void *k, const void *v, const int32_
 namespace bra {
 
 void set_last_error(const std::string &msg) { g_last_error = msg; }
+
+int persistent_grid(long long nitems, int num_sms)
+{
+    long long grid = 2LL * num_sms;
+    const int cap = g_max_ctas.load();
+    if (cap > 0 && grid > cap) grid = cap;
+    if (grid > nitems) grid = nitems;
+    return grid < 1 ? 1 : (int)grid;
+}
 
 bra_status check_route_args(const void *q, const void *k, const int32_t *idx, int B, int H, int W, int C, int n_win,
                             int topk, bra_dtype dtype, Geometry *g)
@@ -306,8 +324,10 @@ bra_status bra_forward(const void *q, const void *k, const void *v, int32_t *idx
         return BRA_ERR_INVALID_ARG;
     if (choose_attend_kernel(g, dtype) < 0) return BRA_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if ((s = route_impl(q, k, idx, g, dtype, st)) != BRA_OK) return s;
-    return attend_impl(q, k, v, idx, out, g, dtype, st);
+    // out is written only by the attention kernel, after routing: until then it holds the means
+    const size_t out_bytes = (size_t)B * H * W * C * (dtype == BRA_BF16 ? 2 : 4);
+    if ((s = route_impl(q, k, idx, g, dtype, st, out, out_bytes)) != BRA_OK) return s;
+    return attend_impl(q, k, v, idx, out, g, dtype, st, true);
 }
 
 bra_status bra_forward_host(const void *q, const void *k, const void *v, int32_t *idx, void *out, int B, int H,
@@ -335,8 +355,8 @@ bra_status bra_forward_host(const void *q, const void *k, const void *v, int32_t
     if (e == cudaSuccess) e = cudaMemcpyAsync(dk, k, tensor, cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = cudaMemcpyAsync(dv, v, tensor, cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) {
-        s = route_impl(dq, dk, didx, g, dtype, st);
-        if (s == BRA_OK) s = attend_impl(dq, dk, dv, didx, dout, g, dtype, st);
+        s = route_impl(dq, dk, didx, g, dtype, st, dout, tensor);
+        if (s == BRA_OK) s = attend_impl(dq, dk, dv, didx, dout, g, dtype, st, true);
         if (s == BRA_OK) e = cudaMemcpyAsync(idx, didx, idx_bytes, cudaMemcpyDeviceToHost, st);
         if (s == BRA_OK && e == cudaSuccess) e = cudaMemcpyAsync(out, dout, tensor, cudaMemcpyDeviceToHost, st);
     }
@@ -353,6 +373,13 @@ bra_status bra_set_attend_kernel(bra_attend_kernel kernel)
 {
     if (kernel < BRA_ATTEND_AUTO || kernel > BRA_ATTEND_REGION_MMA) return BRA_ERR_INVALID_ARG;
     g_forced_kernel.store(kernel);
+    return BRA_OK;
+}
+
+bra_status bra_set_max_ctas(int max_ctas)
+{
+    if (max_ctas < 0) return BRA_ERR_INVALID_ARG;
+    g_max_ctas.store(max_ctas);
     return BRA_OK;
 }
 

@@ -462,8 +462,7 @@ cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &t
     a.idx_chunk = g.topk >= 32 ? 1 : 32 / g.topk;
     const size_t smem = 1024 + tile * (a.qslots + 2 * a.kvslots) + 16 * (a.qslots + a.kvslots) + 4 * a.kvslots +
                         sizeof(ItemInfo) * a.qslots + 4 * (size_t)a.idx_chunk * g.topk;
-    int grid = 2 * num_sms;
-    if (grid > a.nitems) grid = a.nitems;
+    int grid = persistent_grid(a.nitems, num_sms);
     a.per_cta = (a.nitems + grid - 1) / grid;
     grid = (a.nitems + a.per_cta - 1) / a.per_cta;
     switch (g.rs) {
@@ -485,6 +484,7 @@ struct DenseArgs {
     int rows_per_split;  // image rows of queries per CTA
     int nsplit;
     float scale_log2;
+    int inputs_ready;  // q, k, v may be loaded before the wait for the previous kernel
 };
 
 // MIN_CTAS: CTAs per SM the registers are budgeted for (2, or 3 when three CTAs' shared memory
@@ -518,13 +518,15 @@ __global__ void __launch_bounds__(256, MIN_CTAS) attend_dense_mma_kernel(const _
     const int b = (int)(item / a.ncb);
     const int y0 = split * a.rows_per_split;
     const int32_t *routed = a.idx + (int64_t)b * a.R * a.topk;
-    grid_dependency_wait();
 
     if (threadIdx.x == 0) {
         mbar_init(bar, 1);
         mbar_fence_init();
     }
     __syncthreads();
+    // q, k and v: before the wait for the previous kernel when that kernel is the routing step of
+    // the same forward pass (it already waited for their producers), else after it
+    if (!a.inputs_ready) grid_dependency_wait();
     if (threadIdx.x == 0) {
         mbar_arrive_expect_tx(bar, (uint32_t)((nq + 2 * a.N) * kRowBytes));
         tma_load_4d(sQ, &tq, cb * 64, 0, y0, b, bar);
@@ -541,16 +543,28 @@ __global__ void __launch_bounds__(256, MIN_CTAS) attend_dense_mma_kernel(const _
     for (int t = threadIdx.x; t < a.npad; t += blockDim.x)
         reg[t] = t < a.N ? (uint8_t)(((t / a.W) / a.hr) * a.n_win + (t % a.W) / a.wr) : 0;
     for (int e = threadIdx.x; e < a.R * a.R; e += blockDim.x) cnt[e] = 0;
+    if (a.inputs_ready) grid_dependency_wait();  // idx comes from the previous kernel
     __syncthreads();
-    // multiplicity of every routed region: warp w takes query regions w, w + 8, ..., a lane per
-    // idx entry of the row (all loads of a row in flight)
-    for (int r = warp; r < a.R; r += nwarps) {
-        for (int j = lane; j < a.topk; j += 32) {
-            const int s = routed[r * a.topk + j];
-            if (s >= 0 && s < a.R)
-                atomicAdd(&cnt[r * a.R + s], 1);
-            else if (cb == 0 && split == 0)
-                flag_error(a.err, kErrIndex);
+    // multiplicity of every routed region: the image's idx entries, eight loads per thread in
+    // flight at once, then one shared-memory count per entry
+    const int nent = a.R * a.topk;
+    for (int e0 = threadIdx.x; e0 < nent; e0 += 8 * blockDim.x) {
+        int sv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = e0 + u * blockDim.x;
+            sv[u] = e < nent ? routed[e] : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = e0 + u * blockDim.x;
+            if (e < nent) {
+                const int s = sv[u];
+                if (s >= 0 && s < a.R)
+                    atomicAdd(&cnt[(e / a.topk) * a.R + s], 1);
+                else if (cb == 0 && split == 0)
+                    flag_error(a.err, kErrIndex);
+            }
         }
     }
     __syncthreads();
@@ -666,9 +680,10 @@ static size_t dense_smem_bytes(const Geometry &g, int rows_per_split)
 
 cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                     const CUtensorMap &tout, const int32_t *idx, const Geometry &g, int rows_per_split,
-                                    unsigned *err, cudaStream_t stream)
+                                    unsigned *err, bool inputs_ready, cudaStream_t stream)
 {
     DenseArgs a;
+    a.inputs_ready = inputs_ready ? 1 : 0;
     a.idx = idx;
     a.err = err;
     a.H = g.H;

@@ -42,6 +42,7 @@ struct RegionArgs {
     int nsplit;   // CTAs per (image, group); query regions are dealt among them
     int keys;     // 4 topk rounded up to a multiple of 16
     float scale_log2;
+    int inputs_ready;  // q, k, v may be loaded before the wait for the previous kernel
 };
 
 // bytes of one staged tensor (two 64-channel tiles of N rows, then one spare row: zeros, in the
@@ -87,19 +88,22 @@ __global__ void __launch_bounds__(32 * kRegionWarps, 1) attend_region_mma_kernel
     item /= a.nsplit;
     const int grp = item % a.ngroups;
     const int b = item / a.ngroups;
-    grid_dependency_wait();
 
     if (threadIdx.x == 0) {
         mbar_init(bar, 1);
         mbar_fence_init();
     }
     __syncthreads();
+    // q, k and v: before the wait for the previous kernel when that kernel is the routing step of
+    // the same forward pass (it already waited for their producers), else after it
+    if (!a.inputs_ready) grid_dependency_wait();
     if (threadIdx.x == 0) {
         mbar_arrive_expect_tx(bar, (uint32_t)(3 * 2 * a.N * 128));
         tma_load_5d(sQ, &tq, 0, 0, 0, 2 * grp, b, bar);
         tma_load_5d(sK, &tk, 0, 0, 0, 2 * grp, b, bar);
         tma_load_5d(sV, &tv, 0, 0, 0, 2 * grp, b, bar);
     }
+    if (a.inputs_ready) grid_dependency_wait();  // idx comes from the previous kernel
     // V row 2 N: zeros, read for padding keys and skipped regions (their p is 0, and 0 times a
     // non-finite value in a real row would not be)
     if (threadIdx.x < 8) reinterpret_cast<uint4 *>(sV + (size_t)2 * a.N * 128)[threadIdx.x] = make_uint4(0, 0, 0, 0);
@@ -302,9 +306,10 @@ bool region_mma_supports(const Geometry &g)
 
 cudaError_t launch_attend_region_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                      const int32_t *idx, void *out, const Geometry &g, int num_sms, unsigned *err,
-                                     cudaStream_t stream)
+                                     bool inputs_ready, cudaStream_t stream)
 {
     RegionArgs a;
+    a.inputs_ready = inputs_ready ? 1 : 0;
     a.idx = idx;
     a.err = err;
     a.out = static_cast<__nv_bfloat16 *>(out);

@@ -459,8 +459,7 @@ cudaError_t launch_attend_gather_umma(const CUtensorMap &tq, const CUtensorMap &
     a.idx_chunk = g.topk >= 32 ? 1 : 32 / g.topk;
     const size_t smem = 1024 + (size_t)kTile * (a.qslots + 2 * a.kvslots) + 8 * (2 * a.qslots + 2 * a.kvslots + 9) +
                         4 * a.kvslots + 4 + 4 * (size_t)a.idx_chunk * g.topk;
-    int grid = 2 * num_sms;
-    if (grid > a.nitems) grid = a.nitems;
+    int grid = persistent_grid(a.nitems, num_sms);
     a.per_cta = (a.nitems + grid - 1) / grid;
     grid = (a.nitems + a.per_cta - 1) / a.per_cta;
     static int granted[64] = {0};

@@ -46,6 +46,10 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // Sets the message bra_last_error_message returns on this thread.
 void set_last_error(const std::string &msg);
 
+// Grid of a persistent attention kernel over `nitems` work items: two CTAs per SM, at most
+// one CTA per item, and at most the cap set by bra_set_max_ctas (0 = none).
+int persistent_grid(long long nitems, int num_sms);
+
 // The argument checks of bra_route (shape, NULL pointers, alignment); fills g.
 bra_status check_route_args(const void *q, const void *k, const int32_t *idx, int B, int H, int W, int C, int n_win,
                             int topk, bra_dtype dtype, Geometry *g);
@@ -93,9 +97,12 @@ bool dense_mma_supports(const Geometry &g);
 // Stacked-head gather attention for 4-token regions (bf16, hd == 32, C % 128 == 0, N <= 256,
 // topk <= 64). Maps: q, k, v as 5-D views, box (64, W, H, 2, 1).
 bool region_mma_supports(const Geometry &g);
+// inputs_ready (here and for the dense kernel): q, k and v may be loaded before the kernel waits
+// for its predecessor on the stream (true when that predecessor is the routing kernel of the same
+// forward pass, which already waited for their producers); idx is read after the wait.
 cudaError_t launch_attend_region_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                      const int32_t *idx, void *out, const Geometry &g, int num_sms, unsigned *err,
-                                     cudaStream_t stream);
+                                     bool inputs_ready, cudaStream_t stream);
 
 // Box of the gather kernel's q, k and v maps: (64 channels, wr, hr, NCB channel blocks, 1 image)
 // on the 5-D view (channel in block, x, y, channel block, image) of [B, H, W, C], so that one
@@ -117,6 +124,6 @@ cudaError_t launch_attend_gather_umma(const CUtensorMap &tq, const CUtensorMap &
 int dense_mma_rows_per_split(const Geometry &g, int num_sms);
 cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                     const CUtensorMap &tout, const int32_t *idx, const Geometry &g,
-                                    int rows_per_split, unsigned *err, cudaStream_t stream);
+                                    int rows_per_split, unsigned *err, bool inputs_ready, cudaStream_t stream);
 
 }  // namespace bra

@@ -19,6 +19,7 @@
 // overwrite every element they read, so nothing needs clearing between calls. Two calls
 // whose kernels overlap on the GPU (two streams, or two host threads) race on the array:
 // order them on one stream.
+#include <atomic>
 #include <cstdio>
 #include <mutex>
 
@@ -35,7 +36,7 @@ constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
 static __device__ __align__(256) float g_route_scratch[kNoAllocScratchBytes / sizeof(float)];
 
 struct NoAllocDevice {
-    bool ready = false;
+    std::atomic<bool> ready{false};  // set (release) after scratch and num_sms
     float *scratch = nullptr;  // device address of g_route_scratch on this device
     int num_sms = 0;
 };
@@ -58,9 +59,9 @@ bra_status noalloc_setup(NoAllocDevice **out)
         return BRA_ERR_UNSUPPORTED;
     }
     NoAllocDevice &st = g_noalloc_devices[dev];
-    if (!st.ready) {
+    if (!st.ready.load(std::memory_order_acquire)) {
         std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-        if (!st.ready) {
+        if (!st.ready.load(std::memory_order_relaxed)) {
             float *p = nullptr;
             e = cudaGetSymbolAddress((void **)&p, g_route_scratch);
             if (e != cudaSuccess) {
@@ -75,7 +76,7 @@ bra_status noalloc_setup(NoAllocDevice **out)
             }
             st.scratch = p;
             st.num_sms = sms;
-            st.ready = true;
+            st.ready.store(true, std::memory_order_release);
         }
     }
     *out = &st;

@@ -132,6 +132,14 @@ bra_status bra_forward_host(const void *q, const void *k, const void *v, int32_t
    Returns BRA_ERR_INVALID_ARG for an unknown value. */
 bra_status bra_set_attend_kernel(bra_attend_kernel kernel);
 
+/* Caps the grid of the persistent attention kernels (the tcgen05 and the mma.sync gather
+   kernels, which split the work items of a call evenly over at most two CTAs per SM) at
+   max_ctas CTAs for later calls in this process; 0 removes the cap. A small cap gives each
+   CTA many consecutive work items, which tests use to exercise the carried state between
+   items on small inputs. The result does not depend on it. Returns BRA_ERR_INVALID_ARG for
+   max_ctas < 0. */
+bra_status bra_set_max_ctas(int max_ctas);
+
 /* The attention kernel a call with these arguments would use (after any forcing), or -1 if
    the call would be rejected or unsupported. */
 int bra_selected_attend_kernel(int B, int H, int W, int C, int heads, int n_win, int topk, bra_dtype dtype);

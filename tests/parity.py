@@ -73,6 +73,23 @@ def check_routing(gpu_idx: np.ndarray, q: np.ndarray, k: np.ndarray, n_win: int,
     return orc_idx, near
 
 
+def value_relative_rejects(gpu_idx: np.ndarray, orc_idx: np.ndarray, A: np.ndarray) -> int:
+    """Rows the acceptance rule took as near-ties that a rule relative to the affinity VALUES,
+    |A_gpu - A_orc| <= 1e-5 * max(|A_gpu|, |A_orc|) at every differing position, would reject
+    (a report of how much looser the terms-magnitude measure is on real inputs)."""
+    gpu_idx = np.asarray(gpu_idx)
+    rejects = 0
+    for b, r in np.argwhere(np.any(gpu_idx != orc_idx, axis=-1)):
+        for a, o in zip(gpu_idx[b, r], orc_idx[b, r]):
+            if a == o:
+                continue
+            va, vo = A[b, r, a], A[b, r, o]
+            if not abs(va - vo) <= ROUTE_REL_TOL * max(abs(va), abs(vo)):
+                rejects += 1
+                break
+    return rejects
+
+
 def check_output(gpu: np.ndarray, ref: np.ndarray, dtype: str, what: str = "out"):
     gpu = np.asarray(gpu, np.float64)
     ref = np.asarray(ref, np.float64)

@@ -5,8 +5,9 @@ bra_route: a process that hands all of HBM to its own allocator at start-up, or 
 latency-critical loop that must not take allocator locks or risk an out-of-memory error.
 Its scratch is a fixed array inside the library, shared by every call, so this test makes
 two calls in a row on different shapes and checks that each returns exactly bra_route's
-indices (the same kernels run, so the routing must be bit-identical). One-token regions need
-no scratch at all. It sits in a file of its own, collected last.
+indices (the same kernels run, so the routing must be bit-identical). Shapes that route on chip
+(one-token regions, and up to 256 regions of several tokens) need no scratch at all; the others
+use the fixed array. It sits in a file of its own, collected last.
 """
 import ctypes
 
@@ -15,7 +16,7 @@ import torch
 
 import bi_level_routing_b200 as bra
 from bi_level_routing_b200 import api
-from bi_level_routing_b200.workloads import WORKLOADS
+from bi_level_routing_b200.workloads import WORKLOADS, Workload
 from parity import make
 
 pytestmark = pytest.mark.gpu
@@ -35,22 +36,38 @@ def _route_noalloc(L, q, k, idx, n_win, topk):
                                api.DTYPES[q.dtype], torch.cuda.current_stream().cuda_stream)
 
 
+# Shapes the on-chip routing kernel does not take (more than 256 regions) use the fixed scratch;
+# the named workloads route on chip and need none. Both kinds, two calls in a row.
+WIDE = Workload("r400_rs4", 2, 40, 40, 64, 2, 20, 6, "bf16", "region_offset", 31)
+WIDE_F32 = Workload("r324_rs4_f32", 3, 36, 36, 32, 1, 18, 5, "f32", "region_offset", 32)
+
+
 def test_no_alloc_route_matches_bra_route_on_two_calls_in_a_row():
     L = _lib()
-    for w in (WORKLOADS["stage1"].with_(B=16), WORKLOADS["highres"].with_(B=2)):
+    for w in (WIDE, WORKLOADS["stage1"].with_(B=16), WIDE_F32, WORKLOADS["highres"].with_(B=2)):
         _, (q, k, _) = make(w)
         ref = bra.route(q, k, w.n_win, w.topk)
         idx = torch.full_like(ref, -7)
         assert _route_noalloc(L, q, k, idx, w.n_win, w.topk) == 0, L.bra_last_error_message()
         torch.cuda.synchronize()
         assert torch.equal(idx, ref), f"{w.name}: bra_route_noalloc differs from bra_route"
+    # the largest of these that fits the fixed scratch: 2 * 24 * 400 * 64 * 4 bytes = 4.9 MB
+    w = WIDE.with_(B=24)
+    assert 2 * w.B * w.R * w.C * 4 <= 8 << 20
+    _, (q, k, _) = make(w)
+    ref = bra.route(q, k, w.n_win, w.topk)
+    idx = torch.full_like(ref, -7)
+    assert _route_noalloc(L, q, k, idx, w.n_win, w.topk) == 0, L.bra_last_error_message()
+    torch.cuda.synchronize()
+    assert torch.equal(idx, ref), "full-scratch call differs from bra_route"
 
 
 def test_no_alloc_route_rejects_sizes_beyond_its_scratch():
     L = _lib()
-    # four-token regions, so the means need scratch: 2 * 128 * 49 * 256 * 4 bytes = 12.8 MB > 8 MiB
-    w = WORKLOADS["stage3"].with_(B=128)
-    assert w.H // w.n_win * (w.W // w.n_win) > 1
+    # more than 256 four-token regions, so the means go through scratch:
+    # 2 * 16 * 400 * 256 * 4 bytes = 13.1 MB > 8 MiB
+    w = WIDE.with_(B=16, C=256, heads=8)
+    assert w.H // w.n_win * (w.W // w.n_win) > 1 and w.R > 256
     fake = 0x10000  # rejected before any use
     status = L.bra_route_noalloc(fake, fake, fake, w.B, w.H, w.W, w.C, w.n_win, w.topk, 1, None)
     assert status == 2  # BRA_ERR_UNSUPPORTED
