@@ -68,8 +68,16 @@ class Oracle:
         lib.oracle_attend_tokens.argtypes = [_DP, _DP, _DP, _IP, _I, _I, _I, _I, _I, _I, _I, _LP,
                                              ctypes.c_int64, _DP]
         lib.oracle_forward.argtypes = [_DP, _DP, _DP, _I, _I, _I, _I, _I, _I, _I, _IP, _DP]
+        lib.oracle_route_heads.argtypes = [_DP, _DP, _I, _I, _I, _I, _I, _I, _I, _IP, _DP]
+        lib.oracle_attend_heads.argtypes = [_DP, _DP, _DP, _IP, _I, _I, _I, _I, _I, _I, _I, _DP]
+        lib.oracle_lepe.argtypes = [_DP, _DP, _DP, _I, _I, _I, _I, _DP]
+        lib.oracle_attend_backward.argtypes = [_DP, _DP, _DP, _IP, _DP, _I, _I, _I, _I, _I, _I, _I, _DP, _DP, _DP]
+        lib.oracle_forward_auto_pad.argtypes = [_DP, _DP, _DP, _I, _I, _I, _I, _I, _I, _I, _IP, _DP]
+        lib.oracle_attend_auto_pad.argtypes = [_DP, _DP, _DP, _IP, _I, _I, _I, _I, _I, _I, _I, _DP]
         for name in ("oracle_region_means", "oracle_affinity", "oracle_topk", "oracle_route",
-                     "oracle_attend", "oracle_attend_tokens", "oracle_forward"):
+                     "oracle_attend", "oracle_attend_tokens", "oracle_forward", "oracle_route_heads",
+                     "oracle_attend_heads", "oracle_lepe", "oracle_attend_backward", "oracle_forward_auto_pad",
+                     "oracle_attend_auto_pad"):
             getattr(lib, name).restype = _I
         self._lib = lib
         self.path = path
@@ -162,6 +170,77 @@ class Oracle:
                                              idx.ctypes.data_as(_IP), out.ctypes.data_as(_DP)), "forward")
         return out, idx
 
+    def route_heads(self, q, k, n_win: int, topk: int, heads: int, want_affinity: bool = False):
+        """Per-head routing ("医学图像分割模块", §五 steps ③④): idx int32 [B, heads, R, min(topk, R)]
+        (and optionally the per-head affinities [B, heads, R, R], scale head_dim^-1/2)."""
+        q, k = _f64(q), _f64(k)
+        B, H, W, C = q.shape
+        R = n_win * n_win
+        kk = min(topk, R)
+        idx = np.empty((B, heads, R, kk), np.int32)
+        A = np.empty((B, heads, R, R), np.float64) if want_affinity else None
+        self._check(self._lib.oracle_route_heads(q.ctypes.data_as(_DP), k.ctypes.data_as(_DP), B, H, W, C, heads,
+                                                 n_win, topk, idx.ctypes.data_as(_IP),
+                                                 A.ctypes.data_as(_DP) if A is not None else None), "route_heads")
+        return (idx, A) if want_affinity else idx
+
+    def attend_heads(self, q, k, v, idx, n_win: int) -> np.ndarray:
+        """Attention with per-head index rows idx [B, heads, R, topk] ("医学图像分割模块", §五 ⑤-⑦)."""
+        q, k, v, idx = _f64(q), _f64(k), _f64(v), _i32(idx)
+        B, H, W, C = q.shape
+        heads, topk = idx.shape[1], idx.shape[-1]
+        out = np.empty_like(q)
+        self._check(self._lib.oracle_attend_heads(q.ctypes.data_as(_DP), k.ctypes.data_as(_DP),
+                                                  v.ctypes.data_as(_DP), idx.ctypes.data_as(_IP), B, H, W, C,
+                                                  heads, n_win, topk, out.ctypes.data_as(_DP)), "attend_heads")
+        return out
+
+    def lepe(self, x, weight, bias) -> np.ndarray:
+        """x + 5x5 depthwise convolution of x (zero padding 2) + bias ("医学图像分割模块", §五 ⑧);
+        x [B, H, W, C], weight [C, 5, 5], bias [C]."""
+        x, weight, bias = _f64(x), _f64(weight), _f64(bias)
+        B, H, W, C = x.shape
+        assert weight.shape == (C, 5, 5) and bias.shape == (C,)
+        y = np.empty_like(x)
+        self._check(self._lib.oracle_lepe(x.ctypes.data_as(_DP), weight.ctypes.data_as(_DP),
+                                          bias.ctypes.data_as(_DP), B, H, W, C, y.ctypes.data_as(_DP)), "lepe")
+        return y
+
+    def attend_backward(self, q, k, v, idx, dout, heads: int, n_win: int):
+        """(dq, dk, dv): gradients of sum(dout * attend(q, k, v, idx)) with idx held fixed."""
+        q, k, v, idx, dout = _f64(q), _f64(k), _f64(v), _i32(idx), _f64(dout)
+        B, H, W, C = q.shape
+        dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+        self._check(self._lib.oracle_attend_backward(
+            q.ctypes.data_as(_DP), k.ctypes.data_as(_DP), v.ctypes.data_as(_DP), idx.ctypes.data_as(_IP),
+            dout.ctypes.data_as(_DP), B, H, W, C, heads, n_win, idx.shape[-1], dq.ctypes.data_as(_DP),
+            dk.ctypes.data_as(_DP), dv.ctypes.data_as(_DP)), "attend_backward")
+        return dq, dk, dv
+
+    def forward_auto_pad(self, q, k, v, n_win: int, topk: int, heads: int):
+        """auto_pad ("从静态到动态", §4.2): zero-pad to multiples of n_win, route + attend, crop.
+        Returns (out [B, H, W, C], idx [B, R, topk] of the padded map)."""
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        B, H, W, C = q.shape
+        idx = np.empty((B, n_win * n_win, topk), np.int32)
+        out = np.empty_like(q)
+        self._check(self._lib.oracle_forward_auto_pad(q.ctypes.data_as(_DP), k.ctypes.data_as(_DP),
+                                                      v.ctypes.data_as(_DP), B, H, W, C, heads, n_win, topk,
+                                                      idx.ctypes.data_as(_IP), out.ctypes.data_as(_DP)),
+                    "forward_auto_pad")
+        return out, idx
+
+    def attend_auto_pad(self, q, k, v, idx, heads: int, n_win: int) -> np.ndarray:
+        """Step 5 of auto_pad with a given index of the padded map."""
+        q, k, v, idx = _f64(q), _f64(k), _f64(v), _i32(idx)
+        B, H, W, C = q.shape
+        out = np.empty_like(q)
+        self._check(self._lib.oracle_attend_auto_pad(q.ctypes.data_as(_DP), k.ctypes.data_as(_DP),
+                                                     v.ctypes.data_as(_DP), idx.ctypes.data_as(_IP), B, H, W, C,
+                                                     heads, n_win, idx.shape[-1], out.ctypes.data_as(_DP)),
+                    "attend_auto_pad")
+        return out
+
 
 _default: Oracle | None = None
 
@@ -204,3 +283,27 @@ def forward(q, k, v, n_win, topk, heads):
 
 def max_threads():
     return default().max_threads()
+
+
+def route_heads(q, k, n_win, topk, heads, want_affinity=False):
+    return default().route_heads(q, k, n_win, topk, heads, want_affinity)
+
+
+def attend_heads(q, k, v, idx, n_win):
+    return default().attend_heads(q, k, v, idx, n_win)
+
+
+def lepe(x, weight, bias):
+    return default().lepe(x, weight, bias)
+
+
+def attend_backward(q, k, v, idx, dout, heads, n_win):
+    return default().attend_backward(q, k, v, idx, dout, heads, n_win)
+
+
+def forward_auto_pad(q, k, v, n_win, topk, heads):
+    return default().forward_auto_pad(q, k, v, n_win, topk, heads)
+
+
+def attend_auto_pad(q, k, v, idx, heads, n_win):
+    return default().attend_auto_pad(q, k, v, idx, heads, n_win)

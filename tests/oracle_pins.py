@@ -15,7 +15,15 @@ oracle disagrees with an independent statement of the same quantity:
 * closed forms: rs = 1 and topk = 1 returns the routed token's value; constant values
   pass through; attention is linear in v; a worked 2x2 example with a tie
   (tests/golden/tie_break_2x2.json);
-* invariance of the output to the order of a routing row.
+* invariance of the output to the order of a routing row;
+* per-head routing against a numpy restatement (per-head window means, matmul / sqrt(head_dim),
+  brute-force ranking, topk clamped to R) and, with one head, against the shared routing;
+  per-head attention against masked dense attention with one mask per head;
+* LePE against torch's depthwise conv2d (padding 2, bias) plus the input, and two closed forms;
+* the backward pass against central finite differences of the forward oracle and against torch
+  autograd of masked dense attention;
+* auto_pad against numpy zero padding + window means + brute-force ranking + masked dense
+  attention + crop, the ordinary forward on divisible sizes, and a one-token closed form.
 
 The same functions run against mutated copies of the oracle in test_oracle_mutants.py, to
 show that each plausible slip in the oracle fails at least one of them. Run as a script,
@@ -275,9 +283,185 @@ def pin_attend_tokens(orc):
     _close(orc.attend_tokens(q, k, v, idx, heads, n, toks), full[toks], tol=0.0, what="attend_tokens")
 
 
+# ---------------------------------------------------------------- per-head routing, LePE, backward, auto_pad
+
+def numpy_route_heads(q, k, n_win, topk, heads):
+    """Per-head routing restated with numpy: head h's region means are its head_dim channels of
+    the window means, affinities (qm_h km_h^T) / sqrt(head_dim), rows ranked by brute force,
+    min(topk, R) kept."""
+    B, H, W, C = q.shape
+    R, hd = n_win * n_win, C // heads
+    qm = numpy_region_means(q, n_win).reshape(B, R, heads, hd).transpose(0, 2, 1, 3)
+    km = numpy_region_means(k, n_win).reshape(B, R, heads, hd).transpose(0, 2, 1, 3)
+    A = np.matmul(qm, km.transpose(0, 1, 3, 2)) / math.sqrt(hd)
+    kk = min(topk, R)
+    return numpy_topk(A.reshape(B * heads, R, R), kk).reshape(B, heads, R, kk), A
+
+
+def masked_dense_attention_heads(q, k, v, idx, n_win):
+    """masked_dense_attention with one index per head: idx [B, heads, R, topk]."""
+    B, H, W, C = q.shape
+    heads = idx.shape[1]
+    hd = C // heads
+    out = np.empty_like(np.asarray(q, np.float64))
+    for h in range(heads):
+        sl = slice(h * hd, (h + 1) * hd)
+        out[..., sl] = masked_dense_attention(q[..., sl], k[..., sl], v[..., sl], idx[:, h], 1, n_win)
+    return out
+
+
+def pin_route_heads(orc):
+    rng = _rng(21)
+    for (B, H, W, C, heads, n, topk) in [(2, 6, 8, 8, 2, 2, 3), (1, 9, 6, 12, 3, 3, 4), (1, 8, 8, 6, 3, 4, 7)]:
+        q, k = rng.standard_normal((B, H, W, C)), rng.standard_normal((B, H, W, C))
+        idx, A = orc.route_heads(q, k, n, topk, heads, want_affinity=True)
+        nidx, nA = numpy_route_heads(q, k, n, topk, heads)
+        _close(A, nA, what=f"per-head affinity {B,H,W,C,heads,n}")
+        assert np.array_equal(idx, nidx), "per-head routing differs from brute force"
+    # topk above R is clamped to R: every row is the full ranking
+    idx = orc.route_heads(q, k, 4, 20, 3)
+    assert idx.shape == (1, 3, 16, 16) and np.array_equal(idx, numpy_route_heads(q, k, 4, 16, 3)[0])
+    # one head over all channels is the shared routing (same scale C^-1/2)
+    q, k = rng.standard_normal((2, 6, 6, 5)), rng.standard_normal((2, 6, 6, 5))
+    idx1, A1 = orc.route_heads(q, k, 3, 4, 1, want_affinity=True)
+    idx0, A0 = orc.route(q, k, 3, 4, want_affinity=True)
+    assert np.array_equal(idx1[:, 0], idx0)
+    _close(A1[:, 0], A0, what="one head = shared routing")
+
+
+def pin_attend_heads(orc):
+    rng = _rng(22)
+    for (B, H, W, C, heads, n, topk) in [(2, 6, 8, 8, 2, 2, 2), (1, 9, 6, 6, 3, 3, 4)]:
+        q, k, v = (rng.standard_normal((B, H, W, C)) for _ in range(3))
+        R = n * n
+        idx = rng.integers(0, R, size=(B, heads, R, topk)).astype(np.int32)
+        _close(orc.attend_heads(q, k, v, idx, n), masked_dense_attention_heads(q, k, v, idx, n),
+               what=f"per-head masked dense {B,H,W,C,heads,n,topk}")
+        # every head given the same rows: the shared-index attention
+        same = np.repeat(idx[:, :1], heads, axis=1)
+        _close(orc.attend_heads(q, k, v, same, n), orc.attend(q, k, v, idx[:, 0], heads, n), what="same rows")
+        # per-head routing end to end against masked dense over the brute-force index
+        ridx = orc.route_heads(q, k, n, topk, heads)
+        _close(orc.attend_heads(q, k, v, ridx, n),
+               masked_dense_attention_heads(q, k, v, numpy_route_heads(q, k, n, topk, heads)[0], n),
+               what="per-head route + attend")
+
+
+def torch_lepe(x, w, bias):
+    import torch
+    B, H, W, C = x.shape
+    t = torch.from_numpy(np.ascontiguousarray(x)).permute(0, 3, 1, 2)
+    conv = torch.nn.functional.conv2d(t, torch.from_numpy(np.ascontiguousarray(w)).reshape(C, 1, 5, 5),
+                                      torch.from_numpy(np.ascontiguousarray(bias)), padding=2, groups=C)
+    return (t + conv).permute(0, 2, 3, 1).numpy()
+
+
+def pin_lepe(orc):
+    rng = _rng(23)
+    for (B, H, W, C) in [(2, 7, 9, 3), (1, 4, 3, 5), (1, 1, 6, 2)]:
+        x, w, bias = rng.standard_normal((B, H, W, C)), rng.standard_normal((C, 5, 5)), rng.standard_normal(C)
+        _close(orc.lepe(x, w, bias), torch_lepe(x, w, bias), what=f"lepe vs torch conv2d {B,H,W,C}")
+    # a filter that is 1 at the centre doubles x; a zero filter adds the bias
+    x = rng.standard_normal((1, 5, 6, 4))
+    centre = np.zeros((4, 5, 5))
+    centre[:, 2, 2] = 1.0
+    _close(orc.lepe(x, centre, np.zeros(4)), 2.0 * x, what="centre tap")
+    bias = rng.standard_normal(4)
+    _close(orc.lepe(x, np.zeros((4, 5, 5)), bias), x + bias, what="bias only")
+
+
+def torch_masked_attention_grads(q, k, v, idx, dout, heads, n_win):
+    """Gradients of sum(dout * masked dense attention) by torch autograd, float64."""
+    import torch
+    B, H, W, C = q.shape
+    R, N, hd = n_win * n_win, H * W, C // heads
+    reg = torch.from_numpy(region_of_token(H, W, n_win))
+    tq, tk, tv = (torch.from_numpy(np.ascontiguousarray(x)).requires_grad_(True) for x in (q, k, v))
+    outs = []
+    for b in range(B):
+        cnt = torch.zeros((R, R), dtype=torch.float64)
+        for r in range(R):
+            for s in idx[b, r]:
+                cnt[r, s] += 1
+        weight = cnt[reg][:, reg]
+        qb, kb, vb = (t[b].reshape(N, C) for t in (tq, tk, tv))
+        heads_out = []
+        for h in range(heads):
+            sl = slice(h * hd, (h + 1) * hd)
+            logits = (qb[:, sl] @ kb[:, sl].T) / math.sqrt(hd)
+            logits = torch.where(weight > 0, logits, torch.tensor(-math.inf, dtype=torch.float64))
+            p = weight * torch.exp(logits - logits.max(dim=1, keepdim=True).values)
+            p = p / p.sum(dim=1, keepdim=True)
+            heads_out.append(p @ vb[:, sl])
+        outs.append(torch.cat(heads_out, dim=1))
+    out = torch.stack(outs).reshape(B, H, W, C)
+    (out * torch.from_numpy(np.ascontiguousarray(dout))).sum().backward()
+    return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()
+
+
+def pin_backward(orc):
+    rng = _rng(24)
+    # central differences of sum(dout * out) on every coordinate of a tiny case
+    B, H, W, C, heads, n, topk = 1, 4, 4, 4, 2, 2, 2
+    q, k, v = (rng.standard_normal((B, H, W, C)) for _ in range(3))
+    idx = rng.integers(0, n * n, size=(B, n * n, topk)).astype(np.int32)
+    dout = rng.standard_normal((B, H, W, C))
+    grads = orc.attend_backward(q, k, v, idx, dout, heads, n)
+    eps = 1e-6
+    for which, g in enumerate(grads):
+        num = np.zeros_like(g)
+        for i in range(g.size):
+            args = [q.copy(), k.copy(), v.copy()]
+            args[which].reshape(-1)[i] += eps
+            fp = np.sum(dout * orc.attend(*args, idx, heads, n))
+            args[which].reshape(-1)[i] -= 2 * eps
+            fm = np.sum(dout * orc.attend(*args, idx, heads, n))
+            num.reshape(-1)[i] = (fp - fm) / (2 * eps)
+        _close(g, num, tol=1e-7, what=f"finite differences of {'qkv'[which]}")
+    # torch autograd of masked dense attention, duplicated regions included
+    B, H, W, C, heads, n, topk = 2, 6, 8, 8, 2, 2, 3
+    q, k, v, dout = (rng.standard_normal((B, H, W, C)) for _ in range(4))
+    idx = rng.integers(0, n * n, size=(B, n * n, topk)).astype(np.int32)
+    idx[:, :, -1] = idx[:, :, 0]
+    for g, t, name in zip(orc.attend_backward(q, k, v, idx, dout, heads, n),
+                          torch_masked_attention_grads(q, k, v, idx, dout, heads, n), "qkv"):
+        _close(g, t, what=f"autograd d{name}")
+
+
+def pin_auto_pad(orc):
+    rng = _rng(25)
+    # sizes that divide: the ordinary forward pass
+    q, k, v = (rng.standard_normal((2, 6, 9, 4)) for _ in range(3))
+    out, idx = orc.forward_auto_pad(q, k, v, 3, 2, 2)
+    out0, idx0 = orc.forward(q, k, v, 3, 2, 2)
+    assert np.array_equal(idx, idx0)
+    _close(out, out0, tol=0.0, what="auto_pad on divisible sizes")
+    # numpy: zero padding at the bottom and right, window means over the padded windows,
+    # brute-force ranking, masked dense attention, crop
+    for (B, H, W, C, heads, n, topk) in [(2, 5, 7, 4, 2, 3, 2), (1, 9, 4, 6, 3, 4, 5), (1, 3, 3, 2, 1, 2, 4)]:
+        q, k, v = (rng.standard_normal((B, H, W, C)) for _ in range(3))
+        Hp, Wp = -(-H // n) * n, -(-W // n) * n
+        pad = lambda x: np.pad(x, ((0, 0), (0, Hp - H), (0, Wp - W), (0, 0)))
+        qp, kp, vp = pad(q), pad(k), pad(v)
+        A = np.matmul(numpy_region_means(qp, n), numpy_region_means(kp, n).transpose(0, 2, 1)) / math.sqrt(C)
+        nidx = numpy_topk(A, topk)
+        out, idx = orc.forward_auto_pad(q, k, v, n, topk, heads)
+        assert np.array_equal(idx, nidx), f"auto_pad routing {B,H,W,C,n}"
+        _close(out, masked_dense_attention(qp, kp, vp, nidx, heads, n)[:, :H, :W],
+               what=f"auto_pad {B,H,W,C,heads,n,topk}")
+        _close(orc.attend_auto_pad(q, k, v, idx, heads, n), out, tol=0.0, what="attend_auto_pad")
+    # one real token in a 2 x 2 grid of one-token regions: its three routed neighbours are zero
+    # keys (logit 0) with zero values, so out = e^l / (e^l + 3) v, l = q . k / sqrt(C)
+    q, k, v = (rng.standard_normal((1, 1, 1, 3)) for _ in range(3))
+    out, idx = orc.forward_auto_pad(q, k, v, 2, 4, 1)
+    l = float(q.ravel() @ k.ravel()) / math.sqrt(3)
+    _close(out, math.exp(l) / (math.exp(l) + 3.0) * v, tol=1e-14, what="one token, three zero keys")
+
+
 PINS = [pin_region_means, pin_affinity, pin_topk_bruteforce, pin_route_ties, pin_masked_dense,
         pin_global_attention, pin_window_attention, pin_closed_forms, pin_golden_2x2,
-        pin_row_order_invariance, pin_attend_tokens]
+        pin_row_order_invariance, pin_attend_tokens, pin_route_heads, pin_attend_heads, pin_lepe,
+        pin_backward, pin_auto_pad]
 
 
 def run_all(orc):

@@ -58,6 +58,42 @@ MUTANTS = [
     ("last routed region ignored",
      [("for (int j = 0; j < topk; ++j) {\n            const int sy = routed[j] / n_win, sx = routed[j] % n_win;\n            for (int yy = 0; yy < hr; ++yy)\n                for (int xx = 0; xx < wr; ++xx) {\n                    const double *vt",
        "for (int j = 0; j < topk - (topk > 1); ++j) {\n            const int sy = routed[j] / n_win, sx = routed[j] % n_win;\n            for (int yy = 0; yy < hr; ++yy)\n                for (int xx = 0; xx < wr; ++xx) {\n                    const double *vt", 1)]),
+    # per-head routing and attention
+    ("per-head affinity scaled by C",
+     [("const double head_scale = 1.0 / sqrt((double)hd);", "const double head_scale = 1.0 / sqrt((double)C);", 1)]),
+    ("per-head routing without the topk clamp",
+     [("const int k_eff = topk < R ? topk : R;", "const int k_eff = topk;", 1)]),
+    ("per-head keys from head 0",
+     [("km[((int64_t)b * R + s2) * C + h * hd + d];", "km[((int64_t)b * R + s2) * C + d];", 1)]),
+    ("every head attends with head 0's index rows",
+     [("(idx_heads > 1 ? h : 0)", "0", 1)]),
+    # LePE
+    ("LePE without the residual",
+     [("y[token_offset(b, i, j, H, W, C) + c] = x[token_offset(b, i, j, H, W, C) + c] + conv;",
+       "y[token_offset(b, i, j, H, W, C) + c] = conv;", 1)]),
+    ("LePE without the bias", [("double conv = bias[c];", "double conv = 0.0;", 1)]),
+    ("LePE with a flipped filter (convolution, not correlation)",
+     [("w[(int64_t)c * 25 + di * 5 + dj]", "w[(int64_t)c * 25 + (4 - di) * 5 + (4 - dj)]", 1)]),
+    ("LePE with padding 1",
+     [("const int ii = i + di - 2, jj = j + dj - 2;", "const int ii = i + di - 1, jj = j + dj - 1;", 1)]),
+    # backward
+    ("backward without the softmax centring term",
+     [("const double ds = p[i] * (dp[i] - pdp);", "const double ds = p[i] * dp[i];", 1)]),
+    ("backward dk without the scale",
+     [("dk[key[i] + c0 + c] += inv_sqrt_hd * ds", "dk[key[i] + c0 + c] += ds", 1)]),
+    ("backward dq from the values",
+     [("dq[qo + c0 + c] += inv_sqrt_hd * ds * k[key[i] + c0 + c];",
+       "dq[qo + c0 + c] += inv_sqrt_hd * ds * v[key[i] + c0 + c];", 1)]),
+    ("backward dv from the unnormalised weights",
+     [("p[i] /= denom;", "p[i] /= 1.0;", 1)]),
+    # auto_pad
+    ("auto_pad pads at the top and left",
+     [("xp[token_offset(b, i, j, Hp, Wp, C) + c] = x[token_offset(b, i, j, H, W, C) + c];",
+       "xp[token_offset(b, i + Hp - H, j + Wp - W, Hp, Wp, C) + c] = x[token_offset(b, i, j, H, W, C) + c];", 1)]),
+    ("auto_pad crops the bottom right",
+     [("out[token_offset(b, i, j, H, W, C) + c] = op[token_offset(b, i, j, Hp, Wp, C) + c];",
+       "out[token_offset(b, i, j, H, W, C) + c] = op[token_offset(b, i + Hp - H, j + Wp - W, Hp, Wp, C) + c];", 1)]),
+    ("auto_pad rounds down", [("return (n + n_win - 1) / n_win * n_win;", "return n / n_win * n_win;", 1)]),
 ]
 
 
