@@ -55,6 +55,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-per-config", action="store_true", help="time the headline workload only")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip per-head routing, LePE, backward and auto_pad timings")
     ap.add_argument("--eager", action="store_true", help="do not capture CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     ap.add_argument("--cpu-seconds-per-config", type=float, default=2.0,
@@ -427,6 +429,146 @@ def e2e_record(w, host, dev, world, K):
             "steps": ke, "entry_point": "bra_forward_host"}
 
 
+def time_steps(step, nsteps_sets, K, repeats, world, dev):
+    """Median ms per step of K steps (step(i) works on rotation set i % nsets), captured as one
+    CUDA graph with timing events around it; eager if capture is refused."""
+    import torch
+    import torch.distributed as dist
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
+
+    def record():
+        e0.record()
+        for i in range(K):
+            step(i)
+        e1.record()
+
+    g = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            record()
+        run = g.replay
+    except Exception:  # capture refused: eager
+        g = None
+        torch.cuda.synchronize()
+        run = record
+    run()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(max(1, repeats)):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        run()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) / K)
+    ms = sorted(ts)[len(ts) // 2]
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    del g
+    return ms
+
+
+def measure_extras(args, dev, world, rank, pk, pk_kind):
+    """The rows after the forward pass, each timed like the headline: per-head routing + attention,
+    the LePE epilogue (alone and after the forward pass), the backward pass and auto_pad."""
+    import torch
+    import bi_level_routing_b200 as bra
+    from bi_level_routing_b200.workloads import WORKLOADS, Workload, make_inputs
+    hbm = float(pk["hbm_gbs"])
+    K, reps = args.steps, args.repeats
+    l2 = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 * 2**20))
+
+    def tensors(w, seed_shift=0):
+        inp = make_inputs(w, seed=w.seed + 1000 * rank + seed_shift)
+        if w.dtype == "bf16":
+            return [torch.from_numpy(inp[n + "_bits"].view(np.int16)).view(torch.bfloat16).to(dev) for n in "qkv"]
+        return [torch.from_numpy(inp[n]).to(dev) for n in "qkv"]
+
+    def rotation(w, per_set_bytes, make_set):
+        base = tensors(w)
+        nsets = max(2, math.ceil(2 * l2 / per_set_bytes) + 1)
+        return [make_set([torch.roll(t, shifts=i, dims=0).contiguous() for t in base]) for i in range(nsets)]
+
+    def record(name, w, ms, algo_bytes, note):
+        achieved = algo_bytes / (ms * 1e-3) / 1e9
+        return {"value": w.tokens * world / (ms * 1e-3), "unit": UNIT, "step_us": ms * 1e3,
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                             "algorithmic_bytes_per_step": algo_bytes,
+                             "peak_source": f"{pk_kind} hbm_gbs (MEASURED_PEAKS.json)"},
+                "config": w.describe(), "what": note}
+
+    out = {}
+    e = lambda w: w.elem_bytes
+    # per-head routing: bra_forward_heads
+    for name in ("stage1", "stage2", "stage3"):
+        w = WORKLOADS[name]
+        R = w.R
+        sets = rotation(w, w.unique_bytes(), lambda t: (*t, torch.empty_like(t[0]),
+                        torch.empty((w.B, w.heads, R, w.topk), dtype=torch.int32, device=dev)))
+        step = lambda i: bra.forward_heads(*sets[i % len(sets)][:3], w.n_win, w.topk, w.heads,
+                                           out=sets[i % len(sets)][3], idx=sets[i % len(sets)][4])
+        ms = time_steps(step, len(sets), K, reps, world, dev)
+        out[f"per_head_routing/{name}"] = record(name, w, ms, w.unique_bytes(),
+                                                 "bra_forward_heads: per-head means, affinity and top-k, then "
+                                                 "attention with each head's own routed regions")
+        del sets
+    # LePE: the epilogue alone, and bra_forward_lepe
+    w = WORKLOADS["stage1"]
+    rng = np.random.Generator(np.random.PCG64(5))
+    wt = torch.from_numpy(rng.standard_normal((w.C, 5, 5)) * 0.2).float().to(dev)
+    bias = torch.from_numpy(rng.standard_normal(w.C) * 0.1).float().to(dev)
+    sets = rotation(w, 2 * w.B * w.N * w.C * e(w), lambda t: (t[0], torch.empty_like(t[0])))
+    ms = time_steps(lambda i: bra.lepe(sets[i % len(sets)][0], wt, bias, out=sets[i % len(sets)][1]), len(sets), K,
+                    reps, world, dev)
+    out["lepe/stage1"] = record("lepe", w, ms, 2 * w.B * w.N * w.C * e(w), "bra_lepe: x + 5x5 depthwise conv + bias")
+    del sets
+    sets = rotation(w, 5 * w.B * w.N * w.C * e(w), lambda t: (*t, torch.empty_like(t[0]), torch.empty_like(t[0]),
+                    torch.empty((w.B, w.R, w.topk), dtype=torch.int32, device=dev)))
+    ms = time_steps(lambda i: bra.forward_lepe(*sets[i % len(sets)][:3], w.n_win, w.topk, w.heads, wt, bias,
+                                               attn=sets[i % len(sets)][3], out=sets[i % len(sets)][4],
+                                               idx=sets[i % len(sets)][5]), len(sets), K, reps, world, dev)
+    out["forward_lepe/stage1"] = record("forward_lepe", w, ms, 5 * w.B * w.N * w.C * e(w),
+                                        "bra_forward_lepe: routing, attention into attn, LePE epilogue into out")
+    del sets
+    # backward with the index fixed
+    w = WORKLOADS["stage1"]
+    per = (4 * e(w) + 12) * w.B * w.N * w.C
+
+    def back_set(t):
+        q, k, v = t
+        idx = torch.empty((w.B, w.R, w.topk), dtype=torch.int32, device=dev)
+        bra.route(q, k, w.n_win, w.topk, idx=idx)
+        f32 = lambda: torch.empty((w.B, w.H, w.W, w.C), dtype=torch.float32, device=dev)
+        return (q, k, v, idx, torch.flip(v, dims=[0]).contiguous(), f32(), f32(), f32())
+
+    sets = rotation(w, per, back_set)
+    ms = time_steps(lambda i: bra.attend_backward(*sets[i % len(sets)][:5], w.heads, w.n_win,
+                                                  dq=sets[i % len(sets)][5], dk=sets[i % len(sets)][6],
+                                                  dv=sets[i % len(sets)][7]), len(sets), K, reps, world, dev)
+    out["backward/stage1"] = record("backward", w, ms, per, "bra_attend_backward: dq, dk, dv (fp32) of the token "
+                                    "attention with idx fixed; bytes = q, k, v, dout read + dq, dk, dv written")
+    del sets
+    # auto_pad: the stage-1 shape at 54 x 54 (padded to 56 x 56 for the 7 x 7 region grid)
+    w = Workload("stage1_54x54", 64, 54, 54, 64, 2, 7, 1, "bf16", "region_offset", 20267)
+    sets = rotation(w, w.unique_bytes(), lambda t: (*t, torch.empty_like(t[0]),
+                    torch.empty((w.B, w.R, w.topk), dtype=torch.int32, device=dev)))
+    ms = time_steps(lambda i: bra.forward_auto_pad(*sets[i % len(sets)][:3], w.n_win, w.topk, w.heads,
+                                                   out=sets[i % len(sets)][3], idx=sets[i % len(sets)][4]),
+                    len(sets), K, reps, world, dev)
+    out["auto_pad/stage1_54x54"] = record("auto_pad", w, ms, w.unique_bytes(),
+                                          "bra_forward_auto_pad on 54 x 54 (zero padding to 56 x 56 read in place)")
+    del sets
+    torch.cuda.empty_cache()
+    return out
+
+
 def main(argv=None):
     args = parse_args(argv)
     rank = int(os.environ.get("RANK", "0"))
@@ -492,6 +634,9 @@ def main(argv=None):
             if mc is not m:
                 del mc
         line["per_config"] = per
+
+    if not args.no_extras:
+        line["extras"] = measure_extras(args, dev, world, rank, pk, pk_kind)
 
     if world > 1:
         dist.barrier()

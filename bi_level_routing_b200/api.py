@@ -45,6 +45,13 @@ def lib() -> ctypes.CDLL:
     L.bra_attend.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, I, I, I, I, vp]
     L.bra_forward.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, I, I, I, I, vp]
     L.bra_forward_host.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, I, I, I, I, vp]
+    L.bra_route_heads.argtypes = [vp, vp, vp, I, I, I, I, I, I, I, I, vp]
+    L.bra_attend_heads.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, I, I, I, I, vp]
+    L.bra_forward_heads.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, I, I, I, I, vp]
+    L.bra_forward_auto_pad.argtypes = [vp, vp, vp, vp, vp, I, I, I, I, I, I, I, I, vp]
+    L.bra_lepe.argtypes = [vp, vp, vp, vp, I, I, I, I, I, vp]
+    L.bra_forward_lepe.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, I, I, I, I, vp]
+    L.bra_attend_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, I, I, I, I, vp]
     L.bra_set_attend_kernel.argtypes = [I]
     L.bra_set_max_ctas.argtypes = [I]
     L.bra_selected_attend_kernel.argtypes = [I, I, I, I, I, I, I, I]
@@ -56,6 +63,8 @@ def lib() -> ctypes.CDLL:
     L.bra_status_string.restype = ctypes.c_char_p
     L.bra_last_error_message.restype = ctypes.c_char_p
     for name in ("bra_route", "bra_attend", "bra_forward", "bra_forward_host", "bra_set_attend_kernel", "bra_set_max_ctas",
+                 "bra_route_heads", "bra_attend_heads", "bra_forward_heads", "bra_forward_auto_pad", "bra_lepe",
+                 "bra_forward_lepe", "bra_attend_backward",
                  "bra_selected_attend_kernel", "bra_check_device_error", "bra_kernels_per_call"):
         getattr(L, name).restype = I
     _lib = L
@@ -164,6 +173,129 @@ def forward_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_win: int, 
         _check(lib().bra_forward_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), out.data_ptr(), B, H,
                                       W, C, heads, n_win, topk, DTYPES[q.dtype], _stream(device)), "bra_forward_host")
     return out, idx
+
+
+def route_heads(q: torch.Tensor, k: torch.Tensor, n_win: int, topk: int, heads: int,
+                idx: torch.Tensor | None = None) -> torch.Tensor:
+    """Per-head routing index int32 [B, heads, n_win^2, min(topk, n_win^2)] (topk clamped to the
+    number of regions, as the pages do)."""
+    B, H, W, C = _shape(q, "q")
+    _same(q, ("k", k))
+    R = n_win * n_win
+    topk = min(topk, R)
+    if idx is None:
+        idx = torch.empty((B, heads, R, topk), dtype=torch.int32, device=q.device)
+    elif idx.shape != (B, heads, R, topk) or idx.dtype != torch.int32 or not idx.is_contiguous():
+        raise ValueError("idx must be a contiguous int32 [B, heads, n_win^2, min(topk, n_win^2)] tensor")
+    _check(lib().bra_route_heads(q.data_ptr(), k.data_ptr(), idx.data_ptr(), B, H, W, C, heads, n_win, topk,
+                                 DTYPES[q.dtype], _stream(q.device)), "bra_route_heads")
+    return idx
+
+
+def attend_heads(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor, n_win: int,
+                 out: torch.Tensor | None = None) -> torch.Tensor:
+    """Attention where head h gathers the regions of its own rows idx [B, heads, R, topk]."""
+    B, H, W, C = _shape(q, "q")
+    _same(q, ("k", k), ("v", v))
+    if idx.dim() != 4 or idx.dtype != torch.int32 or not idx.is_contiguous() or idx.device != q.device:
+        raise ValueError("idx must be a contiguous int32 [B, heads, n_win^2, topk] tensor on q's device")
+    if out is None:
+        out = torch.empty_like(q)
+    _same(q, ("out", out))
+    _check(lib().bra_attend_heads(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), out.data_ptr(), B, H, W,
+                                  C, idx.shape[1], n_win, idx.shape[-1], DTYPES[q.dtype], _stream(q.device)),
+           "bra_attend_heads")
+    return out
+
+
+def forward_heads(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_win: int, topk: int, heads: int,
+                  out: torch.Tensor | None = None, idx: torch.Tensor | None = None):
+    """The forward pass with per-head routing. Returns (out, idx [B, heads, R, min(topk, R)])."""
+    B, H, W, C = _shape(q, "q")
+    _same(q, ("k", k), ("v", v))
+    R = n_win * n_win
+    topk = min(topk, R)
+    if out is None:
+        out = torch.empty_like(q)
+    _same(q, ("out", out))
+    if idx is None:
+        idx = torch.empty((B, heads, R, topk), dtype=torch.int32, device=q.device)
+    _check(lib().bra_forward_heads(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), out.data_ptr(), B, H,
+                                   W, C, heads, n_win, topk, DTYPES[q.dtype], _stream(q.device)), "bra_forward_heads")
+    return out, idx
+
+
+def forward_auto_pad(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_win: int, topk: int, heads: int,
+                     out: torch.Tensor | None = None, idx: torch.Tensor | None = None):
+    """The forward pass on any H x W: the map is taken as zero-padded at the bottom and right to
+    multiples of n_win (nothing is copied), and out has q's shape. Returns (out, idx)."""
+    B, H, W, C = _shape(q, "q")
+    _same(q, ("k", k), ("v", v))
+    R = n_win * n_win
+    if out is None:
+        out = torch.empty_like(q)
+    _same(q, ("out", out))
+    if idx is None:
+        idx = torch.empty((B, R, topk), dtype=torch.int32, device=q.device)
+    _check(lib().bra_forward_auto_pad(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), out.data_ptr(), B, H,
+                                      W, C, heads, n_win, topk, DTYPES[q.dtype], _stream(q.device)),
+           "bra_forward_auto_pad")
+    return out, idx
+
+
+def lepe(x: torch.Tensor, weight: torch.Tensor, bias: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """x + 5x5 depthwise convolution of x (zero padding 2) + bias; weight fp32 [C, 5, 5], bias fp32 [C]."""
+    B, H, W, C = _shape(x, "x")
+    for name, t, shape in (("weight", weight, (C, 5, 5)), ("bias", bias, (C,))):
+        if t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous() or t.device != x.device:
+            raise ValueError(f"{name} must be a contiguous float32 {shape} tensor on x's device")
+    if out is None:
+        out = torch.empty_like(x)
+    _same(x, ("out", out))
+    _check(lib().bra_lepe(x.data_ptr(), weight.data_ptr(), bias.data_ptr(), out.data_ptr(), B, H, W, C,
+                          DTYPES[x.dtype], _stream(x.device)), "bra_lepe")
+    return out
+
+
+def forward_lepe(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_win: int, topk: int, heads: int,
+                 weight: torch.Tensor, bias: torch.Tensor, attn: torch.Tensor | None = None,
+                 out: torch.Tensor | None = None, idx: torch.Tensor | None = None):
+    """The forward pass followed by the LePE epilogue. Returns (out, attn, idx): attn is the
+    attention output, out = attn + lepe(attn)."""
+    B, H, W, C = _shape(q, "q")
+    _same(q, ("k", k), ("v", v))
+    R = n_win * n_win
+    attn = torch.empty_like(q) if attn is None else attn
+    out = torch.empty_like(q) if out is None else out
+    _same(q, ("attn", attn), ("out", out))
+    if idx is None:
+        idx = torch.empty((B, R, topk), dtype=torch.int32, device=q.device)
+    _check(lib().bra_forward_lepe(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), attn.data_ptr(),
+                                  out.data_ptr(), weight.data_ptr(), bias.data_ptr(), B, H, W, C, heads, n_win, topk,
+                                  DTYPES[q.dtype], _stream(q.device)), "bra_forward_lepe")
+    return out, attn, idx
+
+
+def attend_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor, dout: torch.Tensor,
+                    heads: int, n_win: int, dq: torch.Tensor | None = None, dk: torch.Tensor | None = None,
+                    dv: torch.Tensor | None = None):
+    """(dq, dk, dv), float32 [B, H, W, C]: gradients of sum(dout * attend(q, k, v, idx)), idx fixed."""
+    B, H, W, C = _shape(q, "q")
+    _same(q, ("k", k), ("v", v), ("dout", dout))
+    if idx.dim() != 3 or idx.dtype != torch.int32 or not idx.is_contiguous() or idx.device != q.device:
+        raise ValueError("idx must be a contiguous int32 [B, n_win^2, topk] tensor on q's device")
+    grads = []
+    for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
+        if g is None:
+            g = torch.empty((B, H, W, C), dtype=torch.float32, device=q.device)
+        elif g.shape != (B, H, W, C) or g.dtype != torch.float32 or not g.is_contiguous() or g.device != q.device:
+            raise ValueError(f"{name} must be a contiguous float32 [B, H, W, C] tensor on q's device")
+        grads.append(g)
+    dq, dk, dv = grads
+    _check(lib().bra_attend_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), idx.data_ptr(), dout.data_ptr(),
+                                     dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, W, C, heads, n_win,
+                                     idx.shape[-1], DTYPES[q.dtype], _stream(q.device)), "bra_attend_backward")
+    return dq, dk, dv
 
 
 def check_device_error(device=None) -> int:

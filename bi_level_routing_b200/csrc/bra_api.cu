@@ -369,6 +369,182 @@ bra_status bra_forward_host(const void *q, const void *k, const void *v, int32_t
     return BRA_OK;
 }
 
+// ---------------------------------------------------------------- per-head routing
+
+static bra_status route_heads_impl(const void *q, const void *k, int32_t *idx, const bra::Geometry &g,
+                                   bra_dtype dtype, cudaStream_t stream, void *workspace = nullptr,
+                                   size_t ws_bytes = 0)
+{
+    DeviceState *st = nullptr;
+    bra_status s = device_state(&st);
+    if (s != BRA_OK) return s;
+    const bool bf16 = dtype == BRA_BF16;
+    if (g.rs == 1) {  // one-token regions: the means are the tokens
+        const cudaError_t e = bra::launch_route_heads_tokens(q, k, idx, g, bf16, stream);
+        return e == cudaSuccess ? BRA_OK : cuda_fail(e, "per-head routing kernel");
+    }
+    const size_t bytes = (size_t)2 * g.B * g.R * g.C * sizeof(float);
+    const bool in_workspace = workspace && bytes <= ws_bytes;
+    void *scratch = in_workspace ? workspace : nullptr;
+    cudaError_t e = cudaSuccess;
+    if (!in_workspace && (e = cudaMallocFromPoolAsync(&scratch, bytes, st->pool, stream)) != cudaSuccess)
+        return cuda_fail(e, "cudaMallocFromPoolAsync(route scratch)");
+    float *qm = static_cast<float *>(scratch);
+    float *km = qm + (size_t)g.B * g.R * g.C;
+    e = bra::launch_region_means(q, k, qm, km, g, bf16, st->num_sms, stream);
+    if (e == cudaSuccess) e = bra::launch_route_heads(qm, km, idx, g, stream);
+    cudaError_t f = in_workspace ? cudaSuccess : cudaFreeAsync(scratch, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "per-head routing kernels");
+    if (f != cudaSuccess) return cuda_fail(f, "cudaFreeAsync(route scratch)");
+    return BRA_OK;
+}
+
+static bra_status check_data_ptrs(const void *q, const void *k, const void *v, const int32_t *idx, const void *out)
+{
+    if (!q || !k || !v || !idx || !out) return BRA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(idx, 4))
+        return BRA_ERR_INVALID_ARG;
+    return BRA_OK;
+}
+
+bra_status bra_route_heads(const void *q, const void *k, int32_t *idx, int B, int H, int W, int C, int heads,
+                           int n_win, int topk, bra_dtype dtype, void *stream)
+{
+    bra::Geometry g;
+    bra_status s = check_shape(B, H, W, C, heads, n_win, topk, dtype, &g);
+    if (s != BRA_OK) return s;
+    if (B == 0) return BRA_OK;
+    if (!q || !k || !idx) return BRA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(idx, 4)) return BRA_ERR_INVALID_ARG;
+    if (!bra::route_heads_supports(g, dtype == BRA_BF16)) return BRA_ERR_UNSUPPORTED;
+    return route_heads_impl(q, k, idx, g, dtype, static_cast<cudaStream_t>(stream));
+}
+
+bra_status bra_attend_heads(const void *q, const void *k, const void *v, const int32_t *idx, void *out, int B,
+                            int H, int W, int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream)
+{
+    bra::Geometry g;
+    bra_status s = check_shape(B, H, W, C, heads, n_win, topk, dtype, &g);
+    if (s != BRA_OK) return s;
+    if (B == 0) return BRA_OK;
+    if ((s = check_data_ptrs(q, k, v, idx, out)) != BRA_OK) return s;
+    if (g.hd > bra::kSimtMaxHeadDim) return BRA_ERR_UNSUPPORTED;
+    DeviceState *st = nullptr;
+    if ((s = device_state(&st)) != BRA_OK) return s;
+    const cudaError_t e = bra::launch_attend_staged(q, k, v, idx, out, g, g.H, g.W, true, dtype == BRA_BF16,
+                                                    st->error_word, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BRA_OK : cuda_fail(e, "per-head attention kernel");
+}
+
+bra_status bra_forward_heads(const void *q, const void *k, const void *v, int32_t *idx, void *out, int B, int H,
+                             int W, int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream)
+{
+    bra::Geometry g;
+    bra_status s = check_shape(B, H, W, C, heads, n_win, topk, dtype, &g);
+    if (s != BRA_OK) return s;
+    if (B == 0) return BRA_OK;
+    if ((s = check_data_ptrs(q, k, v, idx, out)) != BRA_OK) return s;
+    if (!bra::route_heads_supports(g, dtype == BRA_BF16) || g.hd > bra::kSimtMaxHeadDim) return BRA_ERR_UNSUPPORTED;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const size_t out_bytes = (size_t)B * H * W * C * (dtype == BRA_BF16 ? 2 : 4);
+    if ((s = route_heads_impl(q, k, idx, g, dtype, cs, out, out_bytes)) != BRA_OK) return s;
+    DeviceState *st = nullptr;
+    if ((s = device_state(&st)) != BRA_OK) return s;
+    const cudaError_t e =
+        bra::launch_attend_staged(q, k, v, idx, out, g, g.H, g.W, true, dtype == BRA_BF16, st->error_word, cs);
+    return e == cudaSuccess ? BRA_OK : cuda_fail(e, "per-head attention kernel");
+}
+
+// ---------------------------------------------------------------- auto_pad
+
+bra_status bra_forward_auto_pad(const void *q, const void *k, const void *v, int32_t *idx, void *out, int B, int H,
+                                int W, int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream)
+{
+    if (H <= 0 || W <= 0 || n_win <= 0) return BRA_ERR_INVALID_ARG;
+    if (H % n_win == 0 && W % n_win == 0)  // nothing to pad: the ordinary forward pass
+        return bra_forward(q, k, v, idx, out, B, H, W, C, heads, n_win, topk, dtype, stream);
+    const long long Hp = (long long)(H + n_win - 1) / n_win * n_win, Wp = (long long)(W + n_win - 1) / n_win * n_win;
+    if (Hp > 0x7fffffffLL || Wp > 0x7fffffffLL) return BRA_ERR_UNSUPPORTED;
+    bra::Geometry g;  // the padded region grid
+    bra_status s = check_shape(B, (int)Hp, (int)Wp, C, heads, n_win, topk, dtype, &g);
+    if (s != BRA_OK) return s;
+    if (B == 0) return BRA_OK;
+    if ((s = check_data_ptrs(q, k, v, idx, out)) != BRA_OK) return s;
+    if (g.hd > bra::kSimtMaxHeadDim) return BRA_ERR_UNSUPPORTED;
+    DeviceState *st = nullptr;
+    if ((s = device_state(&st)) != BRA_OK) return s;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == BRA_BF16;
+    // the fp32 means in out when they fit (it is written only by the attention), else pool scratch
+    const size_t bytes = (size_t)2 * g.B * g.R * g.C * sizeof(float);
+    const size_t out_bytes = (size_t)B * H * W * C * (bf16 ? 2 : 4);
+    const bool in_out = bytes <= out_bytes;
+    void *scratch = in_out ? out : nullptr;
+    cudaError_t e = cudaSuccess;
+    if (!in_out && (e = cudaMallocFromPoolAsync(&scratch, bytes, st->pool, cs)) != cudaSuccess)
+        return cuda_fail(e, "cudaMallocFromPoolAsync(route scratch)");
+    float *qm = static_cast<float *>(scratch);
+    float *km = qm + (size_t)g.B * g.R * g.C;
+    e = bra::launch_region_means_padded(q, k, qm, km, g, H, W, bf16, cs);
+    if (e == cudaSuccess) e = bra::launch_route_topk(qm, km, idx, g, cs);
+    cudaError_t f = in_out ? cudaSuccess : cudaFreeAsync(scratch, cs);
+    if (e == cudaSuccess) e = bra::launch_attend_staged(q, k, v, idx, out, g, H, W, false, bf16, st->error_word, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "auto_pad kernels");
+    if (f != cudaSuccess) return cuda_fail(f, "cudaFreeAsync(route scratch)");
+    return BRA_OK;
+}
+
+// ---------------------------------------------------------------- LePE
+
+bra_status bra_lepe(const void *x, const float *weight, const float *bias, void *y, int B, int H, int W, int C,
+                    bra_dtype dtype, void *stream)
+{
+    if (dtype != BRA_F32 && dtype != BRA_BF16) return BRA_ERR_INVALID_ARG;
+    if (B < 0 || H <= 0 || W <= 0 || C <= 0) return BRA_ERR_INVALID_ARG;
+    if (!bra::lepe_supports(C, dtype == BRA_BF16)) return BRA_ERR_INVALID_ARG;
+    if (B == 0) return BRA_OK;
+    if (!x || !weight || !bias || !y || x == y) return BRA_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(weight, 4) || !aligned(bias, 4)) return BRA_ERR_INVALID_ARG;
+    if ((long long)B * H * W > 0x7fffffffLL) return BRA_ERR_UNSUPPORTED;
+    const cudaError_t e = bra::launch_lepe(x, weight, bias, y, B, H, W, C, dtype == BRA_BF16,
+                                           static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BRA_OK : cuda_fail(e, "LePE kernel");
+}
+
+bra_status bra_forward_lepe(const void *q, const void *k, const void *v, int32_t *idx, void *attn, void *out,
+                            const float *weight, const float *bias, int B, int H, int W, int C, int heads, int n_win,
+                            int topk, bra_dtype dtype, void *stream)
+{
+    bra::Geometry g;
+    bra_status s = check_shape(B, H, W, C, heads, n_win, topk, dtype, &g);
+    if (s != BRA_OK) return s;
+    if (B == 0) return BRA_OK;
+    if (!out || !weight || !bias || !aligned(out, 16) || !aligned(weight, 4) || !aligned(bias, 4) || out == attn)
+        return BRA_ERR_INVALID_ARG;
+    if ((s = bra_forward(q, k, v, idx, attn, B, H, W, C, heads, n_win, topk, dtype, stream)) != BRA_OK) return s;
+    return bra_lepe(attn, weight, bias, out, B, H, W, C, dtype, stream);
+}
+
+// ---------------------------------------------------------------- backward
+
+bra_status bra_attend_backward(const void *q, const void *k, const void *v, const int32_t *idx, const void *dout,
+                               float *dq, float *dk, float *dv, int B, int H, int W, int C, int heads, int n_win,
+                               int topk, bra_dtype dtype, void *stream)
+{
+    bra::Geometry g;
+    bra_status s = check_shape(B, H, W, C, heads, n_win, topk, dtype, &g);
+    if (s != BRA_OK) return s;
+    if (B == 0) return BRA_OK;
+    if ((s = check_data_ptrs(q, k, v, idx, dout)) != BRA_OK) return s;
+    if (!dq || !dk || !dv || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16)) return BRA_ERR_INVALID_ARG;
+    if (!bra::attend_backward_supports(g)) return BRA_ERR_UNSUPPORTED;
+    DeviceState *st = nullptr;
+    if ((s = device_state(&st)) != BRA_OK) return s;
+    const cudaError_t e = bra::launch_attend_backward(q, k, v, idx, dout, dq, dk, dv, g, dtype == BRA_BF16,
+                                                      st->error_word, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BRA_OK : cuda_fail(e, "backward kernel");
+}
+
 bra_status bra_set_attend_kernel(bra_attend_kernel kernel)
 {
     if (kernel < BRA_ATTEND_AUTO || kernel > BRA_ATTEND_REGION_MMA) return BRA_ERR_INVALID_ARG;

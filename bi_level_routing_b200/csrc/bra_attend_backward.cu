@@ -1,0 +1,312 @@
+// bra_attend_backward.cu -- the backward pass of the token attention with the routing index held
+// fixed: given dout = dL/dout, the gradients dq, dk, dv of L = sum(dout * out). The pages train
+// the model ("从静态到动态", §3.2; "BiFormer用双层路由注意力重塑视觉Transformer效率极限", §3.2) but
+// print no backward; top-k passes no gradient, so routing is a constant of the backward. Per
+// query token and head, with logits l_i = hd^-1/2 q . k_i over the gathered keys and p = softmax:
+//   dv_i += p_i dout,  dp_i = dout . v_i,  ds_i = p_i (dp_i - D),  D = sum_j p_j dp_j = dout . out,
+//   dq = hd^-1/2 sum_i ds_i k_i,  dk_i += hd^-1/2 ds_i q.
+//
+// One CTA per (image, query region, group of heads), one thread per (query token, head):
+//  pass 1 recomputes the forward softmax (running max and sum) and out over the staged keys,
+//         and D = dout . out;
+//  pass 2 forms p_i and ds_i chunk by chunk, adds dq in registers (a query's keys are all in its
+//         CTA, so dq is written once, without atomics), and keeps p and ds of the chunk in
+//         shared memory; the CTA then turns around, one thread per (key, 4 channels), and sums
+//         dk and dv of the chunk's keys over the region's queries, which it adds to global
+//         memory with 16-byte atomics (other query regions route to the same keys).
+// dq, dk, dv are fp32 [B, H, W, C] whatever the input type; dk and dv are cleared first.
+#include "bra_device.cuh"
+#include "bra_launch.h"
+
+namespace bra {
+
+namespace {
+
+struct BackArgs {
+    const void *q, *k, *v, *dout;
+    const int32_t *idx;
+    float *dq, *dk, *dv;
+    unsigned *err;
+    int H, W, C, heads, hd, n_win, hr, wr, rs, R, topk;
+    int hpc;     // heads per CTA
+    int kcr;     // routed regions per key chunk
+    float scale;       // hd^-1/2
+    float scale_log2;  // hd^-1/2 log2(e)
+};
+
+}  // namespace
+
+template <typename T, int HDMAX>
+__global__ void __launch_bounds__(256) attend_backward_kernel(const BackArgs a)
+{
+    extern __shared__ float4 smem4[];
+    const int ngroups = a.heads / a.hpc;
+    int64_t blk = blockIdx.x;
+    const int hg = (int)(blk % ngroups);
+    blk /= ngroups;
+    const int r = (int)(blk % a.R);
+    const int64_t b = blk / a.R;
+    const int ry = r / a.n_win, rx = r - ry * a.n_win;
+    const int hd = a.hd, rs = a.rs, hpc = a.hpc;
+    const int kc = a.kcr * rs;  // keys per chunk and head
+    float *Qs = reinterpret_cast<float *>(smem4);      // [hpc][rs][hd]
+    float *Ds = Qs + (size_t)hpc * rs * hd;            // [hpc][rs][hd] dout
+    float *Ks = Ds + (size_t)hpc * rs * hd;            // [hpc][kc][hd]
+    float *Vs = Ks + (size_t)hpc * kc * hd;            // [hpc][kc][hd]
+    float *Ps = Vs + (size_t)hpc * kc * hd;            // [hpc][rs][kc]
+    float *Ss = Ps + (size_t)hpc * rs * kc;            // [hpc][rs][kc]
+    int *sreg = reinterpret_cast<int *>(Ss + (size_t)hpc * rs * kc);  // [hpc][topk]
+    const T *gq = static_cast<const T *>(a.q), *gk = static_cast<const T *>(a.k);
+    const T *gv = static_cast<const T *>(a.v), *gd = static_cast<const T *>(a.dout);
+    const int hl = threadIdx.x / rs, t = threadIdx.x - hl * rs;
+    const bool active = hl < hpc;
+    const int h = hg * hpc + hl;
+    grid_dependency_wait();
+
+    // the region's queries and output gradients, and the routed regions of every head
+    for (int e = threadIdx.x; e < hpc * rs * hd; e += blockDim.x) {
+        const int eh = e / (rs * hd), rem = e - eh * rs * hd, et = rem / hd, c = rem - et * hd;
+        const int y = ry * a.hr + et / a.wr, x = rx * a.wr + et % a.wr;
+        const int64_t off = ((b * a.H + y) * a.W + x) * a.C + (int64_t)(hg * hpc + eh) * hd + c;
+        Qs[e] = to_float(gq[off]);
+        Ds[e] = to_float(gd[off]);
+    }
+    for (int e = threadIdx.x; e < hpc * a.topk; e += blockDim.x) {
+        const int j = e % a.topk;
+        const int s = a.idx[(b * a.R + r) * a.topk + j];
+        const bool ok = s >= 0 && s < a.R;
+        if (!ok && hg == 0 && e < a.topk) flag_error(a.err, kErrIndex);
+        sreg[e] = ok ? s : -1;
+    }
+    __syncthreads();
+
+    const float *qrow = Qs + ((size_t)hl * rs + t) * hd;
+    const float *drow = Ds + ((size_t)hl * rs + t) * hd;
+    float m = -INFINITY, l = 0.f, D = 0.f;
+    float o[HDMAX], dq[HDMAX];
+#pragma unroll
+    for (int c = 0; c < HDMAX; ++c) o[c] = dq[c] = 0.f;
+
+    // stages the key and value rows of routed slots [j0, j0 + nj) of every head of the group
+    auto stage = [&](int j0, int nj) {
+        for (int e = threadIdx.x; e < hpc * nj * rs * hd; e += blockDim.x) {
+            const int eh = e / (nj * rs * hd), rem = e - eh * (nj * rs * hd);
+            const int key = rem / hd, c = rem - key * hd;
+            const int jj = key / rs, tk = key - jj * rs;
+            const int s = sreg[eh * a.topk + j0 + jj];
+            float kv = 0.f, vv = 0.f;
+            if (s >= 0) {
+                const int sy = s / a.n_win, sx = s - sy * a.n_win;
+                const int y = sy * a.hr + tk / a.wr, x = sx * a.wr + tk % a.wr;
+                const int64_t off = ((b * a.H + y) * a.W + x) * a.C + (int64_t)(hg * hpc + eh) * hd + c;
+                kv = to_float(gk[off]);
+                vv = to_float(gv[off]);
+            }
+            Ks[((size_t)eh * kc + key) * hd + c] = kv;
+            Vs[((size_t)eh * kc + key) * hd + c] = vv;
+        }
+    };
+
+    // pass 1: the forward softmax statistics and out, then D = dout . out
+    for (int j0 = 0; j0 < a.topk; j0 += a.kcr) {
+        const int nj = min(a.kcr, a.topk - j0);
+        __syncthreads();
+        stage(j0, nj);
+        __syncthreads();
+        if (!active) continue;
+        for (int key = 0; key < nj * rs; ++key) {
+            if (sreg[hl * a.topk + j0 + key / rs] < 0) continue;
+            const float *kr = Ks + ((size_t)hl * kc + key) * hd;
+            float dot = 0.f;
+#pragma unroll
+            for (int c = 0; c < HDMAX; ++c)
+                if (c < hd) dot = fmaf(qrow[c], kr[c], dot);
+            const float sl = dot * a.scale_log2;
+            if (sl > m) {
+                const float corr = fast_exp2(m - sl);
+                l *= corr;
+#pragma unroll
+                for (int c = 0; c < HDMAX; ++c) o[c] *= corr;
+                m = sl;
+            }
+            const float p = fast_exp2(sl - m);
+            l += p;
+            const float *vr = Vs + ((size_t)hl * kc + key) * hd;
+#pragma unroll
+            for (int c = 0; c < HDMAX; ++c)
+                if (c < hd) o[c] = fmaf(p, vr[c], o[c]);
+        }
+    }
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    if (active) {
+#pragma unroll
+        for (int c = 0; c < HDMAX; ++c)
+            if (c < hd) D = fmaf(drow[c], o[c] * inv_l, D);
+    }
+
+    // pass 2: p and ds per key, dq in registers; dk and dv per chunk through shared memory
+    for (int j0 = 0; j0 < a.topk; j0 += a.kcr) {
+        const int nj = min(a.kcr, a.topk - j0);
+        __syncthreads();
+        stage(j0, nj);
+        __syncthreads();
+        if (active) {
+            float *prow = Ps + ((size_t)hl * rs + t) * kc;
+            float *srow = Ss + ((size_t)hl * rs + t) * kc;
+            for (int key = 0; key < nj * rs; ++key) {
+                if (sreg[hl * a.topk + j0 + key / rs] < 0) {
+                    prow[key] = 0.f;
+                    srow[key] = 0.f;
+                    continue;
+                }
+                const float *kr = Ks + ((size_t)hl * kc + key) * hd;
+                const float *vr = Vs + ((size_t)hl * kc + key) * hd;
+                float dot = 0.f, dp = 0.f;
+#pragma unroll
+                for (int c = 0; c < HDMAX; ++c)
+                    if (c < hd) {
+                        dot = fmaf(qrow[c], kr[c], dot);
+                        dp = fmaf(drow[c], vr[c], dp);
+                    }
+                const float p = fast_exp2(dot * a.scale_log2 - m) * inv_l;
+                const float ds = p * (dp - D);
+#pragma unroll
+                for (int c = 0; c < HDMAX; ++c)
+                    if (c < hd) dq[c] = fmaf(ds, kr[c], dq[c]);
+                prow[key] = p;
+                srow[key] = ds;
+            }
+        }
+        __syncthreads();
+        // dk and dv of the chunk's keys: one thread per (head, key, 4 channels)
+        const int c4n = hd / 4;
+        for (int e = threadIdx.x; e < hpc * nj * rs * c4n; e += blockDim.x) {
+            const int eh = e / (nj * rs * c4n), rem = e - eh * (nj * rs * c4n);
+            const int key = rem / c4n, c = 4 * (rem - key * c4n);
+            const int jj = key / rs, tk = key - jj * rs;
+            const int s = sreg[eh * a.topk + j0 + jj];
+            if (s < 0) continue;
+            float4 gk4 = make_float4(0.f, 0.f, 0.f, 0.f), gv4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int tq = 0; tq < rs; ++tq) {
+                const float ds = Ss[((size_t)eh * rs + tq) * kc + key];
+                const float p = Ps[((size_t)eh * rs + tq) * kc + key];
+                const float4 qq = *reinterpret_cast<const float4 *>(Qs + ((size_t)eh * rs + tq) * hd + c);
+                const float4 dd = *reinterpret_cast<const float4 *>(Ds + ((size_t)eh * rs + tq) * hd + c);
+                gk4.x = fmaf(ds, qq.x, gk4.x);
+                gk4.y = fmaf(ds, qq.y, gk4.y);
+                gk4.z = fmaf(ds, qq.z, gk4.z);
+                gk4.w = fmaf(ds, qq.w, gk4.w);
+                gv4.x = fmaf(p, dd.x, gv4.x);
+                gv4.y = fmaf(p, dd.y, gv4.y);
+                gv4.z = fmaf(p, dd.z, gv4.z);
+                gv4.w = fmaf(p, dd.w, gv4.w);
+            }
+            gk4.x *= a.scale;
+            gk4.y *= a.scale;
+            gk4.z *= a.scale;
+            gk4.w *= a.scale;
+            const int sy = s / a.n_win, sx = s - sy * a.n_win;
+            const int y = sy * a.hr + tk / a.wr, x = sx * a.wr + tk % a.wr;
+            const int64_t off = ((b * a.H + y) * a.W + x) * a.C + (int64_t)(hg * hpc + eh) * hd + c;
+            atomicAdd(reinterpret_cast<float4 *>(a.dk + off), gk4);
+            atomicAdd(reinterpret_cast<float4 *>(a.dv + off), gv4);
+        }
+    }
+    if (active) {
+        const int y = ry * a.hr + t / a.wr, x = rx * a.wr + t % a.wr;
+        float *dst = a.dq + ((b * a.H + y) * a.W + x) * a.C + (int64_t)h * hd;
+#pragma unroll
+        for (int c = 0; c < HDMAX; ++c)
+            if (c < hd) dst[c] = dq[c] * a.scale;
+    }
+}
+
+namespace {
+
+constexpr size_t kBackMaxSmem = 100 * 1024;
+
+size_t back_smem(int hpc, int rs, int hd, int kcr, int topk)
+{
+    const size_t kc = (size_t)kcr * rs;
+    return sizeof(float) * ((size_t)2 * hpc * rs * hd + (size_t)2 * hpc * kc * hd + (size_t)2 * hpc * rs * kc) +
+           4 * (size_t)hpc * topk + 16;
+}
+
+}  // namespace
+
+bool attend_backward_supports(const Geometry &g)
+{
+    return g.rs <= 256 && g.hd % 4 == 0 && g.hd <= kSimtMaxHeadDim && back_smem(1, g.rs, g.hd, 1, g.topk) <= kBackMaxSmem;
+}
+
+cudaError_t launch_attend_backward(const void *q, const void *k, const void *v, const int32_t *idx, const void *dout,
+                                   float *dq, float *dk, float *dv, const Geometry &g, bool bf16, unsigned *err,
+                                   cudaStream_t stream)
+{
+    if (!attend_backward_supports(g)) return cudaErrorInvalidConfiguration;
+    BackArgs a;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.dout = dout;
+    a.idx = idx;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.err = err;
+    a.H = g.H;
+    a.W = g.W;
+    a.C = g.C;
+    a.heads = g.heads;
+    a.hd = g.hd;
+    a.n_win = g.n_win;
+    a.hr = g.hr;
+    a.wr = g.wr;
+    a.rs = g.rs;
+    a.R = g.R;
+    a.topk = g.topk;
+    a.scale = (float)(1.0 / sqrt((double)g.hd));
+    a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)g.hd));
+    // heads per CTA: the largest divisor of heads with hpc * rs <= 256 threads whose smem holds at
+    // least one routed region per chunk; then as many regions per chunk as fit
+    int hpc = 1;
+    for (int d = 1; d <= g.heads; ++d)
+        if (g.heads % d == 0 && (long long)d * g.rs <= 256 && back_smem(d, g.rs, g.hd, 1, g.topk) <= kBackMaxSmem)
+            hpc = d;
+    int kcr = 1;
+    while (kcr < g.topk && back_smem(hpc, g.rs, g.hd, kcr + 1, g.topk) <= kBackMaxSmem) ++kcr;
+    a.hpc = hpc;
+    a.kcr = kcr;
+    const size_t smem = back_smem(hpc, g.rs, g.hd, kcr, g.topk);
+    const int threads = ((hpc * g.rs + 31) / 32) * 32;
+    const long long blocks = (long long)g.B * g.R * (g.heads / hpc);
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const size_t bytes = (size_t)g.B * g.H * g.W * g.C * sizeof(float);
+    cudaError_t e = cudaMemsetAsync(dk, 0, bytes, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, bytes, stream);
+    if (e != cudaSuccess) return e;
+    void (*kernel)(const BackArgs) = nullptr;
+    int slot = 0;
+    if (g.hd <= 32) {
+        kernel = bf16 ? attend_backward_kernel<__nv_bfloat16, 32> : attend_backward_kernel<float, 32>;
+        slot = bf16 ? 0 : 1;
+    } else if (g.hd <= 64) {
+        kernel = bf16 ? attend_backward_kernel<__nv_bfloat16, 64> : attend_backward_kernel<float, 64>;
+        slot = bf16 ? 2 : 3;
+    } else {
+        kernel = bf16 ? attend_backward_kernel<__nv_bfloat16, 128> : attend_backward_kernel<float, 128>;
+        slot = bf16 ? 4 : 5;
+    }
+    static int granted[6][64] = {{0}};
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (smem > 48 * 1024 && (int)smem > granted[slot][dev]) {
+        if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return e;
+        granted[slot][dev] = (int)smem;
+    }
+    return launch_pdl(kernel, dim3((unsigned)blocks), dim3(threads), smem, stream, a);
+}
+
+}  // namespace bra

@@ -1,110 +1,230 @@
 // bra_attend_simt.cu -- token-to-token attention over the routed regions on CUDA cores.
 //
 // For every query token of region r and every head: softmax, scale head_dim^-1/2, over the
-// tokens of the regions idx[b, r, 0..topk-1] (in that order, row-major inside a region),
-// then the weighted sum of their values ("从零构建BiFormer", §2.2 TokenAttention;
-// "医学图像分割模块：BiFormer / 双层路由注意力", §五 steps ⑤-⑦). The gathered K/V is never
-// materialised: keys are read in place.
+// tokens of the routed regions (in idx order, row-major inside a region), then the weighted sum
+// of their values ("从零构建BiFormer", §2.2 TokenAttention; "医学图像分割模块：BiFormer / 双层路由
+// 注意力", §五 steps ⑤-⑦). This is the kernel of every shape the tensor-core kernels do not take:
+// fp32 inputs, head sizes other than 32, per-head routing (each head gathers the regions of its
+// own index row, §五 steps ③④) and padded maps (auto_pad: tokens outside the H x W image are
+// zeros, as keys and values; queries there are not computed).
 //
-// One thread per (query token, head), keeping q and the running output in registers and
-// folding the softmax online (running max and sum, exp2 with a log2(e) pre-scale). All
-// threads of a block share (image, region, head), so their key and value loads are the
-// same addresses (broadcast). This kernel serves every dtype and head size up to
-// kSimtMaxHeadDim; it is the fp32 path and the fallback of the bf16 tensor-core kernels.
+// One CTA per (image, query region, group of heads): the routed regions' key and value rows of
+// those heads are staged in shared memory by the whole CTA (16-byte vectors when a head's
+// channels allow it), a chunk of routed regions at a time; then one thread per (query token,
+// head) keeps q and its output in registers and folds the softmax online over the staged keys
+// (running max and sum, exp2 with a log2(e) pre-scale). The gathered K/V never reach HBM.
 #include "bra_device.cuh"
 #include "bra_launch.h"
 
 namespace bra {
 
-template <typename T, int HDMAX>
-__global__ void __launch_bounds__(128) attend_simt_kernel(const T *__restrict__ q, const T *__restrict__ k,
-                                                          const T *__restrict__ v, const int32_t *__restrict__ idx,
-                                                          T *__restrict__ out, int H, int W, int C, int heads,
-                                                          int n_win, int topk, float scale_log2, unsigned *err)
-{
-    grid_dependency_wait();
-    const int hd = C / heads;
-    const int hr = H / n_win, wr = W / n_win, rs = hr * wr, R = n_win * n_win;
-    const int64_t blk = blockIdx.x;
-    const int h = (int)(blk % heads);
-    const int r = (int)((blk / heads) % R);
-    const int64_t b = blk / ((int64_t)heads * R);
-    const int ry = r / n_win, rx = r % n_win;
-    const int32_t *routed = idx + (b * R + r) * topk;
+namespace {
 
-    for (int tl = threadIdx.x; tl < rs; tl += blockDim.x) {
-        const int y = ry * hr + tl / wr, x = rx * wr + tl % wr;
-        const int64_t qoff = ((b * H + y) * W + x) * C + (int64_t)h * hd;
+struct StagedArgs {
+    const void *q, *k, *v;
+    const int32_t *idx;
+    void *out;
+    unsigned *err;
+    int H, W;  // the image; the region grid may cover more (tokens outside are zeros)
+    int C, heads, hd, n_win, hr, wr, rs, R, topk;
+    int per_head;  // idx is [B, heads, R, topk]; else [B, R, topk], shared by all heads
+    int hpc;       // heads per CTA
+    int tq;        // threads per head (query tokens per pass)
+    int kchunk;    // routed regions staged per chunk
+    int vec;       // head rows staged as 16-byte vectors
+    float scale_log2;
+};
+
+}  // namespace
+
+template <typename T, int HDMAX>
+__global__ void __launch_bounds__(256) attend_staged_kernel(const StagedArgs a)
+{
+    extern __shared__ float4 smem4[];
+    const int ngroups = a.heads / a.hpc;
+    int64_t blk = blockIdx.x;
+    const int hg = (int)(blk % ngroups);
+    blk /= ngroups;
+    const int r = (int)(blk % a.R);
+    const int64_t b = blk / a.R;
+    const int ry = r / a.n_win, rx = r - ry * a.n_win;
+    const int nkc = a.kchunk * a.rs;  // staged keys per head and chunk
+    T *Ks = reinterpret_cast<T *>(smem4);              // [hpc][nkc][hd]
+    T *Vs = Ks + (size_t)a.hpc * nkc * a.hd;           // [hpc][nkc][hd]
+    int *sreg = reinterpret_cast<int *>(Vs + (size_t)a.hpc * nkc * a.hd);  // [hpc][kchunk]: region, or -1
+    const T *gq = static_cast<const T *>(a.q);
+    const T *gk = static_cast<const T *>(a.k);
+    const T *gv = static_cast<const T *>(a.v);
+    T *gout = static_cast<T *>(a.out);
+    const int hl = threadIdx.x / a.tq, tt = threadIdx.x - hl * a.tq;
+    const int h = hg * a.hpc + hl;
+    grid_dependency_wait();
+
+    for (int t0 = 0; t0 < a.rs; t0 += a.tq) {  // passes over the region's query tokens
+        const int t = t0 + tt;
+        const int qy = ry * a.hr + (t < a.rs ? t / a.wr : 0), qx = rx * a.wr + (t < a.rs ? t % a.wr : 0);
+        const bool real = hl < a.hpc && t < a.rs && qy < a.H && qx < a.W;
+        const int64_t qoff = ((b * a.H + qy) * a.W + qx) * a.C + (int64_t)h * a.hd;
         float qv[HDMAX], o[HDMAX];
 #pragma unroll
         for (int c = 0; c < HDMAX; ++c) {
-            qv[c] = (c < hd) ? to_float(q[qoff + c]) : 0.f;
+            qv[c] = (real && c < a.hd) ? to_float(gq[qoff + c]) : 0.f;
             o[c] = 0.f;
         }
         float m = -INFINITY, l = 0.f;
-        for (int j = 0; j < topk; ++j) {
-            const int s = routed[j];
-            if (s < 0 || s >= R) {
-                flag_error(err, kErrIndex);
-                continue;
+        for (int j0 = 0; j0 < a.topk; j0 += a.kchunk) {
+            const int nj = min(a.kchunk, a.topk - j0);
+            __syncthreads();  // the previous chunk is no longer read
+            for (int e = threadIdx.x; e < a.hpc * nj; e += blockDim.x) {
+                const int ehl = e / nj, jj = e - ehl * nj;
+                const int64_t row = a.per_head ? ((b * a.heads + hg * a.hpc + ehl) * a.R + r) : (b * a.R + r);
+                const int s = a.idx[row * a.topk + j0 + jj];
+                const bool ok = s >= 0 && s < a.R;
+                if (!ok && t0 == 0) flag_error(a.err, kErrIndex);
+                sreg[ehl * a.kchunk + jj] = ok ? s : -1;
             }
-            const int sy = s / n_win, sx = s % n_win;
-            for (int kt = 0; kt < rs; ++kt) {
-                const int ky = sy * hr + kt / wr, kx = sx * wr + kt % wr;
-                const int64_t koff = ((b * H + ky) * W + kx) * C + (int64_t)h * hd;
-                float dot = 0.f;
-#pragma unroll
-                for (int c = 0; c < HDMAX; ++c)
-                    if (c < hd) dot = fmaf(qv[c], to_float(k[koff + c]), dot);
-                const float sl = dot * scale_log2;  // logit in log2 units
-                if (sl > m) {
-                    const float corr = exp2f(m - sl);
-                    l *= corr;
-#pragma unroll
-                    for (int c = 0; c < HDMAX; ++c) o[c] *= corr;
-                    m = sl;
+            __syncthreads();
+            // stage the key and value rows (head, routed slot, token) of this chunk
+            const int rows = a.hpc * nj * a.rs;
+            const int per_row = a.vec ? (a.hd * (int)sizeof(T)) / 16 : a.hd;
+            for (int e = threadIdx.x; e < rows * per_row; e += blockDim.x) {
+                const int row = e / per_row, u = e - row * per_row;
+                const int ehl = row / (nj * a.rs), rem = row - ehl * (nj * a.rs);
+                const int jj = rem / a.rs, tk = rem - jj * a.rs;
+                const int s = sreg[ehl * a.kchunk + jj];
+                if (s < 0) continue;
+                const int sy = s / a.n_win, sx = s - sy * a.n_win;
+                const int ky = sy * a.hr + tk / a.wr, kx = sx * a.wr + tk % a.wr;
+                const bool inside = ky < a.H && kx < a.W;
+                const int64_t goff = ((b * a.H + ky) * a.W + kx) * a.C + (int64_t)(hg * a.hpc + ehl) * a.hd;
+                const size_t soff = ((size_t)ehl * nkc + jj * a.rs + tk) * a.hd;
+                if (a.vec) {
+                    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+                    const int per = 16 / (int)sizeof(T);
+                    reinterpret_cast<uint4 *>(Ks + soff)[u] =
+                        inside ? __ldg(reinterpret_cast<const uint4 *>(gk + goff) + u) : zero;
+                    reinterpret_cast<uint4 *>(Vs + soff)[u] =
+                        inside ? __ldg(reinterpret_cast<const uint4 *>(gv + goff) + u) : zero;
+                    (void)per;
+                } else {
+                    Ks[soff + u] = inside ? gk[goff + u] : from_float<T>(0.f);
+                    Vs[soff + u] = inside ? gv[goff + u] : from_float<T>(0.f);
                 }
-                const float p = exp2f(sl - m);
-                l += p;
+            }
+            __syncthreads();
+            if (!real) continue;
+            const T *kh = Ks + (size_t)hl * nkc * a.hd;
+            const T *vh = Vs + (size_t)hl * nkc * a.hd;
+            for (int jj = 0; jj < nj; ++jj) {
+                if (sreg[hl * a.kchunk + jj] < 0) continue;  // a skipped region contributes no key
+                for (int tk = 0; tk < a.rs; ++tk) {
+                    const T *kr = kh + (size_t)(jj * a.rs + tk) * a.hd;
+                    float dot = 0.f;
 #pragma unroll
-                for (int c = 0; c < HDMAX; ++c)
-                    if (c < hd) o[c] = fmaf(p, to_float(v[koff + c]), o[c]);
+                    for (int c = 0; c < HDMAX; ++c)
+                        if (c < a.hd) dot = fmaf(qv[c], to_float(kr[c]), dot);
+                    const float sl = dot * a.scale_log2;  // logit in log2 units
+                    if (sl > m) {
+                        const float corr = fast_exp2(m - sl);
+                        l *= corr;
+#pragma unroll
+                        for (int c = 0; c < HDMAX; ++c) o[c] *= corr;
+                        m = sl;
+                    }
+                    const float p = fast_exp2(sl - m);
+                    l += p;
+                    const T *vr = vh + (size_t)(jj * a.rs + tk) * a.hd;
+#pragma unroll
+                    for (int c = 0; c < HDMAX; ++c)
+                        if (c < a.hd) o[c] = fmaf(p, to_float(vr[c]), o[c]);
+                }
             }
         }
-        const float inv = (l > 0.f) ? 1.f / l : 0.f;
+        if (real) {
+            const float inv = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll
-        for (int c = 0; c < HDMAX; ++c)
-            if (c < hd) out[qoff + c] = from_float<T>(o[c] * inv);
+            for (int c = 0; c < HDMAX; ++c)
+                if (c < a.hd) gout[qoff + c] = from_float<T>(o[c] * inv);
+        }
     }
 }
 
+namespace {
+
+constexpr size_t kStagedMaxSmem = 96 * 1024;
+
 template <typename T>
-static cudaError_t launch_simt_typed(const void *q, const void *k, const void *v, const int32_t *idx, void *out,
-                                     const Geometry &g, unsigned *err, cudaStream_t stream)
+cudaError_t launch_staged_typed(StagedArgs a, const Geometry &g, cudaStream_t stream)
 {
-    const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)g.hd));
-    int threads = ((g.rs + 31) / 32) * 32;
-    if (threads > 128) threads = 128;
-    const long long blocks = (long long)g.B * g.R * g.heads;
+    const int elem = (int)sizeof(T);
+    // heads per CTA: the largest divisor of heads with hpc * rs <= 256 threads
+    int hpc = 1;
+    for (int d = 1; d <= g.heads; ++d)
+        if (g.heads % d == 0 && (long long)d * g.rs <= 256) hpc = d;
+    a.hpc = hpc;
+    a.tq = g.rs <= 256 ? g.rs : 256;
+    int threads = ((hpc * a.tq + 31) / 32) * 32;
+    if (threads > 256) threads = 256;
+    a.vec = ((g.hd * elem) % 16 == 0) ? 1 : 0;
+    // routed regions per chunk: as many as fit
+    const size_t per_region = (size_t)2 * hpc * g.rs * g.hd * elem + 4 * (size_t)hpc;
+    long long kc = (long long)((kStagedMaxSmem - 16) / per_region);
+    if (kc < 1) return cudaErrorInvalidConfiguration;
+    if (kc > g.topk) kc = g.topk;
+    a.kchunk = (int)kc;
+    const size_t smem = (size_t)2 * hpc * a.kchunk * g.rs * g.hd * elem + 4 * (size_t)hpc * a.kchunk + 16;
+    const long long blocks = (long long)g.B * g.R * (g.heads / hpc);
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    const dim3 grid((unsigned)blocks);
-    const T *tq = (const T *)q, *tk = (const T *)k, *tv = (const T *)v;
-    T *to = (T *)out;
-    if (g.hd <= 32)
-        return launch_pdl(attend_simt_kernel<T, 32>, grid, dim3(threads), 0, stream, tq, tk, tv, idx, to, g.H, g.W, g.C,
-                          g.heads, g.n_win, g.topk, scale_log2, err);
-    if (g.hd <= 64)
-        return launch_pdl(attend_simt_kernel<T, 64>, grid, dim3(threads), 0, stream, tq, tk, tv, idx, to, g.H, g.W, g.C,
-                          g.heads, g.n_win, g.topk, scale_log2, err);
-    return launch_pdl(attend_simt_kernel<T, 128>, grid, dim3(threads), 0, stream, tq, tk, tv, idx, to, g.H, g.W, g.C,
-                      g.heads, g.n_win, g.topk, scale_log2, err);
+    void (*kernel)(const StagedArgs) = g.hd <= 32 ? attend_staged_kernel<T, 32>
+                                                  : (g.hd <= 64 ? attend_staged_kernel<T, 64> : attend_staged_kernel<T, 128>);
+    static int granted[3][64] = {{0}};
+    const int slot = g.hd <= 32 ? 0 : (g.hd <= 64 ? 1 : 2);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if ((int)smem > granted[slot][dev] && smem > 48 * 1024) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        granted[slot][dev] = (int)smem;
+    }
+    return launch_pdl(kernel, dim3((unsigned)blocks), dim3(threads), smem, stream, a);
+}
+
+}  // namespace
+
+cudaError_t launch_attend_staged(const void *q, const void *k, const void *v, const int32_t *idx, void *out,
+                                 const Geometry &g, int H, int W, bool per_head, bool bf16, unsigned *err,
+                                 cudaStream_t stream)
+{
+    if (g.hd > kSimtMaxHeadDim) return cudaErrorInvalidConfiguration;
+    StagedArgs a;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.idx = idx;
+    a.out = out;
+    a.err = err;
+    a.H = H;
+    a.W = W;
+    a.C = g.C;
+    a.heads = g.heads;
+    a.hd = g.hd;
+    a.n_win = g.n_win;
+    a.hr = g.hr;
+    a.wr = g.wr;
+    a.rs = g.rs;
+    a.R = g.R;
+    a.topk = g.topk;
+    a.per_head = per_head ? 1 : 0;
+    a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)g.hd));
+    return bf16 ? launch_staged_typed<__nv_bfloat16>(a, g, stream) : launch_staged_typed<float>(a, g, stream);
 }
 
 cudaError_t launch_attend_simt(const void *q, const void *k, const void *v, const int32_t *idx, void *out,
                                const Geometry &g, bool bf16, unsigned *err, cudaStream_t stream)
 {
-    return bf16 ? launch_simt_typed<__nv_bfloat16>(q, k, v, idx, out, g, err, stream)
-                : launch_simt_typed<float>(q, k, v, idx, out, g, err, stream);
+    return launch_attend_staged(q, k, v, idx, out, g, g.H, g.W, false, bf16, err, stream);
 }
 
 }  // namespace bra

@@ -80,6 +80,40 @@ cudaError_t launch_route_topk_tokens(const void *q, const void *k, int32_t *idx,
 cudaError_t launch_route_topk(const float *qm, const float *km, int32_t *idx, const Geometry &g,
                               cudaStream_t stream);
 
+// Per-head routing ("医学图像分割模块", §五 steps ③④): idx [B, heads, R, topk] from the fp32
+// region means (route_heads) or, for one-token regions, from q and k themselves (..._tokens).
+// Needs R <= 256 and head slices on 16-byte boundaries (route_heads_supports).
+bool route_heads_supports(const Geometry &g, bool bf16);
+cudaError_t launch_route_heads(const float *qm, const float *km, int32_t *idx, const Geometry &g, cudaStream_t stream);
+cudaError_t launch_route_heads_tokens(const void *q, const void *k, int32_t *idx, const Geometry &g, bool bf16,
+                                      cudaStream_t stream);
+
+// Region means of a map padded to the region grid g (g.H = n_win hr >= H, g.W = n_win wr >= W):
+// tokens outside the H x W image count as zeros (auto_pad).
+cudaError_t launch_region_means_padded(const void *q, const void *k, float *qm, float *km, const Geometry &g, int H,
+                                       int W, bool bf16, cudaStream_t stream);
+
+// Attention on CUDA cores with the routed key and value rows staged in shared memory: any dtype,
+// head size up to kSimtMaxHeadDim, idx shared ([B, R, topk]) or per head ([B, heads, R, topk]),
+// and maps padded to the region grid g (tokens at y >= H or x >= W are zeros; H = g.H, W = g.W
+// for an unpadded call; q, k, v, out are [B, H, W, C]).
+cudaError_t launch_attend_staged(const void *q, const void *k, const void *v, const int32_t *idx, void *out,
+                                 const Geometry &g, int H, int W, bool per_head, bool bf16, unsigned *err,
+                                 cudaStream_t stream);
+
+// LePE epilogue: y = x + 5x5 depthwise conv(x) (zero padding 2) + bias; x, y [B, H, W, C] of the
+// element type, weight fp32 [C, 5, 5], bias fp32 [C]; C a multiple of 16 bytes of elements.
+bool lepe_supports(int C, bool bf16);
+cudaError_t launch_lepe(const void *x, const float *weight, const float *bias, void *y, int B, int H, int W, int C,
+                        bool bf16, cudaStream_t stream);
+
+// Backward of the token attention with idx fixed: dq, dk, dv (fp32 [B, H, W, C]) of
+// sum(dout * out); clears dk and dv (memset nodes), then one kernel. Needs hd % 4 == 0, rs <= 256.
+bool attend_backward_supports(const Geometry &g);
+cudaError_t launch_attend_backward(const void *q, const void *k, const void *v, const int32_t *idx, const void *dout,
+                                   float *dq, float *dk, float *dv, const Geometry &g, bool bf16, unsigned *err,
+                                   cudaStream_t stream);
+
 // Largest R the routing kernel handles.
 constexpr int kMaxRegions = 1024;
 

@@ -223,6 +223,49 @@ __global__ void __launch_bounds__(256, 2) route_topk_kernel(const S *__restrict_
     if (nr > 0) affinity_select<E, NR, ROUNDS>(acc, nr, R, topk, scale, idx + ((int64_t)b * R + r0 + i0) * topk, lane);
 }
 
+// Per-head routing ("医学图像分割模块", §五 steps ③④): the same rows, staging and selection as
+// route_topk_kernel, for one head at a time: head h's means are channels [h hd, (h + 1) hd) of
+// the region means (row stride C), its affinities are scaled by hd^-1/2, and its index rows go to
+// idx[b, h, :, :]. One CTA per (image, head, block of rows).
+template <int E, bool ROUNDS, typename S>
+__global__ void __launch_bounds__(256, 2) route_heads_kernel(const S *__restrict__ qm, const S *__restrict__ km,
+                                                          int32_t *__restrict__ idx, int R, int C, int hd, int heads,
+                                                          int topk, int rows, int chunk, float scale)
+{
+    extern __shared__ float4 smem4[];
+    grid_dependency_wait();
+    constexpr int NR = RowsPerPass<E>::value;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row_blocks = (R + rows - 1) / rows;
+    const int bh = blockIdx.x / row_blocks;  // image * heads + head
+    const int h = bh % heads, b = bh / heads;
+    const int r0 = (blockIdx.x % row_blocks) * rows;
+    const int nrows = min(rows, R - r0);
+    const int stride = chunk + 4;
+    const S *gkm = km + (int64_t)b * R * C + (int64_t)h * hd;
+    const S *gqm = qm + ((int64_t)b * R + r0) * C + (int64_t)h * hd;
+    float *skm = reinterpret_cast<float *>(smem4);
+    float *sqm = skm + (size_t)R * stride;
+    const int i0 = warp * NR;
+    const int nr = min(NR, nrows - i0);
+    float acc[NR][E][4];
+#pragma unroll
+    for (int i = 0; i < NR; ++i)
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][e][j] = 0.f;
+    for (int c0 = 0; c0 < hd; c0 += chunk) {
+        const int cn = min(chunk, hd - c0);
+        if (c0 > 0) __syncthreads();
+        stage_rows<false, S>(gkm, R, gqm, nrows, skm, C, c0, cn, stride);
+        __syncthreads();
+        if (nr > 0) affinity_accumulate<E, NR>(acc, sqm + (size_t)i0 * stride, stride, nr, skm, stride, R, cn, lane);
+    }
+    if (nr > 0)
+        affinity_select<E, NR, ROUNDS>(acc, nr, R, topk, scale, idx + ((int64_t)bh * R + r0 + i0) * topk, lane);
+}
+
 // Wide rows (R > 256): one warp per row, keys in shared memory, bitonic network there.
 __global__ void __launch_bounds__(256) route_topk_wide_kernel(const float *__restrict__ qm,
                                                               const float *__restrict__ km, int32_t *__restrict__ idx,
@@ -734,6 +777,134 @@ cudaError_t launch_route_topk(const float *qm, const float *km, int32_t *idx, co
     const float scale = (float)(1.0 / sqrt((double)g.C));
     return launch_pdl(route_topk_wide_kernel, dim3((unsigned)blocks), dim3(warps * 32), (size_t)warps * P * 8, stream, qm,
                       km, idx, g.R, g.C, g.topk, P, scale);
+}
+
+}  // namespace bra
+
+namespace bra {
+
+template <int E, bool ROUNDS, typename S>
+static cudaError_t launch_heads_typed(const S *qm, const S *km, int32_t *idx, const Geometry &g, int rows, int chunk,
+                                      float scale, size_t smem, cudaStream_t stream)
+{
+    static int granted[64] = {0};
+    cudaError_t e = raise_smem_limit(route_heads_kernel<E, ROUNDS, S>, smem, granted);
+    if (e != cudaSuccess) return e;
+    const long long blocks = (long long)((g.R + rows - 1) / rows) * g.B * g.heads;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    return launch_pdl(route_heads_kernel<E, ROUNDS, S>, dim3((unsigned)blocks), dim3(256), smem, stream, qm, km, idx,
+                      g.R, g.C, g.hd, g.heads, g.topk, rows, chunk, scale);
+}
+
+template <int E, typename S>
+static cudaError_t launch_heads_e(const S *qm, const S *km, int32_t *idx, const Geometry &g, cudaStream_t stream)
+{
+    const float scale = (float)(1.0 / sqrt((double)g.hd));
+    const int rows = 8 * RowsPerPass<E>::value;
+    const long long per_col = (long long)(g.R + rows) * sizeof(float);
+    constexpr int V = 16 / sizeof(S);
+    int chunk = g.hd;
+    if (per_col * (chunk + 4) > 100 * 1024) {
+        chunk = 32;
+        while (chunk * 2 < g.hd && per_col * (chunk * 2 + 4) <= 100 * 1024) chunk *= 2;
+        if (per_col * (chunk + 4) > 100 * 1024) return cudaErrorInvalidConfiguration;
+    }
+    if (chunk % V != 0) return cudaErrorInvalidConfiguration;
+    const size_t smem = (size_t)per_col * (chunk + 4);
+    return topk_by_rounds(E, g.topk) ? launch_heads_typed<E, true, S>(qm, km, idx, g, rows, chunk, scale, smem, stream)
+                                     : launch_heads_typed<E, false, S>(qm, km, idx, g, rows, chunk, scale, smem, stream);
+}
+
+template <typename S>
+static cudaError_t launch_heads_any(const S *qm, const S *km, int32_t *idx, const Geometry &g, cudaStream_t stream)
+{
+    if (g.R <= 32) return launch_heads_e<1, S>(qm, km, idx, g, stream);
+    if (g.R <= 64) return launch_heads_e<2, S>(qm, km, idx, g, stream);
+    if (g.R <= 128) return launch_heads_e<4, S>(qm, km, idx, g, stream);
+    if (g.R <= 256) return launch_heads_e<8, S>(qm, km, idx, g, stream);
+    return cudaErrorInvalidConfiguration;
+}
+
+bool route_heads_supports(const Geometry &g, bool bf16)
+{
+    // each head's slice of a row starts on a 16-byte boundary: of the fp32 means, and of the
+    // tokens themselves when a region is one token
+    const int elem = (g.rs == 1) ? (bf16 ? 2 : 4) : 4;
+    return g.R <= 256 && (g.hd * elem) % 16 == 0 && (g.hd * 4) % 16 == 0;
+}
+
+cudaError_t launch_route_heads(const float *qm, const float *km, int32_t *idx, const Geometry &g, cudaStream_t stream)
+{
+    return launch_heads_any<float>(qm, km, idx, g, stream);
+}
+
+cudaError_t launch_route_heads_tokens(const void *q, const void *k, int32_t *idx, const Geometry &g, bool bf16,
+                                      cudaStream_t stream)
+{
+    if (g.rs != 1) return cudaErrorInvalidConfiguration;
+    return bf16 ? launch_heads_any<__nv_bfloat16>(static_cast<const __nv_bfloat16 *>(q),
+                                                  static_cast<const __nv_bfloat16 *>(k), idx, g, stream)
+                : launch_heads_any<float>(static_cast<const float *>(q), static_cast<const float *>(k), idx, g, stream);
+}
+
+}  // namespace bra
+
+namespace bra {
+
+// Region means of a padded map (auto_pad, "从静态到动态", §4.2): the region grid covers
+// n_win hr x n_win wr tokens, of which those at y >= H or x >= W lie outside the H x W image and
+// are zeros. One warp per region; lane l sums the channel vectors l, l + 32, ... over the
+// region's tokens inside the image in row-major order, and the sum is divided by hr wr (the
+// zeros count).
+template <typename T>
+__global__ void __launch_bounds__(256) region_means_padded_kernel(const T *__restrict__ q, const T *__restrict__ k,
+                                                                  float *__restrict__ qm, float *__restrict__ km,
+                                                                  int B, int H, int W, int C, int n_win, int hr,
+                                                                  int wr)
+{
+    grid_dependency_wait();
+    constexpr int V = Vec16<T>::N;
+    const int R = n_win * n_win;
+    const long long reg = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (reg >= (long long)B * R) return;
+    const int lane = threadIdx.x & 31;
+    const long long b = reg / R;
+    const int r = (int)(reg - b * R);
+    const int ry = r / n_win, rx = r - ry * n_win;
+    const int y1 = min(H, (ry + 1) * hr), x1 = min(W, (rx + 1) * wr);
+    const float n = (float)(hr * wr);
+    for (int v = lane; v < C / V; v += 32) {
+        float aq[V], ak[V];
+#pragma unroll
+        for (int i = 0; i < V; ++i) aq[i] = ak[i] = 0.f;
+        for (int y = ry * hr; y < y1; ++y)
+            for (int x = rx * wr; x < x1; ++x) {
+                const int64_t off = ((b * H + y) * W + x) * C + (int64_t)v * V;
+                Vec16<T>::accumulate(Vec16<T>::load_raw(q + off), aq);
+                Vec16<T>::accumulate(Vec16<T>::load_raw(k + off), ak);
+            }
+        float4 *dq = reinterpret_cast<float4 *>(qm + reg * C + (int64_t)v * V);
+        float4 *dk = reinterpret_cast<float4 *>(km + reg * C + (int64_t)v * V);
+#pragma unroll
+        for (int i = 0; i < V / 4; ++i) {
+            dq[i] = make_float4(aq[4 * i] / n, aq[4 * i + 1] / n, aq[4 * i + 2] / n, aq[4 * i + 3] / n);
+            dk[i] = make_float4(ak[4 * i] / n, ak[4 * i + 1] / n, ak[4 * i + 2] / n, ak[4 * i + 3] / n);
+        }
+    }
+}
+
+cudaError_t launch_region_means_padded(const void *q, const void *k, float *qm, float *km, const Geometry &g, int H,
+                                       int W, bool bf16, cudaStream_t stream)
+{
+    const long long blocks = ((long long)g.B * g.R + 7) / 8;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    if (bf16)
+        return launch_pdl(region_means_padded_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3(256), 0, stream,
+                          static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), qm, km, g.B, H,
+                          W, g.C, g.n_win, g.hr, g.wr);
+    return launch_pdl(region_means_padded_kernel<float>, dim3((unsigned)blocks), dim3(256), 0, stream,
+                      static_cast<const float *>(q), static_cast<const float *>(k), qm, km, g.B, H, W, g.C, g.n_win,
+                      g.hr, g.wr);
 }
 
 }  // namespace bra

@@ -125,8 +125,11 @@ def _smooth_field(white: np.ndarray, sigma: float) -> np.ndarray:
 
 
 def _region_grid_to_tokens(off: np.ndarray, H: int, W: int, n_win: int) -> np.ndarray:
-    """[B, n, n, C] per-region values -> [B, H, W, C] (each token takes its window's value)."""
-    return np.repeat(np.repeat(off, H // n_win, axis=1), W // n_win, axis=2)
+    """[B, n, n, C] per-region values -> [B, H, W, C] (each token takes its window's value). When
+    H or W is not a multiple of n_win the windows are those of the map padded to the next
+    multiple (ceil(H / n_win) tokens high), cropped back to H x W."""
+    hr, wr = -(-H // n_win), -(-W // n_win)
+    return np.repeat(np.repeat(off, hr, axis=1), wr, axis=2)[:, :H, :W]
 
 
 def make_inputs(w: Workload, seed: int | None = None) -> dict:

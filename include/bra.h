@@ -32,9 +32,11 @@
  * Ownership. Every buffer belongs to the caller. Calls are asynchronous and ordered on
  *   `stream` (a cudaStream_t; NULL = the legacy default stream) on the current device;
  *   the library never synchronises, except bra_check_device_error and bra_forward_host.
- *   bra_route and bra_forward take fp32 scratch for the region means, 2*B*R*C*4 bytes,
- *   from a stream-ordered pool the library keeps per device (cudaMallocAsync /
- *   cudaFreeAsync on `stream`).
+ *   bra_route takes fp32 scratch for the region means, 2*B*R*C*4 bytes, from a
+ *   stream-ordered pool the library keeps per device (cudaMallocAsync / cudaFreeAsync on
+ *   `stream`); bra_forward keeps them in `out` instead, which the attention overwrites
+ *   afterwards, and allocates nothing (when they fit: rs * sizeof(element) >= 8; one-token
+ *   regions need no means).
  * Validation. Every argument is checked on the host before anything is launched; a
  *   rejected call launches nothing and returns BRA_ERR_INVALID_ARG: a NULL pointer (when
  *   B > 0), B < 0, H, W, C, heads, n_win or topk <= 0, H or W not a multiple of n_win,
@@ -74,7 +76,8 @@ typedef enum { BRA_F32 = 0, BRA_BF16 = 1 } bra_dtype;
    BRA_ERR_UNSUPPORTED. */
 typedef enum {
     BRA_ATTEND_AUTO = 0,
-    BRA_ATTEND_SIMT = 1,      /* any dtype, hd <= 128: one thread per (query, head), CUDA cores */
+    BRA_ATTEND_SIMT = 1,      /* any dtype, hd <= 128: routed rows staged in shared memory, one
+                                 thread per (query, head), CUDA cores */
     BRA_ATTEND_GATHER_MMA = 2,/* bf16, hd == 32, C % 64 == 0, rs % 16 == 0, rs <= 64: per-region
                                  tiles staged by TMA, tensor-core QK^T and PV */
     BRA_ATTEND_DENSE_MMA = 3, /* bf16, hd == 32, C % 64 == 0, R <= 64, H*W <= 256: the image's
@@ -119,6 +122,71 @@ bra_status bra_forward(const void *q, const void *k, const void *v, int32_t *idx
    The paper has no counterpart to this entry point: it is a deployment variant. */
 bra_status bra_route_noalloc(const void *q, const void *k, int32_t *idx, int B, int H, int W, int C, int n_win,
                              int topk, bra_dtype dtype, void *stream);
+
+/* Per-head routing ("医学图像分割模块：BiFormer / 双层路由注意力", §五 steps ③④): the region means
+   of head h are its head_dim channels of the region means (hd = C / heads), its affinities
+   A_h = hd^-1/2 qm_h km_h^T, and idx[b, h, r, :] its topk largest in the routing order above.
+   q, k: device [B, H, W, C]. idx: device int32 [B, heads, n_win^2, topk], written. topk <= R
+   (the pages clamp topk to R; the Python binding does, this call rejects a larger topk). Takes
+   fp32 scratch for the means from the pool, like bra_route (none for one-token regions).
+   BRA_ERR_UNSUPPORTED: R > 256, or a head's channels not a whole number of 16-byte vectors of
+   the fp32 means (hd % 4 != 0) or, for one-token regions, of the tokens. */
+bra_status bra_route_heads(const void *q, const void *k, int32_t *idx, int B, int H, int W, int C, int heads,
+                           int n_win, int topk, bra_dtype dtype, void *stream);
+
+/* Step 5 with per-head routing ("医学图像分割模块", §五 steps ⑤-⑦): head h of a query in region r
+   attends over the tokens of regions idx[b, h, r, 0..topk-1]. idx: device int32
+   [B, heads, n_win^2, topk] (out-of-range entries skipped and flagged, duplicates gathered as
+   often as they occur); other arguments as bra_attend. Runs on CUDA cores with the routed rows
+   staged in shared memory. BRA_ERR_UNSUPPORTED: hd > 128. */
+bra_status bra_attend_heads(const void *q, const void *k, const void *v, const int32_t *idx, void *out, int B,
+                            int H, int W, int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream);
+
+/* bra_route_heads then bra_attend_heads on one stream; the means are kept in `out` until the
+   attention overwrites it, so nothing is allocated. */
+bra_status bra_forward_heads(const void *q, const void *k, const void *v, int32_t *idx, void *out, int B, int H,
+                             int W, int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream);
+
+/* auto_pad ("从静态到动态", §4.2: auto_pad handles the edge padding; "从零构建BiFormer", §1: a
+   padding layer in front when the size is not a multiple of the region grid): the forward pass of
+   an H x W map that need not be a multiple of n_win. The map is taken as padded with zeros at the
+   bottom and the right to Hp x Wp, Hp = ceil(H / n_win) n_win (likewise Wp); nothing is copied:
+   the kernels read zeros outside the image. The padded tokens count in the region means (a sum
+   over the region divided by (Hp / n_win) (Wp / n_win)) and take part in the attention as keys
+   with logit 0 and value 0; out holds the H x W queries only. q, k, v, out: device
+   [B, H, W, C]; idx: device int32 [B, n_win^2, topk], written (routing of the padded map). When
+   H and W are multiples of n_win this is bra_forward. Attention runs on CUDA cores
+   (BRA_ERR_UNSUPPORTED: hd > 128); the means use out as scratch when they fit in it, else the
+   pool. */
+bra_status bra_forward_auto_pad(const void *q, const void *k, const void *v, int32_t *idx, void *out, int B, int H,
+                                int W, int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream);
+
+/* LePE epilogue ("医学图像分割模块", §五 step ⑧: the attention output viewed as a [C, H, W] image,
+   plus its 5 x 5 depthwise convolution): y = x + bias + sum_{dy, dx} weight[c, dy, dx]
+   x[b, i + dy - 2, j + dx - 2, c], zeros outside the image (nn.Conv2d(C, C, 5, padding=2,
+   groups=C), cross-correlation). x, y: device [B, H, W, C] of dtype, distinct; weight: device
+   fp32 [C, 5, 5]; bias: device fp32 [C]. Arithmetic in fp32, y rounded to dtype.
+   BRA_ERR_INVALID_ARG also when x == y or C is not a whole number of 16-byte vectors. */
+bra_status bra_lepe(const void *x, const float *weight, const float *bias, void *y, int B, int H, int W, int C,
+                    bra_dtype dtype, void *stream);
+
+/* bra_forward into `attn`, then bra_lepe(attn) into `out` (both caller-owned [B, H, W, C] of dtype,
+   distinct): out = attn + lepe(attn). The epilogue reads attn right after the attention wrote it,
+   while it is in L2. */
+bra_status bra_forward_lepe(const void *q, const void *k, const void *v, int32_t *idx, void *attn, void *out,
+                            const float *weight, const float *bias, int B, int H, int W, int C, int heads, int n_win,
+                            int topk, bra_dtype dtype, void *stream);
+
+/* Backward of step 5 with the routing index held fixed (the pages train the model, "从静态到动态",
+   §3.2; top-k passes no gradient): given dout = dL/dout, the gradients of L = sum(dout * out)
+   with respect to q, k and v. q, k, v, dout: device [B, H, W, C] of dtype; idx: device int32
+   [B, n_win^2, topk] (out-of-range entries skipped and flagged); dq, dk, dv: device fp32
+   [B, H, W, C], written (dk and dv are cleared first, then accumulated with atomics, so their
+   last bits may differ between runs). BRA_ERR_UNSUPPORTED: hd % 4 != 0, hd > 128, or a region of
+   more than 256 tokens. */
+bra_status bra_attend_backward(const void *q, const void *k, const void *v, const int32_t *idx, const void *dout,
+                               float *dq, float *dk, float *dv, int B, int H, int W, int C, int heads, int n_win,
+                               int topk, bra_dtype dtype, void *stream);
 
 /* bra_forward on HOST buffers: copies q, k, v (host, [B, H, W, C]) to device scratch from
    the library's pool, runs the forward pass on `stream`, copies idx and out back to the

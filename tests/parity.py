@@ -107,3 +107,48 @@ def check_output(gpu: np.ndarray, ref: np.ndarray, dtype: str, what: str = "out"
 def make(w: Workload, seed=None):
     inp = make_inputs(w, seed)
     return inp, device_tensors(inp, w)
+
+
+def check_routing_heads(gpu_idx: np.ndarray, q: np.ndarray, k: np.ndarray, n_win: int, topk: int, heads: int):
+    """check_routing for per-head routing: idx [B, heads, R, k]; the tolerance of a near-tie is
+    measured on head h's channels with its scale head_dim^-1/2. Returns (oracle idx, near rows)."""
+    orc_idx, A = oracle.route_heads(q, k, n_win, topk, heads, want_affinity=True)
+    gpu_idx = np.asarray(gpu_idx)
+    assert gpu_idx.shape == orc_idx.shape, (gpu_idx.shape, orc_idx.shape)
+    if np.array_equal(gpu_idx, orc_idx):
+        return orc_idx, 0
+    B, _, R, kk = orc_idx.shape
+    C = q.shape[-1]
+    hd = C // heads
+    qm, km = oracle.region_means(q, n_win), oracle.region_means(k, n_win)
+    near = 0
+    for b, h, r in np.argwhere(np.any(gpu_idx != orc_idx, axis=-1)):
+        row = gpu_idx[b, h, r]
+        assert np.all((row >= 0) & (row < R)) and len(set(row.tolist())) == kk, f"row {b},{h},{r}: {row}"
+        sl = slice(h * hd, (h + 1) * hd)
+        mag = np.abs(qm[b, r, sl]) @ np.abs(km[b, :, sl]).T / math.sqrt(hd)
+        for j in range(kk):
+            a, o = row[j], orc_idx[b, h, r, j]
+            if a != o:
+                va, vo = A[b, h, r, a], A[b, h, r, o]
+                tol = ROUTE_REL_TOL * max(mag[a], mag[o])
+                assert abs(va - vo) <= tol, f"row {b},{h},{r} pos {j}: {a} ({va!r}) vs {o} ({vo!r}), tol {tol:.3e}"
+        near += 1
+    return orc_idx, near
+
+
+# Backward: fp32 arithmetic on the GPU, float64 in the oracle. Each gradient element is a sum of
+# at most topk * rs * (queries of a region) terms of O(1) size formed in fp32 (relative rounding
+# 2^-24 per operation), so its error stays below about 1e-5 of the largest gradient; the bound is
+# 1e-4 of the largest oracle gradient.
+GRAD_REL_TOL = 1e-4
+
+
+def check_grad(gpu: np.ndarray, ref: np.ndarray, what: str):
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert gpu.shape == ref.shape and np.all(np.isfinite(gpu)), what
+    err = float(np.max(np.abs(gpu - ref)))
+    bound = GRAD_REL_TOL * float(np.max(np.abs(ref)))
+    assert err <= bound, f"{what}: max abs err {err:.3e} > {bound:.3e}"
+    return err

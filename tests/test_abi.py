@@ -133,3 +133,60 @@ def test_scratch_and_launch_accounting(L):
     assert L.bra_kernels_per_call(b"bra_forward", *stage4) == 2
     assert L.bra_route_scratch_bytes(64, 7, 7, 512, 7) == 0
     assert L.bra_kernels_per_call(b"nonsense", *stage1) == 0
+
+
+# ------------------------------------------------------------------ the added entry points: rejected before any launch
+
+def _heads(L, q=FAKE, k=FAKE, idx=FAKE, B=1, H=28, W=28, C=64, heads=2, n_win=7, topk=4, dtype=1):
+    return L.bra_route_heads(q, k, idx, B, H, W, C, heads, n_win, topk, dtype, None)
+
+
+@pytest.mark.parametrize("kw", [dict(heads=3), dict(topk=50), dict(heads=0), dict(q=0), dict(idx=FAKE + 2),
+                                dict(H=30), dict(dtype=5)])
+def test_route_heads_rejects(L, kw):
+    assert _heads(L, **kw) == INVALID
+
+
+def test_route_heads_unsupported(L):
+    # one-token bf16 regions with 4-channel heads: a head's slice is not a 16-byte vector
+    assert _heads(L, H=7, W=7, C=8, heads=2, topk=3) == UNSUPPORTED
+    assert _heads(L, H=34, W=34, n_win=17, topk=3) == UNSUPPORTED  # R = 289 > 256
+
+
+def test_attend_heads_and_forward_heads_reject(L):
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE, 1, 28, 28, 64, 2, 7, 4, 1, None)
+    for fn in (L.bra_attend_heads, L.bra_forward_heads):
+        assert fn(0, *args[1:]) == INVALID
+        assert fn(*args[:4], FAKE + 8, *args[5:]) == INVALID
+        assert fn(*args[:8], 3, *args[9:]) == INVALID  # C % heads
+
+
+def test_forward_auto_pad_rejects(L):
+    base = [FAKE, FAKE, FAKE, FAKE, FAKE, 1, 27, 30, 64, 2, 7, 4, 1, None]
+    for pos, val in ((10, 0), (6, 0), (7, -3), (11, 50), (8, 60), (0, 0), (4, FAKE + 8)):
+        a = list(base)
+        a[pos] = val
+        assert L.bra_forward_auto_pad(*a) == INVALID, (pos, val)
+
+
+def test_lepe_rejects(L):
+    assert L.bra_lepe(FAKE, FAKE, FAKE, FAKE, 1, 8, 8, 64, 1, None) == INVALID  # x == y
+    assert L.bra_lepe(FAKE, FAKE, FAKE, FAKE + 4096, 1, 8, 8, 12, 1, None) == INVALID  # bf16 C % 8
+    assert L.bra_lepe(FAKE, 0, FAKE, FAKE + 4096, 1, 8, 8, 64, 1, None) == INVALID
+    assert L.bra_lepe(FAKE, FAKE, FAKE, FAKE + 4096, -1, 8, 8, 64, 1, None) == INVALID
+    assert L.bra_lepe(FAKE, FAKE, FAKE, FAKE + 4096, 0, 8, 8, 64, 1, None) == OK  # empty batch
+    # out == attn is rejected before the forward pass runs
+    assert L.bra_forward_lepe(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 28, 28, 64, 2, 7, 4, 1, None) == INVALID
+
+
+def test_backward_rejects(L):
+    good = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 28, 28, 64, 2, 7, 4, 1, None]
+    a = list(good)
+    a[5] = 0  # dq
+    assert L.bra_attend_backward(*a) == INVALID
+    a = list(good)
+    a[6] = FAKE + 4  # dk not 16-byte aligned
+    assert L.bra_attend_backward(*a) == INVALID
+    a = list(good)
+    a[11], a[12], a[15] = 8, 4, 0  # fp32, C = 8, heads = 4: head_dim 2
+    assert L.bra_attend_backward(*a) == UNSUPPORTED
