@@ -52,6 +52,7 @@ def lib() -> ctypes.CDLL:
     L.bra_lepe.argtypes = [vp, vp, vp, vp, I, I, I, I, I, vp]
     L.bra_forward_lepe.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, I, I, I, I, vp]
     L.bra_attend_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, I, I, I, I, vp]
+    L.bra_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
     L.bra_set_attend_kernel.argtypes = [I]
     L.bra_set_max_ctas.argtypes = [I]
     L.bra_selected_attend_kernel.argtypes = [I, I, I, I, I, I, I, I]
@@ -64,7 +65,7 @@ def lib() -> ctypes.CDLL:
     L.bra_last_error_message.restype = ctypes.c_char_p
     for name in ("bra_route", "bra_attend", "bra_forward", "bra_forward_host", "bra_set_attend_kernel", "bra_set_max_ctas",
                  "bra_route_heads", "bra_attend_heads", "bra_forward_heads", "bra_forward_auto_pad", "bra_lepe",
-                 "bra_forward_lepe", "bra_attend_backward",
+                 "bra_forward_lepe", "bra_attend_backward", "bra_selftest_wait_timeout",
                  "bra_selected_attend_kernel", "bra_check_device_error", "bra_kernels_per_call"):
         getattr(L, name).restype = I
     _lib = L

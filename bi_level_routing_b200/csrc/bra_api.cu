@@ -24,6 +24,7 @@ struct DeviceState {
     unsigned *error_word = nullptr;
     cudaMemPool_t pool = nullptr;
     int num_sms = 0;
+    cudaStream_t copy_in = nullptr, copy_out = nullptr;  // host-copy streams of bra_forward_host
 };
 
 std::mutex g_mutex;
@@ -68,6 +69,9 @@ bra_status device_state(DeviceState **out)
             uint64_t keep = ~0ull;  // keep freed scratch in the pool
             if ((e = cudaMemPoolSetAttribute(st.pool, cudaMemPoolAttrReleaseThreshold, &keep)) != cudaSuccess)
                 return cuda_fail(e, "cudaMemPoolSetAttribute");
+            if ((e = cudaStreamCreateWithFlags(&st.copy_in, cudaStreamNonBlocking)) != cudaSuccess ||
+                (e = cudaStreamCreateWithFlags(&st.copy_out, cudaStreamNonBlocking)) != cudaSuccess)
+                return cuda_fail(e, "cudaStreamCreateWithFlags");
             if (!g_encode) {
                 void *fn = nullptr;
                 cudaDriverEntryPointQueryResult q;
@@ -144,11 +148,12 @@ int choose_attend_kernel(const bra::Geometry &g, bra_dtype dtype)
     return simt_ok ? BRA_ATTEND_SIMT : -1;
 }
 
-// 4-D bf16 tensor map of a [B, H, W, C] array, 128-byte swizzle, box (64, bw, bh, 1).
-bra_status encode_map(CUtensorMap *map, const void *base, const bra::Geometry &g, int bw, int bh)
+// 4-D bf16 tensor map of a [B, H, W, C] array, 128-byte swizzle, box (64, bw, bh, 1); H, W: the
+// image in memory (g.H, g.W unless the map is padded to the region grid).
+bra_status encode_map(CUtensorMap *map, const void *base, const bra::Geometry &g, int bw, int bh, int H, int W)
 {
-    cuuint64_t dims[4] = {(cuuint64_t)g.C, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.B};
-    cuuint64_t strides[3] = {(cuuint64_t)g.C * 2, (cuuint64_t)g.W * g.C * 2, (cuuint64_t)g.H * g.W * g.C * 2};
+    cuuint64_t dims[4] = {(cuuint64_t)g.C, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)g.B};
+    cuuint64_t strides[3] = {(cuuint64_t)g.C * 2, (cuuint64_t)W * g.C * 2, (cuuint64_t)H * W * g.C * 2};
     cuuint32_t box[4] = {64u, (cuuint32_t)bw, (cuuint32_t)bh, 1u};
     cuuint32_t elem_strides[4] = {1u, 1u, 1u, 1u};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
@@ -164,10 +169,11 @@ bra_status encode_map(CUtensorMap *map, const void *base, const bra::Geometry &g
 // 5-D bf16 tensor map of a [B, H, W, C] array viewed as (channel in its 64-channel block, x, y,
 // channel block, image), 128-byte swizzle, box (64, bw, bh, nblk, 1): the nblk channel blocks
 // of a box land in shared memory one after the other, each as its own (bh x bw)-row tile.
-bra_status encode_map_blocks(CUtensorMap *map, const void *base, const bra::Geometry &g, int bw, int bh, int nblk)
+bra_status encode_map_blocks(CUtensorMap *map, const void *base, const bra::Geometry &g, int bw, int bh, int nblk,
+                             int H, int W)
 {
-    cuuint64_t dims[5] = {64u, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)(g.C / 64), (cuuint64_t)g.B};
-    cuuint64_t strides[4] = {(cuuint64_t)g.C * 2, (cuuint64_t)g.W * g.C * 2, 128u, (cuuint64_t)g.H * g.W * g.C * 2};
+    cuuint64_t dims[5] = {64u, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)(g.C / 64), (cuuint64_t)g.B};
+    cuuint64_t strides[4] = {(cuuint64_t)g.C * 2, (cuuint64_t)W * g.C * 2, 128u, (cuuint64_t)H * W * g.C * 2};
     cuuint32_t box[5] = {64u, (cuuint32_t)bw, (cuuint32_t)bh, (cuuint32_t)nblk, 1u};
     cuuint32_t elem_strides[5] = {1u, 1u, 1u, 1u, 1u};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box,
@@ -212,10 +218,17 @@ bra_status route_impl(const void *q, const void *k, int32_t *idx, const bra::Geo
 
 // inputs_ready: the kernel launched just before on `stream` is this library's routing kernel,
 // which has already waited for the producers of q, k and v, so the attention kernel may read
-// them before it waits for its predecessor (only idx comes from that kernel).
+// them before it waits for its predecessor (only idx comes from that kernel). H, W (>= 0): the
+// image in memory when it is smaller than the region grid g (auto_pad); tokens outside it are
+// zeros and are not stored.
 bra_status attend_impl(const void *q, const void *k, const void *v, const int32_t *idx, void *out,
-                       const bra::Geometry &g, bra_dtype dtype, cudaStream_t stream, bool inputs_ready = false)
+                       const bra::Geometry &g, bra_dtype dtype, cudaStream_t stream, bool inputs_ready = false,
+                       int H = -1, int W = -1)
 {
+    if (H < 0) {
+        H = g.H;
+        W = g.W;
+    }
     const int kernel = choose_attend_kernel(g, dtype);
     if (kernel < 0) return BRA_ERR_UNSUPPORTED;
     DeviceState *st = nullptr;
@@ -223,36 +236,37 @@ bra_status attend_impl(const void *q, const void *k, const void *v, const int32_
     if (s != BRA_OK) return s;
     cudaError_t e = cudaSuccess;
     if (kernel == BRA_ATTEND_SIMT) {
-        e = bra::launch_attend_simt(q, k, v, idx, out, g, dtype == BRA_BF16, st->error_word, stream);
+        e = bra::launch_attend_staged(q, k, v, idx, out, g, H, W, false, dtype == BRA_BF16, st->error_word, stream);
     } else if (kernel == BRA_ATTEND_GATHER_UMMA) {
         CUtensorMap tq, tk, tv;
-        if ((s = encode_map(&tq, q, g, g.wr, g.hr)) != BRA_OK) return s;
-        if ((s = encode_map(&tk, k, g, g.wr, g.hr)) != BRA_OK) return s;
-        if ((s = encode_map(&tv, v, g, g.wr, g.hr)) != BRA_OK) return s;
-        e = bra::launch_attend_gather_umma(tq, tk, tv, idx, out, g, st->num_sms, st->error_word, stream);
+        if ((s = encode_map(&tq, q, g, g.wr, g.hr, H, W)) != BRA_OK) return s;
+        if ((s = encode_map(&tk, k, g, g.wr, g.hr, H, W)) != BRA_OK) return s;
+        if ((s = encode_map(&tv, v, g, g.wr, g.hr, H, W)) != BRA_OK) return s;
+        e = bra::launch_attend_gather_umma(tq, tk, tv, idx, out, g, H, W, st->num_sms, st->error_word, stream);
     } else if (kernel == BRA_ATTEND_REGION_MMA) {
         CUtensorMap tq, tk, tv;
-        if ((s = encode_map_blocks(&tq, q, g, g.W, g.H, 2)) != BRA_OK) return s;
-        if ((s = encode_map_blocks(&tk, k, g, g.W, g.H, 2)) != BRA_OK) return s;
-        if ((s = encode_map_blocks(&tv, v, g, g.W, g.H, 2)) != BRA_OK) return s;
-        e = bra::launch_attend_region_mma(tq, tk, tv, idx, out, g, st->num_sms, st->error_word, inputs_ready, stream);
+        if ((s = encode_map_blocks(&tq, q, g, g.W, g.H, 2, H, W)) != BRA_OK) return s;
+        if ((s = encode_map_blocks(&tk, k, g, g.W, g.H, 2, H, W)) != BRA_OK) return s;
+        if ((s = encode_map_blocks(&tv, v, g, g.W, g.H, 2, H, W)) != BRA_OK) return s;
+        e = bra::launch_attend_region_mma(tq, tk, tv, idx, out, g, H, W, st->num_sms, st->error_word, inputs_ready,
+                                          stream);
     } else if (kernel == BRA_ATTEND_GATHER_MMA) {
         CUtensorMap tq, tk, tv, to;
         int box[5];
         bra::gather_mma_box(g, box);
-        if ((s = encode_map_blocks(&tq, q, g, box[1], box[2], box[3])) != BRA_OK) return s;
-        if ((s = encode_map_blocks(&tk, k, g, box[1], box[2], box[3])) != BRA_OK) return s;
-        if ((s = encode_map_blocks(&tv, v, g, box[1], box[2], box[3])) != BRA_OK) return s;
-        if ((s = encode_map(&to, out, g, box[1], box[2])) != BRA_OK) return s;
-        e = bra::launch_attend_gather_mma(tq, tk, tv, to, idx, out, g, st->num_sms, st->error_word, stream);
+        if ((s = encode_map_blocks(&tq, q, g, box[1], box[2], box[3], H, W)) != BRA_OK) return s;
+        if ((s = encode_map_blocks(&tk, k, g, box[1], box[2], box[3], H, W)) != BRA_OK) return s;
+        if ((s = encode_map_blocks(&tv, v, g, box[1], box[2], box[3], H, W)) != BRA_OK) return s;
+        if ((s = encode_map(&to, out, g, box[1], box[2], H, W)) != BRA_OK) return s;
+        e = bra::launch_attend_gather_mma(tq, tk, tv, to, idx, out, g, H, W, st->num_sms, st->error_word, stream);
     } else {
         const int rows = bra::dense_mma_rows_per_split(g, st->num_sms);
         CUtensorMap tq, tk, tv, to;
-        if ((s = encode_map(&tq, q, g, g.W, rows)) != BRA_OK) return s;
-        if ((s = encode_map(&tk, k, g, g.W, g.H)) != BRA_OK) return s;
-        if ((s = encode_map(&tv, v, g, g.W, g.H)) != BRA_OK) return s;
-        if ((s = encode_map(&to, out, g, g.W, rows)) != BRA_OK) return s;
-        e = bra::launch_attend_dense_mma(tq, tk, tv, to, idx, g, rows, st->error_word, inputs_ready, stream);
+        if ((s = encode_map(&tq, q, g, g.W, rows, H, W)) != BRA_OK) return s;
+        if ((s = encode_map(&tk, k, g, g.W, g.H, H, W)) != BRA_OK) return s;
+        if ((s = encode_map(&tv, v, g, g.W, g.H, H, W)) != BRA_OK) return s;
+        if ((s = encode_map(&to, out, g, g.W, rows, H, W)) != BRA_OK) return s;
+        e = bra::launch_attend_dense_mma(tq, tk, tv, to, idx, g, rows, st->error_word, inputs_ready, H, stream);
     }
     if (e != cudaSuccess) return cuda_fail(e, "attention kernel");
     return BRA_OK;
@@ -343,27 +357,79 @@ bra_status bra_forward_host(const void *q, const void *k, const void *v, int32_t
     if ((s = device_state(&dst)) != BRA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t elem = dtype == BRA_BF16 ? 2 : 4;
-    const size_t tensor = (size_t)B * H * W * C * elem;
+    const size_t image = (size_t)H * W * C * elem, image_idx = (size_t)g.R * topk * sizeof(int32_t);
+    const size_t tensor = (size_t)B * image;
     const size_t tensor_padded = (tensor + 255) & ~(size_t)255;
-    const size_t idx_bytes = (size_t)B * g.R * topk * sizeof(int32_t);
+    const size_t idx_bytes = (size_t)B * image_idx;
     uint8_t *buf = nullptr;
     cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&buf), 4 * tensor_padded + idx_bytes, dst->pool, st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync(host staging)");
     uint8_t *dq = buf, *dk = buf + tensor_padded, *dv = buf + 2 * tensor_padded, *dout = buf + 3 * tensor_padded;
     int32_t *didx = reinterpret_cast<int32_t *>(buf + 4 * tensor_padded);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(dq, q, tensor, cudaMemcpyHostToDevice, st);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(dk, k, tensor, cudaMemcpyHostToDevice, st);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(dv, v, tensor, cudaMemcpyHostToDevice, st);
-    if (e == cudaSuccess) {
-        s = route_impl(dq, dk, didx, g, dtype, st, dout, tensor);
-        if (s == BRA_OK) s = attend_impl(dq, dk, dv, didx, dout, g, dtype, st, true);
-        if (s == BRA_OK) e = cudaMemcpyAsync(idx, didx, idx_bytes, cudaMemcpyDeviceToHost, st);
-        if (s == BRA_OK && e == cudaSuccess) e = cudaMemcpyAsync(out, dout, tensor, cudaMemcpyDeviceToHost, st);
+    // The batch in up to kChunks chunks of whole images: the copies in of chunk c + 1 (stream
+    // copy_in) and out of chunk c - 1 (copy_out) overlap the computation of chunk c (`stream`).
+    constexpr int kChunks = 4;
+    const int nchunk = B < kChunks ? B : kChunks;
+    cudaEvent_t ev_start = nullptr, ev_in[kChunks] = {}, ev_done[kChunks] = {}, ev_out = nullptr;
+    auto make_event = [&](cudaEvent_t *ev) {
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    };
+    make_event(&ev_start);
+    make_event(&ev_out);
+    for (int c = 0; c < nchunk; ++c) {
+        make_event(&ev_in[c]);
+        make_event(&ev_done[c]);
+    }
+    // the staging buffer exists from here on `stream`; the copy streams start after it
+    if (e == cudaSuccess) e = cudaEventRecord(ev_start, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(dst->copy_in, ev_start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(dst->copy_out, ev_start, 0);
+    int b0 = 0;
+    for (int c = 0; c < nchunk && e == cudaSuccess && s == BRA_OK; ++c) {
+        const int nb = B / nchunk + (c < B % nchunk ? 1 : 0);
+        const size_t off = (size_t)b0 * image, bytes = (size_t)nb * image;
+        const size_t ioff = (size_t)b0 * image_idx / sizeof(int32_t), ibytes = (size_t)nb * image_idx;
+        const uint8_t *hq = static_cast<const uint8_t *>(q), *hk = static_cast<const uint8_t *>(k);
+        const uint8_t *hv = static_cast<const uint8_t *>(v);
+        e = cudaMemcpyAsync(dq + off, hq + off, bytes, cudaMemcpyHostToDevice, dst->copy_in);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(dk + off, hk + off, bytes, cudaMemcpyHostToDevice, dst->copy_in);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(dv + off, hv + off, bytes, cudaMemcpyHostToDevice, dst->copy_in);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_in[c], dst->copy_in);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev_in[c], 0);
+        if (e != cudaSuccess) break;
+        bra::Geometry gc = g;
+        gc.B = nb;
+        s = route_impl(dq + off, dk + off, didx + ioff, gc, dtype, st, dout + off, bytes);
+        if (s == BRA_OK) s = attend_impl(dq + off, dk + off, dv + off, didx + ioff, dout + off, gc, dtype, st, true);
+        if (s != BRA_OK) break;
+        e = cudaEventRecord(ev_done[c], st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(dst->copy_out, ev_done[c], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(static_cast<uint8_t *>(out) + off, dout + off, bytes, cudaMemcpyDeviceToHost,
+                                dst->copy_out);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(idx + ioff, didx + ioff, ibytes, cudaMemcpyDeviceToHost, dst->copy_out);
+        b0 += nb;
+    }
+    // `stream` resumes after the last copy out; the buffer goes back to the pool then. After an
+    // error the host waits for both copy streams first, so that no copy still uses the buffer.
+    cudaError_t j = ev_out ? cudaEventRecord(ev_out, dst->copy_out) : cudaErrorInvalidValue;
+    if (j == cudaSuccess) j = cudaStreamWaitEvent(st, ev_out, 0);
+    if (j != cudaSuccess || e != cudaSuccess || s != BRA_OK) {
+        cudaStreamSynchronize(dst->copy_in);
+        cudaStreamSynchronize(dst->copy_out);
     }
     cudaError_t f = cudaFreeAsync(buf, st);
     cudaError_t y = cudaStreamSynchronize(st);
+    for (cudaEvent_t ev : {ev_start, ev_out})
+        if (ev) cudaEventDestroy(ev);
+    for (int c = 0; c < nchunk; ++c) {
+        if (ev_in[c]) cudaEventDestroy(ev_in[c]);
+        if (ev_done[c]) cudaEventDestroy(ev_done[c]);
+    }
     if (s != BRA_OK) return s;
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync");
+    if (e != cudaSuccess) return cuda_fail(e, "host copies");
+    if (j != cudaSuccess) return cuda_fail(j, "copy stream join");
     if (f != cudaSuccess) return cuda_fail(f, "cudaFreeAsync(host staging)");
     if (y != cudaSuccess) return cuda_fail(y, "cudaStreamSynchronize");
     return BRA_OK;
@@ -470,7 +536,7 @@ bra_status bra_forward_auto_pad(const void *q, const void *k, const void *v, int
     if (s != BRA_OK) return s;
     if (B == 0) return BRA_OK;
     if ((s = check_data_ptrs(q, k, v, idx, out)) != BRA_OK) return s;
-    if (g.hd > bra::kSimtMaxHeadDim) return BRA_ERR_UNSUPPORTED;
+    if (choose_attend_kernel(g, dtype) < 0) return BRA_ERR_UNSUPPORTED;
     DeviceState *st = nullptr;
     if ((s = device_state(&st)) != BRA_OK) return s;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -488,10 +554,10 @@ bra_status bra_forward_auto_pad(const void *q, const void *k, const void *v, int
     e = bra::launch_region_means_padded(q, k, qm, km, g, H, W, bf16, cs);
     if (e == cudaSuccess) e = bra::launch_route_topk(qm, km, idx, g, cs);
     cudaError_t f = in_out ? cudaSuccess : cudaFreeAsync(scratch, cs);
-    if (e == cudaSuccess) e = bra::launch_attend_staged(q, k, v, idx, out, g, H, W, false, bf16, st->error_word, cs);
-    if (e != cudaSuccess) return cuda_fail(e, "auto_pad kernels");
+    if (e != cudaSuccess) return cuda_fail(e, "auto_pad routing kernels");
     if (f != cudaSuccess) return cuda_fail(f, "cudaFreeAsync(route scratch)");
-    return BRA_OK;
+    // the attention kernels read the padded grid through maps of the H x W image (zeros beyond it)
+    return attend_impl(q, k, v, idx, out, g, dtype, cs, true, H, W);
 }
 
 // ---------------------------------------------------------------- LePE
@@ -543,6 +609,17 @@ bra_status bra_attend_backward(const void *q, const void *k, const void *v, cons
     const cudaError_t e = bra::launch_attend_backward(q, k, v, idx, dout, dq, dk, dv, g, dtype == BRA_BF16,
                                                       st->error_word, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? BRA_OK : cuda_fail(e, "backward kernel");
+}
+
+bra_status bra_selftest_wait_timeout(unsigned limit_us, void *stream)
+{
+    if (limit_us == 0 || limit_us > 1000000u) return BRA_ERR_INVALID_ARG;
+    DeviceState *st = nullptr;
+    bra_status s = device_state(&st);
+    if (s != BRA_OK) return s;
+    const cudaError_t e =
+        bra::launch_wait_timeout(st->error_word, 1000ull * limit_us, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? BRA_OK : cuda_fail(e, "wait self-test kernel");
 }
 
 bra_status bra_set_attend_kernel(bra_attend_kernel kernel)

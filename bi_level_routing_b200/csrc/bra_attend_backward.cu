@@ -7,8 +7,8 @@
 //   dq = hd^-1/2 sum_i ds_i k_i,  dk_i += hd^-1/2 ds_i q.
 //
 // One CTA per (image, query region, group of heads), one thread per (query token, head):
-//  pass 1 recomputes the forward softmax (running max and sum) and out over the staged keys,
-//         and D = dout . out;
+//  pass 1 recomputes the forward softmax (running max and sum) over the staged keys and, with
+//         the same rescaling, D = dout . out = sum_i p_i (dout . v_i);
 //  pass 2 forms p_i and ds_i chunk by chunk, adds dq in registers (a query's keys are all in its
 //         CTA, so dq is written once, without atomics), and keeps p and ds of the chunk in
 //         shared memory; the CTA then turns around, one thread per (key, 4 channels), and sums
@@ -36,6 +36,19 @@ struct BackArgs {
 
 }  // namespace
 
+// Copies one head row of `hd` elements of T (16-byte aligned, hd * sizeof(T) a multiple of 16) to
+// fp32 in shared memory, one 16-byte vector per call: vector u of the row.
+template <typename T>
+__device__ __forceinline__ void row_vec_to_f32(float *dst, const T *src, int u)
+{
+    constexpr int V = Vec16<T>::N;
+    float f[V];
+    Vec16<T>::load(src + u * V, f);
+    float4 *d = reinterpret_cast<float4 *>(dst + u * V);
+#pragma unroll
+    for (int i = 0; i < V / 4; ++i) d[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+}
+
 template <typename T, int HDMAX>
 __global__ void __launch_bounds__(256) attend_backward_kernel(const BackArgs a)
 {
@@ -53,23 +66,25 @@ __global__ void __launch_bounds__(256) attend_backward_kernel(const BackArgs a)
     float *Ds = Qs + (size_t)hpc * rs * hd;            // [hpc][rs][hd] dout
     float *Ks = Ds + (size_t)hpc * rs * hd;            // [hpc][kc][hd]
     float *Vs = Ks + (size_t)hpc * kc * hd;            // [hpc][kc][hd]
-    float *Ps = Vs + (size_t)hpc * kc * hd;            // [hpc][rs][kc]
-    float *Ss = Ps + (size_t)hpc * rs * kc;            // [hpc][rs][kc]
-    int *sreg = reinterpret_cast<int *>(Ss + (size_t)hpc * rs * kc);  // [hpc][topk]
+    float *Ps = Vs + (size_t)hpc * kc * hd;            // [hpc][kc][rs]: p of (key, query)
+    float *Ss = Ps + (size_t)hpc * kc * rs;            // [hpc][kc][rs]: ds of (key, query)
+    int *sreg = reinterpret_cast<int *>(Ss + (size_t)hpc * kc * rs);  // [hpc][topk]
     const T *gq = static_cast<const T *>(a.q), *gk = static_cast<const T *>(a.k);
     const T *gv = static_cast<const T *>(a.v), *gd = static_cast<const T *>(a.dout);
     const int hl = threadIdx.x / rs, t = threadIdx.x - hl * rs;
     const bool active = hl < hpc;
     const int h = hg * hpc + hl;
+    const int nvh = hd / Vec16<T>::N;  // 16-byte vectors per head row
     grid_dependency_wait();
 
     // the region's queries and output gradients, and the routed regions of every head
-    for (int e = threadIdx.x; e < hpc * rs * hd; e += blockDim.x) {
-        const int eh = e / (rs * hd), rem = e - eh * rs * hd, et = rem / hd, c = rem - et * hd;
+    for (int e = threadIdx.x; e < hpc * rs * nvh; e += blockDim.x) {
+        const int row = e / nvh, u = e - row * nvh;
+        const int eh = row / rs, et = row - eh * rs;
         const int y = ry * a.hr + et / a.wr, x = rx * a.wr + et % a.wr;
-        const int64_t off = ((b * a.H + y) * a.W + x) * a.C + (int64_t)(hg * hpc + eh) * hd + c;
-        Qs[e] = to_float(gq[off]);
-        Ds[e] = to_float(gd[off]);
+        const int64_t off = ((b * a.H + y) * a.W + x) * a.C + (int64_t)(hg * hpc + eh) * hd;
+        row_vec_to_f32(Qs + (size_t)row * hd, gq + off, u);
+        row_vec_to_f32(Ds + (size_t)row * hd, gd + off, u);
     }
     for (int e = threadIdx.x; e < hpc * a.topk; e += blockDim.x) {
         const int j = e % a.topk;
@@ -80,34 +95,35 @@ __global__ void __launch_bounds__(256) attend_backward_kernel(const BackArgs a)
     }
     __syncthreads();
 
-    const float *qrow = Qs + ((size_t)hl * rs + t) * hd;
-    const float *drow = Ds + ((size_t)hl * rs + t) * hd;
-    float m = -INFINITY, l = 0.f, D = 0.f;
-    float o[HDMAX], dq[HDMAX];
+    float qv[HDMAX], dov[HDMAX], dq[HDMAX];
 #pragma unroll
-    for (int c = 0; c < HDMAX; ++c) o[c] = dq[c] = 0.f;
+    for (int c = 0; c < HDMAX; ++c) {
+        qv[c] = (active && c < hd) ? Qs[((size_t)hl * rs + t) * hd + c] : 0.f;
+        dov[c] = (active && c < hd) ? Ds[((size_t)hl * rs + t) * hd + c] : 0.f;
+        dq[c] = 0.f;
+    }
+    // running max and sum of the softmax, and sum_i e_i (dout . v_i) relative to the same max
+    float m = -INFINITY, l = 0.f, dsum = 0.f;
 
     // stages the key and value rows of routed slots [j0, j0 + nj) of every head of the group
     auto stage = [&](int j0, int nj) {
-        for (int e = threadIdx.x; e < hpc * nj * rs * hd; e += blockDim.x) {
-            const int eh = e / (nj * rs * hd), rem = e - eh * (nj * rs * hd);
-            const int key = rem / hd, c = rem - key * hd;
+        for (int e = threadIdx.x; e < hpc * nj * rs * nvh; e += blockDim.x) {
+            const int row = e / nvh, u = e - row * nvh;
+            const int eh = row / (nj * rs), key = row - eh * (nj * rs);
             const int jj = key / rs, tk = key - jj * rs;
             const int s = sreg[eh * a.topk + j0 + jj];
-            float kv = 0.f, vv = 0.f;
+            float *kd = Ks + ((size_t)eh * kc + key) * hd, *vd = Vs + ((size_t)eh * kc + key) * hd;
             if (s >= 0) {
                 const int sy = s / a.n_win, sx = s - sy * a.n_win;
                 const int y = sy * a.hr + tk / a.wr, x = sx * a.wr + tk % a.wr;
-                const int64_t off = ((b * a.H + y) * a.W + x) * a.C + (int64_t)(hg * hpc + eh) * hd + c;
-                kv = to_float(gk[off]);
-                vv = to_float(gv[off]);
+                const int64_t off = ((b * a.H + y) * a.W + x) * a.C + (int64_t)(hg * hpc + eh) * hd;
+                row_vec_to_f32(kd, gk + off, u);
+                row_vec_to_f32(vd, gv + off, u);
             }
-            Ks[((size_t)eh * kc + key) * hd + c] = kv;
-            Vs[((size_t)eh * kc + key) * hd + c] = vv;
         }
     };
 
-    // pass 1: the forward softmax statistics and out, then D = dout . out
+    // pass 1: the forward softmax statistics and D = dout . out = sum_i p_i (dout . v_i)
     for (int j0 = 0; j0 < a.topk; j0 += a.kcr) {
         const int nj = min(a.kcr, a.topk - j0);
         __syncthreads();
@@ -117,32 +133,28 @@ __global__ void __launch_bounds__(256) attend_backward_kernel(const BackArgs a)
         for (int key = 0; key < nj * rs; ++key) {
             if (sreg[hl * a.topk + j0 + key / rs] < 0) continue;
             const float *kr = Ks + ((size_t)hl * kc + key) * hd;
-            float dot = 0.f;
+            const float *vr = Vs + ((size_t)hl * kc + key) * hd;
+            float dot = 0.f, dp = 0.f;
 #pragma unroll
             for (int c = 0; c < HDMAX; ++c)
-                if (c < hd) dot = fmaf(qrow[c], kr[c], dot);
+                if (c < hd) {
+                    dot = fmaf(qv[c], kr[c], dot);
+                    dp = fmaf(dov[c], vr[c], dp);
+                }
             const float sl = dot * a.scale_log2;
             if (sl > m) {
                 const float corr = fast_exp2(m - sl);
                 l *= corr;
-#pragma unroll
-                for (int c = 0; c < HDMAX; ++c) o[c] *= corr;
+                dsum *= corr;
                 m = sl;
             }
             const float p = fast_exp2(sl - m);
             l += p;
-            const float *vr = Vs + ((size_t)hl * kc + key) * hd;
-#pragma unroll
-            for (int c = 0; c < HDMAX; ++c)
-                if (c < hd) o[c] = fmaf(p, vr[c], o[c]);
+            dsum = fmaf(p, dp, dsum);
         }
     }
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
-    if (active) {
-#pragma unroll
-        for (int c = 0; c < HDMAX; ++c)
-            if (c < hd) D = fmaf(drow[c], o[c] * inv_l, D);
-    }
+    const float D = dsum * inv_l;
 
     // pass 2: p and ds per key, dq in registers; dk and dv per chunk through shared memory
     for (int j0 = 0; j0 < a.topk; j0 += a.kcr) {
@@ -151,34 +163,31 @@ __global__ void __launch_bounds__(256) attend_backward_kernel(const BackArgs a)
         stage(j0, nj);
         __syncthreads();
         if (active) {
-            float *prow = Ps + ((size_t)hl * rs + t) * kc;
-            float *srow = Ss + ((size_t)hl * rs + t) * kc;
             for (int key = 0; key < nj * rs; ++key) {
-                if (sreg[hl * a.topk + j0 + key / rs] < 0) {
-                    prow[key] = 0.f;
-                    srow[key] = 0.f;
-                    continue;
+                float p = 0.f, ds = 0.f;
+                if (sreg[hl * a.topk + j0 + key / rs] >= 0) {
+                    const float *kr = Ks + ((size_t)hl * kc + key) * hd;
+                    const float *vr = Vs + ((size_t)hl * kc + key) * hd;
+                    float dot = 0.f, dp = 0.f;
+#pragma unroll
+                    for (int c = 0; c < HDMAX; ++c)
+                        if (c < hd) {
+                            dot = fmaf(qv[c], kr[c], dot);
+                            dp = fmaf(dov[c], vr[c], dp);
+                        }
+                    p = fast_exp2(dot * a.scale_log2 - m) * inv_l;
+                    ds = p * (dp - D);
+#pragma unroll
+                    for (int c = 0; c < HDMAX; ++c)
+                        if (c < hd) dq[c] = fmaf(ds, kr[c], dq[c]);
                 }
-                const float *kr = Ks + ((size_t)hl * kc + key) * hd;
-                const float *vr = Vs + ((size_t)hl * kc + key) * hd;
-                float dot = 0.f, dp = 0.f;
-#pragma unroll
-                for (int c = 0; c < HDMAX; ++c)
-                    if (c < hd) {
-                        dot = fmaf(qrow[c], kr[c], dot);
-                        dp = fmaf(drow[c], vr[c], dp);
-                    }
-                const float p = fast_exp2(dot * a.scale_log2 - m) * inv_l;
-                const float ds = p * (dp - D);
-#pragma unroll
-                for (int c = 0; c < HDMAX; ++c)
-                    if (c < hd) dq[c] = fmaf(ds, kr[c], dq[c]);
-                prow[key] = p;
-                srow[key] = ds;
+                Ps[((size_t)hl * kc + key) * rs + t] = p;
+                Ss[((size_t)hl * kc + key) * rs + t] = ds;
             }
         }
         __syncthreads();
-        // dk and dv of the chunk's keys: one thread per (head, key, 4 channels)
+        // dk and dv of the chunk's keys: one thread per (head, key, 4 channels), summed over the
+        // region's queries
         const int c4n = hd / 4;
         for (int e = threadIdx.x; e < hpc * nj * rs * c4n; e += blockDim.x) {
             const int eh = e / (nj * rs * c4n), rem = e - eh * (nj * rs * c4n);
@@ -186,10 +195,10 @@ __global__ void __launch_bounds__(256) attend_backward_kernel(const BackArgs a)
             const int jj = key / rs, tk = key - jj * rs;
             const int s = sreg[eh * a.topk + j0 + jj];
             if (s < 0) continue;
+            const float *pk = Ps + ((size_t)eh * kc + key) * rs, *sk = Ss + ((size_t)eh * kc + key) * rs;
             float4 gk4 = make_float4(0.f, 0.f, 0.f, 0.f), gv4 = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int tq = 0; tq < rs; ++tq) {
-                const float ds = Ss[((size_t)eh * rs + tq) * kc + key];
-                const float p = Ps[((size_t)eh * rs + tq) * kc + key];
+                const float ds = sk[tq], p = pk[tq];
                 const float4 qq = *reinterpret_cast<const float4 *>(Qs + ((size_t)eh * rs + tq) * hd + c);
                 const float4 dd = *reinterpret_cast<const float4 *>(Ds + ((size_t)eh * rs + tq) * hd + c);
                 gk4.x = fmaf(ds, qq.x, gk4.x);
@@ -236,7 +245,8 @@ size_t back_smem(int hpc, int rs, int hd, int kcr, int topk)
 
 bool attend_backward_supports(const Geometry &g)
 {
-    return g.rs <= 256 && g.hd % 4 == 0 && g.hd <= kSimtMaxHeadDim && back_smem(1, g.rs, g.hd, 1, g.topk) <= kBackMaxSmem;
+    // a head row is a whole number of 16-byte vectors of bf16 (hd % 8) and of fp32 (hd % 4)
+    return g.rs <= 256 && g.hd % 8 == 0 && g.hd <= kSimtMaxHeadDim && back_smem(1, g.rs, g.hd, 1, g.topk) <= kBackMaxSmem;
 }
 
 cudaError_t launch_attend_backward(const void *q, const void *k, const void *v, const int32_t *idx, const void *dout,

@@ -119,7 +119,7 @@ struct GatherArgs {
     const int32_t *idx;
     unsigned *err;
     __nv_bfloat16 *out;   // [B, H, W, C]
-    int H, W, C;
+    int H, W, C;          // the image in memory (the region grid may cover more)
     int n_win, topk, R, hr, wr;
     int ncb;          // 64-channel blocks in C
     int ncb_per_cta;  // channel blocks one work item covers (NCB)
@@ -328,11 +328,13 @@ __global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_
     const LaneOffsets off = lane_offsets(rt, hb, lane);
     // element offsets, inside the region's first token, of this lane's two output rows
     // (rows g and g + 8 of the 16-row tile), channel pair 2t of head hb
-    int row_off[2];
+    int row_off[2], row_y[2], row_x[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int ri = rt * 16 + (lane >> 2) + 8 * h;
-        row_off[h] = ((ri / a.wr) * a.W + ri % a.wr) * a.C + hb * 32 + 2 * (lane & 3);
+        row_y[h] = ri / a.wr;
+        row_x[h] = ri % a.wr;
+        row_off[h] = (row_y[h] * a.W + row_x[h]) * a.C + hb * 32 + 2 * (lane & 3);
     }
     int qs = 0, kvs = 0;
     uint32_t qph = 0, kvph = 0;
@@ -378,10 +380,15 @@ __global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_
             const float l0 = quad_sum(l[0]), l1 = quad_sum(l[1]);
             const float inv0 = l0 > 0.f ? __fdividef(1.f, l0) : 0.f, inv1 = l1 > 0.f ? __fdividef(1.f, l1) : 0.f;
             __nv_bfloat16 *dst = a.out + (((int64_t)info.b * a.H + info.qy) * a.W + info.qx) * a.C + (cb0 + cbl) * 64;
+            // rows of a padded map outside the image are not stored
+            const bool in0 = info.qy + row_y[0] < a.H && info.qx + row_x[0] < a.W;
+            const bool in1 = info.qy + row_y[1] < a.H && info.qx + row_x[1] < a.W;
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
-                *reinterpret_cast<uint32_t *>(dst + row_off[0] + nt * 8) = pack_bf16x2(o[nt][0] * inv0, o[nt][1] * inv0);
-                *reinterpret_cast<uint32_t *>(dst + row_off[1] + nt * 8) = pack_bf16x2(o[nt][2] * inv1, o[nt][3] * inv1);
+                if (in0)
+                    *reinterpret_cast<uint32_t *>(dst + row_off[0] + nt * 8) = pack_bf16x2(o[nt][0] * inv0, o[nt][1] * inv0);
+                if (in1)
+                    *reinterpret_cast<uint32_t *>(dst + row_off[1] + nt * 8) = pack_bf16x2(o[nt][2] * inv1, o[nt][3] * inv1);
             }
         }
     }
@@ -426,15 +433,15 @@ static cudaError_t launch_gather_rs(const CUtensorMap &tq, const CUtensorMap &tk
 }
 
 cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                     const CUtensorMap &tout, const int32_t *idx, void *out, const Geometry &g,
-                                     int num_sms, unsigned *err, cudaStream_t stream)
+                                     const CUtensorMap &tout, const int32_t *idx, void *out, const Geometry &g, int H,
+                                     int W, int num_sms, unsigned *err, cudaStream_t stream)
 {
     GatherArgs a;
     a.idx = idx;
     a.err = err;
     a.out = static_cast<__nv_bfloat16 *>(out);
-    a.H = g.H;
-    a.W = g.W;
+    a.H = H;
+    a.W = W;
     a.C = g.C;
     a.n_win = g.n_win;
     a.topk = g.topk;
@@ -485,6 +492,7 @@ struct DenseArgs {
     int nsplit;
     float scale_log2;
     int inputs_ready;  // q, k, v may be loaded before the wait for the previous kernel
+    int Hm;            // image rows in memory (H: the region grid's, which may be more)
 };
 
 // MIN_CTAS: CTAs per SM the registers are budgeted for (2, or 3 when three CTAs' shared memory
@@ -650,7 +658,7 @@ __global__ void __launch_bounds__(256, MIN_CTAS) attend_dense_mma_kernel(const _
     }
     fence_async_shared();
     __syncthreads();
-    if (threadIdx.x == 0 && alive) {
+    if (threadIdx.x == 0 && alive && y0 < a.Hm) {  // a band wholly below a padded image stores nothing
         tma_store_4d(&tout, sQ, cb * 64, 0, y0, b);
         tma_store_commit();
         tma_store_wait_read();
@@ -680,10 +688,11 @@ static size_t dense_smem_bytes(const Geometry &g, int rows_per_split)
 
 cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                     const CUtensorMap &tout, const int32_t *idx, const Geometry &g, int rows_per_split,
-                                    unsigned *err, bool inputs_ready, cudaStream_t stream)
+                                    unsigned *err, bool inputs_ready, int Hm, cudaStream_t stream)
 {
     DenseArgs a;
     a.inputs_ready = inputs_ready ? 1 : 0;
+    a.Hm = Hm;
     a.idx = idx;
     a.err = err;
     a.H = g.H;

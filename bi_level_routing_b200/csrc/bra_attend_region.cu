@@ -41,6 +41,7 @@ struct RegionArgs {
     int ngroups;  // C / 128
     int nsplit;   // CTAs per (image, group); query regions are dealt among them
     int keys;     // 4 topk rounded up to a multiple of 16
+    int Hm, Wm;   // the image in memory (H, W: the region grid, which may cover more)
     float scale_log2;
     int inputs_ready;  // q, k, v may be loaded before the wait for the previous kernel
 };
@@ -290,11 +291,14 @@ __global__ void __launch_bounds__(32 * kRegionWarps, 1) attend_region_mma_kernel
         // normalise and store: row g -> token qrow, channels 128 grp + 32 hA + 8 i + 2 t4
         const float l0 = quad_sum_f(l[0]), l1 = quad_sum_f(l[1]);
         const float inv0 = l0 > 0.f ? __fdividef(1.f, l0) : 0.f, inv1 = l1 > 0.f ? __fdividef(1.f, l1) : 0.f;
-        __nv_bfloat16 *dst = a.out + ((int64_t)b * a.N + qrow) * a.C + 128 * grp + 2 * t4;
+        const int qy = qrow / a.W, qx = qrow - qy * a.W;  // qrow: a row of the staged (grid-sized) map
+        if (qy < a.Hm && qx < a.Wm) {  // tokens of a padded map outside the image are not stored
+            __nv_bfloat16 *dst = a.out + (((int64_t)b * a.Hm + qy) * a.Wm + qx) * a.C + 128 * grp + 2 * t4;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            *reinterpret_cast<uint32_t *>(dst + 32 * hA + 8 * i) = pack_bf16x2(oA[i][0] * inv0, oA[i][1] * inv0);
-            *reinterpret_cast<uint32_t *>(dst + 32 * hB + 8 * i) = pack_bf16x2(oB[i][0] * inv1, oB[i][1] * inv1);
+            for (int i = 0; i < 4; ++i) {
+                *reinterpret_cast<uint32_t *>(dst + 32 * hA + 8 * i) = pack_bf16x2(oA[i][0] * inv0, oA[i][1] * inv0);
+                *reinterpret_cast<uint32_t *>(dst + 32 * hB + 8 * i) = pack_bf16x2(oB[i][0] * inv1, oB[i][1] * inv1);
+            }
         }
     }
 }
@@ -305,11 +309,13 @@ bool region_mma_supports(const Geometry &g)
 }
 
 cudaError_t launch_attend_region_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                     const int32_t *idx, void *out, const Geometry &g, int num_sms, unsigned *err,
-                                     bool inputs_ready, cudaStream_t stream)
+                                     const int32_t *idx, void *out, const Geometry &g, int H, int W, int num_sms,
+                                     unsigned *err, bool inputs_ready, cudaStream_t stream)
 {
     RegionArgs a;
     a.inputs_ready = inputs_ready ? 1 : 0;
+    a.Hm = H;
+    a.Wm = W;
     a.idx = idx;
     a.err = err;
     a.out = static_cast<__nv_bfloat16 *>(out);

@@ -115,14 +115,27 @@ __global__ void __launch_bounds__(256) attend_staged_kernel(const StagedArgs a)
             if (!real) continue;
             const T *kh = Ks + (size_t)hl * nkc * a.hd;
             const T *vh = Vs + (size_t)hl * nkc * a.hd;
+            constexpr int V = Vec16<T>::N;
             for (int jj = 0; jj < nj; ++jj) {
                 if (sreg[hl * a.kchunk + jj] < 0) continue;  // a skipped region contributes no key
                 for (int tk = 0; tk < a.rs; ++tk) {
                     const T *kr = kh + (size_t)(jj * a.rs + tk) * a.hd;
+                    const T *vr = vh + (size_t)(jj * a.rs + tk) * a.hd;
                     float dot = 0.f;
+                    if (a.vec) {  // 16-byte rows: V channels per shared-memory load
 #pragma unroll
-                    for (int c = 0; c < HDMAX; ++c)
-                        if (c < a.hd) dot = fmaf(qv[c], to_float(kr[c]), dot);
+                        for (int c0 = 0; c0 < HDMAX; c0 += V)
+                            if (c0 < a.hd) {
+                                float f[V];
+                                Vec16<T>::load_shared(kr + c0, f);
+#pragma unroll
+                                for (int i = 0; i < V; ++i) dot = fmaf(qv[c0 + i], f[i], dot);
+                            }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < HDMAX; ++c)
+                            if (c < a.hd) dot = fmaf(qv[c], to_float(kr[c]), dot);
+                    }
                     const float sl = dot * a.scale_log2;  // logit in log2 units
                     if (sl > m) {
                         const float corr = fast_exp2(m - sl);
@@ -133,10 +146,20 @@ __global__ void __launch_bounds__(256) attend_staged_kernel(const StagedArgs a)
                     }
                     const float p = fast_exp2(sl - m);
                     l += p;
-                    const T *vr = vh + (size_t)(jj * a.rs + tk) * a.hd;
+                    if (a.vec) {
 #pragma unroll
-                    for (int c = 0; c < HDMAX; ++c)
-                        if (c < a.hd) o[c] = fmaf(p, to_float(vr[c]), o[c]);
+                        for (int c0 = 0; c0 < HDMAX; c0 += V)
+                            if (c0 < a.hd) {
+                                float f[V];
+                                Vec16<T>::load_shared(vr + c0, f);
+#pragma unroll
+                                for (int i = 0; i < V; ++i) o[c0 + i] = fmaf(p, f[i], o[c0 + i]);
+                            }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < HDMAX; ++c)
+                            if (c < a.hd) o[c] = fmaf(p, to_float(vr[c]), o[c]);
+                    }
                 }
             }
         }

@@ -44,7 +44,7 @@ struct UmmaArgs {
     const int32_t *idx;
     unsigned *err;
     __nv_bfloat16 *out;
-    int H, W, C, n_win, topk, R, hr, wr;
+    int H, W, C, n_win, topk, R, hr, wr;  // H, W: the image in memory (the region grid may cover more)
     int ncb;  // 64-channel blocks = work items per (image, region)
     int nitems, per_cta, qslots, kvslots, idx_chunk;
     float scale_log2;
@@ -258,6 +258,7 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
 #pragma unroll
         for (int c = 0; c < 32; ++c) o[c] = 0.f;
         __nv_bfloat16 *dst = nullptr, *dst_prev = nullptr;
+        bool dst_in = false, dst_prev_in = false;  // the row's token lies inside the image
         // Routing indices run three units ahead of use, loaded with a volatile load at a fixed
         // place in the loop: the L2 latency under full HBM load is close to a microsecond.
         // (pb, pc, pj) = (image * R + region, channel block, routed slot) of the next load.
@@ -298,7 +299,9 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
                 if (j == 0) {
                     item_start = true;
                     dst_prev = dst;
+                    dst_prev_in = dst_in;
                     dst = a.out + (((int64_t)ib * a.H + ry * a.hr) * a.W + rx * a.wr) * a.C + ic * 64 + out_row;
+                    dst_in = ry * a.hr + row / a.wr < a.H && rx * a.wr + row % a.wr < a.W;
                     if (++ic == a.ncb) {
                         ic = 0;
                         if (++rx == a.n_win) {
@@ -401,8 +404,9 @@ __global__ void __launch_bounds__(192, 1) attend_gather_umma_kernel(const __grid
                     // PV(u - 1) was the last region of the previous item: normalise and store it
                     const float lf = (u == units) ? l : l_prev;
                     __nv_bfloat16 *out = (u == units) ? dst : dst_prev;
+                    const bool in_image = (u == units) ? dst_in : dst_prev_in;
                     const float inv = lf > 0.f ? __fdividef(1.f, lf) : 0.f;
-                    if (alive) {
+                    if (alive && in_image) {
                         const float2 iv = make_float2(inv, inv);
                         uint32_t pk[16];
 #pragma unroll
@@ -434,15 +438,15 @@ bool gather_umma_supports(const Geometry &g)
 }
 
 cudaError_t launch_attend_gather_umma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                      const int32_t *idx, void *out, const Geometry &g, int num_sms, unsigned *err,
-                                      cudaStream_t stream)
+                                      const int32_t *idx, void *out, const Geometry &g, int H, int W, int num_sms,
+                                      unsigned *err, cudaStream_t stream)
 {
     UmmaArgs a;
     a.idx = idx;
     a.err = err;
     a.out = static_cast<__nv_bfloat16 *>(out);
-    a.H = g.H;
-    a.W = g.W;
+    a.H = H;
+    a.W = W;
     a.C = g.C;
     a.n_win = g.n_win;
     a.topk = g.topk;

@@ -78,6 +78,12 @@ template <> struct Vec16<float> {
         const float4 v = __ldg(reinterpret_cast<const float4 *>(p));
         f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
     }
+    // 16 bytes from shared memory (or any generic address) as floats
+    __device__ __forceinline__ static void load_shared(const float *p, float *f)
+    {
+        const float4 v = *reinterpret_cast<const float4 *>(p);
+        f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+    }
 };
 template <> struct Vec16<__nv_bfloat16> {
     static constexpr int N = 8;
@@ -97,6 +103,17 @@ template <> struct Vec16<__nv_bfloat16> {
     __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float *f)
     {
         const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+    // 16 bytes from shared memory (or any generic address) as floats
+    __device__ __forceinline__ static void load_shared(const __nv_bfloat16 *p, float *f)
+    {
+        const uint4 v = *reinterpret_cast<const uint4 *>(p);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -146,15 +163,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return done != 0;
 }
 
-// Waits for phase `parity` of `bar` to complete; gives up after kWaitLimitNs, flags
-// kErrTimeout and returns false. Each try suspends the thread in hardware (up to
-// kWaitSuspendNs) until the phase completes, so waiting costs no issue slots.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned *err)
+// Waits for phase `parity` of `bar` to complete; gives up after limit_ns nanoseconds (kWaitLimitNs
+// unless given), flags kErrTimeout and returns false. Each try suspends the thread in hardware
+// (up to kWaitSuspendNs) until the phase completes, so waiting costs no issue slots.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned *err,
+                                          unsigned long long limit_ns = kWaitLimitNs)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_timer_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
             flag_error(err, kErrTimeout);
             return false;
         }

@@ -108,11 +108,15 @@ cudaError_t launch_lepe(const void *x, const float *weight, const float *bias, v
                         bool bf16, cudaStream_t stream);
 
 // Backward of the token attention with idx fixed: dq, dk, dv (fp32 [B, H, W, C]) of
-// sum(dout * out); clears dk and dv (memset nodes), then one kernel. Needs hd % 4 == 0, rs <= 256.
+// sum(dout * out); clears dk and dv (memset nodes), then one kernel. Needs hd % 8 == 0, rs <= 256.
 bool attend_backward_supports(const Geometry &g);
 cudaError_t launch_attend_backward(const void *q, const void *k, const void *v, const int32_t *idx, const void *dout,
                                    float *dq, float *dk, float *dv, const Geometry &g, bool bf16, unsigned *err,
                                    cudaStream_t stream);
+
+// One thread waits on an mbarrier that never completes, with the library's bounded wait given
+// limit_ns; it gives up and sets kErrTimeout in *err.
+cudaError_t launch_wait_timeout(unsigned *err, unsigned long long limit_ns, cudaStream_t stream);
 
 // Largest R the routing kernel handles.
 constexpr int kMaxRegions = 1024;
@@ -124,7 +128,10 @@ cudaError_t launch_attend_simt(const void *q, const void *k, const void *v, cons
 
 // Tensor-core attention kernels (bf16, hd == 32, C % 64 == 0). The tensor maps describe
 // q, k, v, out as 4-D (C, W, H, B) bf16 tensors, 128-byte swizzle (except the gather kernel's
-// q, k and v maps, 5-D, below); box sizes as each launcher's comment states.
+// q, k and v maps, 5-D, below); box sizes as each launcher's comment states. g is the region
+// grid; H, W (arguments of the launchers that take them, and the maps' dimensions) the image in
+// memory, smaller than the grid for a padded map (auto_pad): boxes that reach past the image read
+// zeros, and rows outside it are not stored.
 bool gather_mma_supports(const Geometry &g);
 bool dense_mma_supports(const Geometry &g);
 
@@ -135,8 +142,8 @@ bool region_mma_supports(const Geometry &g);
 // for its predecessor on the stream (true when that predecessor is the routing kernel of the same
 // forward pass, which already waited for their producers); idx is read after the wait.
 cudaError_t launch_attend_region_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                     const int32_t *idx, void *out, const Geometry &g, int num_sms, unsigned *err,
-                                     bool inputs_ready, cudaStream_t stream);
+                                     const int32_t *idx, void *out, const Geometry &g, int H, int W, int num_sms,
+                                     unsigned *err, bool inputs_ready, cudaStream_t stream);
 
 // Box of the gather kernel's q, k and v maps: (64 channels, wr, hr, NCB channel blocks, 1 image)
 // on the 5-D view (channel in block, x, y, channel block, image) of [B, H, W, C], so that one
@@ -144,20 +151,21 @@ cudaError_t launch_attend_region_mma(const CUtensorMap &tq, const CUtensorMap &t
 // box (64, wr, hr, 1).
 void gather_mma_box(const Geometry &g, int box[5]);
 cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                     const CUtensorMap &tout, const int32_t *idx, void *out, const Geometry &g,
-                                     int num_sms, unsigned *err, cudaStream_t stream);
+                                     const CUtensorMap &tout, const int32_t *idx, void *out, const Geometry &g, int H,
+                                     int W, int num_sms, unsigned *err, cudaStream_t stream);
 
 // tcgen05 gather attention for 64-token regions (bf16, hd == 32, C % 64 == 0). Maps: q, k, v
 // with box (64, wr, hr, 1).
 bool gather_umma_supports(const Geometry &g);
 cudaError_t launch_attend_gather_umma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                      const int32_t *idx, void *out, const Geometry &g, int num_sms, unsigned *err,
-                                      cudaStream_t stream);
+                                      const int32_t *idx, void *out, const Geometry &g, int H, int W, int num_sms,
+                                      unsigned *err, cudaStream_t stream);
 
 // Boxes of the dense kernel: q and out (64, W, rows_per_split, 1); k and v (64, W, H, 1).
 int dense_mma_rows_per_split(const Geometry &g, int num_sms);
 cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                     const CUtensorMap &tout, const int32_t *idx, const Geometry &g,
-                                    int rows_per_split, unsigned *err, bool inputs_ready, cudaStream_t stream);
+                                    int rows_per_split, unsigned *err, bool inputs_ready, int Hm,
+                                    cudaStream_t stream);
 
 }  // namespace bra

@@ -4,11 +4,13 @@
 // it). x and y are [B, H, W, C] (bf16 or fp32); weight is fp32 [C, 5, 5] (cross-correlation, as
 // nn.Conv2d), bias fp32 [C]. Arithmetic in fp32, y rounded to the element type.
 //
-// One CTA per (image, 8 x 8 output tokens, block of CB channels): the 12 x 12 input tokens of the
+// One CTA per (image, 16 x 8 output tokens, block of CB channels): the 20 x 12 input tokens of the
 // tile and its 2-token halo (zeros outside the image) are staged in shared memory as fp32, with
-// the block's 25 taps and bias; each thread then computes a pair of channels of several output
-// tokens with packed fp32 FMAs, adds the residual and writes the pair. Every input element is
-// read from global memory once per tile it touches (1.0 + halo), every output written once.
+// the block's 25 taps and bias. Thread (column ox, channel pair cp) keeps the pair's 25 taps and
+// the 16 outputs of its column in registers and sweeps the column's 20 input rows once, adding
+// each row's 5 taps into the outputs it reaches (packed fp32 FMAs); then it adds the residual and
+// writes the pairs. Every input element is read from global memory once per tile it touches
+// (halo included), every output written once.
 #include "bra_device.cuh"
 #include "bra_launch.h"
 
@@ -16,8 +18,8 @@ namespace bra {
 
 namespace {
 
-constexpr int kTile = 8;                // output tokens per tile side
-constexpr int kIn = kTile + 4;          // input tokens per tile side (halo 2)
+constexpr int kTileY = 16, kTileX = 8;  // output tokens per tile
+constexpr int kInY = kTileY + 4, kInX = kTileX + 4;  // input tokens per tile (halo 2)
 constexpr int kLepeThreads = 256;
 
 // Two adjacent outputs (an even channel and the next) in one store: bf16 rounded to nearest even.
@@ -38,11 +40,11 @@ __global__ void __launch_bounds__(kLepeThreads) lepe_kernel(const T *__restrict_
                                                             int W, int C, int CB)
 {
     extern __shared__ float4 smem4[];
-    float *sx = reinterpret_cast<float *>(smem4);  // [kIn * kIn][CB]
-    float *sw = sx + kIn * kIn * CB;               // [25][CB]: tap-major, channels contiguous
+    float *sx = reinterpret_cast<float *>(smem4);  // [kInY * kInX][CB]
+    float *sw = sx + kInY * kInX * CB;             // [25][CB]: tap-major, channels contiguous
     float *sb = sw + 25 * CB;                      // [CB]
     const int nblk = C / CB;
-    const int tiles_x = (W + kTile - 1) / kTile, tiles_y = (H + kTile - 1) / kTile;
+    const int tiles_x = (W + kTileX - 1) / kTileX, tiles_y = (H + kTileY - 1) / kTileY;
     int64_t blk = blockIdx.x;
     const int cb = (int)(blk % nblk);
     blk /= nblk;
@@ -50,15 +52,15 @@ __global__ void __launch_bounds__(kLepeThreads) lepe_kernel(const T *__restrict_
     blk /= tiles_x;
     const int ty = (int)(blk % tiles_y);
     const int64_t b = blk / tiles_y;
-    const int y0 = ty * kTile - 2, x0 = tx * kTile - 2, c0 = cb * CB;
+    const int y0 = ty * kTileY - 2, x0 = tx * kTileX - 2, c0 = cb * CB;
     grid_dependency_wait();
 
     // stage the input tile with its halo (16-byte vectors of channels), the taps and the bias
     constexpr int V = Vec16<T>::N;
     const int vpt = CB / V;
-    for (int e = threadIdx.x; e < kIn * kIn * vpt; e += kLepeThreads) {
+    for (int e = threadIdx.x; e < kInY * kInX * vpt; e += kLepeThreads) {
         const int tok = e / vpt, u = e - tok * vpt;
-        const int iy = y0 + tok / kIn, ix = x0 + tok % kIn;
+        const int iy = y0 + tok / kInX, ix = x0 + tok % kInX;
         float f[V];
         if (iy >= 0 && iy < H && ix >= 0 && ix < W) {
             Vec16<T>::load(x + ((b * H + iy) * W + ix) * C + c0 + u * V, f);
@@ -66,38 +68,57 @@ __global__ void __launch_bounds__(kLepeThreads) lepe_kernel(const T *__restrict_
 #pragma unroll
             for (int i = 0; i < V; ++i) f[i] = 0.f;
         }
+        float4 *d = reinterpret_cast<float4 *>(sx + tok * CB + u * V);
 #pragma unroll
-        for (int i = 0; i < V; ++i) sx[tok * CB + u * V + i] = f[i];
+        for (int i = 0; i < V / 4; ++i) d[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
     }
     for (int e = threadIdx.x; e < 25 * CB; e += kLepeThreads) {
-        const int tap = e / CB, c = e - tap * CB;
-        sw[e] = weight[(int64_t)(c0 + c) * 25 + tap];
+        const int c = e / 25, tap = e - c * 25;  // consecutive threads read consecutive taps
+        sw[tap * CB + c] = weight[(int64_t)(c0 + c) * 25 + tap];
     }
     for (int c = threadIdx.x; c < CB; c += kLepeThreads) sb[c] = bias[c0 + c];
     __syncthreads();
 
-    // thread: channel pair cp, output tokens tg, tg + groups, ...
+    // thread: channel pair cp of output column ox (a CTA has CB / 2 x kTileX <= 256 such threads;
+    // with fewer channel pairs the extra threads take a second column half: rows split in two)
     const int pairs = CB / 2;
-    const int cp = threadIdx.x % pairs, groups = kLepeThreads / pairs;
-    const int tg = threadIdx.x / pairs;
-    if (tg >= groups) return;
+    const int cols = kLepeThreads / pairs;  // >= kTileX
+    const int cp = threadIdx.x % pairs, col = threadIdx.x / pairs;
+    const int ox = col % kTileX, half = col / kTileX, nhalf = cols / kTileX;  // nhalf: 1, 2, 4 or 8
+    const int rows = kTileY / nhalf, oy0 = half * rows;  // this thread's output rows
+    float2 wt[25];
+#pragma unroll
+    for (int i = 0; i < 25; ++i) wt[i] = *reinterpret_cast<const float2 *>(&sw[i * CB + 2 * cp]);
+    float2 acc[kTileY];
     const float2 bb = make_float2(sb[2 * cp], sb[2 * cp + 1]);
-    for (int t = tg; t < kTile * kTile; t += groups) {
-        const int oy = t / kTile, ox = t % kTile;
-        const int gy = ty * kTile + oy, gx = tx * kTile + ox;
-        if (gy >= H || gx >= W) continue;
-        float2 acc = bb;
 #pragma unroll
-        for (int dy = 0; dy < 5; ++dy)
+    for (int i = 0; i < kTileY; ++i) acc[i] = bb;
+    // input rows oy0 .. oy0 + rows + 3; row iy reaches outputs oy = iy - dy, dy = 0..4
 #pragma unroll
-            for (int dx = 0; dx < 5; ++dx) {
-                const float2 xv = *reinterpret_cast<const float2 *>(&sx[((oy + dy) * kIn + ox + dx) * CB + 2 * cp]);
-                const float2 wv = *reinterpret_cast<const float2 *>(&sw[(dy * 5 + dx) * CB + 2 * cp]);
-                acc = __ffma2_rn(xv, wv, acc);
+    for (int r = 0; r < kTileY + 4; ++r) {
+        if (r < rows + 4) {
+            const int iy = oy0 + r;
+            float2 xr[5];
+#pragma unroll
+            for (int dx = 0; dx < 5; ++dx) xr[dx] = *reinterpret_cast<const float2 *>(&sx[(iy * kInX + ox + dx) * CB + 2 * cp]);
+#pragma unroll
+            for (int dy = 0; dy < 5; ++dy) {
+                const int o = r - dy;  // output row (relative to oy0) this input row reaches with tap dy
+                if (o >= 0 && o < rows) {
+#pragma unroll
+                    for (int dx = 0; dx < 5; ++dx) acc[o] = __ffma2_rn(xr[dx], wt[dy * 5 + dx], acc[o]);
+                }
             }
-        const float2 xc = *reinterpret_cast<const float2 *>(&sx[((oy + 2) * kIn + ox + 2) * CB + 2 * cp]);
-        const float r0 = xc.x + acc.x, r1 = xc.y + acc.y;
-        store_pair(y + ((b * H + gy) * W + gx) * C + c0 + 2 * cp, r0, r1);
+        }
+    }
+#pragma unroll
+    for (int o = 0; o < kTileY; ++o) {
+        if (o >= rows) break;
+        const int oy = oy0 + o;
+        const int gy = ty * kTileY + oy, gx = tx * kTileX + ox;
+        if (gy >= H || gx >= W) continue;
+        const float2 xc = *reinterpret_cast<const float2 *>(&sx[((oy + 2) * kInX + ox + 2) * CB + 2 * cp]);
+        store_pair(y + ((b * H + gy) * W + gx) * C + c0 + 2 * cp, xc.x + acc[o].x, xc.y + acc[o].y);
     }
 }
 
@@ -111,9 +132,21 @@ cudaError_t launch_lepe(const void *x, const float *weight, const float *bias, v
     int CB = 64;
     while (CB > 4 && C % CB != 0) CB >>= 1;
     if (C % CB != 0 || CB % (bf16 ? 8 : 4) != 0) return cudaErrorInvalidConfiguration;
-    const size_t smem = ((size_t)kIn * kIn * CB + 25 * (size_t)CB + CB) * sizeof(float);
-    const long long blocks = (long long)B * ((H + kTile - 1) / kTile) * ((W + kTile - 1) / kTile) * (C / CB);
+    const size_t smem = ((size_t)kInY * kInX * CB + 25 * (size_t)CB + CB) * sizeof(float);
+    const long long blocks = (long long)B * ((H + kTileY - 1) / kTileY) * ((W + kTileX - 1) / kTileX) * (C / CB);
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    static int granted[2][64] = {{0}};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if ((int)smem > granted[bf16 ? 1 : 0][dev]) {
+        e = bf16 ? cudaFuncSetAttribute(lepe_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)smem)
+                 : cudaFuncSetAttribute(lepe_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        granted[bf16 ? 1 : 0][dev] = (int)smem;
+    }
     if (bf16)
         return launch_pdl(lepe_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3(kLepeThreads), smem, stream,
                           static_cast<const __nv_bfloat16 *>(x), weight, bias, static_cast<__nv_bfloat16 *>(y), H, W,

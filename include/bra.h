@@ -182,7 +182,7 @@ bra_status bra_forward_lepe(const void *q, const void *k, const void *v, int32_t
    with respect to q, k and v. q, k, v, dout: device [B, H, W, C] of dtype; idx: device int32
    [B, n_win^2, topk] (out-of-range entries skipped and flagged); dq, dk, dv: device fp32
    [B, H, W, C], written (dk and dv are cleared first, then accumulated with atomics, so their
-   last bits may differ between runs). BRA_ERR_UNSUPPORTED: hd % 4 != 0, hd > 128, or a region of
+   last bits may differ between runs). BRA_ERR_UNSUPPORTED: hd % 8 != 0, hd > 128, or a region of
    more than 256 tokens. */
 bra_status bra_attend_backward(const void *q, const void *k, const void *v, const int32_t *idx, const void *dout,
                                float *dq, float *dk, float *dv, int B, int H, int W, int C, int heads, int n_win,
@@ -211,6 +211,13 @@ bra_status bra_set_max_ctas(int max_ctas);
 /* The attention kernel a call with these arguments would use (after any forcing), or -1 if
    the call would be rejected or unsupported. */
 int bra_selected_attend_kernel(int B, int H, int W, int C, int heads, int n_win, int topk, bra_dtype dtype);
+
+/* A check of the bounded wait that every pipelined kernel of the library uses: launches one
+   thread that waits on an mbarrier nothing ever completes, with that wait given a limit of
+   limit_us microseconds (1 .. 1000000; the kernels of the forward pass use 2 s). The wait gives
+   up, sets BRA_ERR_TIMEOUT in the device error word and the kernel returns, with nothing else
+   in flight; bra_check_device_error then returns BRA_ERR_TIMEOUT. Computes nothing. */
+bra_status bra_selftest_wait_timeout(unsigned limit_us, void *stream);
 
 /* Synchronises `stream`, then reads and clears the current device's sticky error word:
    BRA_OK, BRA_ERR_INDEX (an idx entry outside [0, R) was skipped) or BRA_ERR_TIMEOUT. */

@@ -147,7 +147,8 @@ def test_backward_duplicates():
 
 PAD_SHAPES = [_w("stage1_54", 8, 54, 54, 64, 2, 7, 1, "bf16"), _w("stage2_27x30", 4, 27, 30, 128, 4, 7, 4, "bf16"),
               _w("stage3_13", 8, 13, 13, 256, 8, 7, 16, "bf16"), _w("tiny_25x26_f32", 1, 25, 26, 64, 2, 7, 4, "f32"),
-              _w("highres_125", 1, 125, 121, 64, 2, 16, 4, "bf16"), _w("divisible", 2, 28, 28, 64, 2, 7, 4, "bf16")]
+              _w("highres_125", 1, 125, 121, 64, 2, 16, 4, "bf16"), _w("divisible", 2, 28, 28, 64, 2, 7, 4, "bf16"),
+              _w("stage4_6x5", 8, 6, 5, 512, 16, 7, 49, "bf16", "iid"), _w("rs4_13x12_c64", 4, 13, 12, 64, 2, 7, 9, "bf16")]
 
 
 @pytest.mark.parametrize("w", PAD_SHAPES, ids=[w.name for w in PAD_SHAPES])

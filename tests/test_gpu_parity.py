@@ -305,6 +305,20 @@ def test_side_stream_and_host_entry_point():
     assert torch.equal(hout, ref_out.cpu()) and torch.equal(hidx, ref_idx.cpu())
 
 
+def test_host_entry_point_in_chunks():
+    """bra_forward_host splits the batch into chunks whose copies overlap the computation: B = 5
+    gives chunks of 2, 1, 1 and 1 images; every chunk must equal bra_forward on the whole batch."""
+    w = WORKLOADS["stage1"].with_(B=5)
+    inp, (q, k, v) = make(w)
+    ref_out, ref_idx = bra.forward(q, k, v, w.n_win, w.topk, w.heads)
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hout, hidx = bra.forward_host(hq, hk, hv, w.n_win, w.topk, w.heads)
+    assert torch.equal(hout, ref_out.cpu()) and torch.equal(hidx, ref_idx.cpu())
+    # pageable host memory works too
+    hout2, hidx2 = bra.forward_host(q.cpu(), k.cpu(), v.cpu(), w.n_win, w.topk, w.heads)
+    assert torch.equal(hout2, ref_out.cpu()) and torch.equal(hidx2, ref_idx.cpu())
+
+
 def test_repeatable():
     """Same inputs, same bits: the kernels use no atomics in their arithmetic."""
     w = WORKLOADS["highres"].with_(B=2)
