@@ -62,11 +62,14 @@ __global__ void __launch_bounds__(256) attend_backward_kernel(const BackArgs a)
     const int ry = r / a.n_win, rx = r - ry * a.n_win;
     const int hd = a.hd, rs = a.rs, hpc = a.hpc;
     const int kc = a.kcr * rs;  // keys per chunk and head
+    // a head's staged key rows start 4 floats past a multiple of 32: the heads that share a warp
+    // (regions of fewer than 32 tokens) read their rows from different banks
+    const size_t hstride = (size_t)kc * hd + 4;
     float *Qs = reinterpret_cast<float *>(smem4);      // [hpc][rs][hd]
     float *Ds = Qs + (size_t)hpc * rs * hd;            // [hpc][rs][hd] dout
-    float *Ks = Ds + (size_t)hpc * rs * hd;            // [hpc][kc][hd]
-    float *Vs = Ks + (size_t)hpc * kc * hd;            // [hpc][kc][hd]
-    float *Ps = Vs + (size_t)hpc * kc * hd;            // [hpc][kc][rs]: p of (key, query)
+    float *Ks = Ds + (size_t)hpc * rs * hd;            // [hpc] x hstride: [kc][hd]
+    float *Vs = Ks + (size_t)hpc * hstride;            // [hpc] x hstride: [kc][hd]
+    float *Ps = Vs + (size_t)hpc * hstride;            // [hpc][kc][rs]: p of (key, query)
     float *Ss = Ps + (size_t)hpc * kc * rs;            // [hpc][kc][rs]: ds of (key, query)
     int *sreg = reinterpret_cast<int *>(Ss + (size_t)hpc * kc * rs);  // [hpc][topk]
     const T *gq = static_cast<const T *>(a.q), *gk = static_cast<const T *>(a.k);
@@ -105,21 +108,46 @@ __global__ void __launch_bounds__(256) attend_backward_kernel(const BackArgs a)
     // running max and sum of the softmax, and sum_i e_i (dout . v_i) relative to the same max
     float m = -INFINITY, l = 0.f, dsum = 0.f;
 
-    // stages the key and value rows of routed slots [j0, j0 + nj) of every head of the group
+    // stages the key and value rows of routed slots [j0, j0 + nj) of every head of the group:
+    // four 16-byte vectors of k and four of v per thread in flight before their conversion
     auto stage = [&](int j0, int nj) {
-        for (int e = threadIdx.x; e < hpc * nj * rs * nvh; e += blockDim.x) {
-            const int row = e / nvh, u = e - row * nvh;
-            const int eh = row / (nj * rs), key = row - eh * (nj * rs);
-            const int jj = key / rs, tk = key - jj * rs;
-            const int s = sreg[eh * a.topk + j0 + jj];
-            float *kd = Ks + ((size_t)eh * kc + key) * hd, *vd = Vs + ((size_t)eh * kc + key) * hd;
-            if (s >= 0) {
+        constexpr int kBatch = 4;
+        constexpr int V = Vec16<T>::N;
+        const int total = hpc * nj * rs * nvh;
+        for (int e0 = threadIdx.x; e0 < total; e0 += kBatch * blockDim.x) {
+            uint4 kv[kBatch], vv[kBatch];
+            int dsto[kBatch];
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+                const int e = e0 + i * blockDim.x;
+                dsto[i] = -1;
+                if (e >= total) continue;
+                const int row = e / nvh, u = e - row * nvh;
+                const int eh = row / (nj * rs), key = row - eh * (nj * rs);
+                const int jj = key / rs, tk = key - jj * rs;
+                const int s = sreg[eh * a.topk + j0 + jj];
+                if (s < 0) continue;
                 const int sy = s / a.n_win, sx = s - sy * a.n_win;
                 const int y = sy * a.hr + tk / a.wr, x = sx * a.wr + tk % a.wr;
-                const int64_t off = ((b * a.H + y) * a.W + x) * a.C + (int64_t)(hg * hpc + eh) * hd;
-                row_vec_to_f32(kd, gk + off, u);
-                row_vec_to_f32(vd, gv + off, u);
+                const int64_t off = ((b * a.H + y) * a.W + x) * a.C + (int64_t)(hg * hpc + eh) * hd + u * V;
+                kv[i] = Vec16<T>::load_raw(gk + off);
+                vv[i] = Vec16<T>::load_raw(gv + off);
+                dsto[i] = (int)(eh * hstride + (size_t)key * hd + u * V);
             }
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i)
+                if (dsto[i] >= 0) {
+                    float fk[V], fv[V];
+                    Vec16<T>::unpack(kv[i], fk);
+                    Vec16<T>::unpack(vv[i], fv);
+                    float4 *dk4 = reinterpret_cast<float4 *>(Ks + dsto[i]);
+                    float4 *dv4 = reinterpret_cast<float4 *>(Vs + dsto[i]);
+#pragma unroll
+                    for (int j = 0; j < V / 4; ++j) {
+                        dk4[j] = make_float4(fk[4 * j], fk[4 * j + 1], fk[4 * j + 2], fk[4 * j + 3]);
+                        dv4[j] = make_float4(fv[4 * j], fv[4 * j + 1], fv[4 * j + 2], fv[4 * j + 3]);
+                    }
+                }
         }
     };
 
@@ -130,10 +158,11 @@ __global__ void __launch_bounds__(256) attend_backward_kernel(const BackArgs a)
         stage(j0, nj);
         __syncthreads();
         if (!active) continue;
-        for (int key = 0; key < nj * rs; ++key) {
-            if (sreg[hl * a.topk + j0 + key / rs] < 0) continue;
-            const float *kr = Ks + ((size_t)hl * kc + key) * hd;
-            const float *vr = Vs + ((size_t)hl * kc + key) * hd;
+        for (int jj = 0; jj < nj; ++jj) {
+            if (sreg[hl * a.topk + j0 + jj] < 0) continue;  // a skipped region adds no key
+            for (int key = jj * rs; key < (jj + 1) * rs; ++key) {
+            const float *kr = Ks + hl * hstride + (size_t)key * hd;
+            const float *vr = Vs + hl * hstride + (size_t)key * hd;
             float dot = 0.f, dp = 0.f;
 #pragma unroll
             for (int c = 0; c < HDMAX; ++c)
@@ -151,6 +180,7 @@ __global__ void __launch_bounds__(256) attend_backward_kernel(const BackArgs a)
             const float p = fast_exp2(sl - m);
             l += p;
             dsum = fmaf(p, dp, dsum);
+            }
         }
     }
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
@@ -163,11 +193,13 @@ __global__ void __launch_bounds__(256) attend_backward_kernel(const BackArgs a)
         stage(j0, nj);
         __syncthreads();
         if (active) {
-            for (int key = 0; key < nj * rs; ++key) {
+            for (int jj = 0; jj < nj; ++jj) {
+            const bool region_ok = sreg[hl * a.topk + j0 + jj] >= 0;
+            for (int key = jj * rs; key < (jj + 1) * rs; ++key) {
                 float p = 0.f, ds = 0.f;
-                if (sreg[hl * a.topk + j0 + key / rs] >= 0) {
-                    const float *kr = Ks + ((size_t)hl * kc + key) * hd;
-                    const float *vr = Vs + ((size_t)hl * kc + key) * hd;
+                if (region_ok) {
+                    const float *kr = Ks + hl * hstride + (size_t)key * hd;
+                    const float *vr = Vs + hl * hstride + (size_t)key * hd;
                     float dot = 0.f, dp = 0.f;
 #pragma unroll
                     for (int c = 0; c < HDMAX; ++c)
@@ -183,6 +215,7 @@ __global__ void __launch_bounds__(256) attend_backward_kernel(const BackArgs a)
                 }
                 Ps[((size_t)hl * kc + key) * rs + t] = p;
                 Ss[((size_t)hl * kc + key) * rs + t] = ds;
+            }
             }
         }
         __syncthreads();
@@ -237,7 +270,7 @@ constexpr size_t kBackMaxSmem = 100 * 1024;
 size_t back_smem(int hpc, int rs, int hd, int kcr, int topk)
 {
     const size_t kc = (size_t)kcr * rs;
-    return sizeof(float) * ((size_t)2 * hpc * rs * hd + (size_t)2 * hpc * kc * hd + (size_t)2 * hpc * rs * kc) +
+    return sizeof(float) * ((size_t)2 * hpc * rs * hd + (size_t)2 * hpc * (kc * hd + 4) + (size_t)2 * hpc * rs * kc) +
            4 * (size_t)hpc * topk + 16;
 }
 

@@ -49,9 +49,13 @@ __global__ void __launch_bounds__(256) attend_staged_kernel(const StagedArgs a)
     const int64_t b = blk / a.R;
     const int ry = r / a.n_win, rx = r - ry * a.n_win;
     const int nkc = a.kchunk * a.rs;  // staged keys per head and chunk
-    T *Ks = reinterpret_cast<T *>(smem4);              // [hpc][nkc][hd]
-    T *Vs = Ks + (size_t)a.hpc * nkc * a.hd;           // [hpc][nkc][hd]
-    int *sreg = reinterpret_cast<int *>(Vs + (size_t)a.hpc * nkc * a.hd);  // [hpc][kchunk]: region, or -1
+    // a head's rows start 16 bytes past a multiple of 128: heads that share a warp (regions of
+    // fewer than 32 tokens) read their rows from different banks
+    const size_t hstride = (size_t)nkc * a.hd + 16 / sizeof(T);
+    T *Ks = reinterpret_cast<T *>(smem4);              // [hpc] x hstride: [nkc][hd]
+    T *Vs = Ks + (size_t)a.hpc * hstride;              // [hpc] x hstride: [nkc][hd]
+    int *sreg = reinterpret_cast<int *>((reinterpret_cast<uintptr_t>(Vs + (size_t)a.hpc * hstride) + 15) &
+                                        ~uintptr_t(15));  // [hpc][kchunk]: region, or -1
     const T *gq = static_cast<const T *>(a.q);
     const T *gk = static_cast<const T *>(a.k);
     const T *gv = static_cast<const T *>(a.v);
@@ -84,37 +88,64 @@ __global__ void __launch_bounds__(256) attend_staged_kernel(const StagedArgs a)
                 sreg[ehl * a.kchunk + jj] = ok ? s : -1;
             }
             __syncthreads();
-            // stage the key and value rows (head, routed slot, token) of this chunk
+            // stage the key and value rows (head, routed slot, token) of this chunk: 16-byte vectors,
+            // four of k and four of v per thread in flight before their shared-memory stores
             const int rows = a.hpc * nj * a.rs;
-            const int per_row = a.vec ? (a.hd * (int)sizeof(T)) / 16 : a.hd;
-            for (int e = threadIdx.x; e < rows * per_row; e += blockDim.x) {
-                const int row = e / per_row, u = e - row * per_row;
-                const int ehl = row / (nj * a.rs), rem = row - ehl * (nj * a.rs);
-                const int jj = rem / a.rs, tk = rem - jj * a.rs;
-                const int s = sreg[ehl * a.kchunk + jj];
-                if (s < 0) continue;
-                const int sy = s / a.n_win, sx = s - sy * a.n_win;
-                const int ky = sy * a.hr + tk / a.wr, kx = sx * a.wr + tk % a.wr;
-                const bool inside = ky < a.H && kx < a.W;
-                const int64_t goff = ((b * a.H + ky) * a.W + kx) * a.C + (int64_t)(hg * a.hpc + ehl) * a.hd;
-                const size_t soff = ((size_t)ehl * nkc + jj * a.rs + tk) * a.hd;
-                if (a.vec) {
-                    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-                    const int per = 16 / (int)sizeof(T);
-                    reinterpret_cast<uint4 *>(Ks + soff)[u] =
-                        inside ? __ldg(reinterpret_cast<const uint4 *>(gk + goff) + u) : zero;
-                    reinterpret_cast<uint4 *>(Vs + soff)[u] =
-                        inside ? __ldg(reinterpret_cast<const uint4 *>(gv + goff) + u) : zero;
-                    (void)per;
-                } else {
+            if (a.vec) {
+                constexpr int kBatch = 4;
+                const int per_row = (a.hd * (int)sizeof(T)) / 16, total = rows * per_row;
+                for (int e0 = threadIdx.x; e0 < total; e0 += kBatch * blockDim.x) {
+                    uint4 kv[kBatch], vv[kBatch];
+                    size_t so[kBatch];
+#pragma unroll
+                    for (int i = 0; i < kBatch; ++i) {
+                        const int e = e0 + i * blockDim.x;
+                        kv[i] = vv[i] = make_uint4(0u, 0u, 0u, 0u);
+                        so[i] = ~size_t(0);
+                        if (e >= total) continue;
+                        const int row = e / per_row, u = e - row * per_row;
+                        const int ehl = row / (nj * a.rs), rem = row - ehl * (nj * a.rs);
+                        const int jj = rem / a.rs, tk = rem - jj * a.rs;
+                        const int s = sreg[ehl * a.kchunk + jj];
+                        if (s < 0) continue;
+                        so[i] = ehl * hstride + (size_t)(jj * a.rs + tk) * a.hd;
+                        const int sy = s / a.n_win, sx = s - sy * a.n_win;
+                        const int ky = sy * a.hr + tk / a.wr, kx = sx * a.wr + tk % a.wr;
+                        so[i] += (size_t)u * (16 / sizeof(T));
+                        if (ky < a.H && kx < a.W) {
+                            const int64_t goff = ((b * a.H + ky) * a.W + kx) * a.C +
+                                                 (int64_t)(hg * a.hpc + ehl) * a.hd + u * (16 / (int)sizeof(T));
+                            kv[i] = __ldg(reinterpret_cast<const uint4 *>(gk + goff));
+                            vv[i] = __ldg(reinterpret_cast<const uint4 *>(gv + goff));
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < kBatch; ++i)
+                        if (so[i] != ~size_t(0)) {
+                            *reinterpret_cast<uint4 *>(Ks + so[i]) = kv[i];
+                            *reinterpret_cast<uint4 *>(Vs + so[i]) = vv[i];
+                        }
+                }
+            } else {
+                for (int e = threadIdx.x; e < rows * a.hd; e += blockDim.x) {
+                    const int row = e / a.hd, u = e - row * a.hd;
+                    const int ehl = row / (nj * a.rs), rem = row - ehl * (nj * a.rs);
+                    const int jj = rem / a.rs, tk = rem - jj * a.rs;
+                    const int s = sreg[ehl * a.kchunk + jj];
+                    if (s < 0) continue;
+                    const int sy = s / a.n_win, sx = s - sy * a.n_win;
+                    const int ky = sy * a.hr + tk / a.wr, kx = sx * a.wr + tk % a.wr;
+                    const bool inside = ky < a.H && kx < a.W;
+                    const int64_t goff = ((b * a.H + ky) * a.W + kx) * a.C + (int64_t)(hg * a.hpc + ehl) * a.hd;
+                    const size_t soff = ehl * hstride + (size_t)(jj * a.rs + tk) * a.hd;
                     Ks[soff + u] = inside ? gk[goff + u] : from_float<T>(0.f);
                     Vs[soff + u] = inside ? gv[goff + u] : from_float<T>(0.f);
                 }
             }
             __syncthreads();
             if (!real) continue;
-            const T *kh = Ks + (size_t)hl * nkc * a.hd;
-            const T *vh = Vs + (size_t)hl * nkc * a.hd;
+            const T *kh = Ks + hl * hstride;
+            const T *vh = Vs + hl * hstride;
             constexpr int V = Vec16<T>::N;
             for (int jj = 0; jj < nj; ++jj) {
                 if (sreg[hl * a.kchunk + jj] < 0) continue;  // a skipped region contributes no key
@@ -174,7 +205,8 @@ __global__ void __launch_bounds__(256) attend_staged_kernel(const StagedArgs a)
 
 namespace {
 
-constexpr size_t kStagedMaxSmem = 96 * 1024;
+constexpr size_t kStagedMaxSmem = 96 * 1024;     // one routed region per chunk must fit
+constexpr size_t kStagedTargetSmem = 32 * 1024;  // more regions per chunk while within this
 
 template <typename T>
 cudaError_t launch_staged_typed(StagedArgs a, const Geometry &g, cudaStream_t stream)
@@ -189,13 +221,16 @@ cudaError_t launch_staged_typed(StagedArgs a, const Geometry &g, cudaStream_t st
     int threads = ((hpc * a.tq + 31) / 32) * 32;
     if (threads > 256) threads = 256;
     a.vec = ((g.hd * elem) % 16 == 0) ? 1 : 0;
-    // routed regions per chunk: as many as fit
+    // routed regions per chunk: as many as keep the CTA within kStagedTargetSmem (several CTAs per
+    // SM), at least one
     const size_t per_region = (size_t)2 * hpc * g.rs * g.hd * elem + 4 * (size_t)hpc;
-    long long kc = (long long)((kStagedMaxSmem - 16) / per_region);
-    if (kc < 1) return cudaErrorInvalidConfiguration;
+    const size_t fixed = (size_t)2 * hpc * 16 + 32;  // the heads' 16-byte offsets, alignment slack
+    if (per_region + fixed > kStagedMaxSmem) return cudaErrorInvalidConfiguration;
+    long long kc = (long long)((kStagedTargetSmem - fixed) / per_region);
+    if (kc < 1) kc = 1;
     if (kc > g.topk) kc = g.topk;
     a.kchunk = (int)kc;
-    const size_t smem = (size_t)2 * hpc * a.kchunk * g.rs * g.hd * elem + 4 * (size_t)hpc * a.kchunk + 16;
+    const size_t smem = (size_t)a.kchunk * per_region + fixed;
     const long long blocks = (long long)g.B * g.R * (g.heads / hpc);
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     void (*kernel)(const StagedArgs) = g.hd <= 32 ? attend_staged_kernel<T, 32>

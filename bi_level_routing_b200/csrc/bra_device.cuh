@@ -84,6 +84,12 @@ template <> struct Vec16<float> {
         const float4 v = *reinterpret_cast<const float4 *>(p);
         f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
     }
+    // the floats of a 16-byte vector loaded with load_raw
+    __device__ __forceinline__ static void unpack(const uint4 &v, float *f)
+    {
+        f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+    }
 };
 template <> struct Vec16<__nv_bfloat16> {
     static constexpr int N = 8;
@@ -113,7 +119,11 @@ template <> struct Vec16<__nv_bfloat16> {
     // 16 bytes from shared memory (or any generic address) as floats
     __device__ __forceinline__ static void load_shared(const __nv_bfloat16 *p, float *f)
     {
-        const uint4 v = *reinterpret_cast<const uint4 *>(p);
+        unpack(*reinterpret_cast<const uint4 *>(p), f);
+    }
+    // the floats of a 16-byte vector loaded with load_raw
+    __device__ __forceinline__ static void unpack(const uint4 &v, float *f)
+    {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {

@@ -34,7 +34,9 @@ __device__ __forceinline__ void store_pair(float *dst, float a, float b)
 
 }  // namespace
 
-template <typename T>
+// ROWS: output rows per thread, CB / 4 (CB / 2 channel pairs x kTileX columns x kTileY / ROWS row
+// groups = 256 threads); a template argument, so that every loop below unrolls completely.
+template <typename T, int ROWS>
 __global__ void __launch_bounds__(kLepeThreads) lepe_kernel(const T *__restrict__ x, const float *__restrict__ weight,
                                                             const float *__restrict__ bias, T *__restrict__ y, int H,
                                                             int W, int C, int CB)
@@ -55,71 +57,102 @@ __global__ void __launch_bounds__(kLepeThreads) lepe_kernel(const T *__restrict_
     const int y0 = ty * kTileY - 2, x0 = tx * kTileX - 2, c0 = cb * CB;
     grid_dependency_wait();
 
-    // stage the input tile with its halo (16-byte vectors of channels), the taps and the bias
+    // stage the input tile with its halo (16-byte vectors of channels; four loads per thread in
+    // flight before their shared-memory stores), the taps (read in their global order, which is
+    // contiguous for the block: channel-major, 25 taps each) and the bias
     constexpr int V = Vec16<T>::N;
-    const int vpt = CB / V;
-    for (int e = threadIdx.x; e < kInY * kInX * vpt; e += kLepeThreads) {
-        const int tok = e / vpt, u = e - tok * vpt;
-        const int iy = y0 + tok / kInX, ix = x0 + tok % kInX;
-        float f[V];
-        if (iy >= 0 && iy < H && ix >= 0 && ix < W) {
-            Vec16<T>::load(x + ((b * H + iy) * W + ix) * C + c0 + u * V, f);
-        } else {
+    constexpr int kBatch = 4;
+    const int vpt = CB / V, nvec = kInY * kInX * vpt;
+    for (int e0 = threadIdx.x; e0 < nvec; e0 += kBatch * kLepeThreads) {
+        uint4 raw[kBatch];
+        bool inside[kBatch];
 #pragma unroll
-            for (int i = 0; i < V; ++i) f[i] = 0.f;
+        for (int i = 0; i < kBatch; ++i) {
+            const int e = e0 + i * kLepeThreads;
+            const int tok = e / vpt, u = e - tok * vpt;
+            const int iy = y0 + tok / kInX, ix = x0 + tok % kInX;
+            inside[i] = e < nvec && iy >= 0 && iy < H && ix >= 0 && ix < W;
+            if (inside[i]) raw[i] = Vec16<T>::load_raw(x + ((b * H + iy) * W + ix) * C + c0 + u * V);
         }
-        float4 *d = reinterpret_cast<float4 *>(sx + tok * CB + u * V);
 #pragma unroll
-        for (int i = 0; i < V / 4; ++i) d[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+        for (int i = 0; i < kBatch; ++i) {
+            const int e = e0 + i * kLepeThreads;
+            if (e >= nvec) break;
+            float f[V];
+            if (inside[i]) {
+                Vec16<T>::unpack(raw[i], f);
+            } else {
+#pragma unroll
+                for (int j = 0; j < V; ++j) f[j] = 0.f;
+            }
+            const int tok = e / vpt, u = e - tok * vpt;
+            float4 *d = reinterpret_cast<float4 *>(sx + tok * CB + u * V);
+#pragma unroll
+            for (int j = 0; j < V / 4; ++j) d[j] = make_float4(f[4 * j], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]);
+        }
     }
     for (int e = threadIdx.x; e < 25 * CB; e += kLepeThreads) {
-        const int c = e / 25, tap = e - c * 25;  // consecutive threads read consecutive taps
-        sw[tap * CB + c] = weight[(int64_t)(c0 + c) * 25 + tap];
+        const int tap = e / CB, c = e - tap * CB;  // consecutive threads: consecutive channels of a tap
+        sw[e] = weight[(int64_t)(c0 + c) * 25 + tap];
     }
     for (int c = threadIdx.x; c < CB; c += kLepeThreads) sb[c] = bias[c0 + c];
     __syncthreads();
 
-    // thread: channel pair cp of output column ox (a CTA has CB / 2 x kTileX <= 256 such threads;
-    // with fewer channel pairs the extra threads take a second column half: rows split in two)
+    // thread: channel pair cp of output column ox and rows [half ROWS, (half + 1) ROWS) of the tile
+    // (a CTA has CB / 2 x kTileX x kTileY / ROWS = 256 such threads)
     const int pairs = CB / 2;
-    const int cols = kLepeThreads / pairs;  // >= kTileX
     const int cp = threadIdx.x % pairs, col = threadIdx.x / pairs;
-    const int ox = col % kTileX, half = col / kTileX, nhalf = cols / kTileX;  // nhalf: 1, 2, 4 or 8
-    const int rows = kTileY / nhalf, oy0 = half * rows;  // this thread's output rows
+    const int ox = col % kTileX, half = col / kTileX;
+    const int oy0 = half * ROWS;
     float2 wt[25];
 #pragma unroll
     for (int i = 0; i < 25; ++i) wt[i] = *reinterpret_cast<const float2 *>(&sw[i * CB + 2 * cp]);
-    float2 acc[kTileY];
+    float2 acc[ROWS];
     const float2 bb = make_float2(sb[2 * cp], sb[2 * cp + 1]);
 #pragma unroll
-    for (int i = 0; i < kTileY; ++i) acc[i] = bb;
-    // input rows oy0 .. oy0 + rows + 3; row iy reaches outputs oy = iy - dy, dy = 0..4
+    for (int i = 0; i < ROWS; ++i) acc[i] = bb;
+    // input rows oy0 .. oy0 + ROWS + 3; input row r reaches output row r - dy with tap row dy
 #pragma unroll
-    for (int r = 0; r < kTileY + 4; ++r) {
-        if (r < rows + 4) {
-            const int iy = oy0 + r;
-            float2 xr[5];
+    for (int r = 0; r < ROWS + 4; ++r) {
+        float2 xr[5];
 #pragma unroll
-            for (int dx = 0; dx < 5; ++dx) xr[dx] = *reinterpret_cast<const float2 *>(&sx[(iy * kInX + ox + dx) * CB + 2 * cp]);
+        for (int dx = 0; dx < 5; ++dx)
+            xr[dx] = *reinterpret_cast<const float2 *>(&sx[((oy0 + r) * kInX + ox + dx) * CB + 2 * cp]);
 #pragma unroll
-            for (int dy = 0; dy < 5; ++dy) {
-                const int o = r - dy;  // output row (relative to oy0) this input row reaches with tap dy
-                if (o >= 0 && o < rows) {
+        for (int dy = 0; dy < 5; ++dy) {
+            if (r - dy >= 0 && r - dy < ROWS) {
 #pragma unroll
-                    for (int dx = 0; dx < 5; ++dx) acc[o] = __ffma2_rn(xr[dx], wt[dy * 5 + dx], acc[o]);
-                }
+                for (int dx = 0; dx < 5; ++dx) acc[r - dy] = __ffma2_rn(xr[dx], wt[dy * 5 + dx], acc[r - dy]);
             }
         }
     }
+    const int gx = tx * kTileX + ox;
 #pragma unroll
-    for (int o = 0; o < kTileY; ++o) {
-        if (o >= rows) break;
-        const int oy = oy0 + o;
-        const int gy = ty * kTileY + oy, gx = tx * kTileX + ox;
-        if (gy >= H || gx >= W) continue;
-        const float2 xc = *reinterpret_cast<const float2 *>(&sx[((oy + 2) * kInX + ox + 2) * CB + 2 * cp]);
-        store_pair(y + ((b * H + gy) * W + gx) * C + c0 + 2 * cp, xc.x + acc[o].x, xc.y + acc[o].y);
+    for (int o = 0; o < ROWS; ++o) {
+        const int oy = oy0 + o, gy = ty * kTileY + oy;
+        if (gy < H && gx < W) {
+            const float2 xc = *reinterpret_cast<const float2 *>(&sx[((oy + 2) * kInX + ox + 2) * CB + 2 * cp]);
+            store_pair(y + ((b * H + gy) * W + gx) * C + c0 + 2 * cp, xc.x + acc[o].x, xc.y + acc[o].y);
+        }
     }
+}
+
+template <typename T, int ROWS>
+static cudaError_t launch_rows(const void *x, const float *weight, const float *bias, void *y, int H, int W, int C,
+                               int CB, long long blocks, size_t smem, cudaStream_t stream)
+{
+    static int granted[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if ((int)smem > granted[dev]) {
+        e = cudaFuncSetAttribute(lepe_kernel<T, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        granted[dev] = (int)smem;
+    }
+    return launch_pdl(lepe_kernel<T, ROWS>, dim3((unsigned)blocks), dim3(kLepeThreads), smem, stream,
+                      static_cast<const T *>(x), weight, bias, static_cast<T *>(y), H, W, C, CB);
 }
 
 bool lepe_supports(int C, bool bf16) { return C % (bf16 ? 8 : 4) == 0; }
@@ -135,24 +168,21 @@ cudaError_t launch_lepe(const void *x, const float *weight, const float *bias, v
     const size_t smem = ((size_t)kInY * kInX * CB + 25 * (size_t)CB + CB) * sizeof(float);
     const long long blocks = (long long)B * ((H + kTileY - 1) / kTileY) * ((W + kTileX - 1) / kTileX) * (C / CB);
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    static int granted[2][64] = {{0}};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if ((int)smem > granted[bf16 ? 1 : 0][dev]) {
-        e = bf16 ? cudaFuncSetAttribute(lepe_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)smem)
-                 : cudaFuncSetAttribute(lepe_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        granted[bf16 ? 1 : 0][dev] = (int)smem;
+    // rows per thread: CB / 2 channel pairs x 8 columns x (16 / ROWS) row groups = 256 threads
+    const int rows = CB * 8 * 16 / (2 * kLepeThreads);
+    switch (rows) {
+    case 16: return bf16 ? launch_rows<__nv_bfloat16, 16>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream)
+                         : launch_rows<float, 16>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream);
+    case 8: return bf16 ? launch_rows<__nv_bfloat16, 8>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream)
+                        : launch_rows<float, 8>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream);
+    case 4: return bf16 ? launch_rows<__nv_bfloat16, 4>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream)
+                        : launch_rows<float, 4>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream);
+    case 2: return bf16 ? launch_rows<__nv_bfloat16, 2>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream)
+                        : launch_rows<float, 2>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream);
+    case 1: return bf16 ? launch_rows<__nv_bfloat16, 1>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream)
+                        : launch_rows<float, 1>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream);
+    default: return cudaErrorInvalidConfiguration;
     }
-    if (bf16)
-        return launch_pdl(lepe_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3(kLepeThreads), smem, stream,
-                          static_cast<const __nv_bfloat16 *>(x), weight, bias, static_cast<__nv_bfloat16 *>(y), H, W,
-                          C, CB);
-    return launch_pdl(lepe_kernel<float>, dim3((unsigned)blocks), dim3(kLepeThreads), smem, stream,
-                      static_cast<const float *>(x), weight, bias, static_cast<float *>(y), H, W, C, CB);
 }
 
 }  // namespace bra

@@ -854,8 +854,8 @@ namespace bra {
 // Region means of a padded map (auto_pad, "从静态到动态", §4.2): the region grid covers
 // n_win hr x n_win wr tokens, of which those at y >= H or x >= W lie outside the H x W image and
 // are zeros. One warp per region; lane l sums the channel vectors l, l + 32, ... over the
-// region's tokens inside the image in row-major order, and the sum is divided by hr wr (the
-// zeros count).
+// region's tokens inside the image in row-major order (four tokens' loads in flight), and the sum
+// is divided by hr wr (the zeros count).
 template <typename T>
 __global__ void __launch_bounds__(256) region_means_padded_kernel(const T *__restrict__ q, const T *__restrict__ k,
                                                                   float *__restrict__ qm, float *__restrict__ km,
@@ -873,16 +873,30 @@ __global__ void __launch_bounds__(256) region_means_padded_kernel(const T *__res
     const int ry = r / n_win, rx = r - ry * n_win;
     const int y1 = min(H, (ry + 1) * hr), x1 = min(W, (rx + 1) * wr);
     const float n = (float)(hr * wr);
+    const int x0 = rx * wr, nx = x1 - x0, y0 = ry * hr;
+    const int ntok = (y1 - y0) * nx;  // the region's tokens inside the image, row-major
+    constexpr int kBatch = 4;         // tokens' loads of q and of k in flight per lane
     for (int v = lane; v < C / V; v += 32) {
         float aq[V], ak[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) aq[i] = ak[i] = 0.f;
-        for (int y = ry * hr; y < y1; ++y)
-            for (int x = rx * wr; x < x1; ++x) {
-                const int64_t off = ((b * H + y) * W + x) * C + (int64_t)v * V;
-                Vec16<T>::accumulate(Vec16<T>::load_raw(q + off), aq);
-                Vec16<T>::accumulate(Vec16<T>::load_raw(k + off), ak);
-            }
+        for (int t0 = 0; t0 < ntok; t0 += kBatch) {
+            uint4 rq[kBatch], rk[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u)
+                if (t0 + u < ntok) {
+                    const int t = t0 + u, y = y0 + t / nx, x = x0 + t % nx;
+                    const int64_t off = ((b * H + y) * W + x) * C + (int64_t)v * V;
+                    rq[u] = Vec16<T>::load_raw(q + off);
+                    rk[u] = Vec16<T>::load_raw(k + off);
+                }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u)
+                if (t0 + u < ntok) {
+                    Vec16<T>::accumulate(rq[u], aq);
+                    Vec16<T>::accumulate(rk[u], ak);
+                }
+        }
         float4 *dq = reinterpret_cast<float4 *>(qm + reg * C + (int64_t)v * V);
         float4 *dk = reinterpret_cast<float4 *>(km + reg * C + (int64_t)v * V);
 #pragma unroll
