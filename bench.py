@@ -64,7 +64,57 @@ def parse_args(argv=None):
     ap.add_argument("--soak-seconds", type=float, default=1.0,
                     help="identical untimed steps before the timed region, while clocks are sampled")
     ap.add_argument("--repeats", type=int, default=5, help="timed runs of K steps; the median is reported")
+    ap.add_argument("--once", choices=ONCE_ROWS, default=None,
+                    help="run one row of the library --reps times on --workload, untimed, and exit (for profilers)")
+    ap.add_argument("--reps", type=int, default=3, help="calls made by --once")
     return ap.parse_args(argv)
+
+
+ONCE_ROWS = ("forward", "route", "attend", "forward_heads", "lepe", "forward_lepe", "backward", "auto_pad")
+
+
+def run_once(args):
+    """Calls one row of the library a few times on a named workload, eagerly, on fresh seeded
+    inputs (auto_pad: the workload cropped by two rows and columns), checks the device error word
+    and prints one line. Nothing is timed: this is the command that ncu captures."""
+    import torch
+    import bi_level_routing_b200 as bra
+    from bi_level_routing_b200.workloads import WORKLOADS, Workload, make_inputs
+    w = WORKLOADS[args.workload]
+    if args.once == "auto_pad":
+        w = Workload(w.name + "_cropped", w.B, w.H - 2, w.W - 2, w.C, w.heads, w.n_win, w.topk, w.dtype, w.values,
+                     w.seed)
+    inp = make_inputs(w)
+    if w.dtype == "bf16":
+        q, k, v = (torch.from_numpy(inp[n + "_bits"].view(np.int16)).view(torch.bfloat16).cuda() for n in "qkv")
+    else:
+        q, k, v = (torch.from_numpy(inp[n]).cuda() for n in "qkv")
+    rng = np.random.Generator(np.random.PCG64(5))
+    wt = torch.from_numpy(rng.standard_normal((w.C, 5, 5)) * 0.2).float().cuda()
+    bias = torch.from_numpy(rng.standard_normal(w.C) * 0.1).float().cuda()
+    idx = bra.route(q, k, w.n_win, w.topk) if args.once in ("attend", "backward") else None
+    for _ in range(max(1, args.reps)):
+        if args.once == "forward":
+            bra.forward(q, k, v, w.n_win, w.topk, w.heads)
+        elif args.once == "route":
+            bra.route(q, k, w.n_win, w.topk)
+        elif args.once == "attend":
+            bra.attend(q, k, v, idx, w.heads, w.n_win)
+        elif args.once == "forward_heads":
+            bra.forward_heads(q, k, v, w.n_win, w.topk, w.heads)
+        elif args.once == "lepe":
+            bra.lepe(q, wt, bias)
+        elif args.once == "forward_lepe":
+            bra.forward_lepe(q, k, v, w.n_win, w.topk, w.heads, wt, bias)
+        elif args.once == "backward":
+            bra.attend_backward(q, k, v, idx, v, w.heads, w.n_win)
+        else:
+            bra.forward_auto_pad(q, k, v, w.n_win, w.topk, w.heads)
+    torch.cuda.synchronize()
+    status = bra.check_device_error()
+    print(json.dumps({"once": args.once, "workload": w.name, "reps": args.reps, "device_error": status}))
+    if status != 0:
+        raise SystemExit(1)
 
 
 def peaks():
@@ -576,6 +626,9 @@ def main(argv=None):
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     from bi_level_routing_b200.workloads import WORKLOADS
     w = WORKLOADS[args.workload]
+    if args.once:
+        run_once(args)
+        return
     if args.impl == "reference":
         run_reference(args, w, rank)
         return

@@ -272,6 +272,36 @@ bra_status attend_impl(const void *q, const void *k, const void *v, const int32_
     return BRA_OK;
 }
 
+// One-token regions that the dense kernel serves: routing runs inside it (one launch).
+bool fused_forward(const bra::Geometry &g, bra_dtype dtype)
+{
+    return choose_attend_kernel(g, dtype) == BRA_ATTEND_DENSE_MMA && bra::route_dense_supports(g, dtype == BRA_BF16);
+}
+
+// The forward pass on device buffers: the fused kernel where it serves the shape, else the
+// routing step (its fp32 means in `out`, which nothing else writes until the attention kernel)
+// followed by the attention kernel.
+bra_status forward_impl(const void *q, const void *k, const void *v, int32_t *idx, void *out, const bra::Geometry &g,
+                        bra_dtype dtype, cudaStream_t stream)
+{
+    if (fused_forward(g, dtype)) {
+        DeviceState *st = nullptr;
+        bra_status s = device_state(&st);
+        if (s != BRA_OK) return s;
+        CUtensorMap tq, tk, tv, to;
+        if ((s = encode_map(&tq, q, g, g.W, g.H, g.H, g.W)) != BRA_OK) return s;
+        if ((s = encode_map(&tk, k, g, g.W, g.H, g.H, g.W)) != BRA_OK) return s;
+        if ((s = encode_map(&tv, v, g, g.W, g.H, g.H, g.W)) != BRA_OK) return s;
+        if ((s = encode_map(&to, out, g, g.W, g.H, g.H, g.W)) != BRA_OK) return s;
+        const cudaError_t e = bra::launch_route_attend_dense(tq, tk, tv, to, idx, g, st->error_word, stream);
+        return e == cudaSuccess ? BRA_OK : cuda_fail(e, "fused routing and attention kernel");
+    }
+    const size_t out_bytes = (size_t)g.B * g.H * g.W * g.C * (dtype == BRA_BF16 ? 2 : 4);
+    bra_status s = route_impl(q, k, idx, g, dtype, stream, out, out_bytes);
+    if (s != BRA_OK) return s;
+    return attend_impl(q, k, v, idx, out, g, dtype, stream, true);
+}
+
 }  // namespace
 
 namespace bra {
@@ -337,11 +367,7 @@ bra_status bra_forward(const void *q, const void *k, const void *v, int32_t *idx
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(idx, 4))
         return BRA_ERR_INVALID_ARG;
     if (choose_attend_kernel(g, dtype) < 0) return BRA_ERR_UNSUPPORTED;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // out is written only by the attention kernel, after routing: until then it holds the means
-    const size_t out_bytes = (size_t)B * H * W * C * (dtype == BRA_BF16 ? 2 : 4);
-    if ((s = route_impl(q, k, idx, g, dtype, st, out, out_bytes)) != BRA_OK) return s;
-    return attend_impl(q, k, v, idx, out, g, dtype, st, true);
+    return forward_impl(q, k, v, idx, out, g, dtype, static_cast<cudaStream_t>(stream));
 }
 
 bra_status bra_forward_host(const void *q, const void *k, const void *v, int32_t *idx, void *out, int B, int H,
@@ -399,8 +425,7 @@ bra_status bra_forward_host(const void *q, const void *k, const void *v, int32_t
         if (e != cudaSuccess) break;
         bra::Geometry gc = g;
         gc.B = nb;
-        s = route_impl(dq + off, dk + off, didx + ioff, gc, dtype, st, dout + off, bytes);
-        if (s == BRA_OK) s = attend_impl(dq + off, dk + off, dv + off, didx + ioff, dout + off, gc, dtype, st, true);
+        s = forward_impl(dq + off, dk + off, dv + off, didx + ioff, dout + off, gc, dtype, st);
         if (s != BRA_OK) break;
         e = cudaEventRecord(ev_done[c], st);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(dst->copy_out, ev_done[c], 0);
@@ -465,6 +490,47 @@ static bra_status route_heads_impl(const void *q, const void *k, int32_t *idx, c
     return BRA_OK;
 }
 
+// The attention kernel of per-head routing: the mma.sync gather kernel (bf16, hd == 32, rs % 16
+// == 0, rs <= 64) in its per-head mode, else the CUDA-core kernel; a forced kernel that does not
+// take per-head indices (or cannot serve the shape) makes the call unsupported.
+static int choose_heads_kernel(const bra::Geometry &g, bra_dtype dtype)
+{
+    const bool simt_ok = g.hd <= bra::kSimtMaxHeadDim;
+    const bool gather_ok = dtype == BRA_BF16 && bra::gather_mma_supports(g);
+    switch (g_forced_kernel.load()) {
+    case BRA_ATTEND_AUTO: return gather_ok ? BRA_ATTEND_GATHER_MMA : (simt_ok ? BRA_ATTEND_SIMT : -1);
+    case BRA_ATTEND_SIMT: return simt_ok ? BRA_ATTEND_SIMT : -1;
+    case BRA_ATTEND_GATHER_MMA: return gather_ok ? BRA_ATTEND_GATHER_MMA : -1;
+    default: return -1;
+    }
+}
+
+static bra_status attend_heads_impl(const void *q, const void *k, const void *v, const int32_t *idx, void *out,
+                                    const bra::Geometry &g, bra_dtype dtype, cudaStream_t stream)
+{
+    const int kernel = choose_heads_kernel(g, dtype);
+    if (kernel < 0) return BRA_ERR_UNSUPPORTED;
+    DeviceState *st = nullptr;
+    bra_status s = device_state(&st);
+    if (s != BRA_OK) return s;
+    cudaError_t e = cudaSuccess;
+    if (kernel == BRA_ATTEND_SIMT) {
+        e = bra::launch_attend_staged(q, k, v, idx, out, g, g.H, g.W, true, dtype == BRA_BF16, st->error_word, stream);
+    } else {
+        // q: the item's NCB blocks in one box; k, v: one block per box (each head its own region)
+        CUtensorMap tq, tk, tv, to;
+        int box[5];
+        bra::gather_mma_box(g, box);
+        if ((s = encode_map_blocks(&tq, q, g, box[1], box[2], box[3], g.H, g.W)) != BRA_OK) return s;
+        if ((s = encode_map_blocks(&tk, k, g, box[1], box[2], 1, g.H, g.W)) != BRA_OK) return s;
+        if ((s = encode_map_blocks(&tv, v, g, box[1], box[2], 1, g.H, g.W)) != BRA_OK) return s;
+        if ((s = encode_map(&to, out, g, box[1], box[2], g.H, g.W)) != BRA_OK) return s;
+        e = bra::launch_attend_gather_mma(tq, tk, tv, to, idx, out, g, g.H, g.W, st->num_sms, st->error_word, stream,
+                                          true);
+    }
+    return e == cudaSuccess ? BRA_OK : cuda_fail(e, "per-head attention kernel");
+}
+
 static bra_status check_data_ptrs(const void *q, const void *k, const void *v, const int32_t *idx, const void *out)
 {
     if (!q || !k || !v || !idx || !out) return BRA_ERR_INVALID_ARG;
@@ -494,12 +560,7 @@ bra_status bra_attend_heads(const void *q, const void *k, const void *v, const i
     if (s != BRA_OK) return s;
     if (B == 0) return BRA_OK;
     if ((s = check_data_ptrs(q, k, v, idx, out)) != BRA_OK) return s;
-    if (g.hd > bra::kSimtMaxHeadDim) return BRA_ERR_UNSUPPORTED;
-    DeviceState *st = nullptr;
-    if ((s = device_state(&st)) != BRA_OK) return s;
-    const cudaError_t e = bra::launch_attend_staged(q, k, v, idx, out, g, g.H, g.W, true, dtype == BRA_BF16,
-                                                    st->error_word, static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? BRA_OK : cuda_fail(e, "per-head attention kernel");
+    return attend_heads_impl(q, k, v, idx, out, g, dtype, static_cast<cudaStream_t>(stream));
 }
 
 bra_status bra_forward_heads(const void *q, const void *k, const void *v, int32_t *idx, void *out, int B, int H,
@@ -510,15 +571,12 @@ bra_status bra_forward_heads(const void *q, const void *k, const void *v, int32_
     if (s != BRA_OK) return s;
     if (B == 0) return BRA_OK;
     if ((s = check_data_ptrs(q, k, v, idx, out)) != BRA_OK) return s;
-    if (!bra::route_heads_supports(g, dtype == BRA_BF16) || g.hd > bra::kSimtMaxHeadDim) return BRA_ERR_UNSUPPORTED;
+    if (!bra::route_heads_supports(g, dtype == BRA_BF16) || choose_heads_kernel(g, dtype) < 0)
+        return BRA_ERR_UNSUPPORTED;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const size_t out_bytes = (size_t)B * H * W * C * (dtype == BRA_BF16 ? 2 : 4);
     if ((s = route_heads_impl(q, k, idx, g, dtype, cs, out, out_bytes)) != BRA_OK) return s;
-    DeviceState *st = nullptr;
-    if ((s = device_state(&st)) != BRA_OK) return s;
-    const cudaError_t e =
-        bra::launch_attend_staged(q, k, v, idx, out, g, g.H, g.W, true, dtype == BRA_BF16, st->error_word, cs);
-    return e == cudaSuccess ? BRA_OK : cuda_fail(e, "per-head attention kernel");
+    return attend_heads_impl(q, k, v, idx, out, g, dtype, cs);
 }
 
 // ---------------------------------------------------------------- auto_pad
@@ -677,7 +735,7 @@ int bra_kernels_per_call(const char *entry_point, int B, int H, int W, int C, in
     if (!std::strcmp(entry_point, "bra_route")) return route;
     if (!std::strcmp(entry_point, "bra_attend")) return attend;
     if (!std::strcmp(entry_point, "bra_forward") || !std::strcmp(entry_point, "bra_forward_host"))
-        return attend ? route + attend : 0;
+        return attend ? (fused_forward(g, dtype) ? 1 : route + attend) : 0;
     return 0;
 }
 

@@ -25,6 +25,7 @@
 //   weight enters as +log2(cnt) on the logit. Needs R <= 64 and H * W <= 256.
 #include "bra_device.cuh"
 #include "bra_launch.h"
+#include "bra_routing.cuh"
 
 namespace bra {
 
@@ -128,8 +129,12 @@ struct GatherArgs {
     int per_cta;      // contiguous work items per CTA
     int ncw;          // consumer warps = NCB * 2 heads * rs / 16 row tiles
     int qslots, kvslots, idx_chunk;
+    int per_head;     // idx is [B, heads, R, topk]: every head gathers its own regions
+    int heads;
     float scale_log2;
 };
+
+constexpr int kGatherMaxHeads = 8;  // heads of one work item (NCB <= 4 blocks of 2 heads)
 
 // Per-lane byte offsets of the ldmatrix rows inside 128-byte-swizzled tiles. Every row a lane
 // addresses has the same (row & 7), so the swizzle XOR depends on the lane only and the
@@ -220,6 +225,10 @@ struct ItemInfo {
 //    routed region, its K and V tiles into a ring of `kvslots` slots; each slot has a
 //    "full" mbarrier (TMA transaction bytes) and an "empty" one (one arrival per consumer
 //    warp). An idx entry outside [0, R) fills its slot with nothing and is flagged.
+//    Per-head routing (per_head): routed slot j of an item holds, for each of its 2 NCB heads,
+//    the K and V tiles (one 64-channel block) of that head's own j-th region; the head's
+//    warps read their 32 channels of it. (The other 32 channels of the tile are loaded too:
+//    a 64-channel box keeps the 128-byte swizzled layout of the shared-index path.)
 //  * Warps 0..ncw-1 (consumers): warp w owns 16 query rows (w % RT) of head (w / RT) % 2 of
 //    channel block w / (2 RT); it runs attend_region per routed region, then writes its
 //    normalised output into one of two output tiles; one thread stores the tile by TMA
@@ -239,14 +248,15 @@ __global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int NCB = a.ncb_per_cta;
+    const int kv_tiles = (a.per_head ? 4 : 2) * NCB;  // tiles of one KV slot
     uint8_t *sQ = smem;
     uint8_t *sKV = sQ + (size_t)a.qslots * NCB * TILE;
-    uint64_t *full_q = reinterpret_cast<uint64_t *>(sKV + (size_t)a.kvslots * 2 * NCB * TILE);
+    uint64_t *full_q = reinterpret_cast<uint64_t *>(sKV + (size_t)a.kvslots * kv_tiles * TILE);
     uint64_t *empty_q = full_q + a.qslots;
     uint64_t *full_kv = empty_q + a.qslots;
     uint64_t *empty_kv = full_kv + a.kvslots;
-    int *kv_ok = reinterpret_cast<int *>(empty_kv + a.kvslots);
-    ItemInfo *qinfo = reinterpret_cast<ItemInfo *>(kv_ok + a.kvslots);
+    int *kv_ok = reinterpret_cast<int *>(empty_kv + a.kvslots);  // [kvslots][kGatherMaxHeads]
+    ItemInfo *qinfo = reinterpret_cast<ItemInfo *>(kv_ok + a.kvslots * kGatherMaxHeads);
     int *sidx = reinterpret_cast<int *>(qinfo + a.qslots);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -275,9 +285,20 @@ __global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_
         for (int c0 = begin; c0 < end; c0 += a.idx_chunk) {
             const int n = min(a.idx_chunk, end - c0);
             __syncwarp();
-            for (int e = lane; e < n * a.topk; e += 32) {
-                const int it = c0 + e / a.topk, j = e % a.topk;
-                sidx[e] = a.idx[(int64_t)(it / a.groups) * a.topk + j];
+            // index rows of the chunk's items: one per item, or (per_head) one per head of it,
+            // -2 for a head past C (nothing to load, nothing to flag)
+            const int hpi = a.per_head ? 2 * NCB : 1;
+            for (int e = lane; e < n * hpi * a.topk; e += 32) {
+                const int il = e / (hpi * a.topk), rem = e - il * (hpi * a.topk);
+                const int hh = rem / a.topk, j = rem - hh * a.topk;
+                const int it = c0 + il;
+                if (a.per_head) {
+                    const int br = it / a.groups, grp = it - br * a.groups;
+                    const int r = br % a.R, b = br / a.R, h = 2 * grp * NCB + hh;
+                    sidx[e] = h < a.heads ? a.idx[(((int64_t)b * a.heads + h) * a.R + r) * a.topk + j] : -2;
+                } else {
+                    sidx[e] = a.idx[(int64_t)(it / a.groups) * a.topk + j];
+                }
             }
             __syncwarp();
             if (lane != 0 || !alive) continue;
@@ -299,19 +320,41 @@ __global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_
                     qph ^= 1;
                 }
                 for (int j = 0; j < a.topk; ++j) {
-                    const int s = sidx[i * a.topk + j];
-                    const bool ok = s >= 0 && s < a.R;
                     if (!(alive = mbar_wait(&empty_kv[kvs], kvph ^ 1, a.err))) break;
-                    kv_ok[kvs] = ok;
-                    if (ok) {
-                        const int sx = (s % a.n_win) * a.wr, sy = (s / a.n_win) * a.hr;
-                        mbar_arrive_expect_tx(&full_kv[kvs], (uint32_t)(2 * NCB * TILE));
-                        uint8_t *kt = sKV + (size_t)kvs * 2 * NCB * TILE;
-                        tma_load_5d(kt, &tk, 0, sx, sy, cb0, b, &full_kv[kvs]);
-                        tma_load_5d(kt + NCB * TILE, &tv, 0, sx, sy, cb0, b, &full_kv[kvs]);
+                    if (a.per_head) {
+                        // K tiles of the item's heads, then their V tiles (box: one block)
+                        uint8_t *kt = sKV + (size_t)kvs * 4 * NCB * TILE;
+                        int nload = 0;
+                        for (int hh = 0; hh < hpi; ++hh) {
+                            const int s = sidx[(i * hpi + hh) * a.topk + j];
+                            const bool ok = s >= 0 && s < a.R;
+                            if (!ok && s != -2) flag_error(a.err, kErrIndex);
+                            kv_ok[kvs * kGatherMaxHeads + hh] = ok;
+                            nload += ok ? 1 : 0;
+                        }
+                        mbar_arrive_expect_tx(&full_kv[kvs], (uint32_t)(2 * nload * TILE));
+                        for (int hh = 0; hh < hpi; ++hh) {
+                            const int s = sidx[(i * hpi + hh) * a.topk + j];
+                            if (s < 0 || s >= a.R) continue;
+                            const int sx = (s % a.n_win) * a.wr, sy = (s / a.n_win) * a.hr;
+                            tma_load_5d(kt + (size_t)hh * TILE, &tk, 0, sx, sy, cb0 + hh / 2, b, &full_kv[kvs]);
+                            tma_load_5d(kt + (size_t)(2 * NCB + hh) * TILE, &tv, 0, sx, sy, cb0 + hh / 2, b,
+                                        &full_kv[kvs]);
+                        }
                     } else {
-                        flag_error(a.err, kErrIndex);
-                        mbar_arrive_expect_tx(&full_kv[kvs], 0);
+                        const int s = sidx[i * a.topk + j];
+                        const bool ok = s >= 0 && s < a.R;
+                        kv_ok[kvs * kGatherMaxHeads] = ok;
+                        if (ok) {
+                            const int sx = (s % a.n_win) * a.wr, sy = (s / a.n_win) * a.hr;
+                            mbar_arrive_expect_tx(&full_kv[kvs], (uint32_t)(2 * NCB * TILE));
+                            uint8_t *kt = sKV + (size_t)kvs * 2 * NCB * TILE;
+                            tma_load_5d(kt, &tk, 0, sx, sy, cb0, b, &full_kv[kvs]);
+                            tma_load_5d(kt + NCB * TILE, &tv, 0, sx, sy, cb0, b, &full_kv[kvs]);
+                        } else {
+                            flag_error(a.err, kErrIndex);
+                            mbar_arrive_expect_tx(&full_kv[kvs], 0);
+                        }
                     }
                     if (++kvs == a.kvslots) {
                         kvs = 0;
@@ -326,6 +369,10 @@ __global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_
     // ----------------------------------------------------------------- consumer warps
     const int rt = warp % RT, hb = (warp / RT) & 1, cbl = warp / (2 * RT);
     const LaneOffsets off = lane_offsets(rt, hb, lane);
+    // this warp's K tile in a KV slot, the distance from it to its V tile, its validity flag
+    const int kt_index = a.per_head ? cbl * 2 + hb : cbl;
+    const int v_dist = a.per_head ? 2 * NCB : NCB;
+    const int ok_index = a.per_head ? cbl * 2 + hb : 0;
     // element offsets, inside the region's first token, of this lane's two output rows
     // (rows g and g + 8 of the 16-row tile), channel pair 2t of head hb
     int row_off[2], row_y[2], row_x[2];
@@ -363,9 +410,9 @@ __global__ void __launch_bounds__(288, 2) attend_gather_mma_kernel(const __grid_
         for (int nt = 0; nt < 4; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
         for (int j = 0; j < a.topk; ++j) {
             if (alive) alive = mbar_wait(&full_kv[kvs], kvph, a.err);
-            if (alive && active && kv_ok[kvs]) {
-                const uint32_t ktile = smem_u32(sKV + (size_t)(kvs * 2 * NCB + cbl) * TILE);
-                attend_region<NT>(o, m, l, qf, ktile, ktile + NCB * TILE, off, a.scale_log2);
+            if (alive && active && kv_ok[kvs * kGatherMaxHeads + ok_index]) {
+                const uint32_t ktile = smem_u32(sKV + (size_t)(kvs * kv_tiles + kt_index) * TILE);
+                attend_region<NT>(o, m, l, qf, ktile, ktile + v_dist * TILE, off, a.scale_log2);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty_kv[kvs]);
@@ -434,9 +481,11 @@ static cudaError_t launch_gather_rs(const CUtensorMap &tq, const CUtensorMap &tk
 
 cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                      const CUtensorMap &tout, const int32_t *idx, void *out, const Geometry &g, int H,
-                                     int W, int num_sms, unsigned *err, cudaStream_t stream)
+                                     int W, int num_sms, unsigned *err, cudaStream_t stream, bool per_head)
 {
     GatherArgs a;
+    a.per_head = per_head ? 1 : 0;
+    a.heads = g.heads;
     a.idx = idx;
     a.err = err;
     a.out = static_cast<__nv_bfloat16 *>(out);
@@ -460,15 +509,18 @@ cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &t
     a.nitems = (int)nitems;
     // Two CTAs per SM: ~111 KB of shared memory each for the rings.
     const size_t tile = (size_t)g.rs * kRowBytes * ncb_per_cta;  // one slot of one tensor
+    const size_t kv_tile = (per_head ? 4 : 2) * tile;                // one KV slot
     const size_t budget = 111 * 1024;
-    a.qslots = g.topk <= 2 ? 4 : 2;
-    long long kv = (long long)((budget - a.qslots * tile) / (2 * tile));
+    a.qslots = per_head ? 2 : (g.topk <= 2 ? 4 : 2);
+    long long kv = (long long)((budget - a.qslots * tile) / kv_tile);
     if (kv > 8) kv = 8;
     if (kv < 2) kv = 2;
     a.kvslots = (int)kv;
     a.idx_chunk = g.topk >= 32 ? 1 : 32 / g.topk;
-    const size_t smem = 1024 + tile * (a.qslots + 2 * a.kvslots) + 16 * (a.qslots + a.kvslots) + 4 * a.kvslots +
-                        sizeof(ItemInfo) * a.qslots + 4 * (size_t)a.idx_chunk * g.topk;
+    const int hpi = per_head ? 2 * ncb_per_cta : 1;  // index rows per item
+    const size_t smem = 1024 + tile * a.qslots + kv_tile * a.kvslots + 16 * (a.qslots + a.kvslots) +
+                        4 * (size_t)kGatherMaxHeads * a.kvslots + sizeof(ItemInfo) * a.qslots +
+                        4 * (size_t)a.idx_chunk * g.topk * hpi;
     int grid = persistent_grid(a.nitems, num_sms);
     a.per_cta = (a.nitems + grid - 1) / grid;
     grid = (a.nitems + a.per_cta - 1) / a.per_cta;
@@ -485,19 +537,82 @@ cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &t
 
 struct DenseArgs {
     const int32_t *idx;
+    int32_t *idx_out;  // ROUTE: the index this kernel selects, [B, R, topk]
     unsigned *err;
     int H, W, n_win, topk, R, hr, wr, N, npad;
     int ncb;             // 64-channel blocks in C
+    int cpb;             // 64-channel blocks per CTA
     int rows_per_split;  // image rows of queries per CTA
     int nsplit;
     float scale_log2;
-    int inputs_ready;  // q, k, v may be loaded before the wait for the previous kernel
-    int Hm;            // image rows in memory (H: the region grid's, which may be more)
+    float route_scale;  // ROUTE: C^-1/2
+    int inputs_ready;   // q, k, v may be loaded before the wait for the previous kernel
+    int Hm;             // image rows in memory (H: the region grid's, which may be more)
 };
 
+constexpr int kDensePartPad = 68;  // row stride (floats) of a partial affinity tile
+constexpr int kDenseMaxBlocks = 16;  // 64-channel blocks of an image the fused routing adds (C <= 1024)
+
+// The routing step of one-token regions inside the dense kernel (ROUTE), for a cluster of CTAs
+// that together hold one image's q and k, each CTA `cpb` 64-channel blocks of it:
+//  1. each CTA forms, per block, the 64 x 64 tile of partial dot products q_i . k_s over the
+//     block's channels with the MMA sequence of route_tokens_mma_kernel (two 32-channel chunks
+//     in order, 8 channels per lane), so every partial is the same bits as that kernel's partial
+//     of the block;
+//  2. after a cluster barrier, CTA `ct` takes rows ct, ct + nct, ...: for each (row, region) it
+//     adds the partials of blocks 0, 1, ... in order from the CTAs' shared memory (distributed
+//     shared memory, plain loads), scales by C^-1/2 and forms the routing key; the keys of a row
+//     are distinct, so the position of region s in the row's descending order is the number of
+//     keys above its own, which one thread per (row, region) counts. A region whose position is
+//     below topk is written there in the index, and cnt[row][s] = 1 is set in every CTA of the
+//     cluster (the selected regions of a row are distinct). This is the order the routing
+//     kernel's sort gives, so the index is the same bits;
+//  3. a second cluster barrier publishes cnt, and no CTA touches another's memory after it.
+__device__ __forceinline__ void dense_route_rows(const DenseArgs &a, const float *part, int *cnt,
+                                                 unsigned long long *skey, int b, int ct, int nct)
+{
+    const uint32_t part0 = smem_u32(part);
+    const int nrows = (a.R - ct + nct - 1) / nct;  // rows ct, ct + nct, ... below R
+    const int npairs = nrows * a.R;
+    for (int e = threadIdx.x; e < npairs; e += blockDim.x) {
+        const int rr = e / a.R, s = e - rr * a.R;
+        const int i = ct + nct * rr;
+        // every block's partial in flight at once, then added in block order
+        float pw[kDenseMaxBlocks];
+#pragma unroll
+        for (int w = 0; w < kDenseMaxBlocks; ++w) {
+            const int r = w / a.cpb, j = w - r * a.cpb;
+            pw[w] = w < a.ncb ? ld_cluster_f32(cluster_map(part0 + 4u * (uint32_t)((j * 64 + i) * kDensePartPad + s),
+                                                            (uint32_t)r))
+                              : 0.f;
+        }
+        float d = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDenseMaxBlocks; ++w)
+            if (w < a.ncb) d += pw[w];
+        skey[rr * 64 + s] = routing_key(d * a.route_scale, s);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < npairs; e += blockDim.x) {
+        const int rr = e / a.R, s = e - rr * a.R;
+        const unsigned long long *row = skey + rr * 64;
+        const unsigned long long mine = row[s];
+        int pos = 0;
+#pragma unroll 4
+        for (int j = 0; j < a.R; ++j) pos += row[j] > mine ? 1 : 0;
+        if (pos < a.topk) {
+            const int i = ct + nct * rr;
+            a.idx_out[((int64_t)b * a.R + i) * a.topk + pos] = s;
+            const uint32_t at = smem_u32(cnt + i * a.R + s);
+            for (int r = 0; r < nct; ++r) st_cluster_u32(cluster_map(at, (uint32_t)r), 1u);
+        }
+    }
+}
+
 // MIN_CTAS: CTAs per SM the registers are budgeted for (2, or 3 when three CTAs' shared memory
-// fits on an SM).
-template <int MIN_CTAS>
+// fits on an SM). ROUTE: one-token regions, the kernel selects the index itself (launched as a
+// cluster of the CTAs of one image; above).
+template <int MIN_CTAS, bool ROUTE>
 __global__ void __launch_bounds__(256, MIN_CTAS) attend_dense_mma_kernel(const __grid_constant__ CUtensorMap tq,
                                                                const __grid_constant__ CUtensorMap tk,
                                                                const __grid_constant__ CUtensorMap tv,
@@ -508,11 +623,19 @@ __global__ void __launch_bounds__(256, MIN_CTAS) attend_dense_mma_kernel(const _
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int nq = a.rows_per_split * a.W;  // query rows of this CTA (the last split may run past H)
     const int nqpad = (nq + 15) & ~15;
-    uint8_t *sQ = smem;
-    uint8_t *sK = sQ + (size_t)nqpad * kRowBytes;
-    uint8_t *sV = sK + (size_t)a.npad * kRowBytes;
+    const int cpb = a.cpb;
+    const size_t qtile = (size_t)nqpad * kRowBytes, kvtile = (size_t)a.npad * kRowBytes;
+    uint8_t *sQ = smem;               // [cpb] x [nqpad rows]
+    uint8_t *sK = sQ + cpb * qtile;   // [cpb] x [npad rows]
+    uint8_t *sV = sK + cpb * kvtile;  // [cpb] x [npad rows]
+    const int nct = a.ncb / cpb;  // CTAs per (image, band of rows); ROUTE: the cluster
+    // ROUTE: [cpb][64][kDensePartPad] partial affinities, then the routing keys of this CTA's
+    // rows, [ceil(R / nct)][64]
+    float *part = reinterpret_cast<float *>(sV + cpb * kvtile);
+    unsigned long long *skey =
+        reinterpret_cast<unsigned long long *>(part + (ROUTE ? cpb * 64 * kDensePartPad : 0));
     // [R][R]: the multiplicity of each (query region, key region) pair, then, in place, its log2
-    int *cnt = reinterpret_cast<int *>(sV + (size_t)a.npad * kRowBytes);
+    int *cnt = reinterpret_cast<int *>(skey + (ROUTE ? ((a.R + nct - 1) / nct) * 64 : 0));
     float *lw = reinterpret_cast<float *>(cnt);
     uint8_t *reg = reinterpret_cast<uint8_t *>(cnt + a.R * a.R);  // [npad] region of each key
     uint64_t *bar = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(reg + a.npad) + 7) & ~uintptr_t(7));
@@ -522,10 +645,10 @@ __global__ void __launch_bounds__(256, MIN_CTAS) attend_dense_mma_kernel(const _
     int64_t item = blockIdx.x;
     const int split = (int)(item % a.nsplit);
     item /= a.nsplit;
-    const int cb = (int)(item % a.ncb);
-    const int b = (int)(item / a.ncb);
+    const int ct = (int)(item % nct);
+    const int b = (int)(item / nct);
+    const int cb0 = ct * cpb;
     const int y0 = split * a.rows_per_split;
-    const int32_t *routed = a.idx + (int64_t)b * a.R * a.topk;
 
     if (threadIdx.x == 0) {
         mbar_init(bar, 1);
@@ -536,59 +659,113 @@ __global__ void __launch_bounds__(256, MIN_CTAS) attend_dense_mma_kernel(const _
     // the same forward pass (it already waited for their producers), else after it
     if (!a.inputs_ready) grid_dependency_wait();
     if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(bar, (uint32_t)((nq + 2 * a.N) * kRowBytes));
-        tma_load_4d(sQ, &tq, cb * 64, 0, y0, b, bar);
-        tma_load_4d(sK, &tk, cb * 64, 0, 0, b, bar);
-        tma_load_4d(sV, &tv, cb * 64, 0, 0, b, bar);
+        mbar_arrive_expect_tx(bar, (uint32_t)(cpb * (nq + 2 * a.N) * kRowBytes));
+        for (int j = 0; j < cpb; ++j) {
+            tma_load_4d(sQ + j * qtile, &tq, (cb0 + j) * 64, 0, y0, b, bar);
+            tma_load_4d(sK + j * kvtile, &tk, (cb0 + j) * 64, 0, 0, b, bar);
+            tma_load_4d(sV + j * kvtile, &tv, (cb0 + j) * 64, 0, 0, b, bar);
+        }
     }
     // zero the padding rows (TMA writes rows [0, nq) and [0, N) only)
-    for (int i = threadIdx.x; i < (nqpad - nq) * 8; i += blockDim.x)
-        reinterpret_cast<uint4 *>(sQ + (size_t)nq * kRowBytes)[i] = make_uint4(0, 0, 0, 0);
-    for (int i = threadIdx.x; i < (a.npad - a.N) * 8; i += blockDim.x) {
-        reinterpret_cast<uint4 *>(sK + (size_t)a.N * kRowBytes)[i] = make_uint4(0, 0, 0, 0);
-        reinterpret_cast<uint4 *>(sV + (size_t)a.N * kRowBytes)[i] = make_uint4(0, 0, 0, 0);
+    for (int j = 0; j < cpb; ++j) {
+        for (int i = threadIdx.x; i < (nqpad - nq) * 8; i += blockDim.x)
+            reinterpret_cast<uint4 *>(sQ + j * qtile + (size_t)nq * kRowBytes)[i] = make_uint4(0, 0, 0, 0);
+        for (int i = threadIdx.x; i < (a.npad - a.N) * 8; i += blockDim.x) {
+            reinterpret_cast<uint4 *>(sK + j * kvtile + (size_t)a.N * kRowBytes)[i] = make_uint4(0, 0, 0, 0);
+            reinterpret_cast<uint4 *>(sV + j * kvtile + (size_t)a.N * kRowBytes)[i] = make_uint4(0, 0, 0, 0);
+        }
     }
     for (int t = threadIdx.x; t < a.npad; t += blockDim.x)
         reg[t] = t < a.N ? (uint8_t)(((t / a.W) / a.hr) * a.n_win + (t % a.W) / a.wr) : 0;
     for (int e = threadIdx.x; e < a.R * a.R; e += blockDim.x) cnt[e] = 0;
-    if (a.inputs_ready) grid_dependency_wait();  // idx comes from the previous kernel
-    __syncthreads();
-    // multiplicity of every routed region: the image's idx entries, eight loads per thread in
-    // flight at once, then one shared-memory count per entry
-    const int nent = a.R * a.topk;
-    for (int e0 = threadIdx.x; e0 < nent; e0 += 8 * blockDim.x) {
-        int sv[8];
+    bool alive = true;
+    if constexpr (ROUTE) {
+        // the partial affinities of this CTA's blocks: task = (block j, 16-row tile, key half)
+        __syncthreads();
+        alive = mbar_wait(bar, 0, a.err);
+        const int g = lane >> 2, c = lane & 3;
+        const int rtn = (a.R + 15) >> 4, ntiles = (a.R + 7) >> 3;
+        for (int task = warp; task < cpb * 8; task += nwarps) {
+            const int j = task >> 3, rt = (task >> 1) & 3, half = task & 1;
+            if (rt >= rtn) continue;
+            const uint8_t *qt = sQ + j * qtile, *kt = sK + j * kvtile;
+            float acc[4][4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int e = e0 + u * blockDim.x;
-            sv[u] = e < nent ? routed[e] : 0;
-        }
+            for (int n = 0; n < 4; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int e = e0 + u * blockDim.x;
-            if (e < nent) {
-                const int s = sv[u];
-                if (s >= 0 && s < a.R)
-                    atomicAdd(&cnt[(e / a.topk) * a.R + s], 1);
-                else if (cb == 0 && split == 0)
-                    flag_error(a.err, kErrIndex);
+            for (int ch = 0; ch < 2; ++ch) {
+                const uint4 xa = *reinterpret_cast<const uint4 *>(qt + sw128(16 * rt + g, 4 * ch + c));
+                const uint4 xb = *reinterpret_cast<const uint4 *>(qt + sw128(16 * rt + g + 8, 4 * ch + c));
+                const uint32_t a0[4] = {xa.x, xb.x, xa.y, xb.y};
+                const uint32_t a1[4] = {xa.z, xb.z, xa.w, xb.w};
+#pragma unroll
+                for (int n = 0; n < 4; ++n) {
+                    const int nt = 4 * half + n;
+                    if (nt < ntiles) {
+                        const uint4 y = *reinterpret_cast<const uint4 *>(kt + sw128(8 * nt + g, 4 * ch + c));
+                        mma_bf16_16816(acc[n], a0, y.x, y.y);
+                        mma_bf16_16816(acc[n], a1, y.z, y.w);
+                    }
+                }
+            }
+            float *pj = part + (size_t)j * 64 * kDensePartPad;
+#pragma unroll
+            for (int n = 0; n < 4; ++n) {
+                const int nt = 4 * half + n;
+                if (nt < ntiles) {
+                    *reinterpret_cast<float2 *>(pj + (16 * rt + g) * kDensePartPad + 8 * nt + 2 * c) =
+                        make_float2(acc[n][0], acc[n][1]);
+                    *reinterpret_cast<float2 *>(pj + (16 * rt + g + 8) * kDensePartPad + 8 * nt + 2 * c) =
+                        make_float2(acc[n][2], acc[n][3]);
+                }
             }
         }
+        cluster_sync();  // every CTA's partials and zeroed cnt, before any remote access
+        dense_route_rows(a, part, cnt, skey, b, ct, nct);
+        cluster_sync();  // cnt complete in every CTA; no remote access after this point
+    } else {
+        if (a.inputs_ready) grid_dependency_wait();  // idx comes from the previous kernel
+        __syncthreads();
+        // multiplicity of every routed region: the image's idx entries, eight loads per thread in
+        // flight at once, then one shared-memory count per entry
+        const int32_t *routed = a.idx + (int64_t)b * a.R * a.topk;
+        const int nent = a.R * a.topk;
+        for (int e0 = threadIdx.x; e0 < nent; e0 += 8 * blockDim.x) {
+            int sv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = e0 + u * blockDim.x;
+                sv[u] = e < nent ? routed[e] : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = e0 + u * blockDim.x;
+                if (e < nent) {
+                    const int s = sv[u];
+                    if (s >= 0 && s < a.R)
+                        atomicAdd(&cnt[(e / a.topk) * a.R + s], 1);
+                    else if (ct == 0 && split == 0)
+                        flag_error(a.err, kErrIndex);
+                }
+            }
+        }
+        __syncthreads();
     }
-    __syncthreads();
     for (int e = threadIdx.x; e < a.R * a.R; e += blockDim.x) {
         const int c = cnt[e];
         lw[e] = c == 1 ? 0.f : (c ? log2f((float)c) : -INFINITY);  // log2(1) = 0 exactly: skip the call
     }
     __syncthreads();
 
-    const bool alive = mbar_wait(bar, 0, a.err);
+    if constexpr (!ROUTE) alive = mbar_wait(bar, 0, a.err);
     const int g = lane >> 2, t = lane & 3;
-    const uint32_t qbase = smem_u32(sQ), kbase = smem_u32(sK), vbase = smem_u32(sV);
-    const int tasks = (nqpad / 16) * 2;
+    const int tasks = (nqpad / 16) * 2 * cpb;  // (16-row tile, block, head of the block)
 
     for (int task = warp; alive && task < tasks; task += nwarps) {
-        const int rt = task >> 1, hb = task & 1;
+        const int rt = task / (2 * cpb), rem = task - rt * 2 * cpb;
+        const int j = rem >> 1, hb = rem & 1;
+        const uint32_t qbase = smem_u32(sQ + j * qtile), kbase = smem_u32(sK + j * kvtile);
+        const uint32_t vbase = smem_u32(sV + j * kvtile);
         uint32_t qf[2][4];
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks)
@@ -659,7 +836,7 @@ __global__ void __launch_bounds__(256, MIN_CTAS) attend_dense_mma_kernel(const _
     fence_async_shared();
     __syncthreads();
     if (threadIdx.x == 0 && alive && y0 < a.Hm) {  // a band wholly below a padded image stores nothing
-        tma_store_4d(&tout, sQ, cb * 64, 0, y0, b);
+        for (int j = 0; j < cpb; ++j) tma_store_4d(&tout, sQ + j * qtile, (cb0 + j) * 64, 0, y0, b);
         tma_store_commit();
         tma_store_wait_read();
     }
@@ -679,21 +856,22 @@ int dense_mma_rows_per_split(const Geometry &g, int num_sms)
     return (g.H + nsplit - 1) / nsplit;
 }
 
-static size_t dense_smem_bytes(const Geometry &g, int rows_per_split)
+static size_t dense_smem_bytes(const Geometry &g, int rows_per_split, int cpb = 1, bool route = false)
 {
     const int nq = rows_per_split * g.W, nqpad = (nq + 15) & ~15;
     const int npad = (g.N + 15) & ~15;
-    return 1024 + (size_t)(nqpad + 2 * npad) * kRowBytes + (size_t)g.R * g.R * 4 + npad + 16;
+    const int nct = g.C / 64 / cpb;
+    const size_t routing = route ? (size_t)cpb * 64 * kDensePartPad * 4 + (size_t)((g.R + nct - 1) / nct) * 64 * 8 : 0;
+    return 1024 + (size_t)cpb * (nqpad + 2 * npad) * kRowBytes + routing + (size_t)g.R * g.R * 4 + npad + 16;
 }
 
-cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                    const CUtensorMap &tout, const int32_t *idx, const Geometry &g, int rows_per_split,
-                                    unsigned *err, bool inputs_ready, int Hm, cudaStream_t stream)
+static void fill_dense_args(DenseArgs &a, const int32_t *idx, const Geometry &g, int rows_per_split, unsigned *err,
+                            bool inputs_ready, int Hm)
 {
-    DenseArgs a;
     a.inputs_ready = inputs_ready ? 1 : 0;
     a.Hm = Hm;
     a.idx = idx;
+    a.idx_out = nullptr;
     a.err = err;
     a.H = g.H;
     a.W = g.W;
@@ -705,24 +883,87 @@ cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk
     a.N = g.N;
     a.npad = (g.N + 15) & ~15;
     a.ncb = g.C / 64;
+    a.cpb = 1;
     a.rows_per_split = rows_per_split;
     a.nsplit = (g.H + rows_per_split - 1) / rows_per_split;
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)g.hd));
+    a.route_scale = (float)(1.0 / sqrt((double)g.C));
+}
+
+cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                    const CUtensorMap &tout, const int32_t *idx, const Geometry &g, int rows_per_split,
+                                    unsigned *err, bool inputs_ready, int Hm, cudaStream_t stream)
+{
+    DenseArgs a;
+    fill_dense_args(a, idx, g, rows_per_split, err, inputs_ready, Hm);
     const size_t smem = dense_smem_bytes(g, rows_per_split);
     const long long blocks = (long long)g.B * a.ncb * a.nsplit;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     // three CTAs per SM when their shared memory fits (227 KB per SM, 1 KB reserved per CTA)
     if (3 * (smem + 1024) <= 227 * 1024) {
         static int granted3[64] = {0};
-        cudaError_t e = ensure_smem_limit(attend_dense_mma_kernel<3>, smem, granted3);
+        cudaError_t e = ensure_smem_limit(attend_dense_mma_kernel<3, false>, smem, granted3);
         if (e != cudaSuccess) return e;
-        return launch_pdl(attend_dense_mma_kernel<3>, dim3((unsigned)blocks), dim3(256), smem, stream, tq, tk, tv, tout,
-                          a);
+        return launch_pdl(attend_dense_mma_kernel<3, false>, dim3((unsigned)blocks), dim3(256), smem, stream, tq, tk,
+                          tv, tout, a);
     }
     static int granted[64] = {0};
-    cudaError_t e = ensure_smem_limit(attend_dense_mma_kernel<2>, smem, granted);
+    cudaError_t e = ensure_smem_limit(attend_dense_mma_kernel<2, false>, smem, granted);
     if (e != cudaSuccess) return e;
-    return launch_pdl(attend_dense_mma_kernel<2>, dim3((unsigned)blocks), dim3(256), smem, stream, tq, tk, tv, tout, a);
+    return launch_pdl(attend_dense_mma_kernel<2, false>, dim3((unsigned)blocks), dim3(256), smem, stream, tq, tk, tv,
+                      tout, a);
+}
+
+// 64-channel blocks per CTA of the fused kernel: two when the channel blocks pair up and two
+// CTAs of that size fit on an SM, so that half as many CTAs (and clusters half as wide) carry
+// the image; else one.
+static int route_dense_cpb(const Geometry &g)
+{
+    const int ncb = g.C / 64;
+    if (ncb % 2 == 0 && ncb / 2 <= kRouteDenseMaxCluster && 2 * (dense_smem_bytes(g, g.H, 2, true) + 1024) <= 227 * 1024)
+        return 2;
+    return 1;
+}
+
+bool route_dense_supports(const Geometry &g, bool bf16)
+{
+    if (!bf16 || !dense_mma_supports(g) || g.rs != 1 || g.R > 64 || !route_tokens_mma_supports(g, bf16)) return false;
+    const int cpb = route_dense_cpb(g);
+    return g.C / 64 <= kDenseMaxBlocks && g.C / 64 / cpb <= kRouteDenseMaxCluster &&
+           dense_smem_bytes(g, g.H, cpb, true) <= 227 * 1024;
+}
+
+cudaError_t launch_route_attend_dense(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                      const CUtensorMap &tout, int32_t *idx, const Geometry &g, unsigned *err,
+                                      cudaStream_t stream)
+{
+    if (!route_dense_supports(g, true)) return cudaErrorInvalidConfiguration;
+    DenseArgs a;
+    fill_dense_args(a, nullptr, g, g.H, err, false, g.H);
+    a.idx_out = idx;
+    a.cpb = route_dense_cpb(g);
+    const int nct = a.ncb / a.cpb;
+    const size_t smem = dense_smem_bytes(g, g.H, a.cpb, true);
+    const long long blocks = (long long)g.B * nct;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    static int granted[64] = {0};
+    cudaError_t e = ensure_smem_limit(attend_dense_mma_kernel<2, true>, smem, granted);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)nct;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, attend_dense_mma_kernel<2, true>, tq, tk, tv, tout, a);
 }
 
 }  // namespace bra

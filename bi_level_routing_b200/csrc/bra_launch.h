@@ -75,6 +75,8 @@ inline bool topk_by_rounds(int E, int topk)
 // the means are the tokens, widened exactly to fp32, so the index is the same as from the means.
 cudaError_t launch_route_topk_tokens(const void *q, const void *k, int32_t *idx, const Geometry &g, bool bf16,
                                      cudaStream_t stream);
+// The shapes the bf16 tensor-core kernel of that step serves (rs == 1, R <= 64, C % 32 == 0).
+bool route_tokens_mma_supports(const Geometry &g, bool bf16);
 
 // Affinity rows and top-k: idx[b, r, :] from qm, km.
 cudaError_t launch_route_topk(const float *qm, const float *km, int32_t *idx, const Geometry &g,
@@ -152,7 +154,8 @@ cudaError_t launch_attend_region_mma(const CUtensorMap &tq, const CUtensorMap &t
 void gather_mma_box(const Geometry &g, int box[5]);
 cudaError_t launch_attend_gather_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                      const CUtensorMap &tout, const int32_t *idx, void *out, const Geometry &g, int H,
-                                     int W, int num_sms, unsigned *err, cudaStream_t stream);
+                                     int W, int num_sms, unsigned *err, cudaStream_t stream,
+                                     bool per_head = false);
 
 // tcgen05 gather attention for 64-token regions (bf16, hd == 32, C % 64 == 0). Maps: q, k, v
 // with box (64, wr, hr, 1).
@@ -167,5 +170,16 @@ cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk
                                     const CUtensorMap &tout, const int32_t *idx, const Geometry &g,
                                     int rows_per_split, unsigned *err, bool inputs_ready, int Hm,
                                     cudaStream_t stream);
+
+// The forward pass of one-token regions (bf16, R <= 64) in one kernel: the dense kernel with the
+// routing step inside, launched as one thread-block cluster per image (at most
+// kRouteDenseMaxCluster CTAs, one or two 64-channel blocks each). It writes idx [B, R, topk]
+// with the same bits as the routing kernel of these shapes and out as the dense kernel does.
+// Maps: q and out with box (64, W, H, 1), k and v likewise.
+constexpr int kRouteDenseMaxCluster = 8;
+bool route_dense_supports(const Geometry &g, bool bf16);
+cudaError_t launch_route_attend_dense(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                      const CUtensorMap &tout, int32_t *idx, const Geometry &g, unsigned *err,
+                                      cudaStream_t stream);
 
 }  // namespace bra

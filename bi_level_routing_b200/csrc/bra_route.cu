@@ -562,8 +562,11 @@ static cudaError_t launch_topk_any(const S *qm, const S *km, int32_t *idx, const
 // routing kernel does.
 //  * bf16 one-token regions (route_tokens_mma_kernel): the means are the tokens, and a product
 //    of two bf16 values is exact in fp32, so m16n8k16 bf16 MMAs with fp32 accumulation add the
-//    same exact products an fp32 FMA path would, in another order (32-channel chunks, 8
-//    channels per lane).
+//    same exact products an fp32 FMA path would, in another order (8 channels per lane). Here
+//    warp w takes the 64-channel blocks w, w + 8, ..., each as its two 32-channel chunks in
+//    order: with C <= 512 a warp's partial is exactly one block's, which is how the fused
+//    route-and-attend kernel of the forward pass (one CTA per block) forms the same partials
+//    and adds them in the same order, so both give the same index bits.
 //  * fp32 means or tokens (route_tf32x3_kernel): each value is split into two tf32 parts,
 //    x = hi + lo with |x - hi - lo| <= 2^-22 |x|, and m16n8k8 tf32 MMAs add lo*hi, hi*lo and
 //    hi*hi (smallest first; lo*lo, below 2^-22 of the product, is left out). Every product is
@@ -632,7 +635,7 @@ __global__ void __launch_bounds__(256, 2) route_tokens_mma_kernel(const __nv_bfl
     for (int n = 0; n < 8; ++n)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[n][j] = 0.f;
-    for (int col = 32 * warp; col < C; col += 32 * kRouteWarps) {
+    for (int col = 64 * warp; col < C; col += (col & 32) ? 64 * kRouteWarps - 32 : 32) {
         const uint4 xa = __ldg(reinterpret_cast<const uint4 *>(qb + ra + col));
         const uint4 xb = __ldg(reinterpret_cast<const uint4 *>(qb + rb + col));
         uint4 y[8];

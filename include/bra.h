@@ -104,7 +104,10 @@ bra_status bra_route(const void *q, const void *k, int32_t *idx, int B, int H, i
 bra_status bra_attend(const void *q, const void *k, const void *v, const int32_t *idx, void *out, int B,
                       int H, int W, int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream);
 
-/* Steps 1-5: bra_route then bra_attend on the same stream. idx is written (and then read). */
+/* Steps 1-5: bra_route then bra_attend on the same stream. idx is written (and then read).
+   Where every region is one token (H = W = n_win), bf16, R <= 64 and the attention kernel in
+   use is BRA_ATTEND_DENSE_MMA, both steps run in one kernel (one thread-block cluster per
+   image); idx and out are then the same bits as from bra_route and bra_attend. */
 bra_status bra_forward(const void *q, const void *k, const void *v, int32_t *idx, void *out, int B, int H,
                        int W, int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream);
 
@@ -137,8 +140,12 @@ bra_status bra_route_heads(const void *q, const void *k, int32_t *idx, int B, in
 /* Step 5 with per-head routing ("医学图像分割模块", §五 steps ⑤-⑦): head h of a query in region r
    attends over the tokens of regions idx[b, h, r, 0..topk-1]. idx: device int32
    [B, heads, n_win^2, topk] (out-of-range entries skipped and flagged, duplicates gathered as
-   often as they occur); other arguments as bra_attend. Runs on CUDA cores with the routed rows
-   staged in shared memory. BRA_ERR_UNSUPPORTED: hd > 128. */
+   often as they occur); other arguments as bra_attend. bf16 with hd == 32, C % 64 == 0 and
+   regions of 16, 32, 48 or 64 tokens runs on the tensor cores (BRA_ATTEND_GATHER_MMA, each head
+   gathering the tiles of its own regions), everything else on CUDA cores with the routed rows
+   staged in shared memory (BRA_ATTEND_SIMT); bra_set_attend_kernel may force either one, and
+   forcing any other kernel makes the call BRA_ERR_UNSUPPORTED. BRA_ERR_UNSUPPORTED: hd > 128
+   on CUDA cores. */
 bra_status bra_attend_heads(const void *q, const void *k, const void *v, const int32_t *idx, void *out, int B,
                             int H, int W, int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream);
 
@@ -155,9 +162,10 @@ bra_status bra_forward_heads(const void *q, const void *k, const void *v, int32_
    over the region divided by (Hp / n_win) (Wp / n_win)) and take part in the attention as keys
    with logit 0 and value 0; out holds the H x W queries only. q, k, v, out: device
    [B, H, W, C]; idx: device int32 [B, n_win^2, topk], written (routing of the padded map). When
-   H and W are multiples of n_win this is bra_forward. Attention runs on CUDA cores
-   (BRA_ERR_UNSUPPORTED: hd > 128); the means use out as scratch when they fit in it, else the
-   pool. */
+   H and W are multiples of n_win this is bra_forward. Attention runs on the kernel bra_attend
+   would use for the padded shape, reading the padded map through tensor maps of the true image
+   (or, on CUDA cores, with guarded loads); the means use out as scratch when they fit in it,
+   else the pool. */
 bra_status bra_forward_auto_pad(const void *q, const void *k, const void *v, int32_t *idx, void *out, int B, int H,
                                 int W, int C, int heads, int n_win, int topk, bra_dtype dtype, void *stream);
 

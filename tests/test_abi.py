@@ -130,7 +130,15 @@ def test_scratch_and_launch_accounting(L):
     assert L.bra_kernels_per_call(b"bra_forward", 1, 30, 28, 64, 2, 7, 4, 1) == 0  # rejected
     stage4 = (64, 7, 7, 512, 16, 7, 49, 1)  # one-token regions: routing reads q and k directly
     assert L.bra_kernels_per_call(b"bra_route", *stage4) == 1
-    assert L.bra_kernels_per_call(b"bra_forward", *stage4) == 2
+    assert L.bra_kernels_per_call(b"bra_forward", *stage4) == 1  # routing inside the dense kernel
+    assert L.bra_kernels_per_call(b"bra_forward_host", *stage4) == 1
+    f32_stage4 = stage4[:-1] + (0,)  # fp32: the CUDA-core kernels, routing then attention
+    assert L.bra_kernels_per_call(b"bra_forward", *f32_stage4) == 2
+    try:  # with another attention kernel forced, the forward pass is routing then attention
+        L.bra_set_attend_kernel(1)
+        assert L.bra_kernels_per_call(b"bra_forward", *stage4) == 2
+    finally:
+        L.bra_set_attend_kernel(0)
     assert L.bra_route_scratch_bytes(64, 7, 7, 512, 7) == 0
     assert L.bra_kernels_per_call(b"nonsense", *stage1) == 0
 

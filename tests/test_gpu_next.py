@@ -40,6 +40,37 @@ def test_forward_heads(w):
     assert torch.equal(idx2, idx) and torch.equal(out2, out)
 
 
+# shapes the tensor-core gather kernel takes in its per-head mode (bf16, hd 32, rs % 16 == 0):
+# one and two 64-channel blocks per item, a last item group with a block past C, 48-token regions
+HEADS_GATHER = [WORKLOADS["stage1"].with_(B=6), WORKLOADS["stage2"].with_(B=6),
+                WORKLOADS["highres"].with_(B=1),
+                _w("rs32_c192", 3, 16, 32, 192, 6, 4, 5, "bf16"), _w("rs48_c64", 2, 24, 32, 64, 2, 4, 3, "bf16")]
+
+
+@pytest.mark.parametrize("w", HEADS_GATHER, ids=[w.name for w in HEADS_GATHER])
+def test_heads_both_kernels(w):
+    """Per-head attention on the tensor cores and on CUDA cores: each against the oracle over the
+    same per-head index; any other forced kernel refuses per-head indices."""
+    inp, (q, k, v) = make(w)
+    idx = bra.route_heads(q, k, w.n_win, w.topk, w.heads)
+    torch.cuda.synchronize()
+    ref = oracle.attend_heads(inp["q"], inp["k"], inp["v"], idx.cpu().numpy(), w.n_win)
+    try:
+        for kname in ("gather_mma", "simt"):
+            bra.set_attend_kernel(kname)
+            out = bra.attend_heads(q, k, v, idx, w.n_win)
+            out2, idx2 = bra.forward_heads(q, k, v, w.n_win, w.topk, w.heads)
+            torch.cuda.synchronize()
+            assert bra.check_device_error() == 0
+            assert torch.equal(idx2, idx) and torch.equal(out2, out), kname
+            check_output(host_values(out), ref, w.dtype, f"{w.name} per-head / {kname}")
+        bra.set_attend_kernel("dense_mma")
+        with pytest.raises(RuntimeError):
+            bra.attend_heads(q, k, v, idx, w.n_win)
+    finally:
+        bra.set_attend_kernel("auto")
+
+
 def test_heads_topk_clamp_and_one_head():
     w = _w("clamp", 2, 16, 16, 64, 2, 4, 20, "bf16")  # topk 20 > R = 16: clamped to 16
     inp, (q, k, v) = make(w)
