@@ -263,6 +263,273 @@ __global__ void __launch_bounds__(256) attend_backward_kernel(const BackArgs a)
     }
 }
 
+// ------------------------------------------------------------------ 64-token regions, hd = 32
+//
+// A register-tiled variant for regions of 64 tokens and heads of 32 channels (the shape of the
+// stage-1 and high-resolution workloads): one CTA of 256 threads per (image, query region,
+// head); the keys arrive one routed region (64 keys) at a time. The same sums as above, as five
+// 64 x 64 x 32 products on CUDA cores in fp32, each with a thread mapping whose shared-memory
+// reads are broadcasts or conflict-free:
+//   S, dP  : warp w owns query rows 8w .. 8w+7, lane l keys l and l + 32; q and dout are read
+//            transposed (one 16-byte broadcast per 4 rows), k and v transposed (consecutive
+//            keys across the lanes). A row's 64 keys sit in one warp, so its max and sums are
+//            warp reductions.
+//   dQ     : lane l owns rows l and l + 32, warp w channels 4w .. 4w+3: ds transposed (padded
+//            rows) and k by rows (a 16-byte broadcast); dq accumulates in registers over all the
+//            routed regions and is stored once.
+//   dK, dV : lane l owns channels 4 (l % 8) .. + 3 of keys 8w + l / 8 and that + 4: ds and p by
+//            rows, q and dout by rows (16-byte loads); the sums over the region's queries go to
+//            dk and dv with one 16-byte atomic per key and tensor.
+// With one routed region the scores stay in registers between the statistics and the
+// gradients; with more, pass 1 gathers the statistics and pass 2 recomputes them per region.
+namespace {
+
+constexpr int kTiledThreads = 256;
+
+// floats of each shared-memory array of the tiled kernel
+constexpr int kT64 = 64 * 32;        // a 64 x 32 tile
+constexpr int kTPS = 64 * 64;        // a 64 x 64 tile
+constexpr int kTdSt = 64 * 65;       // transposed ds, rows padded to 65
+constexpr size_t kTiledSmem = sizeof(float) * (7 * kT64 + 2 * kTPS + kTdSt) + 16 * sizeof(int);
+
+// Loads one 64-token x 32-channel head tile (rows of the region at (y0, x0), channel offset
+// c0) as fp32: into `tr` transposed ([32][64]) and, when `nat` is set, by rows ([64][32]).
+template <typename T>
+__device__ __forceinline__ void stage_head_tile(const T *g, const BackArgs &a, int64_t b, int y0, int x0, int c0,
+                                                float *tr, float *nat)
+{
+    constexpr int V = Vec16<T>::N;  // channels per 16-byte vector
+    constexpr int NV = 32 / V;      // vectors per row
+    for (int e = threadIdx.x; e < 64 * NV; e += kTiledThreads) {
+        const int row = e & 63, u = e >> 6;  // consecutive lanes: consecutive rows
+        const int y = y0 + row / a.wr, x = x0 + row % a.wr;
+        float f[V];
+        Vec16<T>::load(g + ((b * a.H + y) * a.W + x) * a.C + c0 + u * V, f);
+#pragma unroll
+        for (int i = 0; i < V; ++i) tr[(u * V + i) * 64 + row] = f[i];
+        if (nat) {
+            float4 *d = reinterpret_cast<float4 *>(nat + row * 32 + u * V);
+#pragma unroll
+            for (int i = 0; i < V / 4; ++i) d[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+        }
+    }
+}
+
+__device__ __forceinline__ float warp_max(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+
+__device__ __forceinline__ float warp_sum(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+}  // namespace
+
+template <typename T>
+__global__ void __launch_bounds__(kTiledThreads, 2) attend_backward_tiled_kernel(const BackArgs a)
+{
+    extern __shared__ float4 smem4[];
+    float *Qt = reinterpret_cast<float *>(smem4);  // [32][64] q transposed
+    float *Qn = Qt + kT64;                         // [64][32] q
+    float *Dt = Qn + kT64;                         // [32][64] dout transposed
+    float *Dn = Dt + kT64;                         // [64][32] dout
+    float *Kt = Dn + kT64;                         // [32][64] k of the routed region, transposed
+    float *Kn = Kt + kT64;                         // [64][32] k
+    float *Vt = Kn + kT64;                         // [32][64] v transposed
+    float *Ps = Vt + kT64;                         // [64 queries][64 keys] p
+    float *Ss = Ps + kTPS;                         // [64 queries][64 keys] ds
+    float *St = Ss + kTPS;                         // [64 keys][65] ds transposed
+    int *sreg = reinterpret_cast<int *>(St + kTdSt);  // routed regions (topk <= 16 staged here)
+
+    int64_t blk = blockIdx.x;
+    const int h = (int)(blk % a.heads);
+    blk /= a.heads;
+    const int r = (int)(blk % a.R);
+    const int64_t b = blk / a.R;
+    const int ry = r / a.n_win, rx = r - ry * a.n_win;
+    const int c0 = h * 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const T *gq = static_cast<const T *>(a.q), *gk = static_cast<const T *>(a.k);
+    const T *gv = static_cast<const T *>(a.v), *gd = static_cast<const T *>(a.dout);
+    grid_dependency_wait();
+
+    stage_head_tile(gq, a, b, ry * a.hr, rx * a.wr, c0, Qt, Qn);
+    stage_head_tile(gd, a, b, ry * a.hr, rx * a.wr, c0, Dt, Dn);
+    auto region = [&](int j) -> int {
+        const int s = j < 16 ? sreg[j] : a.idx[(b * a.R + r) * a.topk + j];
+        return (s >= 0 && s < a.R) ? s : -1;
+    };
+    if (threadIdx.x < 16 && threadIdx.x < a.topk) {
+        const int s = a.idx[(b * a.R + r) * a.topk + threadIdx.x];
+        sreg[threadIdx.x] = s;
+    }
+    if (h == 0 && threadIdx.x == 0)
+        for (int j = 0; j < a.topk; ++j) {
+            const int s = a.idx[(b * a.R + r) * a.topk + j];
+            if (s < 0 || s >= a.R) flag_error(a.err, kErrIndex);
+        }
+    __syncthreads();
+
+    // S and dP of this thread's 8 rows x 2 keys against the staged region
+    float sc[8][2], dp[8][2];
+    auto scores = [&]() {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sc[i][0] = sc[i][1] = dp[i][0] = dp[i][1] = 0.f;
+#pragma unroll 4
+        for (int c = 0; c < 32; ++c) {
+            const float4 qa = *reinterpret_cast<const float4 *>(Qt + c * 64 + 8 * warp);
+            const float4 qb = *reinterpret_cast<const float4 *>(Qt + c * 64 + 8 * warp + 4);
+            const float4 da = *reinterpret_cast<const float4 *>(Dt + c * 64 + 8 * warp);
+            const float4 db = *reinterpret_cast<const float4 *>(Dt + c * 64 + 8 * warp + 4);
+            const float k0 = Kt[c * 64 + lane], k1 = Kt[c * 64 + lane + 32];
+            const float v0 = Vt[c * 64 + lane], v1 = Vt[c * 64 + lane + 32];
+            const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+            const float dv[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                sc[i][0] = fmaf(qv[i], k0, sc[i][0]);
+                sc[i][1] = fmaf(qv[i], k1, sc[i][1]);
+                dp[i][0] = fmaf(dv[i], v0, dp[i][0]);
+                dp[i][1] = fmaf(dv[i], v1, dp[i][1]);
+            }
+        }
+    };
+    auto stage_kv = [&](int s) {
+        const int sy = (s / a.n_win) * a.hr, sx = (s % a.n_win) * a.wr;
+        stage_head_tile(gk, a, b, sy, sx, c0, Kt, Kn);
+        stage_head_tile(gv, a, b, sy, sx, c0, Vt, static_cast<float *>(nullptr));
+    };
+
+    // pass 1: running max, sum and sum_i e_i (dout . v_i) of each of the warp's rows
+    float m[8], l[8], dsum[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        m[i] = -INFINITY;
+        l[i] = 0.f;
+        dsum[i] = 0.f;
+    }
+    int staged = -1;  // routed slot whose k and v are in shared memory
+    for (int j = 0; j < a.topk; ++j) {
+        const int s = region(j);
+        if (s < 0) continue;
+        __syncthreads();
+        stage_kv(s);
+        staged = j;
+        __syncthreads();
+        scores();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float s0 = sc[i][0] * a.scale_log2, s1 = sc[i][1] * a.scale_log2;
+            const float mn = fmaxf(m[i], warp_max(fmaxf(s0, s1)));
+            const float corr = fast_exp2(m[i] - mn);
+            const float e0 = fast_exp2(s0 - mn), e1 = fast_exp2(s1 - mn);
+            l[i] = l[i] * corr + warp_sum(e0 + e1);
+            dsum[i] = dsum[i] * corr + warp_sum(fmaf(e0, dp[i][0], e1 * dp[i][1]));
+            m[i] = mn;
+        }
+    }
+    float inv_l[8], D[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        inv_l[i] = l[i] > 0.f ? 1.f / l[i] : 0.f;
+        D[i] = dsum[i] * inv_l[i];
+    }
+
+    // pass 2: p and ds per routed region; dq in registers, dk and dv added per region
+    float dq[2][4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) dq[i][0] = dq[i][1] = dq[i][2] = dq[i][3] = 0.f;
+    const int c4 = lane & 7, kk = 8 * warp + (lane >> 3);  // dK / dV: keys kk, kk + 4; channels 4 c4..
+    for (int j = 0; j < a.topk; ++j) {
+        const int s = region(j);
+        if (s < 0) continue;
+        if (staged != j) {  // the last region of pass 1 is still staged, its scores in registers
+            __syncthreads();
+            stage_kv(s);
+            __syncthreads();
+            scores();
+        }
+        staged = -1;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int row = 8 * warp + i;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int key = lane + 32 * t;
+                const float p = fast_exp2(fmaf(sc[i][t], a.scale_log2, -m[i])) * inv_l[i];
+                const float ds = p * (dp[i][t] - D[i]);
+                Ps[row * 64 + key] = p;
+                Ss[row * 64 + key] = ds;
+                St[key * 65 + row] = ds;
+            }
+        }
+        __syncthreads();
+        // dq rows lane, lane + 32, channels 4 warp ..: sum over the region's 64 keys
+#pragma unroll 4
+        for (int key = 0; key < 64; ++key) {
+            const float4 kr = *reinterpret_cast<const float4 *>(Kn + key * 32 + 4 * warp);
+            const float d0 = St[key * 65 + lane], d1 = St[key * 65 + lane + 32];
+            dq[0][0] = fmaf(d0, kr.x, dq[0][0]);
+            dq[0][1] = fmaf(d0, kr.y, dq[0][1]);
+            dq[0][2] = fmaf(d0, kr.z, dq[0][2]);
+            dq[0][3] = fmaf(d0, kr.w, dq[0][3]);
+            dq[1][0] = fmaf(d1, kr.x, dq[1][0]);
+            dq[1][1] = fmaf(d1, kr.y, dq[1][1]);
+            dq[1][2] = fmaf(d1, kr.z, dq[1][2]);
+            dq[1][3] = fmaf(d1, kr.w, dq[1][3]);
+        }
+        // dk, dv of keys kk and kk + 4, channels 4 c4 ..: sums over the region's 64 queries
+        float4 gk4[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+        float4 gv4[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+#pragma unroll 4
+        for (int row = 0; row < 64; ++row) {
+            const float4 qr = *reinterpret_cast<const float4 *>(Qn + row * 32 + 4 * c4);
+            const float4 dr = *reinterpret_cast<const float4 *>(Dn + row * 32 + 4 * c4);
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const float ds = Ss[row * 64 + kk + 4 * t], p = Ps[row * 64 + kk + 4 * t];
+                gk4[t].x = fmaf(ds, qr.x, gk4[t].x);
+                gk4[t].y = fmaf(ds, qr.y, gk4[t].y);
+                gk4[t].z = fmaf(ds, qr.z, gk4[t].z);
+                gk4[t].w = fmaf(ds, qr.w, gk4[t].w);
+                gv4[t].x = fmaf(p, dr.x, gv4[t].x);
+                gv4[t].y = fmaf(p, dr.y, gv4[t].y);
+                gv4[t].z = fmaf(p, dr.z, gv4[t].z);
+                gv4[t].w = fmaf(p, dr.w, gv4[t].w);
+            }
+        }
+        const int sy = (s / a.n_win) * a.hr, sx = (s % a.n_win) * a.wr;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            const int key = kk + 4 * t;
+            const int y = sy + key / a.wr, x = sx + key % a.wr;
+            const int64_t off = ((b * a.H + y) * a.W + x) * a.C + c0 + 4 * c4;
+            gk4[t].x *= a.scale;
+            gk4[t].y *= a.scale;
+            gk4[t].z *= a.scale;
+            gk4[t].w *= a.scale;
+            atomicAdd(reinterpret_cast<float4 *>(a.dk + off), gk4[t]);
+            atomicAdd(reinterpret_cast<float4 *>(a.dv + off), gv4[t]);
+        }
+        __syncthreads();  // p and ds are rewritten by the next region
+    }
+    const int y0 = ry * a.hr, x0 = rx * a.wr;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int row = lane + 32 * i;
+        const int y = y0 + row / a.wr, x = x0 + row % a.wr;
+        float *dst = a.dq + ((b * a.H + y) * a.W + x) * a.C + c0 + 4 * warp;
+        *reinterpret_cast<float4 *>(dst) =
+            make_float4(dq[i][0] * a.scale, dq[i][1] * a.scale, dq[i][2] * a.scale, dq[i][3] * a.scale);
+    }
+}
+
 namespace {
 
 constexpr size_t kBackMaxSmem = 100 * 1024;
@@ -310,6 +577,28 @@ cudaError_t launch_attend_backward(const void *q, const void *k, const void *v, 
     a.topk = g.topk;
     a.scale = (float)(1.0 / sqrt((double)g.hd));
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)g.hd));
+    if (g.rs == 64 && g.hd == 32) {
+        // 64-token regions, heads of 32 channels: the register-tiled kernel
+        const long long blocks = (long long)g.B * g.R * g.heads;
+        if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+        const size_t bytes = (size_t)g.B * g.H * g.W * g.C * sizeof(float);
+        cudaError_t e = cudaMemsetAsync(dk, 0, bytes, stream);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, bytes, stream);
+        if (e != cudaSuccess) return e;
+        void (*kernel)(const BackArgs) =
+            bf16 ? attend_backward_tiled_kernel<__nv_bfloat16> : attend_backward_tiled_kernel<float>;
+        static int granted_tiled[2][64] = {{0}};
+        int dev = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+        if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+        if ((int)kTiledSmem > granted_tiled[bf16][dev]) {
+            if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTiledSmem)) !=
+                cudaSuccess)
+                return e;
+            granted_tiled[bf16][dev] = (int)kTiledSmem;
+        }
+        return launch_pdl(kernel, dim3((unsigned)blocks), dim3(kTiledThreads), kTiledSmem, stream, a);
+    }
     // heads per CTA: the largest divisor of heads with hpc * rs <= 256 threads whose smem holds at
     // least one routed region per chunk; then as many regions per chunk as fit
     int hpc = 1;

@@ -174,6 +174,27 @@ def test_backward_duplicates():
         check_grad(g.cpu().numpy(), r, f"duplicates {n}")
 
 
+def test_backward_tiled_many_regions_and_bad_entries():
+    """The register-tiled kernel of 64-token regions: 18 routed regions (past the 16 it keeps in
+    shared memory), duplicates, then one out-of-range entry that is skipped and flagged."""
+    w = _w("rs64_r25", 2, 40, 40, 64, 2, 5, 18, "bf16", "iid", 21)
+    inp, (q, k, v) = make(w)
+    rng = np.random.Generator(np.random.PCG64(17))
+    idx = rng.integers(0, w.R, size=(w.B, w.R, w.topk)).astype(np.int32)
+    idx[:, :, 5] = idx[:, :, 17]
+    dout = torch.from_numpy(rng.standard_normal((w.B, w.H, w.W, w.C)).astype(np.float32)).to(torch.bfloat16).cuda()
+    rq, rk, rv = oracle.attend_backward(inp["q"], inp["k"], inp["v"], idx, host_values(dout), w.heads, w.n_win)
+    dq, dk, dv = bra.attend_backward(q, k, v, torch.from_numpy(idx).cuda(), dout, w.heads, w.n_win)
+    assert bra.check_device_error() == 0
+    for g, r, n in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
+        check_grad(g.cpu().numpy(), r, f"tiled, 18 regions {n}")
+    bad = np.concatenate([idx[:, :, :9], np.full((w.B, w.R, 1), -3, np.int32), idx[:, :, 9:]], axis=-1)
+    dq, dk, dv = bra.attend_backward(q, k, v, torch.from_numpy(bad).cuda(), dout, w.heads, w.n_win)
+    assert bra.check_device_error() == 4
+    for g, r, n in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
+        check_grad(g.cpu().numpy(), r, f"tiled, bad entry skipped {n}")
+
+
 # ------------------------------------------------------------------ auto_pad
 
 PAD_SHAPES = [_w("stage1_54", 8, 54, 54, 64, 2, 7, 1, "bf16"), _w("stage2_27x30", 4, 27, 30, 128, 4, 7, 4, "bf16"),
