@@ -491,16 +491,23 @@ static bra_status route_heads_impl(const void *q, const void *k, int32_t *idx, c
 }
 
 // The attention kernel of per-head routing: the mma.sync gather kernel (bf16, hd == 32, rs % 16
-// == 0, rs <= 64) in its per-head mode, else the CUDA-core kernel; a forced kernel that does not
-// take per-head indices (or cannot serve the shape) makes the call unsupported.
+// == 0, rs <= 64) in its per-head mode; for small images with few tokens per region the dense
+// kernel with one routing-count plane per head (under the same rule as the shared index);
+// else the CUDA-core kernel. A forced kernel that does not take per-head indices (or cannot
+// serve the shape) makes the call unsupported.
 static int choose_heads_kernel(const bra::Geometry &g, bra_dtype dtype)
 {
     const bool simt_ok = g.hd <= bra::kSimtMaxHeadDim;
     const bool gather_ok = dtype == BRA_BF16 && bra::gather_mma_supports(g);
+    const bool dense_ok = dtype == BRA_BF16 && bra::dense_mma_supports(g);
     switch (g_forced_kernel.load()) {
-    case BRA_ATTEND_AUTO: return gather_ok ? BRA_ATTEND_GATHER_MMA : (simt_ok ? BRA_ATTEND_SIMT : -1);
+    case BRA_ATTEND_AUTO:
+        if (gather_ok) return BRA_ATTEND_GATHER_MMA;
+        if (dense_ok && 4LL * g.topk * g.rs >= g.N) return BRA_ATTEND_DENSE_MMA;
+        return simt_ok ? BRA_ATTEND_SIMT : -1;
     case BRA_ATTEND_SIMT: return simt_ok ? BRA_ATTEND_SIMT : -1;
     case BRA_ATTEND_GATHER_MMA: return gather_ok ? BRA_ATTEND_GATHER_MMA : -1;
+    case BRA_ATTEND_DENSE_MMA: return dense_ok ? BRA_ATTEND_DENSE_MMA : -1;
     default: return -1;
     }
 }
@@ -516,6 +523,14 @@ static bra_status attend_heads_impl(const void *q, const void *k, const void *v,
     cudaError_t e = cudaSuccess;
     if (kernel == BRA_ATTEND_SIMT) {
         e = bra::launch_attend_staged(q, k, v, idx, out, g, g.H, g.W, true, dtype == BRA_BF16, st->error_word, stream);
+    } else if (kernel == BRA_ATTEND_DENSE_MMA) {
+        const int rows = bra::dense_mma_rows_per_split(g, st->num_sms);
+        CUtensorMap tq, tk, tv, to;
+        if ((s = encode_map(&tq, q, g, g.W, rows, g.H, g.W)) != BRA_OK) return s;
+        if ((s = encode_map(&tk, k, g, g.W, g.H, g.H, g.W)) != BRA_OK) return s;
+        if ((s = encode_map(&tv, v, g, g.W, g.H, g.H, g.W)) != BRA_OK) return s;
+        if ((s = encode_map(&to, out, g, g.W, rows, g.H, g.W)) != BRA_OK) return s;
+        e = bra::launch_attend_dense_mma(tq, tk, tv, to, idx, g, rows, st->error_word, false, g.H, stream, true);
     } else {
         // q: the item's NCB blocks in one box; k, v: one block per box (each head its own region)
         CUtensorMap tq, tk, tv, to;

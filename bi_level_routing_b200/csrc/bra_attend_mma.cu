@@ -548,6 +548,8 @@ struct DenseArgs {
     float route_scale;  // ROUTE: C^-1/2
     int inputs_ready;   // q, k, v may be loaded before the wait for the previous kernel
     int Hm;             // image rows in memory (H: the region grid's, which may be more)
+    int per_head;       // idx is [B, heads, R, topk]: each head of the block has its own counts
+    int heads;
 };
 
 constexpr int kDensePartPad = 68;  // row stride (floats) of a partial affinity tile
@@ -634,10 +636,12 @@ __global__ void __launch_bounds__(256, MIN_CTAS) attend_dense_mma_kernel(const _
     float *part = reinterpret_cast<float *>(sV + cpb * kvtile);
     unsigned long long *skey =
         reinterpret_cast<unsigned long long *>(part + (ROUTE ? cpb * 64 * kDensePartPad : 0));
-    // [R][R]: the multiplicity of each (query region, key region) pair, then, in place, its log2
+    // [planes][R][R]: the multiplicity of each (query region, key region) pair, then, in place,
+    // its log2; one plane, or (per-head routing) one per head of the block
+    const int planes = a.per_head ? 2 : 1;
     int *cnt = reinterpret_cast<int *>(skey + (ROUTE ? ((a.R + nct - 1) / nct) * 64 : 0));
     float *lw = reinterpret_cast<float *>(cnt);
-    uint8_t *reg = reinterpret_cast<uint8_t *>(cnt + a.R * a.R);  // [npad] region of each key
+    uint8_t *reg = reinterpret_cast<uint8_t *>(cnt + planes * a.R * a.R);  // [npad] region of each key
     uint64_t *bar = reinterpret_cast<uint64_t *>((reinterpret_cast<uintptr_t>(reg + a.npad) + 7) & ~uintptr_t(7));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -677,7 +681,7 @@ __global__ void __launch_bounds__(256, MIN_CTAS) attend_dense_mma_kernel(const _
     }
     for (int t = threadIdx.x; t < a.npad; t += blockDim.x)
         reg[t] = t < a.N ? (uint8_t)(((t / a.W) / a.hr) * a.n_win + (t % a.W) / a.wr) : 0;
-    for (int e = threadIdx.x; e < a.R * a.R; e += blockDim.x) cnt[e] = 0;
+    for (int e = threadIdx.x; e < planes * a.R * a.R; e += blockDim.x) cnt[e] = 0;
     bool alive = true;
     if constexpr (ROUTE) {
         // the partial affinities of this CTA's blocks: task = (block j, 16-row tile, key half)
@@ -726,10 +730,13 @@ __global__ void __launch_bounds__(256, MIN_CTAS) attend_dense_mma_kernel(const _
     } else {
         if (a.inputs_ready) grid_dependency_wait();  // idx comes from the previous kernel
         __syncthreads();
-        // multiplicity of every routed region: the image's idx entries, eight loads per thread in
-        // flight at once, then one shared-memory count per entry
-        const int32_t *routed = a.idx + (int64_t)b * a.R * a.topk;
-        const int nent = a.R * a.topk;
+        // multiplicity of every routed region: the image's idx entries (per-head routing: the rows
+        // of this block's two heads, one plane each), eight loads per thread in flight at once,
+        // then one shared-memory count per entry
+        const int32_t *routed = a.per_head ? a.idx + ((int64_t)b * a.heads + 2 * cb0) * a.R * a.topk
+                                           : a.idx + (int64_t)b * a.R * a.topk;
+        const int nent = planes * a.R * a.topk;  // a plane's rows follow the previous plane's
+        const bool flagger = split == 0 && (a.per_head || ct == 0);
         for (int e0 = threadIdx.x; e0 < nent; e0 += 8 * blockDim.x) {
             int sv[8];
 #pragma unroll
@@ -743,15 +750,15 @@ __global__ void __launch_bounds__(256, MIN_CTAS) attend_dense_mma_kernel(const _
                 if (e < nent) {
                     const int s = sv[u];
                     if (s >= 0 && s < a.R)
-                        atomicAdd(&cnt[(e / a.topk) * a.R + s], 1);
-                    else if (ct == 0 && split == 0)
+                        atomicAdd(&cnt[(e / a.topk) * a.R + s], 1);  // row e / topk of plane-major rows
+                    else if (flagger)
                         flag_error(a.err, kErrIndex);
                 }
             }
         }
         __syncthreads();
     }
-    for (int e = threadIdx.x; e < a.R * a.R; e += blockDim.x) {
+    for (int e = threadIdx.x; e < planes * a.R * a.R; e += blockDim.x) {
         const int c = cnt[e];
         lw[e] = c == 1 ? 0.f : (c ? log2f((float)c) : -INFINITY);  // log2(1) = 0 exactly: skip the call
     }
@@ -772,8 +779,9 @@ __global__ void __launch_bounds__(256, MIN_CTAS) attend_dense_mma_kernel(const _
             ldmatrix_x4(qbase + sw128(rt * 16 + (lane & 15), hb * 4 + ks * 2 + (lane >> 4)), qf[ks][0], qf[ks][1],
                         qf[ks][2], qf[ks][3]);
         const int tq0 = y0 * a.W + rt * 16 + g, tq1 = tq0 + 8;  // query tokens of rows g, g+8
-        const float *lw0 = lw + (tq0 < a.N ? reg[tq0] : 0) * a.R;
-        const float *lw1 = lw + (tq1 < a.N ? reg[tq1] : 0) * a.R;
+        const float *lwp = lw + (a.per_head ? hb * a.R * a.R : 0);
+        const float *lw0 = lwp + (tq0 < a.N ? reg[tq0] : 0) * a.R;
+        const float *lw1 = lwp + (tq1 < a.N ? reg[tq1] : 0) * a.R;
         float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
         float o[4][4];
 #pragma unroll
@@ -856,13 +864,15 @@ int dense_mma_rows_per_split(const Geometry &g, int num_sms)
     return (g.H + nsplit - 1) / nsplit;
 }
 
-static size_t dense_smem_bytes(const Geometry &g, int rows_per_split, int cpb = 1, bool route = false)
+static size_t dense_smem_bytes(const Geometry &g, int rows_per_split, int cpb = 1, bool route = false,
+                               bool per_head = false)
 {
     const int nq = rows_per_split * g.W, nqpad = (nq + 15) & ~15;
     const int npad = (g.N + 15) & ~15;
     const int nct = g.C / 64 / cpb;
     const size_t routing = route ? (size_t)cpb * 64 * kDensePartPad * 4 + (size_t)((g.R + nct - 1) / nct) * 64 * 8 : 0;
-    return 1024 + (size_t)cpb * (nqpad + 2 * npad) * kRowBytes + routing + (size_t)g.R * g.R * 4 + npad + 16;
+    return 1024 + (size_t)cpb * (nqpad + 2 * npad) * kRowBytes + routing + (size_t)(per_head ? 2 : 1) * g.R * g.R * 4 +
+           npad + 16;
 }
 
 static void fill_dense_args(DenseArgs &a, const int32_t *idx, const Geometry &g, int rows_per_split, unsigned *err,
@@ -886,17 +896,20 @@ static void fill_dense_args(DenseArgs &a, const int32_t *idx, const Geometry &g,
     a.cpb = 1;
     a.rows_per_split = rows_per_split;
     a.nsplit = (g.H + rows_per_split - 1) / rows_per_split;
+    a.per_head = 0;
+    a.heads = g.heads;
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)g.hd));
     a.route_scale = (float)(1.0 / sqrt((double)g.C));
 }
 
 cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                     const CUtensorMap &tout, const int32_t *idx, const Geometry &g, int rows_per_split,
-                                    unsigned *err, bool inputs_ready, int Hm, cudaStream_t stream)
+                                    unsigned *err, bool inputs_ready, int Hm, cudaStream_t stream, bool per_head)
 {
     DenseArgs a;
     fill_dense_args(a, idx, g, rows_per_split, err, inputs_ready, Hm);
-    const size_t smem = dense_smem_bytes(g, rows_per_split);
+    a.per_head = per_head ? 1 : 0;
+    const size_t smem = dense_smem_bytes(g, rows_per_split, 1, false, per_head);
     const long long blocks = (long long)g.B * a.ncb * a.nsplit;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     // three CTAs per SM when their shared memory fits (227 KB per SM, 1 KB reserved per CTA)

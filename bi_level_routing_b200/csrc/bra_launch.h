@@ -165,11 +165,13 @@ cudaError_t launch_attend_gather_umma(const CUtensorMap &tq, const CUtensorMap &
                                       unsigned *err, cudaStream_t stream);
 
 // Boxes of the dense kernel: q and out (64, W, rows_per_split, 1); k and v (64, W, H, 1).
+// per_head: idx is [B, heads, R, topk] and each head of a 64-channel block is masked by its own
+// routing counts.
 int dense_mma_rows_per_split(const Geometry &g, int num_sms);
 cudaError_t launch_attend_dense_mma(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                     const CUtensorMap &tout, const int32_t *idx, const Geometry &g,
                                     int rows_per_split, unsigned *err, bool inputs_ready, int Hm,
-                                    cudaStream_t stream);
+                                    cudaStream_t stream, bool per_head = false);
 
 // The forward pass of one-token regions (bf16, R <= 64) in one kernel: the dense kernel with the
 // routing step inside, launched as one thread-block cluster per image (at most

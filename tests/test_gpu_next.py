@@ -64,9 +64,42 @@ def test_heads_both_kernels(w):
             assert bra.check_device_error() == 0
             assert torch.equal(idx2, idx) and torch.equal(out2, out), kname
             check_output(host_values(out), ref, w.dtype, f"{w.name} per-head / {kname}")
-        bra.set_attend_kernel("dense_mma")
+        bra.set_attend_kernel("region_mma")
         with pytest.raises(RuntimeError):
             bra.attend_heads(q, k, v, idx, w.n_win)
+    finally:
+        bra.set_attend_kernel("auto")
+
+
+# shapes the dense kernel takes with one routing-count plane per head (bf16, hd 32, R <= 64,
+# H W <= 256): 4-token and one-token regions, two and eight 64-channel blocks
+HEADS_DENSE = [WORKLOADS["stage3"].with_(B=4), WORKLOADS["stage4"].with_(B=4),
+               _w("rs4_r16_c128", 3, 8, 8, 128, 4, 4, 5, "bf16")]
+
+
+@pytest.mark.parametrize("w", HEADS_DENSE, ids=[w.name for w in HEADS_DENSE])
+def test_heads_dense_kernel(w):
+    inp, (q, k, v) = make(w)
+    idx = bra.route_heads(q, k, w.n_win, w.topk, w.heads)
+    torch.cuda.synchronize()
+    ref = oracle.attend_heads(inp["q"], inp["k"], inp["v"], idx.cpu().numpy(), w.n_win)
+    try:
+        for kname in ("dense_mma", "simt"):
+            bra.set_attend_kernel(kname)
+            out = bra.attend_heads(q, k, v, idx, w.n_win)
+            torch.cuda.synchronize()
+            assert bra.check_device_error() == 0
+            check_output(host_values(out), ref, w.dtype, f"{w.name} per-head / {kname}")
+        # given rows with duplicates and one bad entry per row: skipped and flagged
+        rng = np.random.Generator(np.random.PCG64(23))
+        given = rng.integers(0, w.R, size=(w.B, w.heads, w.R, 3)).astype(np.int32)
+        given[..., 2] = given[..., 0]
+        gref = oracle.attend_heads(inp["q"], inp["k"], inp["v"], given, w.n_win)
+        bad = np.concatenate([given, np.full((w.B, w.heads, w.R, 1), w.R, np.int32)], axis=-1)
+        bra.set_attend_kernel("dense_mma")
+        out = bra.attend_heads(q, k, v, torch.from_numpy(bad).cuda(), w.n_win)
+        assert bra.check_device_error() == 4
+        check_output(host_values(out), gref, w.dtype, f"{w.name} per-head dense, given rows")
     finally:
         bra.set_attend_kernel("auto")
 
