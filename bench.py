@@ -40,9 +40,27 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = {"attend_gather_umma": "bi_level_routing_b200/csrc/bra_attend_umma.cu",
                   "attend_gather_mma": "bi_level_routing_b200/csrc/bra_attend_mma.cu",
+                  "attend_gather_mma_heads": "bi_level_routing_b200/csrc/bra_attend_mma.cu",
                   "attend_dense_mma": "bi_level_routing_b200/csrc/bra_attend_mma.cu",
+                  "attend_dense_mma_heads": "bi_level_routing_b200/csrc/bra_attend_mma.cu",
                   "attend_region_mma": "bi_level_routing_b200/csrc/bra_attend_region.cu",
-                  "attend_simt": "bi_level_routing_b200/csrc/bra_attend_simt.cu"}
+                  "attend_simt": "bi_level_routing_b200/csrc/bra_attend_simt.cu",
+                  "attend_backward": "bi_level_routing_b200/csrc/bra_attend_backward.cu",
+                  "lepe": "bi_level_routing_b200/csrc/bra_lepe.cu",
+                  "region_means": "bi_level_routing_b200/csrc/bra_route.cu",
+                  "region_means_small": "bi_level_routing_b200/csrc/bra_route.cu",
+                  "region_means_padded": "bi_level_routing_b200/csrc/bra_route.cu",
+                  "route_tf32x3": "bi_level_routing_b200/csrc/bra_route.cu",
+                  "route_tf32x3_wide": "bi_level_routing_b200/csrc/bra_route.cu",
+                  "route_heads": "bi_level_routing_b200/csrc/bra_route.cu"}
+# The kernels one bra_forward step launches on each named workload (the launch lists show them);
+# the step's recorded DRAM traffic is their sum.
+STEP_KERNELS = {"tiny_f32": ("region_means_small", "route_tf32x3", "attend_simt"),
+                "stage1": ("region_means", "route_tf32x3", "attend_gather_umma"),
+                "stage2": ("region_means_small", "route_tf32x3", "attend_gather_mma"),
+                "stage3": ("region_means_small", "route_tf32x3", "attend_region_mma"),
+                "stage4": ("attend_dense_mma",),
+                "highres": ("region_means", "route_tf32x3_wide", "attend_gather_umma")}
 
 
 def parse_args(argv=None):
@@ -260,6 +278,13 @@ def step_roofline_us(w, pk) -> float:
                w.attention_flops() / (float(pk["bf16_tflops"]) * 1e12)) * 1e6
 
 
+def step_traffic(workload: str):
+    """DRAM bytes of one step: the recorded per-launch traffic of each kernel the step launches,
+    summed, if every one was taken on the current source; else None."""
+    parts = [recorded_traffic(k, workload) for k in STEP_KERNELS.get(workload, ())]
+    return float(sum(parts)) if parts and all(p is not None for p in parts) else None
+
+
 def roofline_record(w, pk, pk_kind, step_us, kernel, kernel_us, route_us, breakdown_us):
     """The step against its roofline (frac) and the dominant kernel's own figures (kernel_*)."""
     hbm = float(pk["hbm_gbs"])
@@ -268,7 +293,7 @@ def roofline_record(w, pk, pk_kind, step_us, kernel, kernel_us, route_us, breakd
     kernel_achieved = w.unique_bytes() / (kernel_us * 1e-6) / 1e9
     return {"bound": "hbm", "scope": "bra_forward step (every kernel of the call)",
             "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-            "traffic": None,
+            "traffic": step_traffic(w.name),
             "peak_source": f"{pk_kind} hbm_gbs (MEASURED_PEAKS.json)" if pk_kind == "measured" else "fallback",
             "algorithmic_bytes_per_step": w.unique_bytes(), "step_roofline_us": roof_us, "step_us": step_us,
             "step_frac_vs_8tbs": (w.unique_bytes() / 8e12 * 1e6) / step_us,
