@@ -277,9 +277,11 @@ __global__ void __launch_bounds__(256) attend_backward_kernel(const BackArgs a)
 //   dQ     : lane l owns rows l and l + 32, warp w channels 4w .. 4w+3: ds transposed (padded
 //            rows) and k by rows (a 16-byte broadcast); dq accumulates in registers over all the
 //            routed regions and is stored once.
-//   dK, dV : lane l owns channels 4 (l % 8) .. + 3 of keys 8w + l / 8 and that + 4: ds and p by
-//            rows, q and dout by rows (16-byte loads); the sums over the region's queries go to
-//            dk and dv with one 16-byte atomic per key and tensor.
+//   dK, dV : warps 0-3 form dk, warps 4-7 dv; thread t of a half owns channels 4 (t % 8) .. + 3
+//            of keys 4 (t / 8) .. + 3: ds (or p) and q (or dout) by rows, 16-byte loads; the sums
+//            over the region's queries go to dk and dv with one 16-byte atomic per key.
+// Rows of the tiles read by rows are padded to 36 floats, so that the staging stores of
+// consecutive rows fall in different banks.
 // With one routed region the scores stay in registers between the statistics and the
 // gradients; with more, pass 1 gathers the statistics and pass 2 recomputes them per region.
 namespace {
@@ -287,13 +289,15 @@ namespace {
 constexpr int kTiledThreads = 256;
 
 // floats of each shared-memory array of the tiled kernel
-constexpr int kT64 = 64 * 32;        // a 64 x 32 tile
+constexpr int kT64 = 64 * 32;        // a 64 x 32 tile, transposed ([32][64])
+constexpr int kRow = 36;             // row stride of a 64 x 32 tile kept by rows
+constexpr int kTN = 64 * kRow;       // a 64 x 32 tile by rows, padded
 constexpr int kTPS = 64 * 64;        // a 64 x 64 tile
 constexpr int kTdSt = 64 * 65;       // transposed ds, rows padded to 65
-constexpr size_t kTiledSmem = sizeof(float) * (7 * kT64 + 2 * kTPS + kTdSt) + 16 * sizeof(int);
+constexpr size_t kTiledSmem = sizeof(float) * (4 * kT64 + 3 * kTN + 2 * kTPS + kTdSt) + 16 * sizeof(int);
 
 // Loads one 64-token x 32-channel head tile (rows of the region at (y0, x0), channel offset
-// c0) as fp32: into `tr` transposed ([32][64]) and, when `nat` is set, by rows ([64][32]).
+// c0) as fp32: into `tr` transposed ([32][64]) and, when `nat` is set, by rows ([64][kRow]).
 template <typename T>
 __device__ __forceinline__ void stage_head_tile(const T *g, const BackArgs &a, int64_t b, int y0, int x0, int c0,
                                                 float *tr, float *nat)
@@ -308,7 +312,7 @@ __device__ __forceinline__ void stage_head_tile(const T *g, const BackArgs &a, i
 #pragma unroll
         for (int i = 0; i < V; ++i) tr[(u * V + i) * 64 + row] = f[i];
         if (nat) {
-            float4 *d = reinterpret_cast<float4 *>(nat + row * 32 + u * V);
+            float4 *d = reinterpret_cast<float4 *>(nat + row * kRow + u * V);
 #pragma unroll
             for (int i = 0; i < V / 4; ++i) d[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
         }
@@ -336,12 +340,12 @@ __global__ void __launch_bounds__(kTiledThreads, 2) attend_backward_tiled_kernel
 {
     extern __shared__ float4 smem4[];
     float *Qt = reinterpret_cast<float *>(smem4);  // [32][64] q transposed
-    float *Qn = Qt + kT64;                         // [64][32] q
-    float *Dt = Qn + kT64;                         // [32][64] dout transposed
-    float *Dn = Dt + kT64;                         // [64][32] dout
-    float *Kt = Dn + kT64;                         // [32][64] k of the routed region, transposed
-    float *Kn = Kt + kT64;                         // [64][32] k
-    float *Vt = Kn + kT64;                         // [32][64] v transposed
+    float *Qn = Qt + kT64;                         // [64][kRow] q
+    float *Dt = Qn + kTN;                          // [32][64] dout transposed
+    float *Dn = Dt + kT64;                         // [64][kRow] dout
+    float *Kt = Dn + kTN;                          // [32][64] k of the routed region, transposed
+    float *Kn = Kt + kT64;                         // [64][kRow] k
+    float *Vt = Kn + kTN;                          // [32][64] v transposed
     float *Ps = Vt + kT64;                         // [64 queries][64 keys] p
     float *Ss = Ps + kTPS;                         // [64 queries][64 keys] ds
     float *St = Ss + kTPS;                         // [64 keys][65] ds transposed
@@ -445,7 +449,9 @@ __global__ void __launch_bounds__(kTiledThreads, 2) attend_backward_tiled_kernel
     float dq[2][4];
 #pragma unroll
     for (int i = 0; i < 2; ++i) dq[i][0] = dq[i][1] = dq[i][2] = dq[i][3] = 0.f;
-    const int c4 = lane & 7, kk = 8 * warp + (lane >> 3);  // dK / dV: keys kk, kk + 4; channels 4 c4..
+    // dK (warps 0-3) or dV (warps 4-7): keys 4 kg .. + 3, channels 4 c4 .. + 3
+    const int half = warp >> 2, ht = threadIdx.x & 127;
+    const int c4 = ht & 7, kg = ht >> 3;
     for (int j = 0; j < a.topk; ++j) {
         const int s = region(j);
         if (s < 0) continue;
@@ -473,7 +479,7 @@ __global__ void __launch_bounds__(kTiledThreads, 2) attend_backward_tiled_kernel
         // dq rows lane, lane + 32, channels 4 warp ..: sum over the region's 64 keys
 #pragma unroll 4
         for (int key = 0; key < 64; ++key) {
-            const float4 kr = *reinterpret_cast<const float4 *>(Kn + key * 32 + 4 * warp);
+            const float4 kr = *reinterpret_cast<const float4 *>(Kn + key * kRow + 4 * warp);
             const float d0 = St[key * 65 + lane], d1 = St[key * 65 + lane + 32];
             dq[0][0] = fmaf(d0, kr.x, dq[0][0]);
             dq[0][1] = fmaf(d0, kr.y, dq[0][1]);
@@ -484,38 +490,38 @@ __global__ void __launch_bounds__(kTiledThreads, 2) attend_backward_tiled_kernel
             dq[1][2] = fmaf(d1, kr.z, dq[1][2]);
             dq[1][3] = fmaf(d1, kr.w, dq[1][3]);
         }
-        // dk, dv of keys kk and kk + 4, channels 4 c4 ..: sums over the region's 64 queries
-        float4 gk4[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-        float4 gv4[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+        // dk (or dv) of keys 4 kg .. + 3, channels 4 c4 ..: sums over the region's 64 queries of
+        // ds q (or p dout)
+        {
+            const float *coef = half ? Ps : Ss;
+            const float *rows = half ? Dn : Qn;
+            float4 g4[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) g4[t] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
-        for (int row = 0; row < 64; ++row) {
-            const float4 qr = *reinterpret_cast<const float4 *>(Qn + row * 32 + 4 * c4);
-            const float4 dr = *reinterpret_cast<const float4 *>(Dn + row * 32 + 4 * c4);
+            for (int row = 0; row < 64; ++row) {
+                const float4 x = *reinterpret_cast<const float4 *>(rows + row * kRow + 4 * c4);
+                const float4 w4 = *reinterpret_cast<const float4 *>(coef + row * 64 + 4 * kg);
+                const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                const float ds = Ss[row * 64 + kk + 4 * t], p = Ps[row * 64 + kk + 4 * t];
-                gk4[t].x = fmaf(ds, qr.x, gk4[t].x);
-                gk4[t].y = fmaf(ds, qr.y, gk4[t].y);
-                gk4[t].z = fmaf(ds, qr.z, gk4[t].z);
-                gk4[t].w = fmaf(ds, qr.w, gk4[t].w);
-                gv4[t].x = fmaf(p, dr.x, gv4[t].x);
-                gv4[t].y = fmaf(p, dr.y, gv4[t].y);
-                gv4[t].z = fmaf(p, dr.z, gv4[t].z);
-                gv4[t].w = fmaf(p, dr.w, gv4[t].w);
+                for (int t = 0; t < 4; ++t) {
+                    g4[t].x = fmaf(wv[t], x.x, g4[t].x);
+                    g4[t].y = fmaf(wv[t], x.y, g4[t].y);
+                    g4[t].z = fmaf(wv[t], x.z, g4[t].z);
+                    g4[t].w = fmaf(wv[t], x.w, g4[t].w);
+                }
             }
-        }
-        const int sy = (s / a.n_win) * a.hr, sx = (s % a.n_win) * a.wr;
+            const int sy = (s / a.n_win) * a.hr, sx = (s % a.n_win) * a.wr;
+            const float sc4 = half ? 1.f : a.scale;
+            float *dst = half ? a.dv : a.dk;
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const int key = kk + 4 * t;
-            const int y = sy + key / a.wr, x = sx + key % a.wr;
-            const int64_t off = ((b * a.H + y) * a.W + x) * a.C + c0 + 4 * c4;
-            gk4[t].x *= a.scale;
-            gk4[t].y *= a.scale;
-            gk4[t].z *= a.scale;
-            gk4[t].w *= a.scale;
-            atomicAdd(reinterpret_cast<float4 *>(a.dk + off), gk4[t]);
-            atomicAdd(reinterpret_cast<float4 *>(a.dv + off), gv4[t]);
+            for (int t = 0; t < 4; ++t) {
+                const int key = 4 * kg + t;
+                const int y = sy + key / a.wr, x = sx + key % a.wr;
+                const int64_t off = ((b * a.H + y) * a.W + x) * a.C + c0 + 4 * c4;
+                atomicAdd(reinterpret_cast<float4 *>(dst + off),
+                          make_float4(g4[t].x * sc4, g4[t].y * sc4, g4[t].z * sc4, g4[t].w * sc4));
+            }
         }
         __syncthreads();  // p and ds are rewritten by the next region
     }
