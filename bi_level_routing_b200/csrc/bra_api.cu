@@ -308,9 +308,9 @@ namespace bra {
 
 void set_last_error(const std::string &msg) { g_last_error = msg; }
 
-int persistent_grid(long long nitems, int num_sms)
+int persistent_grid(long long nitems, int num_sms, int per_sm)
 {
-    long long grid = 2LL * num_sms;
+    long long grid = (long long)per_sm * num_sms;
     const int cap = g_max_ctas.load();
     if (cap > 0 && grid > cap) grid = cap;
     if (grid > nitems) grid = nitems;

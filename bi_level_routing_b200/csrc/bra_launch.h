@@ -46,9 +46,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // Sets the message bra_last_error_message returns on this thread.
 void set_last_error(const std::string &msg);
 
-// Grid of a persistent attention kernel over `nitems` work items: two CTAs per SM, at most
+// Grid of a persistent attention kernel over `nitems` work items: `per_sm` CTAs per SM, at most
 // one CTA per item, and at most the cap set by bra_set_max_ctas (0 = none).
-int persistent_grid(long long nitems, int num_sms);
+int persistent_grid(long long nitems, int num_sms, int per_sm = 2);
 
 // The argument checks of bra_route (shape, NULL pointers, alignment); fills g.
 bra_status check_route_args(const void *q, const void *k, const int32_t *idx, int B, int H, int W, int C, int n_win,

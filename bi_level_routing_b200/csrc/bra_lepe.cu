@@ -35,12 +35,14 @@ __device__ __forceinline__ void store_pair(float *dst, float a, float b)
 }  // namespace
 
 // ROWS: output rows per thread, CB / 4 (CB / 2 channel pairs x kTileX columns x kTileY / ROWS row
-// groups = 256 threads); a template argument, so that every loop below unrolls completely.
+// groups = 256 threads); a template argument, so that every loop below unrolls completely and
+// every index division is by a constant.
 template <typename T, int ROWS>
 __global__ void __launch_bounds__(kLepeThreads) lepe_kernel(const T *__restrict__ x, const float *__restrict__ weight,
                                                             const float *__restrict__ bias, T *__restrict__ y, int H,
-                                                            int W, int C, int CB)
+                                                            int W, int C)
 {
+    constexpr int CB = 4 * ROWS;  // channels of the CTA's block
     extern __shared__ float4 smem4[];
     float *sx = reinterpret_cast<float *>(smem4);  // [kInY * kInX][CB]
     float *sw = sx + kInY * kInX * CB;             // [25][CB]: tap-major, channels contiguous
@@ -62,7 +64,7 @@ __global__ void __launch_bounds__(kLepeThreads) lepe_kernel(const T *__restrict_
     // contiguous for the block: channel-major, 25 taps each) and the bias
     constexpr int V = Vec16<T>::N;
     constexpr int kBatch = 4;
-    const int vpt = CB / V, nvec = kInY * kInX * vpt;
+    constexpr int vpt = CB / V, nvec = kInY * kInX * vpt;
     for (int e0 = threadIdx.x; e0 < nvec; e0 += kBatch * kLepeThreads) {
         uint4 raw[kBatch];
         bool inside[kBatch];
@@ -100,7 +102,7 @@ __global__ void __launch_bounds__(kLepeThreads) lepe_kernel(const T *__restrict_
 
     // thread: channel pair cp of output column ox and rows [half ROWS, (half + 1) ROWS) of the tile
     // (a CTA has CB / 2 x kTileX x kTileY / ROWS = 256 such threads)
-    const int pairs = CB / 2;
+    constexpr int pairs = CB / 2;
     const int cp = threadIdx.x % pairs, col = threadIdx.x / pairs;
     const int ox = col % kTileX, half = col / kTileX;
     const int oy0 = half * ROWS;
@@ -139,7 +141,7 @@ __global__ void __launch_bounds__(kLepeThreads) lepe_kernel(const T *__restrict_
 
 template <typename T, int ROWS>
 static cudaError_t launch_rows(const void *x, const float *weight, const float *bias, void *y, int H, int W, int C,
-                               int CB, long long blocks, size_t smem, cudaStream_t stream)
+                               long long blocks, size_t smem, cudaStream_t stream)
 {
     static int granted[64] = {0};
     int dev = 0;
@@ -152,7 +154,7 @@ static cudaError_t launch_rows(const void *x, const float *weight, const float *
         granted[dev] = (int)smem;
     }
     return launch_pdl(lepe_kernel<T, ROWS>, dim3((unsigned)blocks), dim3(kLepeThreads), smem, stream,
-                      static_cast<const T *>(x), weight, bias, static_cast<T *>(y), H, W, C, CB);
+                      static_cast<const T *>(x), weight, bias, static_cast<T *>(y), H, W, C);
 }
 
 bool lepe_supports(int C, bool bf16) { return C % (bf16 ? 8 : 4) == 0; }
@@ -171,16 +173,16 @@ cudaError_t launch_lepe(const void *x, const float *weight, const float *bias, v
     // rows per thread: CB / 2 channel pairs x 8 columns x (16 / ROWS) row groups = 256 threads
     const int rows = CB * 8 * 16 / (2 * kLepeThreads);
     switch (rows) {
-    case 16: return bf16 ? launch_rows<__nv_bfloat16, 16>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream)
-                         : launch_rows<float, 16>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream);
-    case 8: return bf16 ? launch_rows<__nv_bfloat16, 8>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream)
-                        : launch_rows<float, 8>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream);
-    case 4: return bf16 ? launch_rows<__nv_bfloat16, 4>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream)
-                        : launch_rows<float, 4>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream);
-    case 2: return bf16 ? launch_rows<__nv_bfloat16, 2>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream)
-                        : launch_rows<float, 2>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream);
-    case 1: return bf16 ? launch_rows<__nv_bfloat16, 1>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream)
-                        : launch_rows<float, 1>(x, weight, bias, y, H, W, C, CB, blocks, smem, stream);
+    case 16: return bf16 ? launch_rows<__nv_bfloat16, 16>(x, weight, bias, y, H, W, C, blocks, smem, stream)
+                         : launch_rows<float, 16>(x, weight, bias, y, H, W, C, blocks, smem, stream);
+    case 8: return bf16 ? launch_rows<__nv_bfloat16, 8>(x, weight, bias, y, H, W, C, blocks, smem, stream)
+                        : launch_rows<float, 8>(x, weight, bias, y, H, W, C, blocks, smem, stream);
+    case 4: return bf16 ? launch_rows<__nv_bfloat16, 4>(x, weight, bias, y, H, W, C, blocks, smem, stream)
+                        : launch_rows<float, 4>(x, weight, bias, y, H, W, C, blocks, smem, stream);
+    case 2: return bf16 ? launch_rows<__nv_bfloat16, 2>(x, weight, bias, y, H, W, C, blocks, smem, stream)
+                        : launch_rows<float, 2>(x, weight, bias, y, H, W, C, blocks, smem, stream);
+    case 1: return bf16 ? launch_rows<__nv_bfloat16, 1>(x, weight, bias, y, H, W, C, blocks, smem, stream)
+                        : launch_rows<float, 1>(x, weight, bias, y, H, W, C, blocks, smem, stream);
     default: return cudaErrorInvalidConfiguration;
     }
 }
