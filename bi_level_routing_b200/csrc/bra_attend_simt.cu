@@ -10,9 +10,11 @@
 //
 // One CTA per (image, query region, group of heads): the routed regions' key and value rows of
 // those heads are staged in shared memory by the whole CTA (16-byte vectors when a head's
-// channels allow it), a chunk of routed regions at a time; then one thread per (query token,
-// head) keeps q and its output in registers and folds the softmax online over the staged keys
-// (running max and sum, exp2 with a log2(e) pre-scale). The gathered K/V never reach HBM.
+// channels allow it), a chunk of routed regions at a time; then `ks` threads per (query token,
+// head) (consecutive lanes; ks = 1 when the queries and heads of a CTA fill 256 threads, up to 8
+// for small regions) each keep q and a partial output in registers and fold the softmax online
+// over every ks-th staged key (running max and sum, exp2 with a log2(e) pre-scale); the ks
+// partial states are merged by warp shuffles at the end. The gathered K/V never reach HBM.
 #include "bra_device.cuh"
 #include "bra_launch.h"
 
@@ -29,7 +31,8 @@ struct StagedArgs {
     int C, heads, hd, n_win, hr, wr, rs, R, topk;
     int per_head;  // idx is [B, heads, R, topk]; else [B, R, topk], shared by all heads
     int hpc;       // heads per CTA
-    int tq;        // threads per head (query tokens per pass)
+    int tq;        // query tokens per head and pass
+    int ks;        // threads per (query token, head): the keys are dealt among them
     int kchunk;    // routed regions staged per chunk
     int vec;       // head rows staged as 16-byte vectors
     float scale_log2;
@@ -60,7 +63,8 @@ __global__ void __launch_bounds__(256) attend_staged_kernel(const StagedArgs a)
     const T *gk = static_cast<const T *>(a.k);
     const T *gv = static_cast<const T *>(a.v);
     T *gout = static_cast<T *>(a.out);
-    const int hl = threadIdx.x / a.tq, tt = threadIdx.x - hl * a.tq;
+    const int qt = threadIdx.x / a.ks, kq = threadIdx.x - qt * a.ks;  // (head, query) slot; key lane
+    const int hl = qt / a.tq, tt = qt - hl * a.tq;
     const int h = hg * a.hpc + hl;
     grid_dependency_wait();
 
@@ -147,11 +151,12 @@ __global__ void __launch_bounds__(256) attend_staged_kernel(const StagedArgs a)
             const T *kh = Ks + hl * hstride;
             const T *vh = Vs + hl * hstride;
             constexpr int V = Vec16<T>::N;
-            for (int jj = 0; jj < nj; ++jj) {
+            for (int key = kq; key < nj * a.rs; key += a.ks) {  // this thread's keys of the chunk
+                const int jj = key / a.rs;
                 if (sreg[hl * a.kchunk + jj] < 0) continue;  // a skipped region contributes no key
-                for (int tk = 0; tk < a.rs; ++tk) {
-                    const T *kr = kh + (size_t)(jj * a.rs + tk) * a.hd;
-                    const T *vr = vh + (size_t)(jj * a.rs + tk) * a.hd;
+                {
+                    const T *kr = kh + (size_t)key * a.hd;
+                    const T *vr = vh + (size_t)key * a.hd;
                     float dot = 0.f;
                     if (a.vec) {  // 16-byte rows: V channels per shared-memory load
 #pragma unroll
@@ -194,7 +199,19 @@ __global__ void __launch_bounds__(256) attend_staged_kernel(const StagedArgs a)
                 }
             }
         }
-        if (real) {
+        // merge the ks partial states of a (query, head): rescale to the common max, then add
+        // (every lane of the warp takes part; lanes without a query hold m = -inf, l = 0)
+        for (int off = 1; off < a.ks; off <<= 1) {
+            const float mo = __shfl_xor_sync(0xffffffffu, m, off);
+            const float mn = fmaxf(m, mo);
+            const float sc = (m == -INFINITY) ? 0.f : fast_exp2(m - mn);
+            const float so = (mo == -INFINITY) ? 0.f : fast_exp2(mo - mn);
+            l = l * sc + __shfl_xor_sync(0xffffffffu, l, off) * so;
+#pragma unroll
+            for (int c = 0; c < HDMAX; ++c) o[c] = o[c] * sc + __shfl_xor_sync(0xffffffffu, o[c], off) * so;
+            m = mn;
+        }
+        if (real && kq == 0) {
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll
             for (int c = 0; c < HDMAX; ++c)
@@ -218,7 +235,11 @@ cudaError_t launch_staged_typed(StagedArgs a, const Geometry &g, cudaStream_t st
         if (g.heads % d == 0 && (long long)d * g.rs <= 256) hpc = d;
     a.hpc = hpc;
     a.tq = g.rs <= 256 ? g.rs : 256;
-    int threads = ((hpc * a.tq + 31) / 32) * 32;
+    // threads per (query, head): up to 8 while the CTA stays within 256 threads
+    int ks = 1;
+    while (ks < 8 && (long long)hpc * a.tq * ks * 2 <= 256) ks *= 2;
+    a.ks = ks;
+    int threads = ((hpc * a.tq * ks + 31) / 32) * 32;
     if (threads > 256) threads = 256;
     a.vec = ((g.hd * elem) % 16 == 0) ? 1 : 0;
     // routed regions per chunk: as many as keep the CTA within kStagedTargetSmem (several CTAs per
