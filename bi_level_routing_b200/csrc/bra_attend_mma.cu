@@ -579,19 +579,20 @@ __device__ __forceinline__ void dense_route_rows(const DenseArgs &a, const float
 {
     const uint32_t part0 = smem_u32(part);
     const int nrows = (a.R - ct + nct - 1) / nct;  // rows ct, ct + nct, ... below R
-    const int npairs = nrows * a.R;
-    for (int e = threadIdx.x; e < npairs; e += blockDim.x) {
-        const int rr = e / a.R, s = e - rr * a.R;
+    const int cshift = a.cpb == 2 ? 1 : 0;          // block w sits in CTA w >> cshift
+    // (row, region) pairs as rr * 64 + s (shifts, no division); regions s >= R are skipped
+    for (int e = threadIdx.x; e < nrows * 64; e += blockDim.x) {
+        const int rr = e >> 6, s = e & 63;
+        if (s >= a.R) continue;
         const int i = ct + nct * rr;
+        const uint32_t base = part0 + 4u * (uint32_t)(i * kDensePartPad + s);
         // every block's partial in flight at once, then added in block order
         float pw[kDenseMaxBlocks];
 #pragma unroll
-        for (int w = 0; w < kDenseMaxBlocks; ++w) {
-            const int r = w / a.cpb, j = w - r * a.cpb;
-            pw[w] = w < a.ncb ? ld_cluster_f32(cluster_map(part0 + 4u * (uint32_t)((j * 64 + i) * kDensePartPad + s),
-                                                            (uint32_t)r))
+        for (int w = 0; w < kDenseMaxBlocks; ++w)
+            pw[w] = w < a.ncb ? ld_cluster_f32(cluster_map(base + 4u * (uint32_t)((w & (a.cpb - 1)) * 64 * kDensePartPad),
+                                                            (uint32_t)(w >> cshift)))
                               : 0.f;
-        }
         float d = 0.f;
 #pragma unroll
         for (int w = 0; w < kDenseMaxBlocks; ++w)
@@ -599,12 +600,13 @@ __device__ __forceinline__ void dense_route_rows(const DenseArgs &a, const float
         skey[rr * 64 + s] = routing_key(d * a.route_scale, s);
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < npairs; e += blockDim.x) {
-        const int rr = e / a.R, s = e - rr * a.R;
+    for (int e = threadIdx.x; e < nrows * 64; e += blockDim.x) {
+        const int rr = e >> 6, s = e & 63;
+        if (s >= a.R) continue;
         const unsigned long long *row = skey + rr * 64;
         const unsigned long long mine = row[s];
         int pos = 0;
-#pragma unroll 4
+#pragma unroll 7
         for (int j = 0; j < a.R; ++j) pos += row[j] > mine ? 1 : 0;
         if (pos < a.topk) {
             const int i = ct + nct * rr;
