@@ -226,7 +226,9 @@ __global__ void __launch_bounds__(256, 2) route_topk_kernel(const S *__restrict_
 // Per-head routing ("医学图像分割模块", §五 steps ③④): the same rows, staging and selection as
 // route_topk_kernel, for one head at a time: head h's means are channels [h hd, (h + 1) hd) of
 // the region means (row stride C), its affinities are scaled by hd^-1/2, and its index rows go to
-// idx[b, h, :, :]. One CTA per (image, head, block of rows).
+// idx[b, h, :, :]. One CTA per (image, head, block of rows); when a head's channels fit one
+// staging pass, the block may hold more rows than its warps take at once, and the warps then
+// go over them in turn on the same staged key means (fewer CTAs stage the same key rows).
 template <int E, bool ROUNDS, typename S>
 __global__ void __launch_bounds__(256, 2) route_heads_kernel(const S *__restrict__ qm, const S *__restrict__ km,
                                                           int32_t *__restrict__ idx, int R, int C, int hd, int heads,
@@ -249,6 +251,22 @@ __global__ void __launch_bounds__(256, 2) route_heads_kernel(const S *__restrict
     const int i0 = warp * NR;
     const int nr = min(NR, nrows - i0);
     float acc[NR][E][4];
+    if (hd <= chunk) {
+        stage_rows<false, S>(gkm, R, gqm, nrows, skm, C, 0, hd, stride);
+        __syncthreads();
+        for (int p0 = i0; p0 < nrows; p0 += 8 * NR) {  // 8 warps x NR rows per turn
+            const int np = min(NR, nrows - p0);
+#pragma unroll
+            for (int i = 0; i < NR; ++i)
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][e][j] = 0.f;
+            affinity_accumulate<E, NR>(acc, sqm + (size_t)p0 * stride, stride, np, skm, stride, R, hd, lane);
+            affinity_select<E, NR, ROUNDS>(acc, np, R, topk, scale, idx + ((int64_t)bh * R + r0 + p0) * topk, lane);
+        }
+        return;
+    }
 #pragma unroll
     for (int i = 0; i < NR; ++i)
 #pragma unroll
@@ -803,11 +821,26 @@ template <int E, typename S>
 static cudaError_t launch_heads_e(const S *qm, const S *km, int32_t *idx, const Geometry &g, cudaStream_t stream)
 {
     const float scale = (float)(1.0 / sqrt((double)g.hd));
-    const int rows = 8 * RowsPerPass<E>::value;
-    const long long per_col = (long long)(g.R + rows) * sizeof(float);
+    const int turn = 8 * RowsPerPass<E>::value;  // rows the warps take at once
+    int rows = turn;
+    // one staging pass for the whole head: blocks of several turns of rows, about two CTAs per SM
+    // in all (the key means of an (image, head) are then staged by fewer CTAs)
+    {
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const long long pairs = (long long)g.B * g.heads;
+        long long blocks_per_pair = (2LL * sms + pairs - 1) / pairs;
+        if (blocks_per_pair < 1) blocks_per_pair = 1;
+        int want = (int)((g.R + blocks_per_pair - 1) / blocks_per_pair);
+        want = (want + turn - 1) / turn * turn;
+        if ((long long)(g.R + want) * sizeof(float) * (g.hd + 4) <= 100 * 1024 && want > rows) rows = want;
+    }
+    long long per_col = (long long)(g.R + rows) * sizeof(float);
     constexpr int V = 16 / sizeof(S);
     int chunk = g.hd;
     if (per_col * (chunk + 4) > 100 * 1024) {
+        rows = turn;  // several staging passes: one turn of rows per CTA
+        per_col = (long long)(g.R + rows) * sizeof(float);
         chunk = 32;
         while (chunk * 2 < g.hd && per_col * (chunk * 2 + 4) <= 100 * 1024) chunk *= 2;
         if (per_col * (chunk + 4) > 100 * 1024) return cudaErrorInvalidConfiguration;
