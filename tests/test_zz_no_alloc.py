@@ -44,7 +44,9 @@ WIDE_F32 = Workload("r324_rs4_f32", 3, 36, 36, 32, 1, 18, 5, "f32", "region_offs
 
 def test_no_alloc_route_matches_bra_route_on_two_calls_in_a_row():
     L = _lib()
-    for w in (WIDE, WORKLOADS["stage1"].with_(B=16), WIDE_F32, WORKLOADS["highres"].with_(B=2)):
+    # full-size stage3 needs the most scratch of the named workloads (2 * 64 * 49 * 256 * 4 = 6.4 MB)
+    for w in (WIDE, WORKLOADS["stage1"].with_(B=16), WIDE_F32, WORKLOADS["highres"].with_(B=2), WORKLOADS["stage3"],
+              WORKLOADS["highres"]):
         _, (q, k, _) = make(w)
         ref = bra.route(q, k, w.n_win, w.topk)
         idx = torch.full_like(ref, -7)
