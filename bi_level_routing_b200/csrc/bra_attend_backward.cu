@@ -536,6 +536,290 @@ __global__ void __launch_bounds__(kTiledThreads, 2) attend_backward_tiled_kernel
     }
 }
 
+// ------------------------------------------------------------------ tensor cores, bf16
+//
+// The same gradients for bf16 inputs of 64-token regions and 32-channel heads on mma.sync
+// (m16n8k16, fp32 accumulation), one CTA of 4 warps per (image, query region, head):
+//   S = Q K^T and dP = dout V^T take the bf16 inputs as they are (their products are exact in
+//   fp32); P and dS are fp32 and enter the three products that use them as two bf16 terms,
+//   x = hi + lo with hi = x with its low 16 bits cleared (exact) and lo = x - hi rounded to bf16,
+//   so that each such operand carries about 16 significant bits (relative error <= 2^-16)
+//   and every product is again exact in fp32:
+//   dQ = dS K          (A = dS from the S accumulators of the warp's 16 query rows, B = K),
+//   dV = P^T dout, dK = dS^T Q (A = P^T, dS^T read transposed from shared memory, B = dout, Q).
+// Warp w owns query rows 16w .. 16w+15 for S, dP and dQ, and key rows 16w .. 16w+15 of each
+// routed region for dK and dV. Row statistics (running max, sum, D = sum p dp) are quad
+// reductions; with one routed region the scores stay in registers between the passes.
+namespace {
+
+constexpr int kMmaBackWarps = 4;
+constexpr int kTileRow = 40;   // bf16 per row of a 64 x 32 tile (32 + 8: rows 80 bytes apart)
+constexpr int kPRow = 72;      // bf16 per row of a 64 x 64 tile of p or ds (64 + 8)
+constexpr size_t kMmaBackSmem = sizeof(__nv_bfloat16) * (4 * 64 * kTileRow + 4 * 64 * kPRow) + 16 * sizeof(int);
+
+__device__ __forceinline__ void split_pack(float x0, float x1, uint32_t &hi, uint32_t &lo)
+{
+    const float h0 = bf16_trunc(x0), h1 = bf16_trunc(x1);
+    hi = pack_bf16x2_trunc(h0, h1);
+    lo = pack_bf16x2(x0 - h0, x1 - h1);
+}
+
+__device__ __forceinline__ float quad_max_b(float x)
+{
+    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
+    return fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
+}
+
+__device__ __forceinline__ float quad_sum_b(float x)
+{
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    return x + __shfl_xor_sync(0xffffffffu, x, 2);
+}
+
+// One 64-token x 32-channel bf16 head tile of the region at (y0, x0), channel offset c0, into
+// shared memory rows of kTileRow bf16 (16-byte vectors, all threads).
+__device__ __forceinline__ void stage_bf16_tile(const __nv_bfloat16 *g, const BackArgs &a, int64_t b, int y0, int x0,
+                                                int c0, __nv_bfloat16 *dst)
+{
+    for (int e = threadIdx.x; e < 64 * 4; e += 32 * kMmaBackWarps) {
+        const int row = e >> 2, u = e & 3;
+        const int y = y0 + row / a.wr, x = x0 + row % a.wr;
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(g + ((b * a.H + y) * a.W + x) * a.C + c0 + 8 * u));
+        *reinterpret_cast<uint4 *>(dst + row * kTileRow + 8 * u) = v;
+    }
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(32 * kMmaBackWarps) attend_backward_mma_kernel(const BackArgs a)
+{
+    extern __shared__ float4 smem4[];
+    __nv_bfloat16 *sQ = reinterpret_cast<__nv_bfloat16 *>(smem4);  // [64][kTileRow]
+    __nv_bfloat16 *sD = sQ + 64 * kTileRow;                         // dout
+    __nv_bfloat16 *sK = sD + 64 * kTileRow;                         // k of the routed region
+    __nv_bfloat16 *sV = sK + 64 * kTileRow;                         // v of the routed region
+    __nv_bfloat16 *sPh = sV + 64 * kTileRow;                        // [64 queries][kPRow] p, high part
+    __nv_bfloat16 *sPl = sPh + 64 * kPRow;                          // p, low part
+    __nv_bfloat16 *sSh = sPl + 64 * kPRow;                          // ds, high part
+    __nv_bfloat16 *sSl = sSh + 64 * kPRow;                          // ds, low part
+    int *sreg = reinterpret_cast<int *>(sSl + 64 * kPRow);
+
+    int64_t blk = blockIdx.x;
+    const int h = (int)(blk % a.heads);
+    blk /= a.heads;
+    const int r = (int)(blk % a.R);
+    const int64_t b = blk / a.R;
+    const int ry = r / a.n_win, rx = r - ry * a.n_win;
+    const int c0 = h * 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const __nv_bfloat16 *gq = static_cast<const __nv_bfloat16 *>(a.q), *gk = static_cast<const __nv_bfloat16 *>(a.k);
+    const __nv_bfloat16 *gv = static_cast<const __nv_bfloat16 *>(a.v), *gd = static_cast<const __nv_bfloat16 *>(a.dout);
+    grid_dependency_wait();
+
+    stage_bf16_tile(gq, a, b, ry * a.hr, rx * a.wr, c0, sQ);
+    stage_bf16_tile(gd, a, b, ry * a.hr, rx * a.wr, c0, sD);
+    if (threadIdx.x < 16 && threadIdx.x < a.topk) sreg[threadIdx.x] = a.idx[(b * a.R + r) * a.topk + threadIdx.x];
+    if (h == 0 && threadIdx.x == 0)
+        for (int j = 0; j < a.topk; ++j) {
+            const int s = a.idx[(b * a.R + r) * a.topk + j];
+            if (s < 0 || s >= a.R) flag_error(a.err, kErrIndex);
+        }
+    __syncthreads();
+    auto region = [&](int j) -> int {
+        const int s = j < 16 ? sreg[j] : a.idx[(b * a.R + r) * a.topk + j];
+        return (s >= 0 && s < a.R) ? s : -1;
+    };
+
+    // A fragments of this warp's 16 query rows of q and dout (two 16-channel steps each)
+    const uint32_t q0 = smem_u32(sQ), d0 = smem_u32(sD), k0 = smem_u32(sK), v0 = smem_u32(sV);
+    uint32_t qf[2][4], df[2][4];
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        const uint32_t off = (uint32_t)((16 * warp + (lane & 15)) * kTileRow + 16 * ks + 8 * (lane >> 4)) * 2u;
+        ldmatrix_x4(q0 + off, qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+        ldmatrix_x4(d0 + off, df[ks][0], df[ks][1], df[ks][2], df[ks][3]);
+    }
+
+    // S and dP of the warp's rows against the staged region: 8 key tiles of 8
+    float sc[8][4], dp[8][4];
+    auto scores = [&]() {
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+            dp[nt][0] = dp[nt][1] = dp[nt][2] = dp[nt][3] = 0.f;
+            const uint32_t off = (uint32_t)((8 * nt + (lane & 7)) * kTileRow + 8 * (lane >> 3)) * 2u;
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4(k0 + off, b0, b1, b2, b3);
+            mma_bf16_16816(sc[nt], qf[0], b0, b1);
+            mma_bf16_16816(sc[nt], qf[1], b2, b3);
+            ldmatrix_x4(v0 + off, b0, b1, b2, b3);
+            mma_bf16_16816(dp[nt], df[0], b0, b1);
+            mma_bf16_16816(dp[nt], df[1], b2, b3);
+        }
+    };
+    auto stage_kv = [&](int s) {
+        const int sy = (s / a.n_win) * a.hr, sx = (s % a.n_win) * a.wr;
+        stage_bf16_tile(gk, a, b, sy, sx, c0, sK);
+        stage_bf16_tile(gv, a, b, sy, sx, c0, sV);
+    };
+
+    // pass 1: running max, sum and sum e (dout . v) of rows g and g + 8
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, dsum[2] = {0.f, 0.f};
+    int staged = -1;
+    for (int j = 0; j < a.topk; ++j) {
+        const int s = region(j);
+        if (s < 0) continue;
+        __syncthreads();
+        stage_kv(s);
+        staged = j;
+        __syncthreads();
+        scores();
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) mx = fmaxf(mx, fmaxf(sc[nt][2 * hh], sc[nt][2 * hh + 1]));
+            const float mn = fmaxf(m[hh], quad_max_b(mx) * a.scale_log2);
+            const float corr = fast_exp2(m[hh] - mn);
+            float es = 0.f, eds = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float e = fast_exp2(fmaf(sc[nt][2 * hh + i], a.scale_log2, -mn));
+                    es += e;
+                    eds = fmaf(e, dp[nt][2 * hh + i], eds);
+                }
+            l[hh] = l[hh] * corr + quad_sum_b(es);
+            dsum[hh] = dsum[hh] * corr + quad_sum_b(eds);
+            m[hh] = mn;
+        }
+    }
+    float inv_l[2], D[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        inv_l[hh] = l[hh] > 0.f ? 1.f / l[hh] : 0.f;
+        D[hh] = dsum[hh] * inv_l[hh];
+    }
+
+    // pass 2: p and ds per routed region; dq in registers, dk and dv added per region
+    float dq[4][4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) dq[nt][0] = dq[nt][1] = dq[nt][2] = dq[nt][3] = 0.f;
+    for (int j = 0; j < a.topk; ++j) {
+        const int s = region(j);
+        if (s < 0) continue;
+        if (staged != j) {
+            __syncthreads();
+            stage_kv(s);
+            __syncthreads();
+            scores();
+        }
+        staged = -1;
+        // p and ds in place of the scores; their bf16 high and low parts to shared memory
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int hh = i >> 1;
+                const float p = fast_exp2(fmaf(sc[nt][i], a.scale_log2, -m[hh])) * inv_l[hh];
+                sc[nt][i] = p;
+                dp[nt][i] = p * (dp[nt][i] - D[hh]);
+            }
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = 16 * warp + g + 8 * hh, col = 8 * nt + 2 * t;
+                uint32_t hi, lo;
+                split_pack(sc[nt][2 * hh], sc[nt][2 * hh + 1], hi, lo);
+                *reinterpret_cast<uint32_t *>(sPh + row * kPRow + col) = hi;
+                *reinterpret_cast<uint32_t *>(sPl + row * kPRow + col) = lo;
+                split_pack(dp[nt][2 * hh], dp[nt][2 * hh + 1], hi, lo);
+                *reinterpret_cast<uint32_t *>(sSh + row * kPRow + col) = hi;
+                *reinterpret_cast<uint32_t *>(sSl + row * kPRow + col) = lo;
+            }
+        // dQ += dS K: A = ds of the warp's rows (registers, high then low part), B = K by rows
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t ah[4], al[4];
+            split_pack(dp[2 * kk][0], dp[2 * kk][1], ah[0], al[0]);
+            split_pack(dp[2 * kk][2], dp[2 * kk][3], ah[1], al[1]);
+            split_pack(dp[2 * kk + 1][0], dp[2 * kk + 1][1], ah[2], al[2]);
+            split_pack(dp[2 * kk + 1][2], dp[2 * kk + 1][3], ah[3], al[3]);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                const int row = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4_trans(k0 + (uint32_t)(row * kTileRow + 16 * np + 8 * (lane >> 4)) * 2u, b0, b1, b2, b3);
+                mma_bf16_16816(dq[2 * np], al, b0, b1);
+                mma_bf16_16816(dq[2 * np + 1], al, b2, b3);
+                mma_bf16_16816(dq[2 * np], ah, b0, b1);
+                mma_bf16_16816(dq[2 * np + 1], ah, b2, b3);
+            }
+        }
+        __syncthreads();  // p and ds of every warp in shared memory
+        // dV = P^T dout and dK = dS^T Q for the warp's 16 keys: A read transposed, B by rows
+        float gk4[4][4], gv4[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) gk4[nt][i] = gv4[nt][i] = 0.f;
+        const int mrow = (lane >> 4) & 1, mcol = (lane >> 3) & 1;  // which 8 x 8 of the 16 x 16 A tile
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // 16 queries per step
+            const uint32_t aoff = (uint32_t)((16 * kk + (lane & 7) + 8 * mrow) * kPRow + 16 * warp + 8 * mcol) * 2u;
+            uint32_t ph[4], pl[4], sh[4], sl[4];
+            ldmatrix_x4_trans(smem_u32(sPh) + aoff, ph[0], ph[1], ph[2], ph[3]);
+            ldmatrix_x4_trans(smem_u32(sPl) + aoff, pl[0], pl[1], pl[2], pl[3]);
+            ldmatrix_x4_trans(smem_u32(sSh) + aoff, sh[0], sh[1], sh[2], sh[3]);
+            ldmatrix_x4_trans(smem_u32(sSl) + aoff, sl[0], sl[1], sl[2], sl[3]);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                const int row = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const uint32_t boff = (uint32_t)(row * kTileRow + 16 * np + 8 * (lane >> 4)) * 2u;
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4_trans(d0 + boff, b0, b1, b2, b3);
+                mma_bf16_16816(gv4[2 * np], pl, b0, b1);
+                mma_bf16_16816(gv4[2 * np + 1], pl, b2, b3);
+                mma_bf16_16816(gv4[2 * np], ph, b0, b1);
+                mma_bf16_16816(gv4[2 * np + 1], ph, b2, b3);
+                ldmatrix_x4_trans(q0 + boff, b0, b1, b2, b3);
+                mma_bf16_16816(gk4[2 * np], sl, b0, b1);
+                mma_bf16_16816(gk4[2 * np + 1], sl, b2, b3);
+                mma_bf16_16816(gk4[2 * np], sh, b0, b1);
+                mma_bf16_16816(gk4[2 * np + 1], sh, b2, b3);
+            }
+        }
+        const int sy = (s / a.n_win) * a.hr, sx = (s % a.n_win) * a.wr;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int key = 16 * warp + g + 8 * hh;
+            const int y = sy + key / a.wr, x = sx + key % a.wr;
+            const int64_t off = ((b * a.H + y) * a.W + x) * a.C + c0 + 2 * t;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                atomicAdd(reinterpret_cast<float2 *>(a.dk + off + 8 * nt),
+                          make_float2(gk4[nt][2 * hh] * a.scale, gk4[nt][2 * hh + 1] * a.scale));
+                atomicAdd(reinterpret_cast<float2 *>(a.dv + off + 8 * nt),
+                          make_float2(gv4[nt][2 * hh], gv4[nt][2 * hh + 1]));
+            }
+        }
+        __syncthreads();  // p and ds are rewritten by the next region
+    }
+    const int y0 = ry * a.hr, x0 = rx * a.wr;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const int row = 16 * warp + g + 8 * hh;
+        const int y = y0 + row / a.wr, x = x0 + row % a.wr;
+        float *dst = a.dq + ((b * a.H + y) * a.W + x) * a.C + c0 + 2 * t;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+            *reinterpret_cast<float2 *>(dst + 8 * nt) = make_float2(dq[nt][2 * hh] * a.scale, dq[nt][2 * hh + 1] * a.scale);
+    }
+}
+
 namespace {
 
 constexpr size_t kBackMaxSmem = 100 * 1024;
@@ -583,8 +867,29 @@ cudaError_t launch_attend_backward(const void *q, const void *k, const void *v, 
     a.topk = g.topk;
     a.scale = (float)(1.0 / sqrt((double)g.hd));
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)g.hd));
+    if (g.rs == 64 && g.hd == 32 && bf16) {
+        // 64-token regions, heads of 32 channels, bf16: the tensor-core kernel
+        const long long blocks = (long long)g.B * g.R * g.heads;
+        if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+        const size_t bytes = (size_t)g.B * g.H * g.W * g.C * sizeof(float);
+        cudaError_t e = cudaMemsetAsync(dk, 0, bytes, stream);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, bytes, stream);
+        if (e != cudaSuccess) return e;
+        static int granted_mma[64] = {0};
+        int dev = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+        if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+        if ((int)kMmaBackSmem > 48 * 1024 && (int)kMmaBackSmem > granted_mma[dev]) {
+            if ((e = cudaFuncSetAttribute(attend_backward_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)kMmaBackSmem)) != cudaSuccess)
+                return e;
+            granted_mma[dev] = (int)kMmaBackSmem;
+        }
+        return launch_pdl(attend_backward_mma_kernel, dim3((unsigned)blocks), dim3(32 * kMmaBackWarps), kMmaBackSmem,
+                          stream, a);
+    }
     if (g.rs == 64 && g.hd == 32) {
-        // 64-token regions, heads of 32 channels: the register-tiled kernel
+        // 64-token regions, heads of 32 channels, fp32: the register-tiled kernel
         const long long blocks = (long long)g.B * g.R * g.heads;
         if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
         const size_t bytes = (size_t)g.B * g.H * g.W * g.C * sizeof(float);
