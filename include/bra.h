@@ -190,8 +190,10 @@ bra_status bra_forward_lepe(const void *q, const void *k, const void *v, int32_t
    with respect to q, k and v. q, k, v, dout: device [B, H, W, C] of dtype; idx: device int32
    [B, n_win^2, topk] (out-of-range entries skipped and flagged); dq, dk, dv: device fp32
    [B, H, W, C], written (dk and dv are cleared first, then accumulated with atomics, so their
-   last bits may differ between runs). BRA_ERR_UNSUPPORTED: hd % 8 != 0, hd > 128, or a region of
-   more than 256 tokens. */
+   last bits may differ between runs). bf16 with 64-token regions and 32-channel heads runs on the
+   tensor cores (the bf16 inputs as they are, p and ds as two bf16 terms each: about 16
+   significant bits, products exact, fp32 sums); everything else on CUDA cores in fp32.
+   BRA_ERR_UNSUPPORTED: hd % 8 != 0, hd > 128, or a region of more than 256 tokens. */
 bra_status bra_attend_backward(const void *q, const void *k, const void *v, const int32_t *idx, const void *dout,
                                float *dq, float *dk, float *dv, int B, int H, int W, int C, int heads, int n_win,
                                int topk, bra_dtype dtype, void *stream);
