@@ -139,6 +139,12 @@ def test_scratch_and_launch_accounting(L):
         assert L.bra_kernels_per_call(b"bra_forward", *stage4) == 2
     finally:
         L.bra_set_attend_kernel(0)
+    # the fused kernel's limits: a cluster of at most 8 CTAs (C <= 1024 with two 64-channel blocks
+    # per CTA, an odd block count one per CTA up to 8 blocks), at most 64 one-token regions
+    assert L.bra_kernels_per_call(b"bra_forward", 2, 5, 5, 1024, 32, 5, 25, 1) == 1
+    assert L.bra_kernels_per_call(b"bra_forward", 2, 7, 7, 448, 14, 7, 7, 1) == 1   # 7 blocks, cluster of 7
+    assert L.bra_kernels_per_call(b"bra_forward", 2, 7, 7, 576, 18, 7, 7, 1) == 2   # 9 blocks: unfused
+    assert L.bra_kernels_per_call(b"bra_forward", 2, 9, 9, 64, 2, 9, 9, 1) == 2     # R = 81: unfused
     assert L.bra_route_scratch_bytes(64, 7, 7, 512, 7) == 0
     assert L.bra_kernels_per_call(b"nonsense", *stage1) == 0
 
