@@ -30,6 +30,7 @@ struct BackArgs {
     int H, W, C, heads, hd, n_win, hr, wr, rs, R, topk;
     int hpc;     // heads per CTA
     int kcr;     // routed regions per key chunk
+    int nitems;  // (image, region, head) items of the persistent tensor-core kernel
     float scale;       // hd^-1/2
     float scale_log2;  // hd^-1/2 log2(e)
 };
@@ -539,14 +540,19 @@ __global__ void __launch_bounds__(kTiledThreads, 2) attend_backward_tiled_kernel
 // ------------------------------------------------------------------ tensor cores, bf16
 //
 // The same gradients for bf16 inputs of 64-token regions and 32-channel heads on mma.sync
-// (m16n8k16, fp32 accumulation), one CTA of 4 warps per (image, query region, head):
+// (m16n8k16, fp32 accumulation), a persistent grid of CTAs of 4 warps, each taking (image, query
+// region, head) items in turn:
 //   S = Q K^T and dP = dout V^T take the bf16 inputs as they are (their products are exact in
 //   fp32); P and dS are fp32 and enter the three products that use them as two bf16 terms,
 //   x = hi + lo with hi = x with its low 16 bits cleared (exact) and lo = x - hi rounded to bf16,
 //   so that each such operand carries about 16 significant bits (relative error <= 2^-16)
 //   and every product is again exact in fp32:
-//   dQ = dS K          (A = dS from the S accumulators of the warp's 16 query rows, B = K),
-//   dV = P^T dout, dK = dS^T Q (A = P^T, dS^T read transposed from shared memory, B = dout, Q).
+//   dQ = dS K          (A = the warp's 16 query rows of dS, B = K),
+//   dK = dS^T Q, dV = P^T dout (A = dS^T, P^T read transposed from shared memory, B = Q, dout).
+// ds and then p pass through one pair of shared arrays (high and low part) and dq accumulates
+// in shared memory. The next item's q and dout tiles, and k and v of its first routed region,
+// arrive by cp.async in a second set of tiles while the CTA works on the current item, so that
+// the loads' latency is hidden; with the two sets a CTA needs 68 KB, and three share an SM.
 // Warp w owns query rows 16w .. 16w+15 for S, dP and dQ, and key rows 16w .. 16w+15 of each
 // routed region for dK and dV. Row statistics (running max, sum, D = sum p dp) are quad
 // reductions; with one routed region the scores stay in registers between the passes.
@@ -555,7 +561,10 @@ namespace {
 constexpr int kMmaBackWarps = 4;
 constexpr int kTileRow = 40;   // bf16 per row of a 64 x 32 tile (32 + 8: rows 80 bytes apart)
 constexpr int kPRow = 72;      // bf16 per row of a 64 x 64 tile of p or ds (64 + 8)
-constexpr size_t kMmaBackSmem = sizeof(__nv_bfloat16) * (4 * 64 * kTileRow + 4 * 64 * kPRow) + 16 * sizeof(int);
+constexpr int kDqRow = 40;     // fp32 per row of the 64 x 32 dq accumulator (32 + 8)
+constexpr int kMmaBackCtasPerSm = 3;
+constexpr size_t kMmaBackSmem = sizeof(__nv_bfloat16) * (2 * 4 * 64 * kTileRow + 2 * 64 * kPRow) +
+                                sizeof(float) * 64 * kDqRow + 2 * 16 * sizeof(int);
 
 __device__ __forceinline__ void split_pack(float x0, float x1, uint32_t &hi, uint32_t &lo)
 {
@@ -589,234 +598,316 @@ __device__ __forceinline__ void stage_bf16_tile(const __nv_bfloat16 *g, const Ba
     }
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// The same tile as stage_bf16_tile, by asynchronous copies that land while the CTA computes
+__device__ __forceinline__ void fetch_bf16_tile(const __nv_bfloat16 *g, const BackArgs &a, int64_t b, int y0, int x0,
+                                                int c0, __nv_bfloat16 *dst)
+{
+    for (int e = threadIdx.x; e < 64 * 4; e += 32 * kMmaBackWarps) {
+        const int row = e >> 2, u = e & 3;
+        const int y = y0 + row / a.wr, x = x0 + row % a.wr;
+        cp_async16(smem_u32(dst + row * kTileRow + 8 * u), g + ((b * a.H + y) * a.W + x) * a.C + c0 + 8 * u);
+    }
+}
+
 }  // namespace
 
-__global__ void __launch_bounds__(32 * kMmaBackWarps) attend_backward_mma_kernel(const BackArgs a)
+__global__ void __launch_bounds__(32 * kMmaBackWarps, kMmaBackCtasPerSm) attend_backward_mma_kernel(const BackArgs a)
 {
     extern __shared__ float4 smem4[];
-    __nv_bfloat16 *sQ = reinterpret_cast<__nv_bfloat16 *>(smem4);  // [64][kTileRow]
-    __nv_bfloat16 *sD = sQ + 64 * kTileRow;                         // dout
-    __nv_bfloat16 *sK = sD + 64 * kTileRow;                         // k of the routed region
-    __nv_bfloat16 *sV = sK + 64 * kTileRow;                         // v of the routed region
-    __nv_bfloat16 *sPh = sV + 64 * kTileRow;                        // [64 queries][kPRow] p, high part
-    __nv_bfloat16 *sPl = sPh + 64 * kPRow;                          // p, low part
-    __nv_bfloat16 *sSh = sPl + 64 * kPRow;                          // ds, high part
-    __nv_bfloat16 *sSl = sSh + 64 * kPRow;                          // ds, low part
-    int *sreg = reinterpret_cast<int *>(sSl + 64 * kPRow);
+    // two sets of [q, dout, k, v] tiles of [64][kTileRow]: the CTA works on one item while the
+    // next item's tiles land in the other
+    __nv_bfloat16 *tiles = reinterpret_cast<__nv_bfloat16 *>(smem4);
+    __nv_bfloat16 *sPh = tiles + 8 * 64 * kTileRow;                 // [64 queries][kPRow] ds, then p: high part
+    __nv_bfloat16 *sPl = sPh + 64 * kPRow;                          // low part
+    float *sDq = reinterpret_cast<float *>(sPl + 64 * kPRow);       // [64 queries][kDqRow] dq accumulator
+    int *sregs = reinterpret_cast<int *>(sDq + 64 * kDqRow);        // [2][16] routed regions of each set's item
 
-    int64_t blk = blockIdx.x;
-    const int h = (int)(blk % a.heads);
-    blk /= a.heads;
-    const int r = (int)(blk % a.R);
-    const int64_t b = blk / a.R;
-    const int ry = r / a.n_win, rx = r - ry * a.n_win;
-    const int c0 = h * 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
+    float *const dq_own = sDq + (16 * warp + g) * kDqRow + 2 * t;  // this thread's dq: rows g, g + 8
     const __nv_bfloat16 *gq = static_cast<const __nv_bfloat16 *>(a.q), *gk = static_cast<const __nv_bfloat16 *>(a.k);
     const __nv_bfloat16 *gv = static_cast<const __nv_bfloat16 *>(a.v), *gd = static_cast<const __nv_bfloat16 *>(a.dout);
+    // item = (image b, query region r, head h), heads fastest; its index row is item / heads
+    auto fetch_qd = [&](int item, int set) {
+        const int h = item % a.heads, r = (item / a.heads) % a.R;
+        const int64_t b = (item / a.heads) / a.R;
+        const int ry = r / a.n_win, rx = r - ry * a.n_win;
+        __nv_bfloat16 *base = tiles + set * 4 * 64 * kTileRow;
+        fetch_bf16_tile(gq, a, b, ry * a.hr, rx * a.wr, h * 32, base);
+        fetch_bf16_tile(gd, a, b, ry * a.hr, rx * a.wr, h * 32, base + 64 * kTileRow);
+    };
+    auto fetch_kv = [&](int item, int s, int set) {
+        const int h = item % a.heads;
+        const int64_t b = (item / a.heads) / a.R;
+        __nv_bfloat16 *base = tiles + set * 4 * 64 * kTileRow + 2 * 64 * kTileRow;
+        fetch_bf16_tile(gk, a, b, (s / a.n_win) * a.hr, (s % a.n_win) * a.wr, h * 32, base);
+        fetch_bf16_tile(gv, a, b, (s / a.n_win) * a.hr, (s % a.n_win) * a.wr, h * 32, base + 64 * kTileRow);
+    };
+    auto idx_at = [&](int item, int j) -> int { return __ldg(a.idx + (int64_t)(item / a.heads) * a.topk + j); };
     grid_dependency_wait();
 
-    stage_bf16_tile(gq, a, b, ry * a.hr, rx * a.wr, c0, sQ);
-    stage_bf16_tile(gd, a, b, ry * a.hr, rx * a.wr, c0, sD);
-    if (threadIdx.x < 16 && threadIdx.x < a.topk) sreg[threadIdx.x] = a.idx[(b * a.R + r) * a.topk + threadIdx.x];
-    if (h == 0 && threadIdx.x == 0)
-        for (int j = 0; j < a.topk; ++j) {
-            const int s = a.idx[(b * a.R + r) * a.topk + j];
-            if (s < 0 || s >= a.R) flag_error(a.err, kErrIndex);
-        }
-    __syncthreads();
-    auto region = [&](int j) -> int {
-        const int s = j < 16 ? sreg[j] : a.idx[(b * a.R + r) * a.topk + j];
-        return (s >= 0 && s < a.R) ? s : -1;
-    };
-
-    // A fragments of this warp's 16 query rows of q and dout (two 16-channel steps each)
-    const uint32_t q0 = smem_u32(sQ), d0 = smem_u32(sD), k0 = smem_u32(sK), v0 = smem_u32(sV);
-    uint32_t qf[2][4], df[2][4];
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-        const uint32_t off = (uint32_t)((16 * warp + (lane & 15)) * kTileRow + 16 * ks + 8 * (lane >> 4)) * 2u;
-        ldmatrix_x4(q0 + off, qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
-        ldmatrix_x4(d0 + off, df[ks][0], df[ks][1], df[ks][2], df[ks][3]);
+    int item = blockIdx.x;
+    if (item >= a.nitems) return;
+    {  // the first item: its tiles into set 0 (k and v of its first routed region, when valid)
+        const int s0 = idx_at(item, 0);
+        if (threadIdx.x < 16 && threadIdx.x < a.topk) sregs[threadIdx.x] = idx_at(item, threadIdx.x);
+        fetch_qd(item, 0);
+        if (s0 >= 0 && s0 < a.R) fetch_kv(item, s0, 0);
+        cp_async_commit();
     }
-
-    // S and dP of the warp's rows against the staged region: 8 key tiles of 8
-    float sc[8][4], dp[8][4];
-    auto scores = [&]() {
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-            dp[nt][0] = dp[nt][1] = dp[nt][2] = dp[nt][3] = 0.f;
-            const uint32_t off = (uint32_t)((8 * nt + (lane & 7)) * kTileRow + 8 * (lane >> 3)) * 2u;
-            uint32_t b0, b1, b2, b3;
-            ldmatrix_x4(k0 + off, b0, b1, b2, b3);
-            mma_bf16_16816(sc[nt], qf[0], b0, b1);
-            mma_bf16_16816(sc[nt], qf[1], b2, b3);
-            ldmatrix_x4(v0 + off, b0, b1, b2, b3);
-            mma_bf16_16816(dp[nt], df[0], b0, b1);
-            mma_bf16_16816(dp[nt], df[1], b2, b3);
+    for (int cur = 0;; cur ^= 1) {
+        const int64_t next64 = (int64_t)item + gridDim.x;
+        const bool has_next = next64 < a.nitems;
+        const int next = has_next ? (int)next64 : 0;
+        // the next item's index entries: loaded now, used once pass 1 is done
+        int s_next = -1, reg_next = 0;
+        if (has_next) {
+            s_next = idx_at(next, 0);
+            if (threadIdx.x < 16 && threadIdx.x < a.topk) reg_next = idx_at(next, threadIdx.x);
         }
-    };
-    auto stage_kv = [&](int s) {
-        const int sy = (s / a.n_win) * a.hr, sx = (s % a.n_win) * a.wr;
-        stage_bf16_tile(gk, a, b, sy, sx, c0, sK);
-        stage_bf16_tile(gv, a, b, sy, sx, c0, sV);
-    };
+        cp_async_wait_all();
+        __syncthreads();  // this item's tiles are in place; the other set is free
+        if (has_next) fetch_qd(next, cur ^ 1);
+        cp_async_commit();
 
-    // pass 1: running max, sum and sum e (dout . v) of rows g and g + 8
-    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, dsum[2] = {0.f, 0.f};
-    int staged = -1;
-    for (int j = 0; j < a.topk; ++j) {
-        const int s = region(j);
-        if (s < 0) continue;
-        __syncthreads();
-        stage_kv(s);
-        staged = j;
-        __syncthreads();
-        scores();
+        const int h = item % a.heads;
+        const int r = (item / a.heads) % a.R;
+        const int64_t b = (item / a.heads) / a.R;
+        const int ry = r / a.n_win, rx = r - ry * a.n_win;
+        const int c0 = h * 32;
+        const int *sreg = sregs + 16 * cur;
+        __nv_bfloat16 *sQ = tiles + cur * 4 * 64 * kTileRow;
+        __nv_bfloat16 *sD = sQ + 64 * kTileRow, *sK = sD + 64 * kTileRow, *sV = sK + 64 * kTileRow;
+        if (h == 0 && threadIdx.x == 0)
+            for (int j = 0; j < a.topk; ++j) {
+                const int s = j < 16 ? sreg[j] : a.idx[(b * a.R + r) * a.topk + j];
+                if (s < 0 || s >= a.R) flag_error(a.err, kErrIndex);
+            }
+        auto region = [&](int j) -> int {
+            const int s = j < 16 ? sreg[j] : a.idx[(b * a.R + r) * a.topk + j];
+            return (s >= 0 && s < a.R) ? s : -1;
+        };
+
+        // shared-memory addresses of the tiles; the A fragments of q and dout are read per score pass
+        const uint32_t q0 = smem_u32(sQ), d0 = smem_u32(sD), k0 = smem_u32(sK), v0 = smem_u32(sV);
+
+        // S and dP of the warp's rows against the staged region: 8 key tiles of 8
+        float sc[8][4], dp[8][4];
+        auto scores = [&]() {
+            uint32_t qf[2][4], df[2][4];
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+                const uint32_t off = (uint32_t)((16 * warp + (lane & 15)) * kTileRow + 16 * ks + 8 * (lane >> 4)) * 2u;
+                ldmatrix_x4(q0 + off, qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+                ldmatrix_x4(d0 + off, df[ks][0], df[ks][1], df[ks][2], df[ks][3]);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+                dp[nt][0] = dp[nt][1] = dp[nt][2] = dp[nt][3] = 0.f;
+                const uint32_t off = (uint32_t)((8 * nt + (lane & 7)) * kTileRow + 8 * (lane >> 3)) * 2u;
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4(k0 + off, b0, b1, b2, b3);
+                mma_bf16_16816(sc[nt], qf[0], b0, b1);
+                mma_bf16_16816(sc[nt], qf[1], b2, b3);
+                ldmatrix_x4(v0 + off, b0, b1, b2, b3);
+                mma_bf16_16816(dp[nt], df[0], b0, b1);
+                mma_bf16_16816(dp[nt], df[1], b2, b3);
+            }
+        };
+        auto stage_kv = [&](int s) {
+            const int sy = (s / a.n_win) * a.hr, sx = (s % a.n_win) * a.wr;
+            stage_bf16_tile(gk, a, b, sy, sx, c0, sK);
+            stage_bf16_tile(gv, a, b, sy, sx, c0, sV);
+        };
+
+        // pass 1: running max, sum and sum e (dout . v) of rows g and g + 8
+        float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, dsum[2] = {0.f, 0.f};
+        int staged = -1;
+        for (int j = 0; j < a.topk; ++j) {
+            const int s = region(j);
+            if (s < 0) continue;
+            if (j != 0) {  // the first routed region came with the item's tiles
+                __syncthreads();
+                stage_kv(s);
+                __syncthreads();
+            }
+            staged = j;
+            scores();
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float mx = -INFINITY;
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt) mx = fmaxf(mx, fmaxf(sc[nt][2 * hh], sc[nt][2 * hh + 1]));
+                const float mn = fmaxf(m[hh], quad_max_b(mx) * a.scale_log2);
+                const float corr = fast_exp2(m[hh] - mn);
+                float es = 0.f, eds = 0.f;
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const float e = fast_exp2(fmaf(sc[nt][2 * hh + i], a.scale_log2, -mn));
+                        es += e;
+                        eds = fmaf(e, dp[nt][2 * hh + i], eds);
+                    }
+                l[hh] = l[hh] * corr + quad_sum_b(es);
+                dsum[hh] = dsum[hh] * corr + quad_sum_b(eds);
+                m[hh] = mn;
+            }
+        }
+        // the next item's first routed region into the other set, and its index entries
+        if (has_next && s_next >= 0 && s_next < a.R) fetch_kv(next, s_next, cur ^ 1);
+        cp_async_commit();
+        if (has_next && threadIdx.x < 16 && threadIdx.x < a.topk) sregs[16 * (cur ^ 1) + threadIdx.x] = reg_next;
+        float inv_l[2], D[2];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-            float mx = -INFINITY;
+            inv_l[hh] = l[hh] > 0.f ? 1.f / l[hh] : 0.f;
+            D[hh] = dsum[hh] * inv_l[hh];
+        }
+
+        // pass 2: p and ds per routed region; dq in shared memory (each warp its own rows), dk and dv
+        // added per region
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt) mx = fmaxf(mx, fmaxf(sc[nt][2 * hh], sc[nt][2 * hh + 1]));
-            const float mn = fmaxf(m[hh], quad_max_b(mx) * a.scale_log2);
-            const float corr = fast_exp2(m[hh] - mn);
-            float es = 0.f, eds = 0.f;
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+                *reinterpret_cast<float2 *>(dq_own + 8 * hh * kDqRow + 8 * nt) = make_float2(0.f, 0.f);
+        for (int j = 0; j < a.topk; ++j) {
+            const int s = region(j);
+            if (s < 0) continue;
+            if (staged != j) {
+                __syncthreads();
+                stage_kv(s);
+                __syncthreads();
+                scores();
+            }
+            staged = -1;
+            // p and ds in place of the scores; their bf16 high and low parts to shared memory
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const float e = fast_exp2(fmaf(sc[nt][2 * hh + i], a.scale_log2, -mn));
-                    es += e;
-                    eds = fmaf(e, dp[nt][2 * hh + i], eds);
+                for (int i = 0; i < 4; ++i) {
+                    const int hh = i >> 1;
+                    const float p = fast_exp2(fmaf(sc[nt][i], a.scale_log2, -m[hh])) * inv_l[hh];
+                    sc[nt][i] = p;
+                    dp[nt][i] = p * (dp[nt][i] - D[hh]);
                 }
-            l[hh] = l[hh] * corr + quad_sum_b(es);
-            dsum[hh] = dsum[hh] * corr + quad_sum_b(eds);
-            m[hh] = mn;
-        }
-    }
-    float inv_l[2], D[2];
+            const int sy = (s / a.n_win) * a.hr, sx = (s % a.n_win) * a.wr;
+            const int mrow = (lane >> 4) & 1, mcol = (lane >> 3) & 1;  // which 8 x 8 of the 16 x 16 A tile
+            // ds, then p, through one pair of shared arrays (high and low part): dQ += dS K (A = the
+            // warp's own rows of ds), dK = dS^T Q, then dV = P^T dout
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        inv_l[hh] = l[hh] > 0.f ? 1.f / l[hh] : 0.f;
-        D[hh] = dsum[hh] * inv_l[hh];
-    }
-
-    // pass 2: p and ds per routed region; dq in registers, dk and dv added per region
-    float dq[4][4];
+            for (int pass = 0; pass < 2; ++pass) {
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) dq[nt][0] = dq[nt][1] = dq[nt][2] = dq[nt][3] = 0.f;
-    for (int j = 0; j < a.topk; ++j) {
-        const int s = region(j);
-        if (s < 0) continue;
-        if (staged != j) {
-            __syncthreads();
-            stage_kv(s);
-            __syncthreads();
-            scores();
-        }
-        staged = -1;
-        // p and ds in place of the scores; their bf16 high and low parts to shared memory
+                for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int row = 16 * warp + g + 8 * hh, col = 8 * nt + 2 * t;
+                        uint32_t hi, lo;
+                        if (pass == 0)
+                            split_pack(dp[nt][2 * hh], dp[nt][2 * hh + 1], hi, lo);
+                        else
+                            split_pack(sc[nt][2 * hh], sc[nt][2 * hh + 1], hi, lo);
+                        *reinterpret_cast<uint32_t *>(sPh + row * kPRow + col) = hi;
+                        *reinterpret_cast<uint32_t *>(sPl + row * kPRow + col) = lo;
+                    }
+                __syncthreads();
+                if (pass == 0) {
+                    float dq[4][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int hh = i >> 1;
-                const float p = fast_exp2(fmaf(sc[nt][i], a.scale_log2, -m[hh])) * inv_l[hh];
-                sc[nt][i] = p;
-                dp[nt][i] = p * (dp[nt][i] - D[hh]);
-            }
+                    for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
+                        for (int nt = 0; nt < 4; ++nt) {
+                            const float2 v2 = *reinterpret_cast<const float2 *>(dq_own + 8 * hh * kDqRow + 8 * nt);
+                            dq[nt][2 * hh] = v2.x;
+                            dq[nt][2 * hh + 1] = v2.y;
+                        }
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int row = 16 * warp + g + 8 * hh, col = 8 * nt + 2 * t;
-                uint32_t hi, lo;
-                split_pack(sc[nt][2 * hh], sc[nt][2 * hh + 1], hi, lo);
-                *reinterpret_cast<uint32_t *>(sPh + row * kPRow + col) = hi;
-                *reinterpret_cast<uint32_t *>(sPl + row * kPRow + col) = lo;
-                split_pack(dp[nt][2 * hh], dp[nt][2 * hh + 1], hi, lo);
-                *reinterpret_cast<uint32_t *>(sSh + row * kPRow + col) = hi;
-                *reinterpret_cast<uint32_t *>(sSl + row * kPRow + col) = lo;
-            }
-        // dQ += dS K: A = ds of the warp's rows (registers, high then low part), B = K by rows
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t aoff =
+                            (uint32_t)((16 * warp + (lane & 15)) * kPRow + 16 * kk + 8 * (lane >> 4)) * 2u;
+                        uint32_t ah[4], al[4];
+                        ldmatrix_x4(smem_u32(sPh) + aoff, ah[0], ah[1], ah[2], ah[3]);
+                        ldmatrix_x4(smem_u32(sPl) + aoff, al[0], al[1], al[2], al[3]);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            uint32_t ah[4], al[4];
-            split_pack(dp[2 * kk][0], dp[2 * kk][1], ah[0], al[0]);
-            split_pack(dp[2 * kk][2], dp[2 * kk][3], ah[1], al[1]);
-            split_pack(dp[2 * kk + 1][0], dp[2 * kk + 1][1], ah[2], al[2]);
-            split_pack(dp[2 * kk + 1][2], dp[2 * kk + 1][3], ah[3], al[3]);
+                        for (int np = 0; np < 2; ++np) {
+                            const int row = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+                            uint32_t b0, b1, b2, b3;
+                            ldmatrix_x4_trans(k0 + (uint32_t)(row * kTileRow + 16 * np + 8 * (lane >> 4)) * 2u,
+                                              b0, b1, b2, b3);
+                            mma_bf16_16816(dq[2 * np], al, b0, b1);
+                            mma_bf16_16816(dq[2 * np + 1], al, b2, b3);
+                            mma_bf16_16816(dq[2 * np], ah, b0, b1);
+                            mma_bf16_16816(dq[2 * np + 1], ah, b2, b3);
+                        }
+                    }
 #pragma unroll
-            for (int np = 0; np < 2; ++np) {
-                const int row = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
-                uint32_t b0, b1, b2, b3;
-                ldmatrix_x4_trans(k0 + (uint32_t)(row * kTileRow + 16 * np + 8 * (lane >> 4)) * 2u, b0, b1, b2, b3);
-                mma_bf16_16816(dq[2 * np], al, b0, b1);
-                mma_bf16_16816(dq[2 * np + 1], al, b2, b3);
-                mma_bf16_16816(dq[2 * np], ah, b0, b1);
-                mma_bf16_16816(dq[2 * np + 1], ah, b2, b3);
-            }
-        }
-        __syncthreads();  // p and ds of every warp in shared memory
-        // dV = P^T dout and dK = dS^T Q for the warp's 16 keys: A read transposed, B by rows
-        float gk4[4][4], gv4[4][4];
+                    for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+                        for (int nt = 0; nt < 4; ++nt)
+                            *reinterpret_cast<float2 *>(dq_own + 8 * hh * kDqRow + 8 * nt) =
+                                make_float2(dq[nt][2 * hh], dq[nt][2 * hh + 1]);
+                }
+                float g4[4][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) gk4[nt][i] = gv4[nt][i] = 0.f;
-        const int mrow = (lane >> 4) & 1, mcol = (lane >> 3) & 1;  // which 8 x 8 of the 16 x 16 A tile
+                for (int nt = 0; nt < 4; ++nt) g4[nt][0] = g4[nt][1] = g4[nt][2] = g4[nt][3] = 0.f;
+                const uint32_t bbase = pass == 0 ? q0 : d0;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {  // 16 queries per step
-            const uint32_t aoff = (uint32_t)((16 * kk + (lane & 7) + 8 * mrow) * kPRow + 16 * warp + 8 * mcol) * 2u;
-            uint32_t ph[4], pl[4], sh[4], sl[4];
-            ldmatrix_x4_trans(smem_u32(sPh) + aoff, ph[0], ph[1], ph[2], ph[3]);
-            ldmatrix_x4_trans(smem_u32(sPl) + aoff, pl[0], pl[1], pl[2], pl[3]);
-            ldmatrix_x4_trans(smem_u32(sSh) + aoff, sh[0], sh[1], sh[2], sh[3]);
-            ldmatrix_x4_trans(smem_u32(sSl) + aoff, sl[0], sl[1], sl[2], sl[3]);
+                for (int kk = 0; kk < 4; ++kk) {  // 16 queries per step
+                    const uint32_t aoff =
+                        (uint32_t)((16 * kk + (lane & 7) + 8 * mrow) * kPRow + 16 * warp + 8 * mcol) * 2u;
+                    uint32_t ah[4], al[4];
+                    ldmatrix_x4_trans(smem_u32(sPh) + aoff, ah[0], ah[1], ah[2], ah[3]);
+                    ldmatrix_x4_trans(smem_u32(sPl) + aoff, al[0], al[1], al[2], al[3]);
 #pragma unroll
-            for (int np = 0; np < 2; ++np) {
-                const int row = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
-                const uint32_t boff = (uint32_t)(row * kTileRow + 16 * np + 8 * (lane >> 4)) * 2u;
-                uint32_t b0, b1, b2, b3;
-                ldmatrix_x4_trans(d0 + boff, b0, b1, b2, b3);
-                mma_bf16_16816(gv4[2 * np], pl, b0, b1);
-                mma_bf16_16816(gv4[2 * np + 1], pl, b2, b3);
-                mma_bf16_16816(gv4[2 * np], ph, b0, b1);
-                mma_bf16_16816(gv4[2 * np + 1], ph, b2, b3);
-                ldmatrix_x4_trans(q0 + boff, b0, b1, b2, b3);
-                mma_bf16_16816(gk4[2 * np], sl, b0, b1);
-                mma_bf16_16816(gk4[2 * np + 1], sl, b2, b3);
-                mma_bf16_16816(gk4[2 * np], sh, b0, b1);
-                mma_bf16_16816(gk4[2 * np + 1], sh, b2, b3);
+                    for (int np = 0; np < 2; ++np) {
+                        const int row = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+                        uint32_t b0, b1, b2, b3;
+                        ldmatrix_x4_trans(bbase + (uint32_t)(row * kTileRow + 16 * np + 8 * (lane >> 4)) * 2u,
+                                          b0, b1, b2, b3);
+                        mma_bf16_16816(g4[2 * np], al, b0, b1);
+                        mma_bf16_16816(g4[2 * np + 1], al, b2, b3);
+                        mma_bf16_16816(g4[2 * np], ah, b0, b1);
+                        mma_bf16_16816(g4[2 * np + 1], ah, b2, b3);
+                    }
+                }
+                const float sc4 = pass == 0 ? a.scale : 1.f;
+                float *dst = pass == 0 ? a.dk : a.dv;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int key = 16 * warp + g + 8 * hh;
+                    const int y = sy + key / a.wr, x = sx + key % a.wr;
+                    const int64_t off = ((b * a.H + y) * a.W + x) * a.C + c0 + 2 * t;
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt)
+                        atomicAdd(reinterpret_cast<float2 *>(dst + off + 8 * nt),
+                                  make_float2(g4[nt][2 * hh] * sc4, g4[nt][2 * hh + 1] * sc4));
+                }
+                __syncthreads();  // the arrays are rewritten next
             }
         }
-        const int sy = (s / a.n_win) * a.hr, sx = (s % a.n_win) * a.wr;
+        const int y0 = ry * a.hr, x0 = rx * a.wr;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-            const int key = 16 * warp + g + 8 * hh;
-            const int y = sy + key / a.wr, x = sx + key % a.wr;
-            const int64_t off = ((b * a.H + y) * a.W + x) * a.C + c0 + 2 * t;
+            const int row = 16 * warp + g + 8 * hh;
+            const int y = y0 + row / a.wr, x = x0 + row % a.wr;
+            float *dst = a.dq + ((b * a.H + y) * a.W + x) * a.C + c0 + 2 * t;
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
-                atomicAdd(reinterpret_cast<float2 *>(a.dk + off + 8 * nt),
-                          make_float2(gk4[nt][2 * hh] * a.scale, gk4[nt][2 * hh + 1] * a.scale));
-                atomicAdd(reinterpret_cast<float2 *>(a.dv + off + 8 * nt),
-                          make_float2(gv4[nt][2 * hh], gv4[nt][2 * hh + 1]));
+                const float2 v2 = *reinterpret_cast<const float2 *>(dq_own + 8 * hh * kDqRow + 8 * nt);
+                *reinterpret_cast<float2 *>(dst + 8 * nt) = make_float2(v2.x * a.scale, v2.y * a.scale);
             }
         }
-        __syncthreads();  // p and ds are rewritten by the next region
-    }
-    const int y0 = ry * a.hr, x0 = rx * a.wr;
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        const int row = 16 * warp + g + 8 * hh;
-        const int y = y0 + row / a.wr, x = x0 + row % a.wr;
-        float *dst = a.dq + ((b * a.H + y) * a.W + x) * a.C + c0 + 2 * t;
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-            *reinterpret_cast<float2 *>(dst + 8 * nt) = make_float2(dq[nt][2 * hh] * a.scale, dq[nt][2 * hh + 1] * a.scale);
+        if (!has_next) break;
+        item = next;
     }
 }
 
@@ -868,9 +959,10 @@ cudaError_t launch_attend_backward(const void *q, const void *k, const void *v, 
     a.scale = (float)(1.0 / sqrt((double)g.hd));
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)g.hd));
     if (g.rs == 64 && g.hd == 32 && bf16) {
-        // 64-token regions, heads of 32 channels, bf16: the tensor-core kernel
-        const long long blocks = (long long)g.B * g.R * g.heads;
-        if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+        // 64-token regions, heads of 32 channels, bf16: the persistent tensor-core kernel
+        const long long items = (long long)g.B * g.R * g.heads;
+        if (items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+        a.nitems = (int)items;
         const size_t bytes = (size_t)g.B * g.H * g.W * g.C * sizeof(float);
         cudaError_t e = cudaMemsetAsync(dk, 0, bytes, stream);
         if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, bytes, stream);
@@ -879,6 +971,9 @@ cudaError_t launch_attend_backward(const void *q, const void *k, const void *v, 
         int dev = 0;
         if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
         if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+        int sms = 0;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        const long long blocks = std::min(items, (long long)kMmaBackCtasPerSm * std::max(sms, 1));
         if ((int)kMmaBackSmem > 48 * 1024 && (int)kMmaBackSmem > granted_mma[dev]) {
             if ((e = cudaFuncSetAttribute(attend_backward_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           (int)kMmaBackSmem)) != cudaSuccess)
@@ -896,17 +991,16 @@ cudaError_t launch_attend_backward(const void *q, const void *k, const void *v, 
         cudaError_t e = cudaMemsetAsync(dk, 0, bytes, stream);
         if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, bytes, stream);
         if (e != cudaSuccess) return e;
-        void (*kernel)(const BackArgs) =
-            bf16 ? attend_backward_tiled_kernel<__nv_bfloat16> : attend_backward_tiled_kernel<float>;
-        static int granted_tiled[2][64] = {{0}};
+        void (*kernel)(const BackArgs) = attend_backward_tiled_kernel<float>;
+        static int granted_tiled[64] = {0};
         int dev = 0;
         if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
         if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-        if ((int)kTiledSmem > granted_tiled[bf16][dev]) {
+        if ((int)kTiledSmem > granted_tiled[dev]) {
             if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTiledSmem)) !=
                 cudaSuccess)
                 return e;
-            granted_tiled[bf16][dev] = (int)kTiledSmem;
+            granted_tiled[dev] = (int)kTiledSmem;
         }
         return launch_pdl(kernel, dim3((unsigned)blocks), dim3(kTiledThreads), kTiledSmem, stream, a);
     }

@@ -174,7 +174,9 @@ def test_forward_lepe(name):
 
 BACK_SHAPES = [WORKLOADS["stage1"].with_(B=2), WORKLOADS["stage2"].with_(B=2), WORKLOADS["stage3"].with_(B=2),
                WORKLOADS["stage4"].with_(B=2), WORKLOADS["highres"].with_(B=1), WORKLOADS["tiny_f32"],
-               _w("rs15_f32", 2, 12, 20, 32, 4, 4, 3, "f32"), _w("hd64_bf16", 1, 16, 16, 128, 2, 4, 3, "bf16")]
+               _w("rs15_f32", 2, 12, 20, 32, 4, 4, 3, "f32"), _w("hd64_bf16", 1, 16, 16, 128, 2, 4, 3, "bf16"),
+               # 64-token regions of 32-channel heads in fp32: the register-tiled CUDA-core kernel
+               _w("rs64_f32", 2, 32, 32, 64, 2, 4, 3, "f32"), _w("rs64_f32_topk1", 3, 24, 24, 64, 2, 3, 1, "f32")]
 
 
 @pytest.mark.parametrize("w", BACK_SHAPES, ids=[w.name for w in BACK_SHAPES])
@@ -194,6 +196,27 @@ def test_backward(w):
         check_grad(g.cpu().numpy(), r, f"{w.name} {n}")
 
 
+MANY_ITEMS = [WORKLOADS["stage1"].with_(B=24), WORKLOADS["highres"].with_(B=2)]
+
+
+@pytest.mark.parametrize("w", MANY_ITEMS, ids=[w.name for w in MANY_ITEMS])
+def test_backward_many_items_per_cta(w):
+    """Batches large enough that each CTA of the tensor-core kernel (a persistent grid of a few
+    CTAs per SM) takes several (image, region, head) items in turn, with one routed region
+    (stage1, B = 24: 2352 items) and with four (highres, B = 2: 1024 items); every element."""
+    inp, (q, k, v) = make(w)
+    rng = np.random.Generator(np.random.PCG64(19))
+    dout = torch.from_numpy(rng.standard_normal((w.B, w.H, w.W, w.C)).astype(np.float32)).to(torch.bfloat16).cuda()
+    idx = bra.route(q, k, w.n_win, w.topk)
+    dq, dk, dv = bra.attend_backward(q, k, v, idx, dout, w.heads, w.n_win)
+    torch.cuda.synchronize()
+    assert bra.check_device_error() == 0
+    rq, rk, rv = oracle.attend_backward(inp["q"], inp["k"], inp["v"], idx.cpu().numpy(), host_values(dout), w.heads,
+                                        w.n_win)
+    for g, r, n in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
+        check_grad(g.cpu().numpy(), r, f"{w.name} B={w.B} {n}")
+
+
 def test_backward_duplicates():
     w = _w("dup", 2, 16, 16, 64, 2, 4, 4, "bf16", "iid", 12)
     inp, (q, k, v) = make(w)
@@ -207,25 +230,28 @@ def test_backward_duplicates():
         check_grad(g.cpu().numpy(), r, f"duplicates {n}")
 
 
-def test_backward_tiled_many_regions_and_bad_entries():
-    """The register-tiled kernel of 64-token regions: 18 routed regions (past the 16 it keeps in
-    shared memory), duplicates, then one out-of-range entry that is skipped and flagged."""
-    w = _w("rs64_r25", 2, 40, 40, 64, 2, 5, 18, "bf16", "iid", 21)
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_backward_many_regions_and_bad_entries(dt):
+    """The kernels of 64-token regions (tensor cores for bf16, register tiles for fp32): 18 routed
+    regions (past the 16 they keep in shared memory), duplicates, then one out-of-range entry
+    that is skipped and flagged."""
+    w = _w("rs64_r25", 2, 40, 40, 64, 2, 5, 18, dt, "iid", 21)
     inp, (q, k, v) = make(w)
     rng = np.random.Generator(np.random.PCG64(17))
     idx = rng.integers(0, w.R, size=(w.B, w.R, w.topk)).astype(np.int32)
     idx[:, :, 5] = idx[:, :, 17]
-    dout = torch.from_numpy(rng.standard_normal((w.B, w.H, w.W, w.C)).astype(np.float32)).to(torch.bfloat16).cuda()
+    dout = torch.from_numpy(rng.standard_normal((w.B, w.H, w.W, w.C)).astype(np.float32)).to(q.dtype).cuda()
     rq, rk, rv = oracle.attend_backward(inp["q"], inp["k"], inp["v"], idx, host_values(dout), w.heads, w.n_win)
     dq, dk, dv = bra.attend_backward(q, k, v, torch.from_numpy(idx).cuda(), dout, w.heads, w.n_win)
     assert bra.check_device_error() == 0
     for g, r, n in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
-        check_grad(g.cpu().numpy(), r, f"tiled, 18 regions {n}")
-    bad = np.concatenate([idx[:, :, :9], np.full((w.B, w.R, 1), -3, np.int32), idx[:, :, 9:]], axis=-1)
-    dq, dk, dv = bra.attend_backward(q, k, v, torch.from_numpy(bad).cuda(), dout, w.heads, w.n_win)
-    assert bra.check_device_error() == 4
-    for g, r, n in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
-        check_grad(g.cpu().numpy(), r, f"tiled, bad entry skipped {n}")
+        check_grad(g.cpu().numpy(), r, f"{dt}, 18 regions {n}")
+    for at in (9, 0):  # an out-of-range entry in the middle, and first (the region loaded with the item)
+        bad = np.concatenate([idx[:, :, :at], np.full((w.B, w.R, 1), -3, np.int32), idx[:, :, at:]], axis=-1)
+        dq, dk, dv = bra.attend_backward(q, k, v, torch.from_numpy(bad).cuda(), dout, w.heads, w.n_win)
+        assert bra.check_device_error() == 4
+        for g, r, n in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
+            check_grad(g.cpu().numpy(), r, f"{dt}, bad entry {at} skipped {n}")
 
 
 # ------------------------------------------------------------------ auto_pad
