@@ -598,13 +598,6 @@ __device__ __forceinline__ void stage_bf16_tile(const __nv_bfloat16 *g, const Ba
     }
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
 // The same tile as stage_bf16_tile, by asynchronous copies that land while the CTA computes
 __device__ __forceinline__ void fetch_bf16_tile(const __nv_bfloat16 *g, const BackArgs &a, int64_t b, int y0, int x0,
                                                 int c0, __nv_bfloat16 *dst)

@@ -141,7 +141,8 @@ def _lepe_params(C, seed=5):
 
 
 LEPE_SHAPES = [WORKLOADS["stage1"].with_(B=8), WORKLOADS["stage3"].with_(B=4), WORKLOADS["tiny_f32"],
-               _w("odd_f32", 2, 7, 9, 12, 3, 1, 1, "f32"), _w("odd_bf16", 3, 13, 6, 40, 5, 1, 1, "bf16")]
+               _w("odd_f32", 2, 7, 9, 12, 3, 1, 1, "f32"), _w("odd_bf16", 3, 13, 6, 40, 5, 1, 1, "bf16"),
+               _w("ragged_bf16_c64", 3, 21, 13, 64, 2, 1, 1, "bf16")]
 
 
 @pytest.mark.parametrize("w", LEPE_SHAPES, ids=[w.name for w in LEPE_SHAPES])
